@@ -1,0 +1,395 @@
+"""Pins for the CPU oracle: checks it against what the pages and the
+mathematics fix, never against a retyped copy of its own formulas.
+
+Every test here runs without a GPU.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([part.split() for part in line.split("|")])
+    return rows
+
+
+def _row_as_bitstream(words_row):
+    """A row of uint32 words read as one little-endian integer."""
+    return int.from_bytes(np.ascontiguousarray(words_row, dtype="<u4").tobytes(), "little")
+
+
+# ------------------------------------------------------------------ packing
+
+def test_pack_golden_words(orc):
+    """Hand-computed words of the LSB-first b-bit layout (nuvec-nn QuantizedLinear, weight)."""
+    for (bits,), codes, words in _golden_rows("pack_words.txt"):
+        bits = int(bits)
+        q = np.array([[int(c) for c in codes]], np.uint8)
+        want = np.array([[int(w, 16) for w in words]], np.uint32)
+        got = orc.pack(q, bits)
+        assert got.shape == want.shape
+        assert np.array_equal(got, want), (bits, got, want)
+        assert np.array_equal(orc.unpack(got, q.shape[1], bits), q)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_pack_is_a_little_endian_bitstream(orc, bits):
+    """Row of words == sum_k q[k] << (bits*k) as one integer; unpack inverts pack."""
+    rng = np.random.default_rng(bits)
+    q = rng.integers(0, 2 ** bits, size=(5, 256)).astype(np.uint8)
+    words = orc.pack(q, bits)
+    assert words.shape == (5, 256 * bits // 32)
+    for n in range(q.shape[0]):
+        expect = sum(int(c) << (bits * k) for k, c in enumerate(q[n]))
+        assert _row_as_bitstream(words[n]) == expect
+    assert np.array_equal(orc.unpack(words, 256, bits), q)
+
+
+def test_pack_8bit_is_byte_order(orc):
+    q = np.arange(64, dtype=np.uint8).reshape(2, 32) * 3
+    words = orc.pack(q, 8)
+    assert np.array_equal(words.view(np.uint8).reshape(2, 32), q)
+
+
+def test_pack_rejects_out_of_range(orc):
+    with pytest.raises(orc.OracleError):
+        orc.pack(np.full((1, 8), 16, np.uint8), 4)
+
+
+# ------------------------------------------------------------------ bf16 rounding
+
+def test_bf16_rounding_matches_torch(orc):
+    """The oracle's own bf16 rounding agrees with torch's RNE conversion."""
+    v = np.concatenate([synth.normal(5, (4096,), 1.0), synth.normal(6, (4096,), 1e-3),
+                        np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 3.4e38, -1e-40], np.float32)])
+    _, bits_t = synth.to_bf16(v)
+    assert np.array_equal(orc.f32_to_bf16_bits(v), bits_t)
+    # halfway cases: 1 + 2^-8 is a tie between 1 and 1 + 2^-7 -> even (1.0)
+    assert orc.bf16_bits_to_f32(orc.f32_to_bf16_bits(np.array([1.00390625], np.float32)))[0] == 1.0
+
+
+# ------------------------------------------------------------------ affine quantize / dequantize
+
+def _dyadic_case(N, K, g, bits, seed):
+    """w = bias + q*scale exactly, scale a power of two, each group holding
+    both 0 and 2^b-1 so that min-max recovers scale and bias exactly."""
+    rng = np.random.default_rng(seed)
+    G = K // g
+    qmax = 2 ** bits - 1
+    q = rng.integers(0, qmax + 1, size=(N, K)).astype(np.uint8)
+    for n in range(N):
+        for gi in range(G):
+            pos = rng.choice(g, size=2, replace=False) + gi * g
+            q[n, pos[0]] = 0
+            q[n, pos[1]] = qmax
+    e = rng.integers(6, 12, size=(N, G))
+    scale = np.ldexp(1.0, -e).astype(np.float32)
+    bias = (rng.integers(-64, 64, size=(N, G)) * 2.0 ** -6).astype(np.float32)
+    w = np.empty((N, K), np.float32)
+    for n in range(N):
+        for k in range(K):
+            w[n, k] = Fraction(float(bias[n, k // g])) + int(q[n, k]) * Fraction(float(scale[n, k // g]))
+    return q, scale, bias, w
+
+
+@pytest.mark.parametrize("bits,g", [(2, 32), (4, 64), (8, 128), (4, 128)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_quantize_recovers_dyadic_grid(orc, bits, g, bf16):
+    """Weights on an exact grid come back as the same codes, scale and bias."""
+    q, scale, bias, w = _dyadic_case(6, 2 * g, g, bits, seed=bits * 1000 + g)
+    codes, s, b = orc.affine_quantize(w, bits, g, bf16)
+    assert np.array_equal(s, scale)
+    assert np.array_equal(b, bias)
+    assert np.array_equal(orc.unpack(codes, w.shape[1], bits), q)
+    # and dequantize reproduces w exactly
+    assert np.array_equal(orc.affine_dequantize(codes, s, b, w.shape[1], bits, g), w)
+
+
+@pytest.mark.parametrize("bits,g", [(2, 64), (4, 64), (4, 128), (8, 64), (4, 32)])
+def test_quantize_roundtrip_within_half_scale(orc, bits, g):
+    """|w - dequant(quant(w))| <= scale/2 (plus fp32 rounding of the step) for fp32 params."""
+    w = synth.normal(11, (64, 4 * g), 0.02)
+    codes, s, b = orc.affine_quantize(w, bits, g, False)
+    wh = orc.affine_dequantize(codes, s, b, w.shape[1], bits, g)
+    srep = np.repeat(s, g, axis=1).astype(np.float64)
+    err = np.abs(w.astype(np.float64) - wh)
+    bound = srep * (0.5 + 2.0 ** -21 * 2 ** bits) + np.abs(w) * 2.0 ** -22 + 1e-30
+    assert np.all(err <= bound), float((err - bound).max())
+    # the group minimum maps to code 0 and the maximum to 2^b - 1
+    q = orc.unpack(codes, w.shape[1], bits)
+    G = w.shape[1] // g
+    wg = w.reshape(64, G, g)
+    qg = q.reshape(64, G, g)
+    rows = np.arange(64)[:, None]
+    grp = np.arange(G)[None, :]
+    assert np.all(qg[rows, grp, wg.argmin(axis=2)] == 0)
+    assert np.all(qg[rows, grp, wg.argmax(axis=2)] == 2 ** bits - 1)
+    # scale and bias are exactly the min-max pair
+    assert np.array_equal(b, wg.min(axis=2))
+
+
+def test_quantize_roundtrip_bf16_params(orc):
+    """bf16-stored params: unclipped elements stay within scale_p/2; params are bf16 values."""
+    bits, g = 4, 128
+    w = synth.normal(12, (64, 512), 0.02)
+    codes, s, b = orc.affine_quantize(w, bits, g, True)
+    for p in (s, b):
+        assert np.all((p.view(np.uint32) & 0xFFFF) == 0)
+    wh = orc.affine_dequantize(codes, s, b, 512, bits, g)
+    srep = np.repeat(s, g, axis=1).astype(np.float64)
+    brep = np.repeat(b, g, axis=1).astype(np.float64)
+    t = (w - brep) / srep
+    inside = (t >= -0.5) & (t <= 2 ** bits - 1 + 0.5)
+    err = np.abs(w.astype(np.float64) - wh)
+    bound = srep * (0.5 + 2.0 ** -19) + np.abs(w) * 2.0 ** -22
+    assert inside.mean() > 0.9
+    assert np.all(err[inside] <= bound[inside])
+
+
+def test_quantize_constant_group(orc):
+    """A constant group gets scale 1, code 0 and dequantizes to itself."""
+    w = np.full((2, 64), 0.125, np.float32)
+    w[1, :] = -3.0
+    codes, s, b = orc.affine_quantize(w, 4, 64, False)
+    assert np.all(s == 1.0)
+    assert np.array_equal(b[:, 0], np.array([0.125, -3.0], np.float32))
+    assert np.all(codes == 0)
+    assert np.array_equal(orc.affine_dequantize(codes, s, b, 64, 4, 64), w)
+
+
+def test_quantize_rejects_bad_group(orc):
+    with pytest.raises(orc.OracleError):
+        orc.affine_quantize(np.zeros((2, 96), np.float32), 4, 64, False)
+
+
+# ------------------------------------------------------------------ affine matmul
+
+def _bitstream_codes(words_row, K, bits):
+    """Codes of one packed row, read from its little-endian integer (not via orc.unpack)."""
+    v = _row_as_bitstream(words_row)
+    return [(v >> (bits * k)) & ((1 << bits) - 1) for k in range(K)]
+
+
+@pytest.mark.parametrize("bits,g,M,N,K", [(4, 32, 3, 5, 64), (2, 64, 2, 7, 128), (8, 32, 4, 3, 96)])
+def test_affine_matmul_brute_force_exact(orc, bits, g, M, N, K):
+    """Tiny layers with dyadic x and grid weights: the double sums are exact,
+    so the oracle must equal an exact rational brute force."""
+    q, scale, bias, w = _dyadic_case(N, K, g, bits, seed=7 + bits)
+    codes, s, b = orc.affine_quantize(w, bits, g, False)
+    rng = np.random.default_rng(3)
+    x = (rng.integers(-8, 9, size=(M, K)) * 0.25).astype(np.float32)
+    lb = (rng.integers(-8, 9, size=(N,)) * 0.125).astype(np.float32)
+    y, mag = orc.affine_matmul(x, codes, s, b, bits, g, lb)
+    for n in range(N):
+        qn = _bitstream_codes(codes[n], K, bits)
+        for m in range(M):
+            acc = Fraction(float(lb[n]))
+            absacc = Fraction(0)
+            for k in range(K):
+                wk = Fraction(float(s[n, k // g])) * qn[k] + Fraction(float(b[n, k // g]))
+                acc += Fraction(float(x[m, k])) * wk
+                absacc += abs(Fraction(float(x[m, k])) * wk)
+            assert y[m, n] == float(acc)
+            assert mag[m, n] == float(absacc)
+
+
+def test_affine_matmul_vs_torch_float64(orc):
+    """Random layer: oracle y == torch float64 x @ w_hat^T + bias (w_hat = oracle dequant)."""
+    case = synth.AffineCase("t", 3, 256, 40, 4, 64, "f32", "f32", True, seed=21)
+    w = case.weight()
+    codes, s, b = orc.affine_quantize(w, 4, 64, False)
+    wh = orc.affine_dequantize(codes, s, b, 256, 4, 64)
+    x = case.x().vals
+    lb = case.layer_bias().vals
+    y, _ = orc.affine_matmul(x, codes, s, b, 4, 64, lb)
+    ref = (torch.from_numpy(x).double() @ torch.from_numpy(wh).double().T
+           + torch.from_numpy(lb).double()).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-14)
+    # and without bias
+    y0, _ = orc.affine_matmul(x, codes, s, b, 4, 64, None)
+    assert np.allclose(y0, y - lb[None, :].astype(np.float64), rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------------ BitLinear
+
+def _ternary_case(M, K, N, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.integers(-16, 17, size=(M, K)).astype(np.float32)
+    return x
+
+
+@pytest.mark.parametrize("invert", [False, True])
+def test_bitlinear_code1_is_zero(orc, invert):
+    M, K, N = 3, 64, 16
+    x = _ternary_case(M, K, N, 1)
+    P = orc.pack_ternary(np.ones((N, K), np.uint8))
+    assert np.all(P == 0x55)
+    y, _ = orc.bitlinear(x, P, N, 0.5, invert)
+    assert np.all(y == 0.0)
+    lb = np.linspace(-1, 1, N).astype(np.float32)
+    yb, _ = orc.bitlinear(x, P, N, 0.5, invert, lb)
+    assert np.array_equal(yb, np.broadcast_to(lb.astype(np.float64), (M, N)))
+
+
+@pytest.mark.parametrize("invert,factor", [(False, 0.5), (True, 2.0)])
+def test_bitlinear_code2_and_code0_are_rowsums(orc, invert, factor):
+    M, K, N = 4, 128, 8
+    x = _ternary_case(M, K, N, 2)
+    rows = x.astype(np.float64).sum(axis=1)
+    P2 = orc.pack_ternary(np.full((N, K), 2, np.uint8))
+    P0 = orc.pack_ternary(np.zeros((N, K), np.uint8))
+    y2, _ = orc.bitlinear(x, P2, N, 0.5, invert)
+    y0, _ = orc.bitlinear(x, P0, N, 0.5, invert)
+    assert np.array_equal(y2, np.repeat(rows[:, None] * factor, N, axis=1))
+    assert np.array_equal(y0, np.repeat(-rows[:, None] * factor, N, axis=1))
+
+
+def test_bitlinear_one_hot_row_mapping(orc):
+    """Code j of byte P[r, k] drives output r + j*N/4 (BitLinear kernel source)."""
+    M, K, N = 2, 16, 12
+    R = N // 4
+    x = _ternary_case(M, K, N, 3)
+    for r in range(R):
+        for j in range(4):
+            for k in (0, 5, K - 1):
+                P = np.full((R, K), 0x55, np.uint8)
+                P[r, k] = (0x55 & ~(3 << (2 * j))) | (2 << (2 * j))
+                y, _ = orc.bitlinear(x, P, N, 1.0, False)
+                expect = np.zeros((M, N))
+                expect[:, r + j * R] = x[:, k]
+                assert np.array_equal(y, expect), (r, j, k)
+
+
+def test_bitlinear_random_vs_torch(orc):
+    """Random ternary codes, packed by the oracle, vs a float64 dense matmul of (code - 1)."""
+    M, K, N = 3, 256, 32
+    codes = synth.ternary_codes(4, N, K)
+    P = orc.pack_ternary(codes)
+    x = synth.normal(5, (M, K), 1.0)
+    y, mag = orc.bitlinear(x, P, N, 0.75, False)
+    wd = torch.from_numpy(codes.astype(np.float64) - 1.0)
+    ref = (torch.from_numpy(x).double() @ wd.T).numpy() * 0.75
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(mag, (torch.from_numpy(np.abs(x)).double() @ wd.abs().T).numpy() * 0.75)
+    yi, _ = orc.bitlinear(x, P, N, 0.75, True)
+    assert np.allclose(yi, ref / 0.75 * float(np.float32(1.0) / np.float32(0.75)), rtol=1e-12)
+
+
+def test_bitlinear_rejects_ragged_n(orc):
+    with pytest.raises(orc.OracleError):
+        orc.bitlinear(np.zeros((1, 8), np.float32), np.zeros((1, 8), np.uint8), 6, 1.0, False)
+
+
+# ------------------------------------------------------------------ int8 / int4
+
+def test_int8_rows_golden(orc):
+    (R, Cc), w, q, s = _golden_rows("int8_rows.txt")[0]
+    R, Cc = int(R), int(Cc)
+    w = np.array([float(v) for v in w], np.float32).reshape(R, Cc)
+    got_q, got_s = orc.quantize_int8_rows(w)
+    assert np.array_equal(got_q, np.array([int(v) for v in q], np.int8).reshape(R, Cc))
+    assert np.array_equal(got_s, np.array([float(v) for v in s], np.float32))
+
+
+def test_int8_rows_properties(orc):
+    w = synth.normal(8, (128, 1000), 0.02)
+    w[7] = 0.0
+    q, s = orc.quantize_int8_rows(w)
+    amax = np.abs(w).max(axis=1)
+    nz = amax > 0
+    assert np.array_equal(s[nz], (amax[nz] / np.float32(127.0)).astype(np.float32))
+    assert s[7] == 1.0 and np.all(q[7] == 0)
+    arg = np.abs(w).argmax(axis=1)
+    picked = q[np.arange(128), arg]
+    assert np.all(np.abs(picked[nz]) == 127)
+    assert np.all(np.sign(picked[nz]) == np.sign(w[np.arange(128), arg][nz]))
+    err = np.abs(w.astype(np.float64) - q.astype(np.float64) * s[:, None])
+    assert np.all(err <= s[:, None] * (0.5 + 2.0 ** -16))
+
+
+def test_int4_golden_nibbles(orc):
+    (K, N), w, packed, s = _golden_rows("int4_nibbles.txt")[0]
+    K, N = int(K), int(N)
+    w = np.array([float(v) for v in w], np.float32).reshape(K, N)
+    P, sc = orc.pack_int4_cols(w)
+    assert np.array_equal(P, np.array([int(v, 16) for v in packed], np.uint8).reshape(K // 2, N))
+    assert np.array_equal(sc, np.array([float(v) for v in s], np.float32))
+
+
+def test_int4_properties(orc):
+    w = synth.normal(9, (256, 96), 0.02)
+    P, s = orc.pack_int4_cols(w)
+    hi = (P >> 4).astype(np.int64)
+    lo = (P & 15).astype(np.int64)
+    c = np.empty((256, 96), np.int64)
+    c[0::2] = hi
+    c[1::2] = lo
+    arg = np.abs(w).argmax(axis=0)
+    picked = c[arg, np.arange(96)]
+    assert np.all(np.where(w[arg, np.arange(96)] > 0, picked == 15, picked == 1))
+    err = np.abs(w.astype(np.float64) - (c - 8) * s[None, :].astype(np.float64))
+    assert np.all(err <= s[None, :] * (0.5 + 2.0 ** -16))
+    assert c.min() >= 1  # round(w/scale) lies in [-7, 7]
+
+
+def test_int8_matmul_exact(orc):
+    rng = np.random.default_rng(10)
+    a = rng.integers(-128, 128, size=(17, 300)).astype(np.int8)
+    b = rng.integers(-128, 128, size=(23, 300)).astype(np.int8)
+    c = orc.int8_matmul(a, b)
+    assert np.array_equal(c.astype(np.int64), a.astype(np.int64) @ b.astype(np.int64).T)
+
+
+def test_w8a8_vs_float64_library(orc):
+    M, K, N = 5, 512, 24
+    x = synth.normal(11, (M, K), 1.0)
+    w = synth.normal(12, (N, K), 0.02)
+    qw, sw = orc.quantize_int8_rows(w)
+    lb = synth.normal(13, (N,), 0.01)
+    y, mag, qx, sx = orc.w8a8_linear(x, qw, sw, lb)
+    qx2, sx2 = orc.quantize_int8_rows(x)
+    assert np.array_equal(qx, qx2) and np.array_equal(sx, sx2)
+    acc = qx.astype(np.float64) @ qw.astype(np.float64).T
+    ref = acc * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64) + lb[None, :]
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-13)
+    # the dequantized product approximates the float product
+    assert np.allclose(y - lb, x.astype(np.float64) @ w.astype(np.float64).T, atol=0.05 * np.abs(y).max())
+
+
+def test_w4a8_matches_w8a8_on_integer_weights(orc):
+    """Integer weights in [-7, 7] with a +-7 in every column pack with scale 1,
+    so W4A8 must equal W8A8 on the same integers (nibble order and zero point)."""
+    rng = np.random.default_rng(14)
+    M, K, N = 4, 64, 10
+    wint = rng.integers(-7, 8, size=(K, N)).astype(np.float32)
+    wint[rng.integers(0, K, size=N), np.arange(N)] = 7.0
+    P, s4 = orc.pack_int4_cols(wint)
+    assert np.all(s4 == 1.0)
+    x = synth.normal(15, (M, K), 1.0)
+    y4, m4, qx4, sx4 = orc.w4a8_linear(x, P, s4)
+    y8, m8, qx8, sx8 = orc.w8a8_linear(x, wint.T.astype(np.int8), np.ones(N, np.float32))
+    assert np.array_equal(y4, y8) and np.array_equal(m4, m8)
+
+
+def test_quantize_golden_ties(orc):
+    """Half steps round to even (hand-computed fixture)."""
+    (bits, g), w, codes = _golden_rows("affine_ties.txt")[0]
+    bits, g = int(bits), int(g)
+    w = np.array([[float(v) for v in w]], np.float32)
+    want = np.array([[int(v) for v in codes]], np.uint8)
+    for bf16 in (False, True):
+        c, s, b = orc.affine_quantize(w, bits, g, bf16)
+        assert s[0, 0] == 1.0 and b[0, 0] == 0.0
+        assert np.array_equal(orc.unpack(c, g, bits), want)
