@@ -1,0 +1,384 @@
+// k_quant.cu -- quantisers and the dequantiser (bandwidth-bound, bit-exact).
+//
+//  * affine group quantize / dequantize of the MLX format
+//    [nuvec-nn QuantizedLinear: from_linear, dequantized_weight;
+//     cider/ops.py pergroup_linear docstring: quantize and dequantize formulas]
+//  * per-row symmetric int8 (weights and per-token activations)
+//    [cider/ops.py quantize_weight_int8; quant_a of perchannel_linear / w4a8_linear]
+//  * per-column int4 with zero point 8, two codes per byte
+//    [cider/ops.py pack_weight_int4]
+//
+// Every quantisation decision is taken in fp32 with IEEE operations that
+// cannot be contracted (__fsub_rn / __fdiv_rn / __fmaf_rn) and rintf (round
+// half to even), so codes match the CPU reference bit for bit.
+#include "qlin_common.cuh"
+
+namespace qlin {
+namespace {
+
+template <typename T> struct Vec;  // loads of N consecutive elements as floats
+
+QLIN_DEV float load_elem(const float* p, int64_t i) { return p[i]; }
+QLIN_DEV float load_elem(const __nv_bfloat16* p, int64_t i) { return __bfloat162float(p[i]); }
+
+// ---------------------------------------------------------------- affine quantize
+// One warp per (row, group).  Lane l holds CPL = g/32 consecutive values.
+template <typename TW, typename TP, int BITS, int G>
+__global__ void __launch_bounds__(256) affine_quantize_kernel(const TW* __restrict__ w, int64_t N, int64_t K,
+                                                              uint32_t* __restrict__ codes, TP* __restrict__ scales,
+                                                              TP* __restrict__ biases)
+{
+    constexpr int CPL = G / 32;          // codes per lane
+    constexpr int CPW = 32 / BITS;       // codes per word
+    constexpr int LPW = CPW / CPL;       // lanes sharing one word
+    constexpr float QMAX = float((1 << BITS) - 1);
+    const int64_t groups_per_row = K / G;
+    const int64_t gid = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    if (gid >= N * groups_per_row)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int64_t n = gid / groups_per_row;
+    const int64_t gi = gid % groups_per_row;
+    const TW* wg = w + n * K + gi * G + lane * CPL;
+    float v[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i)
+        v[i] = load_elem(wg, i);
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 1; i < CPL; ++i) {
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    float scale = __fdiv_rn(__fsub_rn(mx, mn), QMAX);
+    float bias = mn;
+    scale = to_float(from_float<TP>(scale));
+    bias = to_float(from_float<TP>(bias));
+    if (scale == 0.0f)
+        scale = 1.0f;
+    if (lane == 0) {
+        scales[n * groups_per_row + gi] = from_float<TP>(scale);
+        biases[n * groups_per_row + gi] = from_float<TP>(bias);
+    }
+    uint32_t part = 0;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        float t = rintf(__fdiv_rn(__fsub_rn(v[i], bias), scale));
+        t = fminf(fmaxf(t, 0.0f), QMAX);
+        const int k_in_word = (lane * CPL + i) % CPW;
+        part |= static_cast<uint32_t>(t) << (BITS * k_in_word);
+    }
+#pragma unroll
+    for (int off = 1; off < LPW; off <<= 1)
+        part |= __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane % LPW == 0) {
+        const int64_t words_per_row = K * BITS / 32;
+        codes[n * words_per_row + gi * (G * BITS / 32) + (lane * CPL) / CPW] = part;
+    }
+}
+
+// ---------------------------------------------------------------- affine dequantize
+// One thread per packed word.
+template <typename TP, typename TO, int BITS>
+__global__ void __launch_bounds__(256) affine_dequantize_kernel(const uint32_t* __restrict__ codes,
+                                                                const TP* __restrict__ scales,
+                                                                const TP* __restrict__ biases, int64_t N, int64_t K,
+                                                                int g, TO* __restrict__ out)
+{
+    constexpr int CPW = 32 / BITS;
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    const int64_t words_per_row = K / CPW;
+    const int64_t total = N * words_per_row;
+    const int64_t groups_per_row = K / g;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = idx / words_per_row;
+        const int64_t wi = idx % words_per_row;
+        const int64_t k0 = wi * CPW;
+        const float s = to_float(scales[n * groups_per_row + k0 / g]);
+        const float b = to_float(biases[n * groups_per_row + k0 / g]);
+        const uint32_t word = __ldg(codes + idx);
+        TO vals[CPW];
+#pragma unroll
+        for (int i = 0; i < CPW; ++i)
+            vals[i] = from_float<TO>(__fmaf_rn(static_cast<float>((word >> (BITS * i)) & MASK), s, b));
+        // CPW * sizeof(TO) is 8..64 bytes and out + n*K + k0 is aligned to it.
+        constexpr int BYTES = CPW * (int)sizeof(TO);
+        TO* dst = out + n * K + k0;
+        if constexpr (BYTES >= 16) {
+#pragma unroll
+            for (int c = 0; c < BYTES / 16; ++c)
+                reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(vals)[c];
+        } else {
+            *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(vals);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- per-row int8
+// One block per row: absmax, then quantise (second read comes from L1/L2).
+template <typename TW>
+__global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __restrict__ w, int64_t C,
+                                                                 int8_t* __restrict__ q, float* __restrict__ scale,
+                                                                 int32_t* __restrict__ rowsum)
+{
+    __shared__ float red[8];
+    __shared__ int ired[8];
+    const int64_t r = blockIdx.x;
+    const TW* row = w + r * C;
+    float amax = 0.0f;
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x)
+        amax = fmaxf(amax, fabsf(load_elem(row, c)));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x / 32] = amax;
+    __syncthreads();
+    amax = red[0];
+    for (int i = 1; i < (int)(blockDim.x / 32); ++i)
+        amax = fmaxf(amax, red[i]);
+    float s = __fdiv_rn(amax, 127.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    if (threadIdx.x == 0)
+        scale[r] = s;
+    int sum = 0;
+    int8_t* qrow = q + r * C;
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
+        float t = rintf(__fdiv_rn(load_elem(row, c), s));
+        t = fminf(fmaxf(t, -128.0f), 127.0f);
+        const int qi = static_cast<int>(t);
+        qrow[c] = static_cast<int8_t>(qi);
+        sum += qi;
+    }
+    if (rowsum) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if ((threadIdx.x & 31) == 0)
+            ired[threadIdx.x / 32] = sum;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int t = 0;
+            for (int i = 0; i < (int)(blockDim.x / 32); ++i)
+                t += ired[i];
+            rowsum[r] = t;
+        }
+    }
+}
+
+// Vectorised variant for bf16 rows with C % 8 == 0 (16-byte loads, 8-byte stores).
+__global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                        int64_t C, int8_t* __restrict__ q,
+                                                                        float* __restrict__ scale,
+                                                                        int32_t* __restrict__ rowsum)
+{
+    __shared__ float red[8];
+    __shared__ int ired[8];
+    const int64_t r = blockIdx.x;
+    const uint4* row = reinterpret_cast<const uint4*>(w + r * C);
+    const int64_t C8 = C / 8;
+    float amax = 0.0f;
+    for (int64_t c = threadIdx.x; c < C8; c += blockDim.x) {
+        const uint4 v = __ldg(row + c);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] << 16)));
+            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] & 0xffff0000u)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x / 32] = amax;
+    __syncthreads();
+    amax = red[0];
+    for (int i = 1; i < (int)(blockDim.x / 32); ++i)
+        amax = fmaxf(amax, red[i]);
+    float s = __fdiv_rn(amax, 127.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    if (threadIdx.x == 0)
+        scale[r] = s;
+    int sum = 0;
+    uint2* qrow = reinterpret_cast<uint2*>(q + r * C);
+    for (int64_t c = threadIdx.x; c < C8; c += blockDim.x) {
+        const uint4 v = __ldg(row + c);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t bits = (i & 1) ? (u[i / 2] & 0xffff0000u) : (u[i / 2] << 16);
+            float t = rintf(__fdiv_rn(__uint_as_float(bits), s));
+            t = fminf(fmaxf(t, -128.0f), 127.0f);
+            const int qi = static_cast<int>(t);
+            sum += qi;
+            packed[i / 4] |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * (i % 4));
+        }
+        qrow[c] = make_uint2(packed[0], packed[1]);
+    }
+    if (rowsum) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if ((threadIdx.x & 31) == 0)
+            ired[threadIdx.x / 32] = sum;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int t = 0;
+            for (int i = 0; i < (int)(blockDim.x / 32); ++i)
+                t += ired[i];
+            rowsum[r] = t;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- per-column int4
+// Block = 32 columns x 8 row slices.
+template <typename TW>
+__global__ void __launch_bounds__(256) pack_int4_cols_kernel(const TW* __restrict__ w, int64_t K, int64_t N,
+                                                             uint8_t* __restrict__ packed, float* __restrict__ scale)
+{
+    __shared__ float red[8][32];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int64_t n = (int64_t)blockIdx.x * 32 + tx;
+    float amax = 0.0f;
+    if (n < N)
+        for (int64_t k = ty; k < K; k += 8)
+            amax = fmaxf(amax, fabsf(load_elem(w, k * N + n)));
+    red[ty][tx] = amax;
+    __syncthreads();
+    amax = red[0][tx];
+#pragma unroll
+    for (int i = 1; i < 8; ++i)
+        amax = fmaxf(amax, red[i][tx]);
+    float s = __fdiv_rn(amax, 7.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    if (n >= N)
+        return;
+    if (ty == 0)
+        scale[n] = s;
+    for (int64_t i = ty; i < K / 2; i += 8) {
+        uint32_t c[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float t = __fadd_rn(rintf(__fdiv_rn(load_elem(w, (2 * i + h) * N + n), s)), 8.0f);
+            t = fminf(fmaxf(t, 0.0f), 15.0f);
+            c[h] = static_cast<uint32_t>(t);
+        }
+        packed[i * N + n] = static_cast<uint8_t>((c[0] << 4) | c[1]);
+    }
+}
+
+template <typename TW, typename TP, int BITS>
+cudaError_t quantize_dispatch_g(const TW* w, int64_t N, int64_t K, int g, uint32_t* codes, TP* s, TP* b,
+                                cudaStream_t st)
+{
+    const int64_t groups = N * (K / g);
+    const unsigned blocks = (unsigned)((groups + 7) / 8);
+    switch (g) {
+    case 32: affine_quantize_kernel<TW, TP, BITS, 32><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b); break;
+    case 64: affine_quantize_kernel<TW, TP, BITS, 64><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b); break;
+    default: affine_quantize_kernel<TW, TP, BITS, 128><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b); break;
+    }
+    return cudaGetLastError();
+}
+
+template <typename TW, typename TP>
+cudaError_t quantize_dispatch_b(const void* w, int64_t N, int64_t K, int bits, int g, uint32_t* codes, void* s,
+                                void* b, cudaStream_t st)
+{
+    const TW* wp = static_cast<const TW*>(w);
+    TP* sp = static_cast<TP*>(s);
+    TP* bp = static_cast<TP*>(b);
+    switch (bits) {
+    case 2: return quantize_dispatch_g<TW, TP, 2>(wp, N, K, g, codes, sp, bp, st);
+    case 4: return quantize_dispatch_g<TW, TP, 4>(wp, N, K, g, codes, sp, bp, st);
+    default: return quantize_dispatch_g<TW, TP, 8>(wp, N, K, g, codes, sp, bp, st);
+    }
+}
+
+template <typename TP, typename TO>
+cudaError_t dequantize_dispatch(const uint32_t* codes, const void* s, const void* b, int64_t N, int64_t K, int bits,
+                                int g, void* out, cudaStream_t st, const DeviceInfo& dev)
+{
+    const int64_t words = N * K * bits / 32;
+    const int64_t want = (words + 255) / 256;
+    const unsigned blocks = (unsigned)(want < (int64_t)dev.sm_count * 16 ? want : (int64_t)dev.sm_count * 16);
+    const TP* sp = static_cast<const TP*>(s);
+    const TP* bp = static_cast<const TP*>(b);
+    TO* op = static_cast<TO*>(out);
+    switch (bits) {
+    case 2: affine_dequantize_kernel<TP, TO, 2><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    case 4: affine_dequantize_kernel<TP, TO, 4><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    default: affine_dequantize_kernel<TP, TO, 8><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_affine_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int bits, int g,
+                                   uint32_t* codes, void* scales, void* biases, qlin_dtype p_dt, cudaStream_t st,
+                                   const DeviceInfo&)
+{
+    if (w_dt == QLIN_F32)
+        return p_dt == QLIN_F32 ? quantize_dispatch_b<float, float>(w, N, K, bits, g, codes, scales, biases, st)
+                                : quantize_dispatch_b<float, __nv_bfloat16>(w, N, K, bits, g, codes, scales, biases, st);
+    return p_dt == QLIN_F32
+               ? quantize_dispatch_b<__nv_bfloat16, float>(w, N, K, bits, g, codes, scales, biases, st)
+               : quantize_dispatch_b<__nv_bfloat16, __nv_bfloat16>(w, N, K, bits, g, codes, scales, biases, st);
+}
+
+cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, const void* biases, qlin_dtype p_dt,
+                                     int64_t N, int64_t K, int bits, int g, void* out, qlin_dtype o_dt,
+                                     cudaStream_t st, const DeviceInfo& dev)
+{
+    if (p_dt == QLIN_F32)
+        return o_dt == QLIN_F32
+                   ? dequantize_dispatch<float, float>(codes, scales, biases, N, K, bits, g, out, st, dev)
+                   : dequantize_dispatch<float, __nv_bfloat16>(codes, scales, biases, N, K, bits, g, out, st, dev);
+    return o_dt == QLIN_F32
+               ? dequantize_dispatch<__nv_bfloat16, float>(codes, scales, biases, N, K, bits, g, out, st, dev)
+               : dequantize_dispatch<__nv_bfloat16, __nv_bfloat16>(codes, scales, biases, N, K, bits, g, out, st,
+                                                                   dev);
+}
+
+cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
+                                      int32_t* rowsum, cudaStream_t st, const DeviceInfo&)
+{
+    if (w_dt == QLIN_BF16 && C % 8 == 0 && (reinterpret_cast<uintptr_t>(w) & 15) == 0 &&
+        (reinterpret_cast<uintptr_t>(q) & 7) == 0)
+        quantize_int8_rows_bf16x8_kernel<<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
+                                                                       scale, rowsum);
+    else if (w_dt == QLIN_BF16)
+        quantize_int8_rows_kernel<__nv_bfloat16>
+            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q, scale, rowsum);
+    else
+        quantize_int8_rows_kernel<float><<<(unsigned)R, 256, 0, st>>>(static_cast<const float*>(w), C, q, scale,
+                                                                      rowsum);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64_t N, uint8_t* packed, float* scale,
+                                  cudaStream_t st, const DeviceInfo&)
+{
+    const unsigned blocks = (unsigned)((N + 31) / 32);
+    if (w_dt == QLIN_BF16)
+        pack_int4_cols_kernel<__nv_bfloat16>
+            <<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), K, N, packed, scale);
+    else
+        pack_int4_cols_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(w), K, N, packed, scale);
+    return cudaGetLastError();
+}
+
+}  // namespace qlin

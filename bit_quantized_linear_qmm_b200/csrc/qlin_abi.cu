@@ -1,0 +1,314 @@
+// qlin_abi.cu -- the extern "C" boundary of libqlin.so: argument validation,
+// device checks, workspace sizing and dispatch to the kernel launchers.
+// No exception crosses this file's functions; every failure is a qlin_status.
+#include <mutex>
+
+#include "qlin_common.cuh"
+
+namespace qlin {
+
+// Device status word: kernels OR kStatusTimeout into it when a bounded wait
+// gives up; qlin_get_device_status() reads and clears it.
+__device__ unsigned g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceSlot {
+    std::once_flag once;
+    qlin_status state = QLIN_ERR_DEVICE;
+    DeviceInfo info = {0, nullptr};
+};
+
+DeviceSlot g_slots[kMaxDevices];
+
+// Checks (once per device) that the current device is an sm_100 part, and
+// records its SM count and the address of the status word.  Must run with
+// that device current, outside stream capture (the first call per device).
+qlin_status current_device(DeviceInfo& out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return QLIN_ERR_DEVICE;
+    }
+    DeviceSlot& slot = g_slots[dev];
+    std::call_once(slot.once, [&slot, dev]() {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+            cudaGetLastError();
+            slot.state = QLIN_ERR_DEVICE;
+            return;
+        }
+        if (prop.major != 10 || prop.minor != 0) {
+            slot.state = QLIN_ERR_DEVICE;
+            return;
+        }
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            slot.state = QLIN_ERR_CUDA;
+            return;
+        }
+        slot.info.sm_count = prop.multiProcessorCount;
+        slot.info.status = static_cast<unsigned*>(p);
+        slot.state = QLIN_OK;
+    });
+    out = slot.info;
+    return slot.state;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dtype_ok(qlin_dtype d) { return d == QLIN_F32 || d == QLIN_BF16; }
+size_t dtype_size(qlin_dtype d) { return d == QLIN_F32 ? 4 : 2; }
+bool bits_ok(int b) { return b == 2 || b == 4 || b == 8; }
+bool group_ok(int g) { return g == 32 || g == 64 || g == 128; }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+qlin_status from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        return QLIN_OK;
+    cudaGetLastError();  // clear a non-sticky launch error
+    return e == cudaErrorNotSupported ? QLIN_ERR_UNSUPPORTED : QLIN_ERR_CUDA;
+}
+
+// Shape/type rules common to the affine-format calls.
+qlin_status check_affine(int64_t N, int64_t K, int bits, int g, qlin_dtype p_dt)
+{
+    if (N <= 0 || K <= 0 || N > INT32_MAX || K > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (!bits_ok(bits) || !group_ok(g) || !dtype_ok(p_dt))
+        return QLIN_ERR_UNSUPPORTED;
+    if (K % g != 0)
+        return QLIN_ERR_INVALID_ARG;
+    return QLIN_OK;
+}
+
+}  // namespace
+}  // namespace qlin
+
+using namespace qlin;
+
+extern "C" {
+
+const char* qlin_status_string(qlin_status s)
+{
+    switch (s) {
+    case QLIN_OK: return "QLIN_OK";
+    case QLIN_ERR_INVALID_ARG: return "QLIN_ERR_INVALID_ARG: invalid argument";
+    case QLIN_ERR_UNSUPPORTED: return "QLIN_ERR_UNSUPPORTED: unsupported bits/group/dtype combination";
+    case QLIN_ERR_MISALIGNED: return "QLIN_ERR_MISALIGNED: pointer or row pitch not 16-byte aligned";
+    case QLIN_ERR_DEVICE: return "QLIN_ERR_DEVICE: no sm_100 CUDA device current";
+    case QLIN_ERR_CUDA: return "QLIN_ERR_CUDA: CUDA runtime error";
+    case QLIN_ERR_TIMEOUT: return "QLIN_ERR_TIMEOUT: a bounded device wait expired";
+    case QLIN_ERR_WORKSPACE: return "QLIN_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "QLIN_ERR_?: unknown status";
+}
+
+int qlin_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size)
+{
+    (void)N;
+    (void)bits;
+    (void)group_size;
+    if (M <= 0 || K <= 0)
+        return 0;
+    switch (op) {
+    case QLIN_OP_W8A8: return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
+    case QLIN_OP_W4A8: return align256((size_t)M * (size_t)K) + 2 * align256((size_t)M * 4);
+    default: return 0;
+    }
+}
+
+qlin_status qlin_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int bits, int group_size,
+                          uint32_t* codes, void* scales, void* biases, qlin_dtype param_dt, void* stream)
+{
+    if (!w || !codes || !scales || !biases)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(w_dt))
+        return QLIN_ERR_UNSUPPORTED;
+    qlin_status s = check_affine(N, K, bits, group_size, param_dt);
+    if (s != QLIN_OK)
+        return s;
+    DeviceInfo dev;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    return from_cuda(launch_affine_quantize(w, w_dt, N, K, bits, group_size, codes, scales, biases, param_dt,
+                                            static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status qlin_dequantize(const uint32_t* codes, const void* scales, const void* biases, qlin_dtype param_dt,
+                            int64_t N, int64_t K, int bits, int group_size, void* w_out, qlin_dtype out_dt,
+                            void* stream)
+{
+    if (!codes || !scales || !biases || !w_out)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(out_dt))
+        return QLIN_ERR_UNSUPPORTED;
+    qlin_status s = check_affine(N, K, bits, group_size, param_dt);
+    if (s != QLIN_OK)
+        return s;
+    // one word's outputs go out as 8- or 16-byte vector stores
+    if (!aligned16(w_out) || (reinterpret_cast<uintptr_t>(codes) & 3u) != 0)
+        return QLIN_ERR_MISALIGNED;
+    DeviceInfo dev;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    return from_cuda(launch_affine_dequantize(codes, scales, biases, param_dt, N, K, bits, group_size, w_out, out_dt,
+                                              static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const uint32_t* codes,
+                        const void* scales, const void* biases, qlin_dtype param_dt, int64_t N, int bits,
+                        int group_size, const void* bias, void* y, void* workspace, size_t ws_bytes, void* stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (!x || !codes || !scales || !biases || !y || M <= 0 || M > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(x_dt))
+        return QLIN_ERR_UNSUPPORTED;
+    qlin_status s = check_affine(N, K, bits, group_size, param_dt);
+    if (s != QLIN_OK)
+        return s;
+    if (bits == 2 && group_size == 32)
+        return QLIN_ERR_UNSUPPORTED;
+    if (!aligned16(codes) || !aligned16(x) || (K * bits / 8) % 16 != 0 || (K * (int64_t)dtype_size(x_dt)) % 16 != 0)
+        return QLIN_ERR_MISALIGNED;
+    DeviceInfo dev;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    AffineGemvArgs a;
+    a.x = x;
+    a.x_dt = x_dt;
+    a.M = M;
+    a.K = K;
+    a.N = N;
+    a.codes = codes;
+    a.scales = scales;
+    a.biases = biases;
+    a.p_dt = param_dt;
+    a.bits = bits;
+    a.g = group_size;
+    a.bias = bias;
+    a.y = y;
+    return from_cuda(launch_affine_gemv(a, static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status bitlinear_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const uint8_t* packed, int64_t N,
+                             const float* weight_scale, int invert_weight_scale, const void* bias, void* y,
+                             void* stream)
+{
+    if (!x || !packed || !weight_scale || !y || M <= 0 || K <= 0 || N <= 0 || M > INT32_MAX || K > INT32_MAX ||
+        N > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (N % 4 != 0 || K % 16 != 0)
+        return QLIN_ERR_INVALID_ARG;
+    if (x_dt != QLIN_BF16)
+        return QLIN_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(packed))
+        return QLIN_ERR_MISALIGNED;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    BitlinearArgs a;
+    a.x = x;
+    a.x_dt = x_dt;
+    a.M = M;
+    a.K = K;
+    a.N = N;
+    a.packed = packed;
+    a.weight_scale = weight_scale;
+    a.invert = invert_weight_scale ? 1 : 0;
+    a.bias = bias;
+    a.y = y;
+    return from_cuda(launch_bitlinear_gemv(a, static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status qlin_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
+                                    void* stream)
+{
+    if (!w || !q || !scale || R <= 0 || C <= 0 || R > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(w_dt))
+        return QLIN_ERR_UNSUPPORTED;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    return from_cuda(
+        launch_quantize_int8_rows(w, w_dt, R, C, q, scale, nullptr, static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status qlin_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64_t N, uint8_t* packed, float* scale,
+                                void* stream)
+{
+    if (!w || !packed || !scale || K <= 0 || N <= 0 || K % 2 != 0 || N > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(w_dt))
+        return QLIN_ERR_UNSUPPORTED;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    return from_cuda(launch_pack_int4_cols(w, w_dt, K, N, packed, scale, static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status qlin_int8_matmul_int32(const int8_t* a, const int8_t* b, int64_t M, int64_t N, int64_t K, int32_t* c,
+                                   void* stream)
+{
+    (void)stream;
+    if (!a || !b || !c || M <= 0 || N <= 0 || K <= 0)
+        return QLIN_ERR_INVALID_ARG;
+    return QLIN_ERR_UNSUPPORTED;
+}
+
+qlin_status w8a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const int8_t* w, const float* scale_w,
+                        int64_t N, const void* bias, void* y, void* workspace, size_t ws_bytes, void* stream)
+{
+    (void)x_dt, (void)bias, (void)workspace, (void)ws_bytes, (void)stream;
+    if (!x || !w || !scale_w || !y || M <= 0 || N <= 0 || K <= 0)
+        return QLIN_ERR_INVALID_ARG;
+    return QLIN_ERR_UNSUPPORTED;
+}
+
+qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const uint8_t* packed_w,
+                        const float* scale_w, int64_t N, const void* bias, void* y, void* workspace, size_t ws_bytes,
+                        void* stream)
+{
+    (void)x_dt, (void)bias, (void)workspace, (void)ws_bytes, (void)stream;
+    if (!x || !packed_w || !scale_w || !y || M <= 0 || N <= 0 || K <= 0)
+        return QLIN_ERR_INVALID_ARG;
+    return QLIN_ERR_UNSUPPORTED;
+}
+
+qlin_status qlin_get_device_status(void* stream)
+{
+    DeviceInfo dev;
+    qlin_status s = current_device(dev);
+    if (s != QLIN_OK)
+        return s;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return QLIN_ERR_CUDA;
+    }
+    unsigned word = 0;
+    if (cudaMemcpy(&word, dev.status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return QLIN_ERR_CUDA;
+    }
+    if (word != 0) {
+        const unsigned zero = 0;
+        cudaMemcpy(dev.status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        return QLIN_ERR_TIMEOUT;
+    }
+    return QLIN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,240 @@
+// qlin_common.cuh -- shared device helpers of the sm_100a kernels (inline PTX
+// for mbarriers, bulk copies and the legacy warp MMA) and the internal launch
+// interface between the C ABI (qlin_abi.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "qlin.h"
+
+#define QLIN_DEV __device__ __forceinline__
+
+namespace qlin {
+
+// Bit set in the device status word when a bounded wait gave up.
+constexpr unsigned kStatusTimeout = 1u;
+// Bounded waits give up after this many nanoseconds of %globaltimer.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// ---------------------------------------------------------------- small device utilities
+
+QLIN_DEV unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+QLIN_DEV uint32_t smem_u32(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+QLIN_DEV float bf16_bits_to_float(uint16_t h)
+{
+    return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+template <typename T> QLIN_DEV float to_float(T v);
+template <> QLIN_DEV float to_float<float>(float v) { return v; }
+template <> QLIN_DEV float to_float<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> QLIN_DEV T from_float(float v);
+template <> QLIN_DEV float from_float<float>(float v) { return v; }
+template <> QLIN_DEV __nv_bfloat16 from_float<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// ---------------------------------------------------------------- mbarrier
+
+QLIN_DEV void mbar_init(uint64_t* bar, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+QLIN_DEV void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+QLIN_DEV void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+QLIN_DEV void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+QLIN_DEV bool mbar_try_wait(uint64_t* bar, unsigned parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up after
+// kWaitLimitNs, sets the timeout bit in *status and returns false.
+QLIN_DEV bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned* status)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity))
+                return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- bulk copies (1-D TMA)
+
+// Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte
+// aligned) completing as transaction bytes on `bar`.
+QLIN_DEV void bulk_g2s(void* smem_dst, const void* gmem_src, unsigned bytes, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------- cluster helpers
+
+QLIN_DEV unsigned cluster_ctarank()
+{
+    unsigned r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+QLIN_DEV void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+QLIN_DEV uint32_t map_shared_rank(uint32_t local_addr, unsigned rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+    return r;
+}
+
+QLIN_DEV float ld_shared_cluster_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+
+QLIN_DEV void pdl_wait_prior_grids()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+QLIN_DEV void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- warp MMA (m16n8k16 bf16, m16n8k32 s8)
+
+QLIN_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+QLIN_DEV void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+QLIN_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+QLIN_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv)
+{
+    // (a & mask) | orv
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));
+    return r;
+}
+
+}  // namespace qlin
+
+// ---------------------------------------------------------------- internal launch interface
+// Each launcher validates nothing (qlin_abi.cu did) and returns the launch status.
+namespace qlin {
+
+struct DeviceInfo {
+    int sm_count;
+    unsigned* status;  // device status word
+};
+
+cudaError_t launch_affine_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int bits, int g,
+                                   uint32_t* codes, void* scales, void* biases, qlin_dtype p_dt,
+                                   cudaStream_t st, const DeviceInfo& dev);
+cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, const void* biases,
+                                     qlin_dtype p_dt, int64_t N, int64_t K, int bits, int g, void* out,
+                                     qlin_dtype o_dt, cudaStream_t st, const DeviceInfo& dev);
+cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
+                                      float* scale, int32_t* rowsum, cudaStream_t st, const DeviceInfo& dev);
+cudaError_t launch_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64_t N, uint8_t* packed,
+                                  float* scale, cudaStream_t st, const DeviceInfo& dev);
+
+struct AffineGemvArgs {
+    const void* x;
+    qlin_dtype x_dt;
+    int64_t M, K, N;
+    const uint32_t* codes;
+    const void* scales;
+    const void* biases;
+    qlin_dtype p_dt;
+    int bits, g;
+    const void* bias;
+    void* y;
+};
+cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
+
+struct BitlinearArgs {
+    const void* x;
+    qlin_dtype x_dt;
+    int64_t M, K, N;
+    const uint8_t* packed;
+    const float* weight_scale;
+    int invert;
+    const void* bias;
+    void* y;
+};
+cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const DeviceInfo& dev);
+
+}  // namespace qlin

@@ -1,0 +1,210 @@
+/*
+ * qlin.h -- C ABI of libqlin.so: quantized linear layers on an NVIDIA B200
+ * (sm_100a), computed straight from packed low-bit weights.
+ *
+ *     y = x * dequant(Wq)^T + bias
+ *
+ * Formats (cited by page title and section):
+ *   - MLX affine groups [docs.rs nuvec-nn 0.1.0 "Struct QuantizedLinear",
+ *     fields weight / scales / biases / group_size / bits; cider/ops.py
+ *     pergroup_linear docstring, quantize/dequantize formulas]:
+ *     codes uint32 [N, K*bits/32], element k of a row in bits
+ *     bits*(k mod 32/bits) of word k*bits/32 (LSB first); one scale and one
+ *     bias per group of group_size inputs, [N, K/group_size];
+ *     w = q*scale + bias.
+ *   - BitLinear ternary [mlx_lm/models/bitlinear_layers.py,
+ *     make_bitlinear_kernel and class BitLinear]: uint8 [N/4, K]; bits 2j..2j+1
+ *     of byte [r, k] hold the code of output row r + j*N/4; w = code - 1; one
+ *     tensor scale, multiplied in, or its reciprocal multiplied in.
+ *   - per-row symmetric INT8 [cider/ops.py quantize_weight_int8,
+ *     perchannel_linear]: int8 [N, K] + fp32 scale [N].
+ *   - per-column INT4 [cider/ops.py pack_weight_int4, w4a8_linear]: uint8
+ *     [K/2, N], high nibble = even k, low nibble = odd k, w = (code - 8) *
+ *     scale[n].
+ *
+ * Conventions for every entry point:
+ *   - Tensors are caller-owned DEVICE pointers, row-major and contiguous.
+ *     The library never allocates device memory: scratch, where an operation
+ *     needs it, comes from the caller's `workspace` (size from
+ *     qlin_workspace_size()).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise, except qlin_get_device_status().
+ *   - Every call validates its arguments before launching anything and
+ *     returns a qlin_status; nothing is launched when it is not QLIN_OK.
+ *     No C++ exception crosses this interface.
+ *   - The device is the CUDA device current on the calling thread; it must
+ *     be an sm_100 GPU (QLIN_ERR_DEVICE otherwise).
+ *   - Pointers that the kernels stream with bulk copies (codes, packed
+ *     weights, x, int8 weights) must be 16-byte aligned and their row pitch a
+ *     multiple of 16 bytes; otherwise QLIN_ERR_MISALIGNED.
+ *   - Floating-point results use fp32 accumulation; integer codes and int32
+ *     accumulations are exact.
+ */
+#ifndef QLIN_H_
+#define QLIN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QLIN_OK = 0,
+    QLIN_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, shape rule broken */
+    QLIN_ERR_UNSUPPORTED = 2,  /* bits / group_size / dtype combination not provided */
+    QLIN_ERR_MISALIGNED = 3,   /* a pointer or row pitch breaks the 16-byte rule */
+    QLIN_ERR_DEVICE = 4,       /* no CUDA device, or not sm_100 */
+    QLIN_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    QLIN_ERR_TIMEOUT = 6,      /* a bounded on-device wait gave up (see qlin_get_device_status) */
+    QLIN_ERR_WORKSPACE = 7     /* workspace missing or smaller than qlin_workspace_size() */
+} qlin_status;
+
+typedef enum {
+    QLIN_F32 = 0,
+    QLIN_BF16 = 1
+} qlin_dtype;
+
+typedef enum {
+    QLIN_OP_MATMUL = 0,     /* qlin_matmul */
+    QLIN_OP_BITLINEAR = 1,  /* bitlinear_matmul */
+    QLIN_OP_W8A8 = 2,       /* w8a8_linear */
+    QLIN_OP_W4A8 = 3        /* w4a8_linear */
+} qlin_op;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* qlin_status_string(qlin_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int qlin_version(void);
+
+/*
+ * Bytes of device workspace `op` needs for the given sizes (0 = none).
+ * bits / group_size matter only for QLIN_OP_MATMUL and may be 0 otherwise.
+ */
+size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size);
+
+/*
+ * Affine group quantisation of a dense weight [nuvec-nn QuantizedLinear,
+ * from_linear; cider/ops.py pergroup_linear docstring, quantize formula].
+ * Per group of `group_size` consecutive inputs of one output row:
+ *   scale = (max - min) / (2^bits - 1), bias = min  (fp32; min-max choice),
+ *   both rounded to param_dt; a stored scale of 0 becomes 1;
+ *   q = clip(round_half_even((w - bias) / scale), 0, 2^bits - 1) from the
+ *   STORED scale and bias, fp32 subtract and IEEE divide.
+ * w: [N, K] of w_dt.  codes: uint32 [N, K*bits/32].  scales, biases:
+ * [N, K/group_size] of param_dt.  bits in {2, 4, 8}; group_size in
+ * {32, 64, 128}; K % group_size == 0.  Bit-exact with the CPU reference.
+ */
+qlin_status qlin_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int bits,
+                          int group_size, uint32_t* codes, void* scales, void* biases,
+                          qlin_dtype param_dt, void* stream);
+
+/*
+ * Dequantised weight [nuvec-nn QuantizedLinear, dequantized_weight; cider
+ * pergroup_linear docstring, dequantize formula]: w_out[n, k] =
+ * fma(q, scale, bias) in fp32, rounded once to out_dt.  w_out: [N, K].
+ * Bit-exact with the CPU reference.
+ */
+qlin_status qlin_dequantize(const uint32_t* codes, const void* scales, const void* biases,
+                            qlin_dtype param_dt, int64_t N, int64_t K, int bits, int group_size,
+                            void* w_out, qlin_dtype out_dt, void* stream);
+
+/*
+ * Quantized linear layer [nuvec-nn QuantizedLinear, forward: x W^T + b
+ * computed from the packed weight, its scales and biases].
+ * x: [M, K] of x_dt (which is also the dtype of bias and y).  bias: [N] or
+ * NULL.  y: [M, N].  M <= 16 runs the decode kernel (bulk-copy streamed
+ * codes, register dequantisation, tensor-core MACs, split-K reduced through
+ * cluster shared memory); larger M runs the prefill GEMM (codes dequantised
+ * to bf16 in shared memory feeding tcgen05 MMA with fp32 accumulation in
+ * tensor memory).  Requires (K*bits/8) % 16 == 0 and, for x, (K*sizeof(x_dt))
+ * % 16 == 0.  `workspace` may be NULL when qlin_workspace_size() is 0.
+ */
+qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
+                        const uint32_t* codes, const void* scales, const void* biases,
+                        qlin_dtype param_dt, int64_t N, int bits, int group_size,
+                        const void* bias, void* y, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * BitLinear ternary layer [mlx_lm bitlinear_layers.py, make_bitlinear_kernel
+ * and BitLinear.__call__]:
+ *   y[m, r + j*N/4] = s * sum_k x[m, k] * (((packed[r, k] >> 2j) & 3) - 1) + bias
+ * with s = invert_weight_scale ? 1/weight_scale[0] : weight_scale[0] (an fp32
+ * reciprocal, then a multiply).  x: [M, K] of x_dt; packed: uint8 [N/4, K];
+ * weight_scale: DEVICE pointer to one fp32; bias: [N] of x_dt or NULL (added
+ * in fp32 before the single rounding to x_dt); y: [M, N] of x_dt.
+ * Requires N % 4 == 0 and K % 16 == 0.
+ */
+qlin_status bitlinear_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
+                             const uint8_t* packed, int64_t N, const float* weight_scale,
+                             int invert_weight_scale, const void* bias, void* y, void* stream);
+
+/*
+ * Per-row symmetric int8 quantisation [cider/ops.py quantize_weight_int8]:
+ * scale[r] = max_c |w[r, c]| / 127 (zero -> 1), q = clip(round_half_even(w /
+ * scale), -128, 127).  Used for weights (rows = output features) and, with
+ * the same rule, for activations (rows = tokens; the pages' quant_a).
+ * w: [R, C] of w_dt; q: int8 [R, C]; scale: fp32 [R].  Bit-exact.
+ */
+qlin_status qlin_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C,
+                                    int8_t* q, float* scale, void* stream);
+
+/*
+ * Per-column int4 with zero point 8 [cider/ops.py pack_weight_int4]:
+ * scale[n] = max_k |w[k, n]| / 7 (zero -> 1), c = clip(round_half_even(w /
+ * scale) + 8, 0, 15); packed[i, n] = (c[2i, n] << 4) | c[2i+1, n].
+ * w: [K, N] of w_dt (K even); packed: uint8 [K/2, N]; scale: fp32 [N].
+ * Bit-exact.
+ */
+qlin_status qlin_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64_t N,
+                                uint8_t* packed, float* scale, void* stream);
+
+/*
+ * Raw int8 x int8 -> int32 product [cider/ops.py int8_matmul_int32]:
+ * c[m, n] = sum_k a[m, k] * b[n, k], exact (callers keep |c| < 2^31).
+ * a: int8 [M, K]; b: int8 [N, K]; c: int32 [M, N].  K % 16 == 0.
+ */
+qlin_status qlin_int8_matmul_int32(const int8_t* a, const int8_t* b, int64_t M, int64_t N,
+                                   int64_t K, int32_t* c, void* stream);
+
+/*
+ * W8A8 linear [cider/ops.py perchannel_linear]: y = dequant(quant_a(x) @
+ * w^T) + bias, quant_a = per-token qlin_quantize_int8_rows of x (kept in the
+ * workspace), int32 accumulation, then y = acc * s_x[m] * scale_w[n] + bias
+ * in fp32 and one rounding to x_dt.  x: [M, K] of x_dt; w: int8 [N, K];
+ * scale_w: fp32 [N]; bias: [N] of x_dt or NULL; y: [M, N] of x_dt.
+ * K % 16 == 0.  workspace >= qlin_workspace_size(QLIN_OP_W8A8, M, N, K, 0, 0).
+ */
+qlin_status w8a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const int8_t* w,
+                        const float* scale_w, int64_t N, const void* bias, void* y,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * W4A8 linear [cider/ops.py w4a8_linear]: y = dequant(quant_a(x) @
+ * unpack4(w)), unpack4 reading code c[k, n] from packed[k/2, n] (high
+ * nibble for even k) with weight c - 8; int32 accumulation; y = acc *
+ * s_x[m] * scale_w[n] (+ bias, an extension: the page has none) rounded to
+ * x_dt.  packed: uint8 [K/2, N]; other arguments as w8a8_linear.
+ * K % 32 == 0, N % 16 == 0.
+ */
+qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
+                        const uint8_t* packed_w, const float* scale_w, int64_t N,
+                        const void* bias, void* y, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) the library's device
+ * status word: QLIN_ERR_TIMEOUT if a bounded on-device wait in any kernel
+ * gave up since the last call, QLIN_ERR_CUDA if the stream holds an error,
+ * QLIN_OK otherwise.
+ */
+qlin_status qlin_get_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLIN_H_ */

@@ -1,0 +1,67 @@
+"""Shared helpers for the GPU parity tests (the tolerance, device transfer)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+# Floating-point bar: |y - y_ref| <= REL * (sum_k |x_k w_k| + |bias_n|) + ABS, with
+# y_ref the oracle's unrounded double result.  The |bias| term covers the
+# final rounding of a bias-dominated output.
+REL = 2e-3
+ABS = 1e-5
+
+
+def build_lib():
+    from bit_quantized_linear_qmm_b200 import build
+    build.build()
+    from bit_quantized_linear_qmm_b200 import qlin
+    return qlin
+
+
+def to_dev(a: np.ndarray, dtype=None) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+def u32_dev(a: np.ndarray) -> torch.Tensor:
+    """uint32 numpy -> int32 CUDA tensor with the same bytes."""
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).cuda()
+
+
+def bf16_dev_from_f32_values(v: np.ndarray) -> torch.Tensor:
+    """fp32 values that are exactly bf16 -> bf16 CUDA tensor (exact)."""
+    return torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(torch.bfloat16).cuda()
+
+
+def params_dev(vals: np.ndarray, dtype: str) -> torch.Tensor:
+    if dtype == "bf16":
+        return bf16_dev_from_f32_values(vals)
+    return to_dev(vals.astype(np.float32))
+
+
+def host_f32(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float32)
+
+
+def host_bits16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def assert_fp_close(y_gpu: torch.Tensor, y_ref: np.ndarray, absdot: np.ndarray, bias=None, what=""):
+    y = y_gpu.double().cpu().numpy()
+    assert y.shape == y_ref.shape, (y.shape, y_ref.shape)
+    scale = absdot.copy()
+    if bias is not None:
+        scale = scale + np.abs(np.asarray(bias, np.float64))[None, :]
+    tol = REL * scale + ABS
+    err = np.abs(y - y_ref)
+    bad = err > tol
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        worst = float((err / tol).max())
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} outside tolerance (worst err/tol {worst:.3g}); "
+            f"first {[(tuple(i), float(y[tuple(i)]), float(y_ref[tuple(i)])) for i in idx]}")
+    return float((err / tol).max())

@@ -1,0 +1,67 @@
+"""Host-only checks of the C ABI: the library builds, loads and exports every
+function include/qlin.h declares, and argument validation answers before any
+device work (no GPU needed)."""
+import ctypes as C
+
+import pytest
+
+from helpers import build_lib
+
+
+@pytest.fixture(scope="module")
+def ql():
+    return build_lib()
+
+
+def test_exports_every_declared_function(ql):
+    names = ql.header_functions()
+    assert len(names) >= 13
+    L = ql.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(ql):
+    for s in range(8):
+        assert ql.status_string(s).startswith("QLIN_")
+    assert "unknown" in ql.status_string(99)
+
+
+def test_workspace_sizes(ql):
+    assert ql.workspace_size(ql.QLIN_OP_MATMUL, 16, 4096, 4096, 4, 128) == 0
+    assert ql.workspace_size(ql.QLIN_OP_BITLINEAR, 8, 4096, 4096) == 0
+    assert ql.workspace_size(ql.QLIN_OP_W8A8, 4096, 8192, 8192) == 4096 * 8192 + 4096 * 4
+    assert ql.workspace_size(ql.QLIN_OP_W8A8, 1, 8192, 8192) == 8192 + 256
+    assert ql.workspace_size(ql.QLIN_OP_W4A8, 1, 8192, 8192) == 8192 + 512
+
+
+P16 = C.c_void_p(256)  # a non-null, 16-byte aligned stand-in; never dereferenced on these paths
+
+
+def test_validation_before_device(ql):
+    L = ql.lib()
+    # null pointers
+    assert L.qlin_quantize(None, 0, 4, 64, 4, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_INVALID_ARG
+    # unsupported bits / group
+    assert L.qlin_quantize(P16, 0, 4, 64, 3, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize(P16, 0, 4, 64, 4, 48, P16, P16, P16, 0, None) == ql.QLIN_ERR_UNSUPPORTED
+    # K not a multiple of the group
+    assert L.qlin_dequantize(P16, P16, P16, 0, 4, 96, 4, 64, P16, 0, None) == ql.QLIN_ERR_INVALID_ARG
+    # misaligned codes pointer
+    assert L.qlin_matmul(P16, 1, 1, 128, C.c_void_p(260), P16, P16, 1, 64, 4, 64, None, P16, None, 0,
+                         None) == ql.QLIN_ERR_MISALIGNED
+    # BitLinear needs N % 4 == 0 and K % 16 == 0
+    assert L.bitlinear_matmul(P16, 1, 1, 64, P16, 6, P16, 0, None, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.bitlinear_matmul(P16, 1, 1, 60, P16, 8, P16, 0, None, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    # int4 needs even K
+    assert L.qlin_pack_int4_cols(P16, 0, 3, 8, P16, P16, None) == ql.QLIN_ERR_INVALID_ARG
+
+
+def test_valid_call_without_gpu_reports_device(ql):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    L = ql.lib()
+    assert L.qlin_matmul(P16, 1, 1, 128, P16, P16, P16, 1, 64, 4, 64, None, P16, None, 0,
+                         None) == ql.QLIN_ERR_DEVICE
+    assert L.qlin_get_device_status(None) == ql.QLIN_ERR_DEVICE

@@ -1,0 +1,78 @@
+"""GPU parity of qlin_matmul (MLX affine format) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import assert_fp_close, build_lib, params_dev, u32_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ql():
+    return build_lib()
+
+
+def _run_case(ql, orc, case: synth.AffineCase, rows=None):
+    """Runs the layer on the GPU; compares all outputs, or the sampled rows `rows`."""
+    w = case.weight()
+    codes, s, b = orc.affine_quantize(w, case.bits, case.group_size, case.param_dtype == "bf16")
+    x = case.x()
+    lb = case.layer_bias()
+    y = ql.matmul(x.torch("cuda"), u32_dev(codes), params_dev(s, case.param_dtype),
+                  params_dev(b, case.param_dtype), case.bits, case.group_size,
+                  None if lb is None else lb.torch("cuda"))
+    torch.cuda.synchronize()
+    assert y.dtype == (torch.bfloat16 if case.x_dtype == "bf16" else torch.float32)
+    if rows is not None:
+        codes, s, b = codes[rows], s[rows], b[rows]
+        y = y[:, torch.as_tensor(rows, device=y.device)]
+    bias_v = None if lb is None else lb.vals if rows is None else lb.vals[rows]
+    yr, mag = orc.affine_matmul(x.vals, codes, s, b, case.bits, case.group_size, bias_v)
+    return assert_fp_close(y, yr, mag, bias_v, case.name)
+
+
+SMALL = [
+    synth.AffineCase(f"b{b}_g{g}_M{M}_{xd}_{pd}{'_bias' if bias else ''}", M, K, 197, b, g, xd, pd, bias, seed=7)
+    for (b, g, K) in [(4, 32, 640), (4, 64, 640), (4, 128, 1280), (2, 64, 768), (2, 128, 1280),
+                      (8, 32, 544), (8, 64, 640), (8, 128, 1280)]
+    for M in (1, 3, 8, 9, 16)
+    for (xd, pd, bias) in [("bf16", "bf16", True), ("f32", "f32", False)]
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c.name for c in SMALL])
+def test_affine_small_shapes(ql, orc, case):
+    _run_case(ql, orc, case)
+
+
+def test_affine_small_layer_full(ql, orc):
+    """The 4-bit g64 fp32 layer x[4,512] . W[512,512]^T + bias, every output."""
+    _run_case(ql, orc, synth.AFFINE_SMALL)
+
+
+@pytest.mark.parametrize("case", synth.AFFINE_DECODE, ids=[c.name for c in synth.AFFINE_DECODE])
+def test_affine_decode_configs_sampled(ql, orc, case):
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(case.N, size=256, replace=False))
+    rows[-1] = case.N - 1
+    _run_case(ql, orc, case, rows)
+
+
+def test_affine_m_above_16(ql, orc):
+    case = synth.AffineCase("b4_g64_M40", 40, 512, 130, 4, 64, "bf16", "bf16", True, seed=3)
+    _run_case(ql, orc, case)
+
+
+def test_affine_rejects_bad_args(ql):
+    x = torch.zeros((1, 96), dtype=torch.bfloat16, device="cuda")
+    codes = torch.zeros((4, 12), dtype=torch.int32, device="cuda")
+    s = torch.zeros((4, 1), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ql.QlinError) as e:
+        ql.matmul(x, codes, s, s, 4, 64)  # K % g != 0
+    assert e.value.status == ql.QLIN_ERR_INVALID_ARG
+    with pytest.raises(ql.QlinError) as e:
+        ql.matmul(x, codes, s, s, 3, 32)
+    assert e.value.status == ql.QLIN_ERR_UNSUPPORTED
+    assert ql.device_status() == ql.QLIN_OK

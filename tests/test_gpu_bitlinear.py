@@ -1,0 +1,71 @@
+"""GPU parity of bitlinear_matmul (ternary weights packed 4:1 along N)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import assert_fp_close, build_lib, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ql():
+    return build_lib()
+
+
+def _run(ql, orc, case: synth.BitLinearCase):
+    P = case.packed()
+    x = case.x()
+    lb = case.layer_bias()
+    ws = torch.tensor([case.weight_scale], dtype=torch.float32, device="cuda")
+    y = ql.bitlinear_matmul(x.torch("cuda"), to_dev(P), case.N, ws, case.invert,
+                            None if lb is None else lb.torch("cuda"))
+    torch.cuda.synchronize()
+    yr, mag = orc.bitlinear(x.vals, P, case.N, case.weight_scale, case.invert,
+                            None if lb is None else lb.vals)
+    return assert_fp_close(y, yr, mag, None if lb is None else lb.vals, case.name)
+
+
+SMALL = [synth.BitLinearCase(f"M{M}_K{K}_N{N}_{'div' if inv else 'mul'}{'_bias' if b else ''}", M, K, N, 0.75,
+                             inv, b, seed=11)
+         for M in (1, 5, 8, 16) for (K, N) in [(512, 204), (1040, 64), (4096, 260)]
+         for inv in (False, True) for b in (False, True)]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c.name for c in SMALL])
+def test_bitlinear_small(ql, orc, case):
+    _run(ql, orc, case)
+
+
+@pytest.mark.parametrize("case", synth.BITLINEAR_DECODE, ids=[c.name for c in synth.BITLINEAR_DECODE])
+def test_bitlinear_decode_config_full(ql, orc, case):
+    _run(ql, orc, case)
+
+
+def test_bitlinear_code1_gives_exact_zero(ql):
+    x = torch.randn((8, 512), device="cuda").to(torch.bfloat16)
+    P = torch.full((64, 512), 0x55, dtype=torch.uint8, device="cuda")
+    ws = torch.tensor([0.5], device="cuda")
+    y = ql.bitlinear_matmul(x, P, 256, ws, False)
+    assert torch.count_nonzero(y).item() == 0
+
+
+def test_bitlinear_code2_rowsum(ql):
+    """All codes 2: y = rowsum(x) * scale, exact for small-integer x."""
+    x = torch.randint(-4, 5, (3, 1024), device="cuda").to(torch.bfloat16)
+    P = torch.full((16, 1024), 0xAA, dtype=torch.uint8, device="cuda")
+    ws = torch.tensor([0.5], device="cuda")
+    for inv, f in ((False, 0.5), (True, 2.0)):
+        y = ql.bitlinear_matmul(x, P, 64, ws, inv).float()
+        expect = x.float().sum(dim=1, keepdim=True).expand(3, 64) * f
+        assert torch.equal(y, expect)
+
+
+def test_bitlinear_rejects_ragged(ql):
+    x = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")
+    P = torch.zeros((2, 64), dtype=torch.uint8, device="cuda")
+    ws = torch.ones(1, device="cuda")
+    with pytest.raises(ql.QlinError) as e:
+        ql.bitlinear_matmul(x, P, 6, ws, False)
+    assert e.value.status == ql.QLIN_ERR_INVALID_ARG

@@ -1,0 +1,99 @@
+"""GPU parity of the quantisers and the dequantiser (bit-exact with the oracle)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import build_lib, host_bits16, host_f32, params_dev, to_dev, u32_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ql():
+    return build_lib()
+
+
+def _w_dev(w, w_dt):
+    if w_dt == "bf16":
+        vals, bits = synth.to_bf16(w)
+        return vals, torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    return w, to_dev(w)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("g", [32, 64, 128])
+@pytest.mark.parametrize("p_dt", ["f32", "bf16"])
+@pytest.mark.parametrize("w_dt", ["f32", "bf16"])
+def test_quantize_bit_exact(ql, orc, bits, g, p_dt, w_dt):
+    N, K = 75, 6 * g
+    w = synth.outlier_weights(100 + bits + g, N, K, frac=0.01)
+    w[3, :g] = 0.25  # a constant group
+    wv, wd = _w_dev(w, w_dt)
+    codes, s, b = ql.quantize(wd, bits, g, torch.bfloat16 if p_dt == "bf16" else torch.float32)
+    torch.cuda.synchronize()
+    rc, rs, rb = orc.affine_quantize(wv, bits, g, p_dt == "bf16")
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), rc)
+    assert np.array_equal(host_f32(s), rs)
+    assert np.array_equal(host_f32(b), rb)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("g", [32, 128])
+@pytest.mark.parametrize("p_dt", ["f32", "bf16"])
+@pytest.mark.parametrize("o_dt", ["f32", "bf16"])
+def test_dequantize_bit_exact(ql, orc, bits, g, p_dt, o_dt):
+    N, K = 53, 4 * g
+    w = synth.normal(200 + bits, (N, K), 0.02)
+    rc, rs, rb = orc.affine_quantize(w, bits, g, p_dt == "bf16")
+    out = ql.dequantize(u32_dev(rc), params_dev(rs, p_dt), params_dev(rb, p_dt), K, bits, g,
+                        torch.bfloat16 if o_dt == "bf16" else torch.float32)
+    torch.cuda.synchronize()
+    ref = orc.affine_dequantize(rc, rs, rb, K, bits, g)
+    if o_dt == "bf16":
+        assert np.array_equal(host_bits16(out), orc.f32_to_bf16_bits(ref))
+    else:
+        assert np.array_equal(out.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("w_dt", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 8192), (7, 1000), (33, 4096), (3, 24)])
+def test_quantize_int8_rows_bit_exact(ql, orc, w_dt, shape):
+    R, Cc = shape
+    w = synth.normal(300 + R, (R, Cc), 1.0)
+    if R > 2:
+        w[1] = 0.0
+        w[2, 5] = 1e4
+    wv, wd = _w_dev(w, w_dt)
+    q, s = ql.quantize_int8_rows(wd)
+    torch.cuda.synchronize()
+    rq, rs = orc.quantize_int8_rows(wv)
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy(), rs)
+
+
+@pytest.mark.parametrize("w_dt", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 4), (64, 96), (512, 300), (8192, 64)])
+def test_pack_int4_cols_bit_exact(ql, orc, w_dt, shape):
+    K, N = shape
+    w = synth.normal(400 + K, (K, N), 0.02)
+    if N > 3:
+        w[:, 2] = 0.0
+    wv, wd = _w_dev(w, w_dt)
+    P, s = ql.pack_int4_cols(wd)
+    torch.cuda.synchronize()
+    rP, rs = orc.pack_int4_cols(wv)
+    assert np.array_equal(P.cpu().numpy(), rP)
+    assert np.array_equal(s.cpu().numpy(), rs)
+
+
+def test_quantize_full_prefill_weight_bit_exact(ql, orc):
+    """The 14336 x 4096 prefill weight (outliers, 4-bit g64, bf16 params): every code."""
+    case = synth.AFFINE_PREFILL
+    w = case.weight()
+    codes, s, b = ql.quantize(to_dev(w), 4, 64, torch.bfloat16)
+    torch.cuda.synchronize()
+    rc, rs, rb = orc.affine_quantize(w, 4, 64, True)
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), rc)
+    assert np.array_equal(host_f32(s), rs)
+    assert np.array_equal(host_f32(b), rb)
