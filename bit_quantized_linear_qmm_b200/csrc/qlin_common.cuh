@@ -3,6 +3,7 @@
 // interface between the C ABI (qlin_abi.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -113,6 +114,48 @@ QLIN_DEV void bulk_g2s(void* smem_dst, const void* gmem_src, unsigned bytes, uin
         : "memory");
 }
 
+// Hint: bring `bytes` (multiple of 16, 16-byte aligned) of global memory into
+// L2.  Safe before griddepcontrol.wait: L2 is the coherence point, so a later
+// load still sees any write an earlier kernel makes to these bytes.
+QLIN_DEV void bulk_prefetch_l2(const void* gmem_src, unsigned bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes) : "memory");
+}
+
+QLIN_DEV void prefetch_l2(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// ---------------------------------------------------------------- tensor-map TMA (2-D tiles)
+
+// Loads the 2-D box at (c0, c1) of `tmap` (a __grid_constant__ kernel
+// parameter) into shared memory, completing as transaction bytes on `bar`.
+// c0 * element size must be a multiple of 16 bytes.  Out-of-range elements
+// of the box are written as zeros.
+QLIN_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* tmap, int c0, int c1, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// L2 prefetch of the same box (a hint; coherent with earlier writes).
+QLIN_DEV void tma_prefetch_2d(const CUtensorMap* tmap, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+// Byte offset of the 16-byte unit `unit` (0..7) of row `row` inside a box
+// written with CU_TENSOR_MAP_SWIZZLE_128B whose rows are 128 bytes (box
+// base 1024-byte aligned): units are XOR-permuted by row mod 8.
+QLIN_DEV int swz128(int row, int unit) { return row * 128 + ((unit ^ (row & 7)) << 4); }
+
 // ---------------------------------------------------------------- cluster helpers
 
 QLIN_DEV unsigned cluster_ctarank()
@@ -125,6 +168,59 @@ QLIN_DEV unsigned cluster_ctarank()
 QLIN_DEV void cluster_sync()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+QLIN_DEV void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+QLIN_DEV void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+QLIN_DEV void st_shared_cluster_v4(uint32_t addr, float4 v)
+{
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (remote address from
+// map_shared_rank), releasing this thread's prior writes at cluster scope.
+QLIN_DEV void mbar_remote_arrive_cluster(uint32_t remote_bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
+QLIN_DEV bool mbar_try_wait_cluster(uint64_t* bar, unsigned parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// As mbar_wait_bounded, with acquire at cluster scope (for arrivals from other CTAs).
+QLIN_DEV bool mbar_wait_cluster_bounded(uint64_t* bar, unsigned parity, unsigned* status)
+{
+    if (mbar_try_wait_cluster(bar, parity))
+        return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_cluster(bar, parity))
+                return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(status, kStatusTimeout);
+            return false;
+        }
+    }
 }
 
 // Address of the same shared-memory location in CTA `rank` of the cluster.
@@ -158,7 +254,7 @@ QLIN_DEV void pdl_launch_dependents()
 
 QLIN_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -167,7 +263,7 @@ QLIN_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
 
 QLIN_DEV void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -199,6 +295,13 @@ struct DeviceInfo {
     int sm_count;
     unsigned* status;  // device status word
 };
+
+// Host: encodes a 2-D tiled tensor map (row-major [dim1][dim0] elements,
+// row pitch `pitch_bytes`) with box {box0, box1}, 128-byte swizzle, zero
+// fill.  Returns false if the driver entry point is unavailable or rejects
+// the description.
+bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t dim0, uint64_t dim1,
+                    uint64_t pitch_bytes, uint32_t box0, uint32_t box1);
 
 cudaError_t launch_affine_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int bits, int g,
                                    uint32_t* codes, void* scales, void* biases, qlin_dtype p_dt,
