@@ -7,23 +7,24 @@
 //              [mlx_lm bitlinear_layers.py, make_bitlinear_kernel, BitLinear.__call__]
 //
 // Design (B200, HBM- and latency-bound):
-//  * A CTA owns 64 output rows x a K-range.  K is split over the CTAs of a
-//    thread-block cluster; each CTA pushes its fp32 partial tile into the
-//    leader CTA's shared memory (st.shared::cluster) and arrives on the
-//    leader's mbarrier; the leader sums, adds the layer bias and stores y.
-//    No workspace, no atomics in global memory, one cluster barrier.
-//  * One producer thread streams the tile through a 4-stage shared-memory
-//    ring with 2-D tensor-map TMA (cp.async.bulk.tensor, 128-byte swizzle,
-//    completion on mbarriers): one instruction moves a 128-byte column block
-//    of all 64 weight rows, one a 128-byte column block of all tokens of x
-//    (tokens >= M and bytes past the row end arrive as zeros).  With
-//    programmatic dependent launch the first stages' weights are prefetched
-//    into L2 before griddepcontrol.wait, so back-to-back layers overlap one
-//    kernel's DRAM fetch with the previous kernel's tail.
-//  * Eight consumer warps (4 row tiles of 16 rows x 2 K-lanes) dequantise in
-//    registers and run the MACs on the tensor cores with the legacy
-//    mma.sync.m16n8k16 (weights as the 16-row A operand, x as the n=8 B
-//    operand, fp32 accumulation).
+//  * A CTA owns a block of output rows over the whole of K (about one CTA
+//    per SM), so the only reduction is inside the CTA: no clusters, no
+//    workspace, no global atomics.  A small footprint leaves room on each SM
+//    for the next kernel in the stream.
+//  * One producer thread streams the block through a shared-memory ring with
+//    2-D tensor-map TMA (cp.async.bulk.tensor, 128-byte swizzle, completion
+//    on mbarriers): one instruction moves a 128-byte column block of all the
+//    CTA's weight rows, one the same columns of the M token rows of x (the
+//    remaining token rows of the ring stay zero).  With programmatic
+//    dependent launch the next kernel is released at once, and each kernel
+//    prefetches its first stages into L2 before griddepcontrol.wait, so a
+//    layer's DRAM fetch overlaps the previous layer's tail.
+//  * Eight consumer warps split K (whole groups / k16 steps round robin);
+//    each covers all the CTA's 16-row tiles, so every x fragment serves them
+//    all.  They dequantise in registers and run the MACs on the tensor cores
+//    with the legacy mma.sync.m16n8k16 (weights as the 16-row A operand, x as
+//    the n=8 B operand, fp32 accumulation); partial tiles are summed through
+//    shared memory.
 //  * affine: codes become bf16 with one LOP3 per pair: (w >> s) & 0x000F000F
 //    | 0x43004300 is the bf16 pair (128 + q_i, 128 + q_j), exact.  The 128
 //    offset and the group bias fold out per group with the group sums of x,
@@ -33,8 +34,9 @@
 //    (8-bit codes use no offset: bf16 holds 0..255 exactly.)  Because a dot
 //    product over a group does not depend on the order of k, each lane pairs
 //    codes in the order the LOP3 yields them and permutes x to match (PRMT).
-//  * bitlinear: (c + 128) pairs from the same LOP3, then one bf16x2 add of
-//    -129 gives the exact weights c - 1, so a code-1 weight contributes an
+//  * bitlinear: each 2-bit field is read in place by one LOP3 as the bf16
+//    128 + 4^j c and turned into the exact weight c - 1 by one bf16x2 FMA
+//    (times 4^-j, minus 128 4^-j + 1), so a code-1 weight contributes an
 //    exact zero.
 //  * Every mbarrier wait is bounded (qlin::kWaitLimitNs); on expiry the
 //    kernel records the timeout in the status word, stops issuing copies,
@@ -45,13 +47,11 @@ namespace qlin {
 namespace {
 
 constexpr int kRowTiles = 4;                       // 16-row MMA tiles per CTA
-constexpr int kKLanes = 2;                         // consumer warps sharing a row tile along K
-constexpr int kConsumerWarps = kRowTiles * kKLanes;
+constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;    // + one producer warp
 constexpr int kRowsPerCta = 16 * kRowTiles;
-constexpr int kStages = 4;
-constexpr int kMaxCluster = 8;
+constexpr int kStages = 6;                          // barrier slots; a kernel uses NS <= kStages
 constexpr int kRedStride = kRowsPerCta + 4;        // padded row of the partial tile (bank spread)
 
 __host__ __device__ constexpr int round_up(int a, int b) { return (a + b - 1) / b * b; }
@@ -59,7 +59,6 @@ __host__ __device__ constexpr int round_up(int a, int b) { return (a + b - 1) / 
 struct alignas(8) Barriers {
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t reduce;  // leader: one arrival per CTA of the cluster
     int abort_flag;
 };
 
@@ -71,14 +70,6 @@ QLIN_DEV uint32_t pair_lo(uint32_t a, uint32_t b) { return prmt(a, b, 0x5410); }
 QLIN_DEV uint32_t pair_hi(uint32_t a, uint32_t b) { return prmt(a, b, 0x7632); }  // (a.hi, b.hi)
 
 constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;      // (1.0, 1.0)
-constexpr uint32_t kMinus129Bf16x2 = 0xC301C301u;  // (-129.0, -129.0)
-
-QLIN_DEV uint32_t bf16x2_add(uint32_t a, uint32_t b)
-{
-    uint32_t r;
-    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
 
 // Split fp32 pairs into bf16 hi/lo parts: x = hi + lo + O(2^-17 |x|).
 QLIN_DEV void split_f32_pair(float a, float b, uint32_t& hi, uint32_t& lo)
@@ -99,13 +90,16 @@ QLIN_DEV void split_f32_pair(float a, float b, uint32_t& hi, uint32_t& lo)
 // griddepcontrol.wait only L2 prefetches of weights are issued (coherent
 // with any earlier kernel's writes); every load into shared memory follows
 // the wait.
-template <typename IssueFn, typename PFn, typename BytesFn>
+template <int NS, typename IssueFn, typename PFn, typename BytesFn>
 QLIN_DEV void producer_loop(Barriers& bars, int nst, unsigned* status, IssueFn issue, PFn prefetch,
                             BytesFn stage_bytes)
 {
     if ((threadIdx.x & 31) == 0) {
-        const int pre = nst < kStages ? nst : kStages;
-        const int npf = nst < 2 * kStages ? nst : 2 * kStages;
+        // let the next kernel in the stream start its own prologue and L2
+        // prefetch on whatever SM room is left
+        pdl_launch_dependents();
+        const int pre = nst < NS ? nst : NS;
+        const int npf = nst < 2 * NS ? nst : 2 * NS;
         for (int it = 0; it < npf; ++it)
             prefetch(it);
         pdl_wait_prior_grids();
@@ -113,121 +107,116 @@ QLIN_DEV void producer_loop(Barriers& bars, int nst, unsigned* status, IssueFn i
             mbar_arrive_expect_tx(&bars.full[it], stage_bytes(it));
             issue(it, it);
         }
-        pdl_launch_dependents();
         int issued = pre;
         for (int it = pre; it < nst; ++it) {
-            const int slot = it % kStages;
-            if (!mbar_wait_bounded(&bars.empty[slot], ((it / kStages) & 1) ^ 1, status) || volatile_abort(bars))
+            const int slot = it % NS;
+            if (!mbar_wait_bounded(&bars.empty[slot], ((it / NS) & 1) ^ 1, status) || volatile_abort(bars))
                 break;
             mbar_arrive_expect_tx(&bars.full[slot], stage_bytes(it));
             issue(it, slot);
             ++issued;
         }
         // Drain: no TMA load may still target this CTA's shared memory at exit.
-        for (int it = issued - kStages < 0 ? 0 : issued - kStages; it < issued; ++it)
-            mbar_wait_bounded(&bars.full[it % kStages], (it / kStages) & 1, status);
+        for (int it = issued - NS < 0 ? 0 : issued - NS; it < issued; ++it)
+            mbar_wait_bounded(&bars.full[it % NS], (it / NS) & 1, status);
     }
     __syncwarp();
 }
 
-// ---------------------------------------------------------------- cluster reduction
+// ---------------------------------------------------------------- CTA reduction
 
-// Called by all kThreads threads.  Consumers have accumulated this CTA's
-// partial tile in red[token * kRedStride + row].  Every CTA pushes it into
-// slot `rank` of the leader's recv buffer and arrives on the leader's reduce
-// barrier; the leader's consumers wait for all S slots, sum them and call
-// store(token, row, value).
-template <typename StoreFn>
-QLIN_DEV void cluster_reduce(Barriers& bars, float* red, float* recv, int M, int S, unsigned* status,
-                             StoreFn store)
+// Sums, over the consumer warps that cover the same rows, the F fragment
+// values each lane holds (val(j)) and writes them to red[token * kRedStride +
+// row] (pos(rg, j, lane, row, token)).  Warp w covers row group w % RG.  The
+// stage ring (idle once every warp has left the main loop) is the scratch;
+// no shared-memory atomics.
+template <int F, int RG, typename ValFn, typename PosFn>
+QLIN_DEV void cta_reduce(float* scratch, float* red, ValFn val, PosFn pos)
 {
-    const int rank = blockIdx.x;  // the cluster spans gridDim.x
-    cluster_wait();               // every CTA's barriers are initialised before any remote access
-    if (threadIdx.x >= kConsumerThreads)
-        return;
-    consumer_bar();  // red complete
-    const int tile = M * kRowsPerCta;
-    const uint32_t dst = map_shared_rank(smem_u32(recv + rank * tile), 0);
-    for (int e4 = threadIdx.x; e4 < tile / 4; e4 += kConsumerThreads) {
-        const int e = e4 * 4;
-        const int tok = e / kRowsPerCta, r = e % kRowsPerCta;
-        const float* src = red + tok * kRedStride + r;
-        st_shared_cluster_v4(dst + 16u * (uint32_t)e4, make_float4(src[0], src[1], src[2], src[3]));
-    }
-    consumer_bar();  // all of this CTA's pushes issued
-    if (threadIdx.x == 0)
-        mbar_remote_arrive_cluster(map_shared_rank(smem_u32(&bars.reduce), 0));
-    if (rank != 0)
-        return;
-    if (!mbar_wait_cluster_bounded(&bars.reduce, 0, status))
-        return;
-    pdl_wait_prior_grids();  // (already satisfied) no global write before the prior grid completed
-    for (int e = threadIdx.x; e < tile; e += kConsumerThreads) {
+    constexpr int KL = kConsumerWarps / RG;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    consumer_bar();  // every consumer warp is done with the stage ring
+#pragma unroll
+    for (int j = 0; j < F; ++j)
+        scratch[(warp * F + j) * 32 + lane] = val(j);
+    consumer_bar();
+    for (int e = threadIdx.x; e < RG * F * 32; e += kConsumerThreads) {
+        const int rg = e / (F * 32), j = (e / 32) % F, ln = e % 32;
         float v = 0.f;
-        for (int q = 0; q < S; ++q)
-            v += recv[q * tile + e];
-        store(e / kRowsPerCta, e % kRowsPerCta, v);
+#pragma unroll
+        for (int k = 0; k < KL; ++k)
+            v += scratch[((k * RG + rg) * F + j) * 32 + ln];
+        int row, tok;
+        pos(rg, j, ln, row, tok);
+        red[tok * kRedStride + row] = v;
     }
 }
 
-QLIN_DEV void init_barriers(Barriers& bars, int S)
+QLIN_DEV void init_barriers(Barriers& bars)
 {
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bars.full[s], 1);
             mbar_init(&bars.empty[s], kConsumerWarps);
         }
-        mbar_init(&bars.reduce, (unsigned)S);
         bars.abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    cluster_arrive_relaxed();
+}
+
+// Zeroes the token rows [m0, MMAX) of every x box of every stage: the TMA
+// only writes the first M rows, and tokens past M must read as zero.
+QLIN_DEV void zero_x_tail(uint8_t* stages, int ns, int stage_bytes, int w_stage, int nxb, int mmax, int m0)
+{
+    const int per_box = (mmax - m0) * 128 / 16;  // 16-byte units
+    const int total = ns * nxb * per_box;
+    for (int e = threadIdx.x; e < total; e += kConsumerThreads) {
+        const int s = e / (nxb * per_box), b = (e / per_box) % nxb, u = e % per_box;
+        *reinterpret_cast<uint4*>(stages + s * stage_bytes + w_stage + b * (mmax * 128) + m0 * 128 + u * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
 }
 
 // ---------------------------------------------------------------- affine decode kernel
 
-template <int BITS, int G, typename XT, typename PT, int NT>
+template <int BITS, int G, typename XT, typename PT, int NT, int RT>
 struct AffineCfg {
+    static constexpr int ROWS = 16 * RT;                   // output rows per CTA
     static constexpr int KST = 1024 / BITS > 256 ? 1024 / BITS : 256;  // k per stage
     static constexpr int NWB = KST * BITS / 8 / 128;       // 128-byte weight boxes per stage
     static constexpr int XE = 128 / (int)sizeof(XT);       // x elements per 128-byte box row
     static constexpr int NXB = KST / XE;                   // x boxes per stage
     static constexpr int MMAX = 8 * NT;
-    static constexpr int W_STAGE = NWB * kRowsPerCta * 128;
+    static constexpr int W_STAGE = NWB * ROWS * 128;
     static constexpr int X_STAGE = NXB * MMAX * 128;
     static constexpr int STAGE = W_STAGE + X_STAGE;       // multiple of 1024
+    static constexpr int NS = (64 * 1024 / STAGE) < 2 ? 2 : ((64 * 1024 / STAGE) > kStages ? kStages : (64 * 1024 / STAGE));
     static constexpr int CPW = 32 / BITS;                  // codes per 32-bit word
     static constexpr int WPG = G * BITS / 32;              // words per row per group
     static constexpr int WPL = WPG / 4;                    // words per lane per row per group
     static constexpr int NP = CPW / 2;                     // bf16 pairs per word
-    static constexpr int MAX_GROUPS = 64;                  // param groups per row kept in smem
-    static constexpr int PARAMS_PER_THREAD = kRowsPerCta * MAX_GROUPS / kConsumerThreads;
+    static constexpr int GPS = KST / G;                    // groups per full stage
     static_assert(WPL >= 1, "group too small for the decode lane mapping");
     static_assert(STAGE % 1024 == 0, "swizzled boxes need 1024-byte alignment");
     // bf16 holds 0..255 exactly but not 128 + q for q >= 128: 8-bit codes go unbiased
     static constexpr float OFFSET = BITS == 8 ? 0.0f : 128.0f;
     static constexpr int RED = MMAX * kRedStride * 4;
-    static constexpr int recv_bytes(int S) { return S * MMAX * kRowsPerCta * 4; }
-    static constexpr int smem_bytes(int gstride, int S)
+    static constexpr int params_bytes(int groups) { return round_up(ROWS * groups * 8, 16); }
+    static constexpr int smem_bytes(int groups)
     {
-        return kStages * STAGE + round_up(kRowsPerCta * gstride * 8, 16) + RED + recv_bytes(S) +
-               (int)sizeof(Barriers) + 1024;
+        return NS * STAGE + params_bytes(groups) + RED + (int)sizeof(Barriers) + 1024;
     }
 };
 
 struct AffineParams {
-    CUtensorMap tm_w;  // codes as bytes [N][K*BITS/8], box {128 B, 64 rows}
-    CUtensorMap tm_x;  // x [M][K], box {128 B, 8*NT tokens}
-    const uint8_t* codes;  // bytes of the uint32 words
-    const void* x;
+    CUtensorMap tm_w;  // codes as bytes [N][K*BITS/8], box {128 B, ROWS rows}
+    CUtensorMap tm_x;  // x [M][K], box {128 B, M tokens}
     const void* scales;
     const void* biases;
     const void* bias;
     void* y;
     int M, K, N;
-    int k_per_split;  // multiple of KST
-    int gstride;      // groups per row held in the smem parameter block (k_per_split / G)
     unsigned* status;
 };
 
@@ -341,196 +330,209 @@ QLIN_DEV uint32_t w_word(const uint8_t* wst, int rows, int row, int wi)
     return *reinterpret_cast<const uint32_t*>(wst + b * (rows * 128) + swz128(row, w >> 2) + ((w & 3) << 2));
 }
 
-template <int BITS, int G, typename XT, typename PT, int NT>
+template <int BITS, int G, typename XT, typename PT, int NT, int RT>
 __global__ void __launch_bounds__(kThreads, 2) affine_gemv_kernel(const __grid_constant__ AffineParams p)
 {
-    using Cfg = AffineCfg<BITS, G, XT, PT, NT>;
+    using Cfg = AffineCfg<BITS, G, XT, PT, NT, RT>;
+    constexpr int ROWS = Cfg::ROWS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
-    const int params_bytes = round_up(kRowsPerCta * p.gstride * 8, 16);
-    float2* params = reinterpret_cast<float2*>(smem + kStages * Cfg::STAGE);
-    float* red = reinterpret_cast<float*>(smem + kStages * Cfg::STAGE + params_bytes);
-    float* recv = red + Cfg::RED / 4;
-    Barriers& bars = *reinterpret_cast<Barriers*>(reinterpret_cast<uint8_t*>(recv) + Cfg::recv_bytes(gridDim.x));
+    const int ng = p.K / G;  // groups per row
+    float2* params = reinterpret_cast<float2*>(smem + Cfg::NS * Cfg::STAGE);
+    float* red = reinterpret_cast<float*>(smem + Cfg::NS * Cfg::STAGE + Cfg::params_bytes(ng));
+    Barriers& bars = *reinterpret_cast<Barriers*>(reinterpret_cast<uint8_t*>(red) + Cfg::RED);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = gridDim.x;
-    const int split = blockIdx.x;  // == rank in the cluster
-    const int n0 = blockIdx.y * kRowsPerCta;
-    const int kbeg = split * p.k_per_split;
-    const int kend = min(p.K, kbeg + p.k_per_split);
-    const int nst = kend > kbeg ? (kend - kbeg + Cfg::KST - 1) / Cfg::KST : 0;
-    const int rows_valid = min(kRowsPerCta, p.N - n0);
+    const int n0 = blockIdx.x * ROWS;
+    const int nst = (p.K + Cfg::KST - 1) / Cfg::KST;
+    const int rows_valid = min(ROWS, p.N - n0);
     const int M = p.M;
 
-    init_barriers(bars, S);
+    init_barriers(bars);
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------ producer warp
-        producer_loop(
+        producer_loop<Cfg::NS>(
             bars, nst, p.status,
             [&](int it, int slot) {
-                const int k0 = kbeg + it * Cfg::KST;
+                const int k0 = it * Cfg::KST;
                 uint8_t* wst = stages + slot * Cfg::STAGE;
                 uint8_t* xst = wst + Cfg::W_STAGE;
 #pragma unroll
                 for (int b = 0; b < Cfg::NWB; ++b)
-                    tma_load_2d(wst + b * (kRowsPerCta * 128), &p.tm_w, k0 * BITS / 8 + b * 128, n0,
-                                &bars.full[slot]);
+                    tma_load_2d(wst + b * (ROWS * 128), &p.tm_w, k0 * BITS / 8 + b * 128, n0, &bars.full[slot]);
 #pragma unroll
                 for (int b = 0; b < Cfg::NXB; ++b)
                     tma_load_2d(xst + b * (Cfg::MMAX * 128), &p.tm_x, k0 + b * Cfg::XE, 0, &bars.full[slot]);
             },
             [&](int it) {
-                const int k0 = kbeg + it * Cfg::KST;
 #pragma unroll
                 for (int b = 0; b < Cfg::NWB; ++b)
-                    tma_prefetch_2d(&p.tm_w, k0 * BITS / 8 + b * 128, n0);
+                    tma_prefetch_2d(&p.tm_w, it * Cfg::KST * BITS / 8 + b * 128, n0);
             },
-            [&](int) { return (unsigned)Cfg::STAGE; });
+            [&](int) { return (unsigned)(Cfg::W_STAGE + Cfg::NXB * M * 128); });
     } else {
         // ------------------------------------------------ consumer warps
-        // zero the partial tile; group parameters of this CTA's rows and K-range -> smem as
-        // {s, b - OFFSET s}: all loads issued before any store (one round trip)
-        for (int e = threadIdx.x; e < Cfg::RED / 4; e += kConsumerThreads)
-            red[e] = 0.f;
+        zero_x_tail(stages, Cfg::NS, Cfg::STAGE, Cfg::W_STAGE, Cfg::NXB, Cfg::MMAX, M);
+        // group parameters of the CTA's rows -> smem as {s, b - OFFSET s}: all loads of a
+        // batch issued before its stores
         {
-            const int g0 = kbeg / G;
-            const int ng = (kend - kbeg) / G;
-            const int gpr = p.K / G;
             const PT* sc = static_cast<const PT*>(p.scales);
             const PT* bi = static_cast<const PT*>(p.biases);
-            PT sv[Cfg::PARAMS_PER_THREAD], bv[Cfg::PARAMS_PER_THREAD];
-#pragma unroll
-            for (int i = 0; i < Cfg::PARAMS_PER_THREAD; ++i) {
-                const int e = threadIdx.x + i * kConsumerThreads;
-                const int r = e / ng, gl = e % ng;
-                if (r < rows_valid && e < kRowsPerCta * ng && gl == 0) {
-                    prefetch_l2(sc + (size_t)(n0 + r) * gpr + g0);
-                    prefetch_l2(bi + (size_t)(n0 + r) * gpr + g0);
-                }
+            const int pbytes = rows_valid * ng * (int)sizeof(PT);  // the CTA's params are contiguous
+            for (int off = threadIdx.x * 128; off < pbytes; off += kConsumerThreads * 128) {
+                prefetch_l2(reinterpret_cast<const uint8_t*>(sc + (size_t)n0 * ng) + off);
+                prefetch_l2(reinterpret_cast<const uint8_t*>(bi + (size_t)n0 * ng) + off);
             }
             pdl_wait_prior_grids();
+            constexpr int B = 8;
+            for (int e0 = threadIdx.x; e0 < ROWS * ng; e0 += B * kConsumerThreads) {
+                PT sv[B], bv[B];
 #pragma unroll
-            for (int i = 0; i < Cfg::PARAMS_PER_THREAD; ++i) {
-                const int e = threadIdx.x + i * kConsumerThreads;
-                const int r = e / ng, gl = e % ng;
-                if (r < rows_valid && e < kRowsPerCta * ng) {
-                    sv[i] = sc[(size_t)(n0 + r) * gpr + g0 + gl];
-                    bv[i] = bi[(size_t)(n0 + r) * gpr + g0 + gl];
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < Cfg::PARAMS_PER_THREAD; ++i) {
-                const int e = threadIdx.x + i * kConsumerThreads;
-                const int r = e / ng, gl = e % ng;
-                if (e < kRowsPerCta * ng) {
-                    float s = 0.f, b = 0.f;
-                    if (r < rows_valid) {
-                        s = to_float(sv[i]);
-                        b = to_float(bv[i]);
+                for (int i = 0; i < B; ++i) {
+                    const int e = e0 + i * kConsumerThreads;
+                    if (e < rows_valid * ng) {
+                        sv[i] = sc[(size_t)n0 * ng + e];
+                        bv[i] = bi[(size_t)n0 * ng + e];
                     }
-                    params[r * p.gstride + gl] = make_float2(s, fmaf(-Cfg::OFFSET, s, b));
+                }
+#pragma unroll
+                for (int i = 0; i < B; ++i) {
+                    const int e = e0 + i * kConsumerThreads;
+                    if (e < ROWS * ng) {
+                        float s = 0.f, b = 0.f;
+                        if (e < rows_valid * ng) {
+                            s = to_float(sv[i]);
+                            b = to_float(bv[i]);
+                        }
+                        params[e] = make_float2(s, fmaf(-Cfg::OFFSET, s, b));
+                    }
                 }
             }
         }
         consumer_bar();
 
+        // every warp covers all RT row tiles (sharing each x fragment and the
+        // group-sum MMA among them) and takes whole groups round robin
         const int gid = lane >> 2, tig = lane & 3;
-        const int rt = warp % kRowTiles, kl_lane = warp / kRowTiles;
-        const int row0 = rt * 16 + gid;  // local rows row0, row0 + 8
-        float acc[NT][4];
+        float acc[RT][NT][4];
 #pragma unroll
-        for (int t = 0; t < NT; ++t)
+        for (int i = 0; i < RT; ++i)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                acc[t][i] = 0.f;
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[i][t][e] = 0.f;
         const uint32_t ones[4] = {kOnesBf16x2, kOnesBf16x2, kOnesBf16x2, kOnesBf16x2};
         for (int it = 0; it < nst; ++it) {
-            const int slot = it % kStages;
-            if (!mbar_wait_bounded(&bars.full[slot], (it / kStages) & 1, p.status)) {
+            const int slot = it % Cfg::NS;
+            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status)) {
                 bars.abort_flag = 1;
                 break;
             }
             const uint8_t* wst = stages + slot * Cfg::STAGE;
             const uint8_t* xst = wst + Cfg::W_STAGE;
-            const int kst = min(Cfg::KST, kend - (kbeg + it * Cfg::KST));
+            const int kst = min(Cfg::KST, p.K - it * Cfg::KST);
             const int groups = kst / G;
-            for (int gl = kl_lane; gl < groups; gl += kKLanes) {
-                float d[NT][4], dx[NT][4];
+            for (int gl = (warp - it * Cfg::GPS % kConsumerWarps + kConsumerWarps) % kConsumerWarps; gl < groups;
+                 gl += kConsumerWarps) {
+                float d[RT][NT][4], dx[NT][4];
 #pragma unroll
-                for (int t = 0; t < NT; ++t)
+                for (int t = 0; t < NT; ++t) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        d[t][i] = dx[t][i] = 0.f;
+                    for (int e = 0; e < 4; ++e)
+                        dx[t][e] = 0.f;
+#pragma unroll
+                    for (int i = 0; i < RT; ++i)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            d[i][t][e] = 0.f;
+                }
 #pragma unroll
                 for (int j = 0; j < Cfg::WPL; ++j) {
                     const int wi = gl * Cfg::WPG + j * 4 + tig;  // word index in the stage row
-                    const uint32_t w0 = w_word(wst, kRowsPerCta, row0, wi);
-                    const uint32_t w1 = w_word(wst, kRowsPerCta, row0 + 8, wi);
-                    const int kl = wi * Cfg::CPW;                // k offset of the word in the stage
+                    uint32_t w[RT][2];
+#pragma unroll
+                    for (int i = 0; i < RT; ++i) {
+                        w[i][0] = w_word(wst, ROWS, i * 16 + gid, wi);
+                        w[i][1] = w_word(wst, ROWS, i * 16 + gid + 8, wi);
+                    }
+                    const int kl = wi * Cfg::CPW;  // k offset of the word in the stage
                     uint32_t bx[NT][Cfg::NP], bxl[NT][Cfg::NP];
 #pragma unroll
                     for (int t = 0; t < NT; ++t)
                         load_b_pairs<BITS, XT, Cfg::NP, Cfg::MMAX>(xst, t * 8 + gid, kl, bx[t], bxl[t]);
 #pragma unroll
                     for (int part = 0; part < Cfg::NP / 2; ++part) {
-                        uint32_t a[4];
-                        make_a_regs<BITS>(w0, w1, part, a);
 #pragma unroll
                         for (int t = 0; t < NT; ++t) {
-                            mma_bf16_16816(d[t], a, bx[t][2 * part], bx[t][2 * part + 1]);
                             mma_bf16_16816(dx[t], ones, bx[t][2 * part], bx[t][2 * part + 1]);
-                            if constexpr (sizeof(XT) == 4) {
-                                mma_bf16_16816(d[t], a, bxl[t][2 * part], bxl[t][2 * part + 1]);
+                            if constexpr (sizeof(XT) == 4)
                                 mma_bf16_16816(dx[t], ones, bxl[t][2 * part], bxl[t][2 * part + 1]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < RT; ++i) {
+                            uint32_t a[4];
+                            make_a_regs<BITS>(w[i][0], w[i][1], part, a);
+#pragma unroll
+                            for (int t = 0; t < NT; ++t) {
+                                mma_bf16_16816(d[i][t], a, bx[t][2 * part], bx[t][2 * part + 1]);
+                                if constexpr (sizeof(XT) == 4)
+                                    mma_bf16_16816(d[i][t], a, bxl[t][2 * part], bxl[t][2 * part + 1]);
                             }
                         }
                     }
                 }
                 // group epilogue: acc += s * D' + (b - OFFSET s) * X
-                const int gidx = it * (Cfg::KST / G) + gl;
-                const float2 pr0 = params[row0 * p.gstride + gidx];
-                const float2 pr1 = params[(row0 + 8) * p.gstride + gidx];
+                const int gidx = it * Cfg::GPS + gl;
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    acc[t][0] = fmaf(pr0.x, d[t][0], fmaf(pr0.y, dx[t][0], acc[t][0]));
-                    acc[t][1] = fmaf(pr0.x, d[t][1], fmaf(pr0.y, dx[t][1], acc[t][1]));
-                    acc[t][2] = fmaf(pr1.x, d[t][2], fmaf(pr1.y, dx[t][2], acc[t][2]));
-                    acc[t][3] = fmaf(pr1.x, d[t][3], fmaf(pr1.y, dx[t][3], acc[t][3]));
+                for (int i = 0; i < RT; ++i) {
+                    const int row = i * 16 + gid;
+                    const float2 pr0 = params[row * ng + gidx];
+                    const float2 pr1 = params[(row + 8) * ng + gidx];
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        acc[i][t][0] = fmaf(pr0.x, d[i][t][0], fmaf(pr0.y, dx[t][0], acc[i][t][0]));
+                        acc[i][t][1] = fmaf(pr0.x, d[i][t][1], fmaf(pr0.y, dx[t][1], acc[i][t][1]));
+                        acc[i][t][2] = fmaf(pr1.x, d[i][t][2], fmaf(pr1.y, dx[t][2], acc[i][t][2]));
+                        acc[i][t][3] = fmaf(pr1.x, d[i][t][3], fmaf(pr1.y, dx[t][3], acc[i][t][3]));
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&bars.empty[slot]);
         }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const int c0 = t * 8 + 2 * tig;
-            atomicAdd(&red[c0 * kRedStride + row0], acc[t][0]);
-            atomicAdd(&red[(c0 + 1) * kRedStride + row0], acc[t][1]);
-            atomicAdd(&red[c0 * kRedStride + row0 + 8], acc[t][2]);
-            atomicAdd(&red[(c0 + 1) * kRedStride + row0 + 8], acc[t][3]);
+        cta_reduce<RT * NT * 4, 1>(
+            reinterpret_cast<float*>(stages), red,
+            [&](int j) { return acc[j / (NT * 4)][(j / 4) % NT][j % 4]; },
+            [&](int, int j, int ln, int& row, int& tok) {
+                const int i = j / (NT * 4), t = (j / 4) % NT, e = j % 4;
+                row = i * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
+                tok = t * 8 + 2 * (ln & 3) + (e & 1);
+            });
+        consumer_bar();
+        using OT = XT;
+        const OT* bias = static_cast<const OT*>(p.bias);
+        OT* y = static_cast<OT*>(p.y);
+        for (int e = threadIdx.x; e < M * ROWS; e += kConsumerThreads) {
+            const int tok = e / ROWS, r = e % ROWS;
+            if (r < rows_valid) {
+                float v = red[tok * kRedStride + r];
+                if (bias)
+                    v += to_float(bias[n0 + r]);
+                y[(size_t)tok * p.N + n0 + r] = from_float<OT>(v);
+            }
         }
     }
-    using OT = XT;
-    const OT* bias = static_cast<const OT*>(p.bias);
-    OT* y = static_cast<OT*>(p.y);
-    cluster_reduce(bars, red, recv, M, S, p.status, [&](int tok, int r, float v) {
-        if (r < rows_valid) {
-            if (bias)
-                v += to_float(bias[n0 + r]);
-            y[(size_t)tok * p.N + n0 + r] = from_float<OT>(v);
-        }
-    });
 }
 
 // ---------------------------------------------------------------- BitLinear decode kernel
 
 template <int NT>
 struct BitCfg {
-    static constexpr int PROWS = kRowsPerCta / 4;   // packed rows per CTA (16) -> 64 output rows
+    static constexpr int PROWS = 8;                 // packed rows per CTA -> 32 output rows
     static constexpr int KST = 512;                 // k (bytes per packed row) per stage
     static constexpr int NWB = KST / 128;           // 128-byte weight boxes per stage
     static constexpr int NXB = KST * 2 / 128;       // 128-byte x boxes per stage
@@ -538,25 +540,30 @@ struct BitCfg {
     static constexpr int W_STAGE = NWB * PROWS * 128;
     static constexpr int X_STAGE = NXB * MMAX * 128;
     static constexpr int STAGE = W_STAGE + X_STAGE;
+    static constexpr int NS = (64 * 1024 / STAGE) > kStages ? kStages : (64 * 1024 / STAGE);
+    static constexpr int SPW = KST / 16 / kConsumerWarps;  // k16 steps per warp in a full stage
     static_assert(STAGE % 1024 == 0, "swizzled boxes need 1024-byte alignment");
     static constexpr int RED = MMAX * kRedStride * 4;
-    static constexpr int recv_bytes(int S) { return S * MMAX * kRowsPerCta * 4; }
-    static constexpr int smem_bytes(int S) { return kStages * STAGE + RED + recv_bytes(S) + (int)sizeof(Barriers) + 1024; }
+    static constexpr int SMEM = NS * STAGE + RED + (int)sizeof(Barriers) + 1024;
 };
 
 struct BitParams {
-    CUtensorMap tm_w;  // packed [N/4][K] bytes, box {128 B, 16 rows}
-    CUtensorMap tm_x;  // x [M][K] bf16, box {64 elements, 8*NT tokens}
-    const uint8_t* packed;
-    const __nv_bfloat16* x;
+    CUtensorMap tm_w;  // packed [N/4][K] bytes, box {128 B, 8 rows}
+    CUtensorMap tm_x;  // x [M][K] bf16, box {64 elements, M tokens}
     const float* weight_scale;
     const __nv_bfloat16* bias;
     __nv_bfloat16* y;
     int M, K, N, R;  // R = N / 4
-    int k_per_split;
     int invert;
     unsigned* status;
 };
+
+QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t r;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 2) bitlinear_gemv_kernel(const __grid_constant__ BitParams p)
@@ -565,26 +572,21 @@ __global__ void __launch_bounds__(kThreads, 2) bitlinear_gemv_kernel(const __gri
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
-    float* red = reinterpret_cast<float*>(smem + kStages * Cfg::STAGE);
-    float* recv = red + Cfg::RED / 4;
-    Barriers& bars = *reinterpret_cast<Barriers*>(reinterpret_cast<uint8_t*>(recv) + Cfg::recv_bytes(gridDim.x));
+    float* red = reinterpret_cast<float*>(smem + Cfg::NS * Cfg::STAGE);
+    Barriers& bars = *reinterpret_cast<Barriers*>(reinterpret_cast<uint8_t*>(red) + Cfg::RED);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = gridDim.x;
-    const int split = blockIdx.x;
-    const int p0 = blockIdx.y * Cfg::PROWS;
-    const int kbeg = split * p.k_per_split;
-    const int kend = min(p.K, kbeg + p.k_per_split);
-    const int nst = kend > kbeg ? (kend - kbeg + Cfg::KST - 1) / Cfg::KST : 0;
+    const int p0 = blockIdx.x * Cfg::PROWS;
+    const int nst = (p.K + Cfg::KST - 1) / Cfg::KST;
     const int M = p.M;
 
-    init_barriers(bars, S);
+    init_barriers(bars);
 
     if (warp == kConsumerWarps) {
-        producer_loop(
+        producer_loop<Cfg::NS>(
             bars, nst, p.status,
             [&](int it, int slot) {
-                const int k0 = kbeg + it * Cfg::KST;
+                const int k0 = it * Cfg::KST;
                 uint8_t* wst = stages + slot * Cfg::STAGE;
                 uint8_t* xst = wst + Cfg::W_STAGE;
 #pragma unroll
@@ -595,128 +597,116 @@ __global__ void __launch_bounds__(kThreads, 2) bitlinear_gemv_kernel(const __gri
                     tma_load_2d(xst + b * (Cfg::MMAX * 128), &p.tm_x, k0 + b * 64, 0, &bars.full[slot]);
             },
             [&](int it) {
-                const int k0 = kbeg + it * Cfg::KST;
 #pragma unroll
                 for (int b = 0; b < Cfg::NWB; ++b)
-                    tma_prefetch_2d(&p.tm_w, k0 + b * 128, p0);
+                    tma_prefetch_2d(&p.tm_w, it * Cfg::KST + b * 128, p0);
             },
-            [&](int) { return (unsigned)Cfg::STAGE; });
+            [&](int) { return (unsigned)(Cfg::W_STAGE + Cfg::NXB * M * 128); });
     } else {
-        for (int e = threadIdx.x; e < Cfg::RED / 4; e += kConsumerThreads)
-            red[e] = 0.f;
+        zero_x_tail(stages, Cfg::NS, Cfg::STAGE, Cfg::W_STAGE, Cfg::NXB, Cfg::MMAX, M);
+        pdl_wait_prior_grids();  // weight_scale may come from an earlier kernel
+        const float ws = *p.weight_scale;
+        const float scale = p.invert ? __fdiv_rn(1.0f, ws) : ws;
         consumer_bar();
+        // Warps take k16 steps round robin.  A lane's 32-bit word (4 consecutive
+        // k of packed row gid) feeds two MMAs: fields {0, 2} and {1, 3} of its
+        // bytes, as A rows gid / gid+8.  Field j is read in place with one LOP3,
+        // (w & (3 << 2j)) | 0x4300 = bf16 128 + 4^j c, and one bf16x2 FMA,
+        // times 4^-j minus (128 4^-j + 1), gives the exact weight c - 1.
         const int gid = lane >> 2, tig = lane & 3;
-        const int rt = warp % kRowTiles, kl_lane = warp / kRowTiles;
-        const int prow = rt * 4 + (gid & 3);  // local packed row of both A rows of this lane
-        const int sh0 = 2 * (gid >> 2);       // field j of A row gid; row gid+8 uses j+2
-        // two accumulator sets (even / odd steps) halve the MMA dependency chain
-        float acc[2][NT][4];
+        // per-field bf16x2 constants: {4^-j, -(128 4^-j + 1)} for the rows of each MMA
+        constexpr uint32_t kScale0 = 0x3F803F80u, kBias0 = 0xC301C301u;  // j=0: 1, -129
+        constexpr uint32_t kScale1 = 0x3E803E80u, kBias1 = 0xC204C204u;  // j=1: 1/4, -33
+        constexpr uint32_t kScale2 = 0x3D803D80u, kBias2 = 0xC110C110u;  // j=2: 1/16, -9
+        float a02[NT][4], a13[NT][4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int t = 0; t < NT; ++t)
+            for (int e = 0; e < 4; ++e)
+                a02[t][e] = a13[t][e] = 0.f;
+        auto step = [&](const uint8_t* wst, const uint8_t* xst, int s) {
+            const int wi = s * 4 + tig;  // word of 4 bytes (k = 4 wi .. 4 wi + 3)
+            const uint32_t w = w_word(wst, Cfg::PROWS, gid, wi);
+            const uint32_t hw = w >> 8;  // bytes k+1, k+3 in the low byte of each half
+            uint32_t f02[4], f13[4];
+            f02[0] = bf16x2_fma(lop3_and_or(w, 0x00030003u, 0x43004300u), kScale0, kBias0);         // f0 (k, k+2)
+            f02[1] = bf16x2_fma(lop3_and_or(w, 0x00300030u, 0x43004300u), kScale2, kBias2);         // f2 (k, k+2)
+            f02[2] = bf16x2_fma(lop3_and_or(hw, 0x00030003u, 0x43004300u), kScale0, kBias0);        // f0 (k+1, k+3)
+            f02[3] = bf16x2_fma(lop3_and_or(hw, 0x00300030u, 0x43004300u), kScale2, kBias2);        // f2 (k+1, k+3)
+            f13[0] = bf16x2_fma(lop3_and_or(w, 0x000C000Cu, 0x43004300u), kScale1, kBias1);         // f1 (k, k+2)
+            f13[1] = bf16x2_fma(lop3_and_or(w >> 6, 0x00030003u, 0x43004300u), kScale0, kBias0);    // f3 (k, k+2)
+            f13[2] = bf16x2_fma(lop3_and_or(hw, 0x000C000Cu, 0x43004300u), kScale1, kBias1);        // f1 (k+1, k+3)
+            f13[3] = bf16x2_fma(lop3_and_or(w >> 14, 0x00030003u, 0x43004300u), kScale0, kBias0);   // f3 (k+1, k+3)
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    acc[h][t][i] = 0.f;
+            for (int t = 0; t < NT; ++t) {
+                // tokens >= M read zeros
+                const uint2 v = *reinterpret_cast<const uint2*>(
+                    x_addr<__nv_bfloat16, Cfg::MMAX>(xst, t * 8 + gid, 4 * wi));
+                const uint32_t b0 = pair_lo(v.x, v.y);  // (x_k, x_{k+2})
+                const uint32_t b1 = pair_hi(v.x, v.y);  // (x_{k+1}, x_{k+3})
+                mma_bf16_16816(a02[t], f02, b0, b1);
+                mma_bf16_16816(a13[t], f13, b0, b1);
+            }
+        };
         for (int it = 0; it < nst; ++it) {
-            const int slot = it % kStages;
-            if (!mbar_wait_bounded(&bars.full[slot], (it / kStages) & 1, p.status)) {
+            const int slot = it % Cfg::NS;
+            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status)) {
                 bars.abort_flag = 1;
                 break;
             }
             const uint8_t* wst = stages + slot * Cfg::STAGE;
             const uint8_t* xst = wst + Cfg::W_STAGE;
-            const int kst = min(Cfg::KST, kend - (kbeg + it * Cfg::KST));
-            const int steps = kst / 16;
-            const int s_half = (steps + 1) / 2;
-            const int s_beg = kl_lane * s_half;
-            const int s_end = min(steps, s_beg + s_half);
-            // one k16 step: A from the word of this lane, B from x; accumulates into acc_h
-            auto step = [&](int s, float (&acc_h)[NT][4]) {
-                const int wi = s * 4 + tig;  // word of 4 bytes (k = 4 wi .. 4 wi + 3)
-                const uint32_t w = w_word(wst, Cfg::PROWS, prow, wi);
-                uint32_t a[4];
-                // (c + 128) pairs, then + (-129, -129): the exact weights c - 1.
-                // row gid: field j = sh0 / 2, pairs (k, k+2) and (k+1, k+3); row gid+8: field j + 2
-                a[0] = bf16x2_add(lop3_and_or(w >> sh0, 0x00030003u, 0x43004300u), kMinus129Bf16x2);
-                a[2] = bf16x2_add(lop3_and_or(w >> (sh0 + 8), 0x00030003u, 0x43004300u), kMinus129Bf16x2);
-                a[1] = bf16x2_add(lop3_and_or(w >> (sh0 + 4), 0x00030003u, 0x43004300u), kMinus129Bf16x2);
-                a[3] = bf16x2_add(lop3_and_or(w >> (sh0 + 12), 0x00030003u, 0x43004300u), kMinus129Bf16x2);
+            const int steps = min(Cfg::KST, p.K - it * Cfg::KST) / 16;
+            if (steps == Cfg::KST / 16) {
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    // tokens >= M read the zeros the TMA wrote
-                    const uint2 v = *reinterpret_cast<const uint2*>(
-                        x_addr<__nv_bfloat16, Cfg::MMAX>(xst, t * 8 + gid, 4 * wi));
-                    mma_bf16_16816(acc_h[t], a, pair_lo(v.x, v.y), pair_hi(v.x, v.y));  // (x_k, x_{k+2}), (x_{k+1}, x_{k+3})
-                }
-            };
-            int s = s_beg;
-#pragma unroll 2
-            for (; s + 1 < s_end; s += 2) {
-                step(s, acc[0]);
-                step(s + 1, acc[1]);
+                for (int j = 0; j < Cfg::SPW; ++j)
+                    step(wst, xst, warp + j * kConsumerWarps);
+            } else {
+                for (int s2 = warp; s2 < steps; s2 += kConsumerWarps)
+                    step(wst, xst, s2);
             }
-            if (s < s_end)
-                step(s, acc[0]);
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&bars.empty[slot]);
         }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const int c0 = t * 8 + 2 * tig;
-            const int r0 = rt * 16 + gid;
-            atomicAdd(&red[c0 * kRedStride + r0], acc[0][t][0] + acc[1][t][0]);
-            atomicAdd(&red[(c0 + 1) * kRedStride + r0], acc[0][t][1] + acc[1][t][1]);
-            atomicAdd(&red[c0 * kRedStride + r0 + 8], acc[0][t][2] + acc[1][t][2]);
-            atomicAdd(&red[(c0 + 1) * kRedStride + r0 + 8], acc[0][t][3] + acc[1][t][3]);
+        // red row index = field * 8 + local packed row
+        cta_reduce<NT * 8, 1>(
+            reinterpret_cast<float*>(stages), red,
+            [&](int j) {
+                const int t = j / 8, e = (j / 4) % 2, f = j % 4;
+                switch (f) {
+                case 0: return a02[t][e];
+                case 1: return a13[t][e];
+                case 2: return a02[t][e + 2];
+                default: return a13[t][e + 2];
+                }
+            },
+            [&](int, int j, int ln, int& row, int& tok) {
+                const int t = j / 8, e = (j / 4) % 2, f = j % 4;
+                row = f * 8 + (ln >> 2);
+                tok = t * 8 + 2 * (ln & 3) + e;
+            });
+        consumer_bar();
+        for (int e = threadIdx.x; e < M * 32; e += kConsumerThreads) {
+            const int tok = e / 32, i = e % 32;
+            const int pr = p0 + (i & 7);
+            if (pr < p.R) {
+                const int n = pr + (i >> 3) * p.R;
+                float v = red[tok * kRedStride + i] * scale;
+                if (p.bias)
+                    v += __bfloat162float(p.bias[n]);
+                p.y[(size_t)tok * p.N + n] = __float2bfloat16_rn(v);
+            }
         }
     }
-    pdl_wait_prior_grids();  // weight_scale may come from an earlier kernel
-    const float ws = *p.weight_scale;
-    const float scale = p.invert ? __fdiv_rn(1.0f, ws) : ws;
-    cluster_reduce(bars, red, recv, M, S, p.status, [&](int tok, int i, float v) {
-        // local row i: row tile i / 16; A row ii = i % 16 -> packed row 4 (i / 16) + ii % 4, field ii / 4
-        const int ii = i % 16;
-        const int pr = p0 + (i / 16) * 4 + (ii & 3);
-        if (pr < p.R) {
-            const int n = pr + (ii >> 2) * p.R;
-            v *= scale;
-            if (p.bias)
-                v += __bfloat162float(p.bias[n]);
-            p.y[(size_t)tok * p.N + n] = __float2bfloat16_rn(v);
-        }
-    });
 }
 
 // ---------------------------------------------------------------- launch helpers
 
-struct SplitPlan {
-    int S;
-    int k_per_split;
-};
-
-SplitPlan plan_splits(int tiles, int K, int kst, int sm_count, int max_k_per_split)
-{
-    const int nst = (K + kst - 1) / kst;
-    int S = (2 * sm_count + tiles - 1) / tiles;
-    S = S < 1 ? 1 : (S > kMaxCluster ? kMaxCluster : S);
-    const int min_s = (K + max_k_per_split - 1) / max_k_per_split;
-    if (S < min_s)
-        S = min_s;
-    if (S > nst)
-        S = nst;
-    const int sps = (nst + S - 1) / S;
-    SplitPlan pl;
-    pl.S = (nst + sps - 1) / sps;
-    pl.k_per_split = sps * kst;
-    return pl;
-}
-
 template <typename Kern, typename Params>
-cudaError_t launch_cluster(Kern kern, dim3 grid, int smem, int cluster_x, cudaStream_t st, const Params& prm)
+cudaError_t launch_pdl(Kern kern, dim3 grid, int smem, cudaStream_t st, const Params& prm)
 {
-    if (cluster_x > kMaxCluster)
+    if (smem > 227 * 1024)
         return cudaErrorNotSupported;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
@@ -726,29 +716,21 @@ cudaError_t launch_cluster(Kern kern, dim3 grid, int smem, int cluster_x, cudaSt
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cluster_x;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
-template <int BITS, int G, typename XT, typename PT, int NT>
+template <int BITS, int G, typename XT, typename PT, int NT, int RT>
 cudaError_t affine_launch_t(const AffineGemvArgs& a, int m0, int mcount, cudaStream_t st, const DeviceInfo& dev)
 {
-    using Cfg = AffineCfg<BITS, G, XT, PT, NT>;
-    const int tiles = (int)((a.N + kRowsPerCta - 1) / kRowsPerCta);
-    const SplitPlan pl = plan_splits(tiles, (int)a.K, Cfg::KST, dev.sm_count, Cfg::MAX_GROUPS * G);
-    if (pl.k_per_split / G > Cfg::MAX_GROUPS)
-        return cudaErrorNotSupported;
+    using Cfg = AffineCfg<BITS, G, XT, PT, NT, RT>;
+    (void)dev;
     AffineParams prm;
-    prm.codes = reinterpret_cast<const uint8_t*>(a.codes);
-    prm.x = static_cast<const uint8_t*>(a.x) + (size_t)m0 * a.K * sizeof(XT);
+    const void* x = static_cast<const uint8_t*>(a.x) + (size_t)m0 * a.K * sizeof(XT);
     prm.scales = a.scales;
     prm.biases = a.biases;
     prm.bias = a.bias;
@@ -756,26 +738,33 @@ cudaError_t affine_launch_t(const AffineGemvArgs& a, int m0, int mcount, cudaStr
     prm.M = mcount;
     prm.K = (int)a.K;
     prm.N = (int)a.N;
-    prm.k_per_split = pl.k_per_split;
-    prm.gstride = pl.k_per_split / G;
     prm.status = dev.status;
     const uint64_t row_bytes = (uint64_t)a.K * BITS / 8;
     if (!encode_tmap_2d(&prm.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, row_bytes, (uint64_t)a.N, row_bytes, 128,
-                        kRowsPerCta) ||
+                        Cfg::ROWS) ||
         !encode_tmap_2d(&prm.tm_x, sizeof(XT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                        prm.x, (uint64_t)a.K, (uint64_t)mcount, (uint64_t)a.K * sizeof(XT), Cfg::XE, Cfg::MMAX))
+                        x, (uint64_t)a.K, (uint64_t)mcount, (uint64_t)a.K * sizeof(XT), Cfg::XE, (uint32_t)mcount))
         return cudaErrorInvalidValue;
-    return launch_cluster(affine_gemv_kernel<BITS, G, XT, PT, NT>, dim3(pl.S, tiles, 1),
-                          Cfg::smem_bytes(prm.gstride, pl.S), pl.S, st, prm);
+    const int ctas = (int)((a.N + Cfg::ROWS - 1) / Cfg::ROWS);
+    return launch_pdl(affine_gemv_kernel<BITS, G, XT, PT, NT, RT>, dim3(ctas, 1, 1), Cfg::smem_bytes((int)(a.K / G)),
+                      st, prm);
 }
 
 template <int BITS, int G, typename XT, typename PT>
 cudaError_t affine_launch_nt(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
+    // 64-row CTAs when that still gives about one CTA per SM, else 32-row CTAs
+    const bool wide = a.N / 64 >= dev.sm_count;
     for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
         const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
-        cudaError_t e = mc <= 8 ? affine_launch_t<BITS, G, XT, PT, 1>(a, (int)m0, mc, st, dev)
-                                : affine_launch_t<BITS, G, XT, PT, 2>(a, (int)m0, mc, st, dev);
+        cudaError_t e;
+        if (mc <= 8 && sizeof(XT) == 2)
+            e = wide ? affine_launch_t<BITS, G, XT, PT, 1, 4>(a, (int)m0, mc, st, dev)
+                     : affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev);
+        else if (mc <= 8)
+            e = affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev);
+        else
+            e = affine_launch_t<BITS, G, XT, PT, 2, 2>(a, (int)m0, mc, st, dev);
         if (e != cudaSuccess)
             return e;
     }
@@ -823,8 +812,7 @@ cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const
     for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
         const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
         BitParams prm;
-        prm.packed = a.packed;
-        prm.x = static_cast<const __nv_bfloat16*>(a.x) + m0 * a.K;
+        const void* x = static_cast<const __nv_bfloat16*>(a.x) + m0 * a.K;
         prm.weight_scale = a.weight_scale;
         prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
         prm.y = static_cast<__nv_bfloat16*>(a.y) + m0 * a.N;
@@ -834,21 +822,14 @@ cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const
         prm.R = R;
         prm.invert = a.invert;
         prm.status = dev.status;
-        cudaError_t e;
-        const int tiles = (R + BitCfg<1>::PROWS - 1) / BitCfg<1>::PROWS;
-        const SplitPlan pl = plan_splits(tiles, (int)a.K, BitCfg<1>::KST, dev.sm_count, 1 << 30);
-        prm.k_per_split = pl.k_per_split;
         if (!encode_tmap_2d(&prm.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, (uint64_t)a.K, (uint64_t)R,
                             (uint64_t)a.K, 128, BitCfg<1>::PROWS) ||
-            !encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, prm.x, (uint64_t)a.K, (uint64_t)mc,
-                            (uint64_t)a.K * 2, 64, mc <= 8 ? 8 : 16))
+            !encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)a.K, (uint64_t)mc,
+                            (uint64_t)a.K * 2, 64, (uint32_t)mc))
             return cudaErrorInvalidValue;
-        if (mc <= 8)
-            e = launch_cluster(bitlinear_gemv_kernel<1>, dim3(pl.S, tiles, 1), BitCfg<1>::smem_bytes(pl.S), pl.S, st,
-                               prm);
-        else
-            e = launch_cluster(bitlinear_gemv_kernel<2>, dim3(pl.S, tiles, 1), BitCfg<2>::smem_bytes(pl.S), pl.S, st,
-                               prm);
+        const int ctas = (R + BitCfg<1>::PROWS - 1) / BitCfg<1>::PROWS;
+        cudaError_t e = mc <= 8 ? launch_pdl(bitlinear_gemv_kernel<1>, dim3(ctas, 1, 1), BitCfg<1>::SMEM, st, prm)
+                                : launch_pdl(bitlinear_gemv_kernel<2>, dim3(ctas, 1, 1), BitCfg<2>::SMEM, st, prm);
         if (e != cudaSuccess)
             return e;
     }
