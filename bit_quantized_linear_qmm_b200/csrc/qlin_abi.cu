@@ -118,8 +118,8 @@ size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits
     if (M <= 0 || K <= 0)
         return 0;
     switch (op) {
-    case QLIN_OP_W8A8: return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
-    case QLIN_OP_W4A8: return align256((size_t)M * (size_t)K) + 2 * align256((size_t)M * 4);
+    case QLIN_OP_W8A8:
+    case QLIN_OP_W4A8: return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
     default: return 0;
     }
 }
@@ -182,6 +182,20 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
     DeviceInfo dev;
     if ((s = current_device(dev)) != QLIN_OK)
         return s;
+    if (M > 16 && bits == 4 && x_dt == QLIN_BF16 && param_dt == QLIN_BF16) {
+        TcGemmArgs t = {};
+        t.M = M;
+        t.N = N;
+        t.K = K;
+        t.a = x;
+        t.b = codes;
+        t.out = y;
+        t.bias = bias;
+        t.scales = scales;
+        t.biases = biases;
+        t.g = group_size;
+        return from_cuda(launch_tc_gemm(TC_AFFINE4, t, static_cast<cudaStream_t>(stream), dev));
+    }
     AffineGemvArgs a;
     a.x = x;
     a.x_dt = x_dt;
@@ -262,29 +276,82 @@ qlin_status qlin_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64
 qlin_status qlin_int8_matmul_int32(const int8_t* a, const int8_t* b, int64_t M, int64_t N, int64_t K, int32_t* c,
                                    void* stream)
 {
-    (void)stream;
-    if (!a || !b || !c || M <= 0 || N <= 0 || K <= 0)
+    if (!a || !b || !c || M <= 0 || N <= 0 || K <= 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
         return QLIN_ERR_INVALID_ARG;
-    return QLIN_ERR_UNSUPPORTED;
+    if (K % 16 != 0)
+        return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(c))
+        return QLIN_ERR_MISALIGNED;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    TcGemmArgs t = {};
+    t.M = M;
+    t.N = N;
+    t.K = K;
+    t.a = a;
+    t.b = b;
+    t.out = c;
+    return from_cuda(launch_tc_gemm(TC_I8_RAW, t, static_cast<cudaStream_t>(stream), dev));
 }
+
+namespace {
+
+// Shared body of the W8A8 / W4A8 layers: per-token int8 activation quant
+// into the workspace, then the tcgen05 GEMM with the scaled epilogue.
+qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const void* w,
+                       const float* scale_w, int64_t N, const void* bias, void* y, void* workspace, size_t ws_bytes,
+                       void* stream)
+{
+    if (!x || !w || !scale_w || !y || M <= 0 || N <= 0 || K <= 0 || M > INT32_MAX || N > INT32_MAX ||
+        K > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (op == TC_W4A8 ? (K % 32 != 0 || N % 16 != 0) : (K % 16 != 0))
+        return QLIN_ERR_INVALID_ARG;
+    if (x_dt != QLIN_BF16)
+        return QLIN_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(y))
+        return QLIN_ERR_MISALIGNED;
+    const size_t need = qlin_workspace_size(op == TC_W4A8 ? QLIN_OP_W4A8 : QLIN_OP_W8A8, M, N, K, 0, 0);
+    if (!workspace || ws_bytes < need || !aligned16(workspace))
+        return QLIN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    int8_t* qx = static_cast<int8_t*>(workspace);
+    float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)M * (size_t)K));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, nullptr, st, dev);
+    if (e != cudaSuccess)
+        return from_cuda(e);
+    TcGemmArgs t = {};
+    t.M = M;
+    t.N = N;
+    t.K = K;
+    t.a = qx;
+    t.b = w;
+    t.out = y;
+    t.s_x = sx;
+    t.s_w = scale_w;
+    t.bias = bias;
+    return from_cuda(launch_tc_gemm(op, t, st, dev));
+}
+
+}  // namespace
 
 qlin_status w8a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const int8_t* w, const float* scale_w,
                         int64_t N, const void* bias, void* y, void* workspace, size_t ws_bytes, void* stream)
 {
-    (void)x_dt, (void)bias, (void)workspace, (void)ws_bytes, (void)stream;
-    if (!x || !w || !scale_w || !y || M <= 0 || N <= 0 || K <= 0)
-        return QLIN_ERR_INVALID_ARG;
-    return QLIN_ERR_UNSUPPORTED;
+    return int_linear(TC_W8A8, x, x_dt, M, K, w, scale_w, N, bias, y, workspace, ws_bytes, stream);
 }
 
 qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const uint8_t* packed_w,
                         const float* scale_w, int64_t N, const void* bias, void* y, void* workspace, size_t ws_bytes,
                         void* stream)
 {
-    (void)x_dt, (void)bias, (void)workspace, (void)ws_bytes, (void)stream;
-    if (!x || !packed_w || !scale_w || !y || M <= 0 || N <= 0 || K <= 0)
-        return QLIN_ERR_INVALID_ARG;
-    return QLIN_ERR_UNSUPPORTED;
+    return int_linear(TC_W4A8, x, x_dt, M, K, packed_w, scale_w, N, bias, y, workspace, ws_bytes, stream);
 }
 
 qlin_status qlin_get_device_status(void* stream)
@@ -319,7 +386,7 @@ qlin_status qlin_get_device_status(void* stream)
 namespace qlin {
 
 bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t dim0, uint64_t dim1,
-                    uint64_t pitch_bytes, uint32_t box0, uint32_t box1)
+                    uint64_t pitch_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle swizzle)
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -338,9 +405,8 @@ bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, u
     cuuint64_t strides[1] = {pitch_bytes};
     cuuint32_t box[2] = {box0, box1};
     cuuint32_t estr[2] = {1, 1};
-    return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace qlin

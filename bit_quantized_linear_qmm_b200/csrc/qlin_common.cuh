@@ -156,6 +156,76 @@ QLIN_DEV void tma_prefetch_2d(const CUtensorMap* tmap, int c0, int c1)
 // base 1024-byte aligned): units are XOR-permuted by row mod 8.
 QLIN_DEV int swz128(int row, int unit) { return row * 128 + ((unit ^ (row & 7)) << 4); }
 
+// ---------------------------------------------------------------- tcgen05 (5th-generation tensor cores, TMEM)
+
+QLIN_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+QLIN_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Whole warp: allocate `ncols` TMEM columns (power of two >= 32); the base
+// address is written to *dst (shared memory).
+QLIN_DEV void tmem_alloc(uint32_t* dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+QLIN_DEV void tmem_dealloc(uint32_t base, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, one elected thread.  KIND is
+// "f16" (bf16/f16 inputs, f32 accumulate) or "i8" (s8/u8 inputs, s32).
+template <bool I8>
+QLIN_DEV void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate)
+{
+    if constexpr (I8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+            : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
+QLIN_DEV void tc_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit TMEM columns -> 16 registers per thread.
+QLIN_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile written with the
+// 128-byte swizzle (rows of 128 bytes, 8-row groups 1024 bytes apart).
+QLIN_DEV uint64_t umma_desc_sw128(uint32_t smem_addr)
+{
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the
+// async proxy (TMA, tensor cores).
+QLIN_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ---------------------------------------------------------------- cluster helpers
 
 QLIN_DEV unsigned cluster_ctarank()
@@ -298,10 +368,11 @@ struct DeviceInfo {
 
 // Host: encodes a 2-D tiled tensor map (row-major [dim1][dim0] elements,
 // row pitch `pitch_bytes`) with box {box0, box1}, 128-byte swizzle, zero
-// fill.  Returns false if the driver entry point is unavailable or rejects
+// fill (or the given swizzle).  Returns false if the driver entry point is unavailable or rejects
 // the description.
 bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t dim0, uint64_t dim1,
-                    uint64_t pitch_bytes, uint32_t box0, uint32_t box1);
+                    uint64_t pitch_bytes, uint32_t box0, uint32_t box1,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 cudaError_t launch_affine_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int bits, int g,
                                    uint32_t* codes, void* scales, void* biases, qlin_dtype p_dt,
@@ -339,5 +410,26 @@ struct BitlinearArgs {
     void* y;
 };
 cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const DeviceInfo& dev);
+
+}  // namespace qlin
+
+namespace qlin {
+
+// tcgen05 GEMM launches (k_tc_gemm.cu).  A is [M][K] row-major (int8 or
+// bf16), the output [M][N] row-major.
+struct TcGemmArgs {
+    int64_t M, N, K;
+    const void* a;            // int8 (qx / raw a) or bf16 (x)
+    const void* b;            // int8 w [N][K], packed int4 [K/2][N] or affine codes [N][K*bits/32]
+    void* out;                // int32 or bf16 [M][N]
+    const float* s_x;         // [M] (W8A8 / W4A8)
+    const float* s_w;         // [N] (W8A8 / W4A8)
+    const void* bias;         // bf16 [N] or null
+    const void* scales;       // affine: bf16 [N][K/g]
+    const void* biases;
+    int g;
+};
+enum TcOp { TC_I8_RAW = 0, TC_W8A8 = 1, TC_W4A8 = 2, TC_AFFINE4 = 3 };
+cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev);
 
 }  // namespace qlin

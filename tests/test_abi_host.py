@@ -32,7 +32,7 @@ def test_workspace_sizes(ql):
     assert ql.workspace_size(ql.QLIN_OP_BITLINEAR, 8, 4096, 4096) == 0
     assert ql.workspace_size(ql.QLIN_OP_W8A8, 4096, 8192, 8192) == 4096 * 8192 + 4096 * 4
     assert ql.workspace_size(ql.QLIN_OP_W8A8, 1, 8192, 8192) == 8192 + 256
-    assert ql.workspace_size(ql.QLIN_OP_W4A8, 1, 8192, 8192) == 8192 + 512
+    assert ql.workspace_size(ql.QLIN_OP_W4A8, 1, 8192, 8192) == 8192 + 256
 
 
 P16 = C.c_void_p(256)  # a non-null, 16-byte aligned stand-in; never dereferenced on these paths

@@ -76,3 +76,33 @@ def test_affine_rejects_bad_args(ql):
         ql.matmul(x, codes, s, s, 3, 32)
     assert e.value.status == ql.QLIN_ERR_UNSUPPORTED
     assert ql.device_status() == ql.QLIN_OK
+
+
+PREFILL_SMALL = [
+    synth.AffineCase(f"prefill_b4_g{g}_M{M}_K{K}_N{N}", M, K, N, 4, g, "bf16", "bf16", True, seed=17)
+    for (M, K, N, g) in [(17, 256, 128, 64), (128, 512, 256, 128), (200, 1024, 300, 32), (300, 2048, 640, 64)]
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_SMALL, ids=[c.name for c in PREFILL_SMALL])
+def test_affine_prefill_small(ql, orc, case):
+    _run_case(ql, orc, case)
+
+
+def test_affine_prefill_config_sampled(ql, orc):
+    """2048 x 4096 x 14336 (outlier weights), one call; sampled tokens x features."""
+    case = synth.AFFINE_PREFILL
+    w = case.weight()
+    codes, s, b = orc.affine_quantize(w, 4, 64, True)
+    x = case.x()
+    lb = case.layer_bias()
+    y = ql.matmul(x.torch("cuda"), u32_dev(codes), params_dev(s, "bf16"), params_dev(b, "bf16"), 4, 64,
+                  lb.torch("cuda"))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(9)
+    toks = np.sort(rng.choice(case.M, size=48, replace=False))
+    feats = np.sort(rng.choice(case.N, size=96, replace=False))
+    feats[-1] = case.N - 1
+    yr, mag = orc.affine_matmul(x.vals[toks], codes[feats], s[feats], b[feats], 4, 64, lb.vals[feats])
+    ys = y[torch.as_tensor(toks, device="cuda")][:, torch.as_tensor(feats, device="cuda")]
+    assert_fp_close(ys, yr, mag, lb.vals[feats], case.name)

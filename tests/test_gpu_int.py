@@ -1,0 +1,122 @@
+"""GPU parity of the int8 paths: raw int8 GEMM (bit-exact), W8A8 and W4A8 layers."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import assert_fp_close, build_lib, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ql():
+    return build_lib()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (130, 200, 272), (256, 384, 512), (5, 1000, 4096),
+                                   (128, 128, 16), (333, 129, 1040)])
+def test_int8_matmul_int32_bit_exact(ql, orc, M, N, K):
+    rng = np.random.default_rng(M * 7 + N)
+    a = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+    b = rng.integers(-128, 128, size=(N, K)).astype(np.int8)
+    c = ql.int8_matmul_int32(to_dev(a), to_dev(b))
+    torch.cuda.synchronize()
+    assert np.array_equal(c.cpu().numpy(), orc.int8_matmul(a, b))
+
+
+def test_int8_matmul_extremes(ql, orc):
+    """All -128 times all -128 over K = 4096 -> 2^26 per element (exact int32)."""
+    a = np.full((130, 4096), -128, np.int8)
+    b = np.full((140, 4096), -128, np.int8)
+    c = ql.int8_matmul_int32(to_dev(a), to_dev(b))
+    torch.cuda.synchronize()
+    assert np.all(c.cpu().numpy() == 128 * 128 * 4096)
+
+
+def _w8a8(ql, orc, case, rows=None, bias=False):
+    w = case.weight()
+    qw, sw = orc.quantize_int8_rows(w)
+    x = case.x()
+    lb = synth.activations(case.seed + 2, (case.N,), "bf16", 0.01) if bias else None
+    y = ql.w8a8_linear(x.torch("cuda"), to_dev(qw), to_dev(sw), None if lb is None else lb.torch("cuda"))
+    torch.cuda.synchronize()
+    if rows is not None:
+        qw, sw = qw[rows], sw[rows]
+        y = y[:, torch.as_tensor(rows, device=y.device)]
+    bias_v = None if lb is None else (lb.vals if rows is None else lb.vals[rows])
+    yr, mag, _, _ = orc.w8a8_linear(x.vals, qw, sw, bias_v)
+    return assert_fp_close(y, yr, mag, bias_v, case.name)
+
+
+def _w4a8(ql, orc, case, cols=None):
+    w = case.weight()                       # [N, K]; W4 quantizes its transpose [K, N]
+    P, sw = orc.pack_int4_cols(np.ascontiguousarray(w.T))
+    x = case.x()
+    y = ql.w4a8_linear(x.torch("cuda"), to_dev(P), to_dev(sw))
+    torch.cuda.synchronize()
+    if cols is not None:
+        P, sw = P[:, cols], sw[cols]
+        y = y[:, torch.as_tensor(cols, device=y.device)]
+    yr, mag, _, _ = orc.w4a8_linear(x.vals, P, sw)
+    return assert_fp_close(y, yr, mag, None, case.name)
+
+
+SMALL = [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
+         [(1, 256, 128), (3, 512, 272), (17, 1024, 384), (200, 768, 144), (256, 4096, 256)]]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c.name for c in SMALL])
+@pytest.mark.parametrize("bias", [False, True])
+def test_w8a8_small(ql, orc, case, bias):
+    _w8a8(ql, orc, case, bias=bias)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c.name for c in SMALL])
+def test_w4a8_small(ql, orc, case):
+    _w4a8(ql, orc, case)
+
+
+@pytest.mark.parametrize("case", synth.INT_LINEAR, ids=[c.name for c in synth.INT_LINEAR])
+def test_w8a8_config_sampled(ql, orc, case):
+    rng = np.random.default_rng(2)
+    rows = np.sort(rng.choice(case.N, size=96, replace=False))
+    sub = synth.IntCase(case.name, min(case.M, 256), case.K, case.N, seed=case.seed)
+    _w8a8(ql, orc, sub if case.M > 256 else case, rows)
+
+
+@pytest.mark.parametrize("case", synth.INT_LINEAR, ids=[c.name for c in synth.INT_LINEAR])
+def test_w4a8_config_sampled(ql, orc, case):
+    rng = np.random.default_rng(3)
+    cols = np.sort(rng.choice(case.N, size=96, replace=False))
+    sub = synth.IntCase(case.name, min(case.M, 256), case.K, case.N, seed=case.seed)
+    _w4a8(ql, orc, sub if case.M > 256 else case, cols)
+
+
+def test_w8a8_full_m4096_sampled_rows_and_tokens(ql, orc):
+    """The M=4096 layer through one call; checked on sampled tokens x sampled features."""
+    case = synth.INT_LINEAR[2]
+    w = case.weight()
+    qw, sw = orc.quantize_int8_rows(w)
+    x = case.x()
+    y = ql.w8a8_linear(x.torch("cuda"), to_dev(qw), to_dev(sw))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(4)
+    toks = np.sort(rng.choice(case.M, size=64, replace=False))
+    feats = np.sort(rng.choice(case.N, size=64, replace=False))
+    yr, mag, _, _ = orc.w8a8_linear(x.vals[toks], qw[feats], sw[feats])
+    ys = y[torch.as_tensor(toks, device="cuda")][:, torch.as_tensor(feats, device="cuda")]
+    assert_fp_close(ys, yr, mag, None, "w8a8 M4096 sampled")
+
+
+def test_int_linear_rejects(ql):
+    x = torch.zeros((2, 100), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((16, 100), dtype=torch.int8, device="cuda")
+    s = torch.ones(16, device="cuda")
+    with pytest.raises(ql.QlinError) as e:
+        ql.w8a8_linear(x, w, s)   # K % 16 != 0
+    assert e.value.status == ql.QLIN_ERR_INVALID_ARG
+    with pytest.raises(ql.QlinError) as e:
+        ql.w8a8_linear(x[:, :96].contiguous(), w[:, :96].contiguous(), s, workspace=torch.empty(8, dtype=torch.uint8,
+                                                                                                device="cuda"))
+    assert e.value.status == ql.QLIN_ERR_WORKSPACE
