@@ -2,16 +2,20 @@
 """Throughput benchmark of the quantized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qlin|reference]
-                    [--workload NAME] [--no-suite]
+                    [--no-suite]
 
-One step = one pass of the workload's hot path over one batch of synthetic
-input (for the default workload, the four BitLinear ternary decode layers
-K = N = 4096, M in {1, 8}, multiply and divide scale modes).  Weights rotate
-over device copies whose total exceeds the L2 cache, so every launch streams
-its weights from HBM.  The K timed steps run as CUDA-graph replays between
-CUDA events on the launching stream, bracketed by a barrier and a device
-synchronise; multi-GPU runs take the maximum time over ranks (weak scaling:
-every rank runs its own copy of the workload, no collective on the data path).
+Headline workload (the JSON line's value): BitLinear ternary decode GEMV,
+K = N = 4096, M in {1, 8}, multiply and divide scale modes.  One step = the
+four layer calls.  Weights rotate over device copies whose total exceeds the
+L2 cache, so every launch streams its weights from HBM.  The K timed steps run
+as CUDA-graph replays between CUDA events on the launching stream, bracketed
+by a barrier and a device synchronise; multi-GPU runs take the maximum time
+over ranks (weak scaling: every rank runs its own copy of the workload, no
+collective on the data path).
+
+The "suite" key times every other hot-path operation (MLX-affine decode and
+prefill, W8A8 / W4A8 at M in {1, 256, 4096}, the raw int8 GEMM, quantize /
+dequantize and the per-token activation quantiser) with its own roofline.
 
 Prints ONE JSON line on rank 0.
 """
@@ -38,6 +42,7 @@ import synth  # noqa: E402
 
 METRIC = "qlinear weight-GB/s at M≤16 & TFLOP/s (TOPS) at M≥256, % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense int8 : bf16 tensor-core ratio on B200 (4.5 : 2.25 POPS)
 
 
 # ---------------------------------------------------------------- environment
@@ -65,8 +70,8 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(kernel_key: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    """DRAM bytes per launch from a committed ncu summary, if taken on the
+    current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -135,115 +140,6 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
 
 
-# ---------------------------------------------------------------- workloads
-
-def _rotation_copies(bytes_per_copy: int, l2_bytes: int, minimum: int = 8) -> int:
-    """Copies whose total is at least twice the L2 size."""
-    return max(minimum, int(math.ceil(2 * l2_bytes / bytes_per_copy)))
-
-
-class BitlinearDecode:
-    """BitLinear ternary decode GEMV: x bf16 [M, 4096], packed uint8 [1024, 4096],
-    M in {1, 8}, weight_scale 0.5, multiply and divide modes; no bias."""
-    key = "bitlinear_gemv_kernel"
-    unit = "GB/s"
-    bound = "hbm"
-
-    def __init__(self, l2_bytes: int):
-        from bit_quantized_linear_qmm_b200 import qlin
-        self.ql = qlin
-        self.cases = synth.BITLINEAR_DECODE
-        c0 = self.cases[0]
-        self.K, self.N = c0.K, c0.N
-        self.wbytes = self.N // 4 * self.K
-        packed = torch.from_numpy(c0.packed()).cuda()
-        self.copies = _rotation_copies(self.wbytes, l2_bytes)
-        self.pool = [packed.clone() for _ in range(self.copies)]
-        self.xs = [c.x().torch("cuda") for c in self.cases]
-        self.ys = [torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda") for c in self.cases]
-        self.ws = torch.tensor([c0.weight_scale], dtype=torch.float32, device="cuda")
-        self.launches_per_step = len(self.cases)
-        self.units_per_step = self.wbytes * len(self.cases)
-        self.alg_bytes_per_launch = self.wbytes
-        self.config = {
-            "workload": "bitlinear ternary decode GEMV: x bf16 [M,4096] ~N(0,1), M in {1,8}; packed uint8 "
-                        "[1024,4096] (codes uniform {0,1,2}, 4 per byte along N); weight_scale 0.5, multiply and "
-                        "divide modes; no bias; y bf16 [M,4096]",
-            "layers_per_step": len(self.cases), "K": self.K, "N": self.N, "M": [c.M for c in self.cases],
-            "weight_bytes_per_layer": self.wbytes,
-            "x_plus_y_bytes_per_step": int(sum(c.M * (c.K + c.N) * 2 for c in self.cases)),
-            "l2": f"inputs larger than L2: weights rotate over {self.copies} device copies "
-                  f"({self.copies * self.wbytes / 1e6:.0f} MB > {l2_bytes / 1e6:.0f} MB L2)",
-        }
-
-    def step(self, i: int):
-        for c, case in enumerate(self.cases):
-            w = self.pool[(i * len(self.cases) + c) % self.copies]
-            self.ql.bitlinear_matmul(self.xs[c], w, case.N, self.ws, case.invert, out=self.ys[c])
-
-    # end-to-end: host x in, host y out, every step
-    def e2e_prepare(self):
-        self.hx = [x.cpu().pin_memory() for x in self.xs]
-        self.hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in self.ys]
-        self.h2d = sum(t.numel() * t.element_size() for t in self.hx)
-        self.d2h = sum(t.numel() * t.element_size() for t in self.hy)
-
-    def e2e_step(self, i: int):
-        for c in range(len(self.cases)):
-            self.xs[c].copy_(self.hx[c], non_blocking=True)
-        self.step(i)
-        for c in range(len(self.cases)):
-            self.hy[c].copy_(self.ys[c], non_blocking=True)
-
-    # the oracle on the host cores
-    def cpu_step(self):
-        import oracle
-        P = self.cases[0].packed()
-        done = 0
-        for case in self.cases:
-            x = case.x().vals
-            oracle.bitlinear(x, P, case.N, case.weight_scale, case.invert)
-            done += self.wbytes
-        return done
-
-
-class AffineDecodeSuite:
-    """Each MLX-affine decode layer of the Llama-7B-shaped set, timed alone."""
-
-    def __init__(self, l2_bytes: int):
-        from bit_quantized_linear_qmm_b200 import qlin
-        self.ql = qlin
-        self.l2 = l2_bytes
-
-    def run(self, steps: int):
-        out = []
-        for case in synth.AFFINE_DECODE:
-            w = case.weight()
-            wd = torch.from_numpy(w).cuda()
-            codes, s, b = self.ql.quantize(wd, case.bits, case.group_size, torch.bfloat16)
-            del wd
-            wbytes = codes.numel() * 4 + s.numel() * 2 + b.numel() * 2
-            copies = _rotation_copies(wbytes, self.l2)
-            pool = [(codes.clone(), s.clone(), b.clone()) for _ in range(copies)]
-            x = case.x().torch("cuda")
-            bias = case.layer_bias().torch("cuda")
-            y = torch.empty((case.M, case.N), dtype=torch.bfloat16, device="cuda")
-
-            def step(i, pool=pool, x=x, bias=bias, y=y, case=case, copies=copies):
-                c, sc, bi = pool[i % copies]
-                self.ql.matmul(x, c, sc, bi, case.bits, case.group_size, bias, out=y)
-            ms = time_steps(step, steps, 5)
-            gbs = wbytes / (ms * 1e-3) / 1e9
-            out.append({"case": case.name, "weight_bytes": int(wbytes), "us": round(ms * 1e3, 3),
-                        "GB/s": round(gbs, 1)})
-            del pool
-            torch.cuda.empty_cache()
-        return out
-
-
-WORKLOADS = {"bitlinear_decode": BitlinearDecode}
-
-
 # ---------------------------------------------------------------- timing
 
 def _graphs(step_fn, steps: int, per_graph: int):
@@ -295,22 +191,300 @@ def time_steps(step_fn, steps: int, warmup: int, per_graph: int = 200, soak_s: f
     return ms / steps
 
 
-# ---------------------------------------------------------------- main
+def _copies(bytes_per_copy: int, l2_bytes: int, minimum: int = 2) -> int:
+    """Copies whose total is at least twice the L2 size."""
+    return max(minimum, int(math.ceil(2 * l2_bytes / max(1, bytes_per_copy))))
 
-def cpu_baseline(workload, budget_s: float = 12.0):
+
+# ---------------------------------------------------------------- headline workload
+
+class BitlinearDecode:
+    """BitLinear ternary decode GEMV: x bf16 [M, 4096], packed uint8 [1024, 4096],
+    M in {1, 8}, weight_scale 0.5, multiply and divide modes; no bias."""
+    key = "bitlinear_gemv_kernel"
+    unit = "GB/s"
+    bound = "hbm"
+
+    def __init__(self, l2_bytes: int):
+        from bit_quantized_linear_qmm_b200 import qlin
+        self.ql = qlin
+        self.cases = synth.BITLINEAR_DECODE
+        c0 = self.cases[0]
+        self.K, self.N = c0.K, c0.N
+        self.wbytes = self.N // 4 * self.K
+        packed = torch.from_numpy(c0.packed()).cuda()
+        self.copies = _copies(self.wbytes, l2_bytes, 8)
+        self.pool = [packed.clone() for _ in range(self.copies)]
+        self.xs = [c.x().torch("cuda") for c in self.cases]
+        self.ys = [torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda") for c in self.cases]
+        self.ws = torch.tensor([c0.weight_scale], dtype=torch.float32, device="cuda")
+        self.launches_per_step = len(self.cases)
+        self.units_per_step = self.wbytes * len(self.cases)
+        self.alg_bytes_per_launch = self.wbytes
+        self.config = {
+            "workload": "bitlinear ternary decode GEMV: x bf16 [M,4096] ~N(0,1), M in {1,8}; packed uint8 "
+                        "[1024,4096] (codes uniform {0,1,2}, 4 per byte along N); weight_scale 0.5, multiply and "
+                        "divide modes; no bias; y bf16 [M,4096]",
+            "layers_per_step": len(self.cases), "K": self.K, "N": self.N, "M": [c.M for c in self.cases],
+            "weight_bytes_per_layer": self.wbytes,
+            "x_plus_y_bytes_per_step": int(sum(c.M * (c.K + c.N) * 2 for c in self.cases)),
+            "l2": f"inputs larger than L2: weights rotate over {self.copies} device copies "
+                  f"({self.copies * self.wbytes / 1e6:.0f} MB > {l2_bytes / 1e6:.0f} MB L2)",
+        }
+
+    def step(self, i: int):
+        for c, case in enumerate(self.cases):
+            w = self.pool[(i * len(self.cases) + c) % self.copies]
+            self.ql.bitlinear_matmul(self.xs[c], w, case.N, self.ws, case.invert, out=self.ys[c])
+
+    def e2e_prepare(self):
+        self.hx = [x.cpu().pin_memory() for x in self.xs]
+        self.hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in self.ys]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.hx)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.hy)
+
+    def e2e_step(self, i: int):
+        for c in range(len(self.cases)):
+            self.xs[c].copy_(self.hx[c], non_blocking=True)
+        self.step(i)
+        for c in range(len(self.cases)):
+            self.hy[c].copy_(self.ys[c], non_blocking=True)
+
+
+def cpu_bitlinear_step():
+    """One step of the headline workload on the host cores with the oracle; returns weight bytes."""
+    import oracle
+    cases = synth.BITLINEAR_DECODE
+    P = cases[0].packed()
+    done = 0
+    for case in cases:
+        oracle.bitlinear(case.x().vals, P, case.N, case.weight_scale, case.invert)
+        done += case.N // 4 * case.K
+    return done
+
+
+def cpu_baseline(budget_s: float = 12.0):
     import oracle
     oracle.build()
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     t0 = time.perf_counter()
-    units = workload.cpu_step()  # one full step at least
+    units = cpu_bitlinear_step()
     steps = 1
     while time.perf_counter() - t0 < budget_s * 0.5:
-        units += workload.cpu_step()
+        units += cpu_bitlinear_step()
         steps += 1
     dt = time.perf_counter() - t0
-    return {"value": round(units / dt / 1e9, 3), "unit": workload.unit, "cores": threads, "kind": "oracle",
-            "sample": f"{steps} full step(s) of the workload on the host cores ({dt:.1f} s)"}
+    return {"value": round(units / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{steps} full step(s) of the workload (4 BitLinear layers) on the host cores, {dt:.1f} s"}
 
+
+# ---------------------------------------------------------------- suite
+
+def _entry(name, us, units, unit, bound, peak, note=None):
+    val = units / (us * 1e-6) / (1e9 if unit == "GB/s" else 1e12)
+    e = {"case": name, "us": round(us, 3), "value": round(val, 1), "unit": unit, "bound": bound,
+         "frac": round(val / peak, 4), "peak": peak}
+    if note:
+        e["note"] = note
+    return e
+
+
+def suite(l2: int, peaks: dict, int8_peak: float):
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    hbm = float(peaks["hbm_gbs"])
+    bf16 = float(peaks["bf16_tflops"])
+    out = []
+    dev = "cuda"
+
+    # --- MLX-affine layer, small (fp32)
+    c = synth.AFFINE_SMALL
+    w = torch.from_numpy(c.weight()).to(dev)
+    codes, s, b = ql.quantize(w, 4, 64, torch.float32)
+    x = c.x().torch(dev)
+    bias = c.layer_bias().torch(dev)
+    y = torch.empty((c.M, c.N), dtype=torch.float32, device=dev)
+    wb = codes.numel() * 4 + s.numel() * 8
+    us = time_steps(lambda i: ql.matmul(x, codes, s, b, 4, 64, bias, out=y), 200, 5) * 1e3
+    out.append(_entry(c.name, us, wb, "GB/s", "hbm", hbm, "launch-bound (0.16 MB)"))
+
+    # --- BitLinear, each case alone
+    P = torch.from_numpy(synth.BITLINEAR_DECODE[0].packed()).to(dev)
+    pool = [P.clone() for _ in range(_copies(P.numel(), l2, 8))]
+    ws = torch.tensor([0.5], device=dev)
+    for c in synth.BITLINEAR_DECODE:
+        x = c.x().torch(dev)
+        y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        us = time_steps(lambda i: ql.bitlinear_matmul(x, pool[i % len(pool)], c.N, ws, c.invert, out=y), 400, 5) * 1e3
+        out.append(_entry(c.name, us, P.numel(), "GB/s", "hbm", hbm))
+    del pool
+
+    # --- MLX-affine decode
+    for c in synth.AFFINE_DECODE:
+        wd = torch.from_numpy(c.weight()).to(dev)
+        codes, s, b = ql.quantize(wd, c.bits, c.group_size, torch.bfloat16)
+        del wd
+        wb = codes.numel() * 4 + s.numel() * 2 + b.numel() * 2
+        pool = [(codes.clone(), s.clone(), b.clone()) for _ in range(_copies(wb, l2, 8))]
+        x = c.x().torch(dev)
+        bias = c.layer_bias().torch(dev)
+        y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+
+        def st(i, pool=pool, x=x, bias=bias, y=y, c=c):
+            cc, ss, bb = pool[i % len(pool)]
+            ql.matmul(x, cc, ss, bb, c.bits, c.group_size, bias, out=y)
+        us = time_steps(st, 200, 5) * 1e3
+        out.append(_entry(c.name, us, wb, "GB/s", "hbm", hbm))
+        del pool
+        torch.cuda.empty_cache()
+
+    # --- MLX-affine prefill (tcgen05 bf16)
+    c = synth.AFFINE_PREFILL
+    wd = torch.from_numpy(c.weight()).to(dev)
+    codes, s, b = ql.quantize(wd, 4, 64, torch.bfloat16)
+    us_q = time_steps(lambda i: ql.quantize(wd, 4, 64, torch.bfloat16), 10, 2) * 1e3
+    qbytes = wd.numel() * 4 + codes.numel() * 4 + s.numel() * 4
+    out.append(_entry("quantize_f32_b4_g64_N14336_K4096", us_q, qbytes, "GB/s", "hbm", hbm,
+                      "reads fp32 W, writes codes + bf16 params"))
+    wdq = torch.empty((c.N, c.K), dtype=torch.bfloat16, device=dev)
+    us_d = time_steps(lambda i: ql.dequantize(codes, s, b, c.K, 4, 64, torch.bfloat16), 10, 2) * 1e3
+    dbytes = codes.numel() * 4 + s.numel() * 4 + wdq.numel() * 2
+    out.append(_entry("dequantize_b4_g64_N14336_K4096_bf16", us_d, dbytes, "GB/s", "hbm", hbm))
+    del wd, wdq
+    x = c.x().torch(dev)
+    bias = c.layer_bias().torch(dev)
+    y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+    pool = [(codes.clone(), s.clone(), b.clone()) for _ in range(3)]
+
+    def stp(i):
+        cc, ss, bb = pool[i % 3]
+        ql.matmul(x, cc, ss, bb, 4, 64, bias, out=y)
+    us = time_steps(stp, 20, 3) * 1e3
+    flops = 2.0 * c.M * c.N * c.K
+    out.append(_entry(c.name, us, flops, "TFLOP/s", "tensor", bf16, "bf16 tcgen05, fp32 accumulate; dequant fused"))
+    del pool, x, y
+    torch.cuda.empty_cache()
+
+    # --- W8A8 / W4A8, K = N = 8192, M in {1, 256, 4096}
+    base = synth.INT_LINEAR[0]
+    wf = torch.from_numpy(base.weight()).to(dev)
+    qw, sw = ql.quantize_int8_rows(wf)
+    P4, s4 = ql.pack_int4_cols(wf.t().contiguous())
+    del wf
+    for c in synth.INT_LINEAR:
+        x = c.x().torch(dev)
+        y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        wsz = ql.workspace_size(ql.QLIN_OP_W8A8, c.M, c.N, c.K)
+        ws_ = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        n8 = 4 if c.M == 1 else 2
+        p8 = [qw.clone() for _ in range(n8)]
+        p4 = [P4.clone() for _ in range(n8)]
+        for name, fn, wbytes in (
+                ("w8a8", lambda i: ql.w8a8_linear(x, p8[i % n8], sw, out=y, workspace=ws_), qw.numel() + 4 * c.N),
+                ("w4a8", lambda i: ql.w4a8_linear(x, p4[i % n8], s4, out=y, workspace=ws_), P4.numel() + 4 * c.N)):
+            us = time_steps(fn, 50 if c.M < 4096 else 10, 3) * 1e3
+            if c.M <= 16:
+                out.append(_entry(f"{name}_{c.name}", us, wbytes, "GB/s", "hbm", hbm,
+                                  "includes the activation-quant kernel"))
+            else:
+                ops = 2.0 * c.M * c.N * c.K
+                roof = min(int8_peak, hbm * 1e9 * ops / (wbytes + c.M * c.K * 3 + c.M * c.N * 2) / 1e12)
+                out.append(_entry(f"{name}_{c.name}", us, ops, "TFLOP/s", "tensor", round(roof, 1),
+                                  "TOPS; includes the activation-quant kernel; peak = min(int8 peak, BW x AI)"))
+        # activation quantiser alone at this M
+        if c.M == 4096:
+            qx = torch.empty((c.M, c.K), dtype=torch.int8, device=dev)
+            us = time_steps(lambda i: ql.quantize_int8_rows(x), 10, 3) * 1e3
+            out.append(_entry("act_quant_M4096_K8192", us, c.M * c.K * 3 + c.M * 4, "GB/s", "hbm", hbm))
+            del qx
+        del p8, p4, ws_, x, y
+        torch.cuda.empty_cache()
+
+    # --- raw int8 GEMM 4096 x 8192 x 8192
+    a8 = torch.randint(-128, 128, (4096, 8192), dtype=torch.int8, device=dev)
+    b8 = torch.randint(-128, 128, (8192, 8192), dtype=torch.int8, device=dev)
+    c32 = torch.empty((4096, 8192), dtype=torch.int32, device=dev)
+    us = time_steps(lambda i: ql.int8_matmul_int32(a8, b8, out=c32), 10, 3) * 1e3
+    out.append(_entry("int8_matmul_int32_M4096_N8192_K8192", us, 2.0 * 4096 * 8192 * 8192, "TFLOP/s", "tensor",
+                      int8_peak, "TOPS"))
+    return out
+
+
+def measure_int8_peak():
+    """torch._int_mm (cuBLASLt) int8 8192^3, best of 10: context for the int8 denominators."""
+    try:
+        a = torch.randint(-128, 128, (8192, 8192), dtype=torch.int8, device="cuda")
+        b = torch.randint(-128, 128, (8192, 8192), dtype=torch.int8, device="cuda").t()
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        best = 1e9
+        for _ in range(10):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(a, b)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return 2.0 * 8192 ** 3 / (best * 1e-3) / 1e12
+    except Exception:  # noqa: BLE001 - context only
+        return None
+
+
+# ---------------------------------------------------------------- profiling entry (for ncu)
+
+def _prof_bitlinear(M):
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    c = synth.BitLinearCase("p", M, 4096, 4096)
+    P = torch.from_numpy(c.packed()).cuda()
+    x = c.x().torch("cuda")
+    ws = torch.tensor([0.5], device="cuda")
+    return lambda: ql.bitlinear_matmul(x, P, 4096, ws, False)
+
+
+def _prof_affine(M, K, N):
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    c = synth.AffineCase("p", M, K, N, 4, 128 if M <= 16 else 64, "bf16", "bf16", True,
+                         outliers=M > 16)
+    codes, s, b = ql.quantize(torch.from_numpy(c.weight()).cuda(), 4, c.group_size, torch.bfloat16)
+    x = c.x().torch("cuda")
+    bias = c.layer_bias().torch("cuda")
+    return lambda: ql.matmul(x, codes, s, b, 4, c.group_size, bias)
+
+
+def _prof_int(kind, M):
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    c = synth.IntCase("p", M, 8192, 8192)
+    wf = torch.from_numpy(c.weight()).cuda()
+    x = c.x().torch("cuda")
+    if kind == "w8a8":
+        qw, sw = ql.quantize_int8_rows(wf)
+        return lambda: ql.w8a8_linear(x, qw, sw)
+    P, s4 = ql.pack_int4_cols(wf.t().contiguous())
+    return lambda: ql.w4a8_linear(x, P, s4)
+
+
+PROFILE_CASES = {
+    "bitlinear_m1": lambda: _prof_bitlinear(1),
+    "bitlinear_m8": lambda: _prof_bitlinear(8),
+    "affine_decode_m1": lambda: _prof_affine(1, 4096, 4096),
+    "affine_prefill_m512": lambda: _prof_affine(512, 4096, 14336),
+    "w8a8_m4096": lambda: _prof_int("w8a8", 4096),
+    "w4a8_m4096": lambda: _prof_int("w4a8", 4096),
+    "w8a8_m1": lambda: _prof_int("w8a8", 1),
+}
+
+
+def profile_case(name):
+    fn = PROFILE_CASES[name]()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for i in range(4):
+        flush.fill_(i)  # cold L2 for each launch
+        fn()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- main
 
 def main():
     ap = argparse.ArgumentParser()
@@ -318,11 +492,13 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="qlin", choices=["qlin", "reference"])
-    ap.add_argument("--workload", default="bitlinear_decode", choices=sorted(WORKLOADS))
     ap.add_argument("--no-suite", action="store_true")
+    ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
+                    help="run a few launches of one case (for ncu), print nothing else")
     args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
+    args.warmup = max(args.warmup, 3)
+    if args.profile:
+        return profile_case(args.profile)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -332,8 +508,9 @@ def main():
         return main_reference(args, world, rank)
 
     from bit_quantized_linear_qmm_b200 import build
-    if rank == 0 and not os.path.exists(os.path.join(ROOT, "bit_quantized_linear_qmm_b200", "libqlin.so")):
-        build.build()
+    if not os.path.exists(os.path.join(ROOT, "bit_quantized_linear_qmm_b200", "libqlin.so")):
+        if rank == 0:
+            build.build()
     torch.cuda.set_device(local_rank)
     dist = None
     if world > 1:
@@ -347,7 +524,7 @@ def main():
 
     peaks = load_peaks()
     l2 = torch.cuda.get_device_properties(local_rank).L2_cache_size
-    wl = WORKLOADS[args.workload](l2)
+    wl = BitlinearDecode(l2)
 
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -366,9 +543,8 @@ def main():
     peak = float(peaks["hbm_gbs"])
     roofline = {"bound": wl.bound, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(wl.key),
-                "kernel": wl.key, "peak_source": f"{peaks['source']} hbm_gbs"}
+                "kernel": wl.key, "peak_source": f"{peaks['source']} hbm_gbs (of measured)"}
 
-    # end to end through the public API: host x in, host y out, every step
     wl.e2e_prepare()
     ms_e2e = time_steps(wl.e2e_step, max(1, min(args.steps, 1000)), args.warmup, barrier=barrier)
     t = torch.tensor([ms_e2e], dtype=torch.float64, device="cuda")
@@ -376,13 +552,16 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     e2e_value = world * wl.units_per_step / (float(t.item()) * 1e-3) / 1e9
 
-    suite = None
+    suite_out = None
+    int8_meas = None
     if not args.no_suite:
-        suite = {"affine_decode": AffineDecodeSuite(l2).run(200)}
+        int8_meas = measure_int8_peak()
+        int8_peak = round(float(peaks["bf16_tflops"]) * INT8_OVER_BF16, 1)
+        suite_out = suite(l2, peaks, int8_peak)
 
     cpu = None
     if rank == 0 and world == 1:
-        cpu = cpu_baseline(wl)
+        cpu = cpu_baseline()
 
     if dist is not None:
         dist.barrier()
@@ -398,45 +577,37 @@ def main():
                 "d2h_bytes_per_step": wl.d2h},
         "clocks": clocks, "gpu_launches": wl.launches_per_step * args.steps,
     }
-    if suite is not None:
-        line["suite"] = suite
+    if suite_out is not None:
+        line["suite"] = suite_out
+        line["int8_peak_tops"] = {"used": round(float(peaks["bf16_tflops"]) * INT8_OVER_BF16, 1),
+                                  "rule": "measured bf16 burst x nominal int8/bf16 ratio 2",
+                                  "torch_int_mm_8192_measured": None if int8_meas is None else round(int8_meas, 1)}
     print(json.dumps(line), flush=True)
 
 
 def main_reference(args, world, rank):
-    """The oracle (CPU) on the same workload and metric, on the host cores."""
+    """The oracle (CPU) on the headline workload and metric, on the host cores."""
     if rank != 0:
         return
-    wl_cls = WORKLOADS[args.workload]
     import oracle
     oracle.build()
-
-    class Host:  # CPU-only view of the workload (no device memory)
-        pass
-    h = Host()
-    cases = synth.BITLINEAR_DECODE
-    h.unit = "GB/s"
-    h.wbytes = cases[0].N // 4 * cases[0].K
-    h.cases = cases
-    h.cpu_step = lambda: wl_cls.cpu_step(h)
-    for _ in range(args.warmup):
-        pass
+    steps = max(1, min(args.steps, 5))
+    cpu_bitlinear_step()  # warm the OpenMP pool and the page cache
     t0 = time.perf_counter()
     units = 0
-    for _ in range(args.steps if args.steps <= 5 else 5):
-        units += h.cpu_step()
+    for _ in range(steps):
+        units += cpu_bitlinear_step()
     dt = time.perf_counter() - t0
-    steps_done = args.steps if args.steps <= 5 else 5
     value = units / dt / 1e9
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": h.unit, "n_gpus": world,
-        "steps": steps_done, "warmup": args.warmup, "ms_per_step": round(dt / steps_done * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "bitlinear ternary decode GEMV (same as the CUDA arm), CPU oracle"},
-        "cpu_baseline": {"value": round(value, 3), "unit": h.unit, "cores": threads, "kind": "oracle",
-                         "sample": f"{steps_done} full steps"},
-        "e2e": {"value": round(value, 3), "unit": h.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": 1, "ms_per_step": round(dt / steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "bitlinear ternary decode GEMV (the CUDA arm's workload), CPU oracle"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{steps} full step(s) of the workload (4 BitLinear layers)"},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
