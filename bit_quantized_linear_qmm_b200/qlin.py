@@ -73,6 +73,7 @@ def lib():
         "qlin_int8_matmul_int32": ([P, P, I64, I64, I64, P, P], I),
         "w8a8_linear": ([P, I, I64, I64, P, P, I64, P, P, P, SZ, P], I),
         "w4a8_linear": ([P, I, I64, I64, P, P, I64, P, P, P, SZ, P], I),
+        "w8a8_linear_noalloc": ([P, I, I64, I64, P, P, I64, P, P, P], I),
         "qlin_get_device_status": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -228,6 +229,18 @@ def w4a8_linear(x, packed_w, scale_w, bias=None, out=None, workspace=None):
         workspace = torch.empty(workspace_size(QLIN_OP_W4A8, M, N, K), dtype=torch.uint8, device=x.device)
     _check(lib().w4a8_linear(_ptr(x), _dt(x), M, K, _ptr(packed_w), _ptr(scale_w), N, _ptr(bias), _ptr(out),
                              _ptr(workspace), workspace.numel(), _stream(x.device)), "w4a8_linear")
+    return out
+
+
+def w8a8_linear_noalloc(x, w, scale_w, bias=None, out=None):
+    """w8a8_linear with the activation scratch inside the library (no workspace)."""
+    _cuda(x, w, scale_w, bias)
+    M, K = x.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    _check(lib().w8a8_linear_noalloc(_ptr(x), _dt(x), M, K, _ptr(w), _ptr(scale_w), N, _ptr(bias), _ptr(out),
+                                     _stream(x.device)), "w8a8_linear_noalloc")
     return out
 
 

@@ -196,6 +196,29 @@ qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
                         void* stream);
 
 /*
+ * W8A8 linear without caller memory (no counterpart on the source pages).
+ * Same operation, arguments and results as w8a8_linear, for callers that
+ * cannot give the library device memory: a host that reserved the GPU's
+ * memory for its own pool, a serving loop that allows no allocator calls
+ * after start-up, or a C program with nothing to borrow scratch from.  The
+ * per-token int8 activations and their scales live in an 8 MiB buffer built
+ * into libqlin.so (each GPU that loads the library holds it until exit);
+ * the call itself allocates and frees nothing.
+ *   - Limit: qlin_workspace_size(QLIN_OP_W8A8, M, N, K, 0, 0) must be at most
+ *     8 MiB (M*K rounded up to 256 bytes, plus 4*M rounded up to 256);
+ *     larger problems return QLIN_ERR_WORKSPACE and launch nothing.
+ *   - The buffer's device address is looked up on the first call made with
+ *     a given device current; make that first call before any stream
+ *     capture on that device.
+ *   - All calls share the one buffer and it keeps the last call's contents
+ *     (every call rewrites what it reads, so nothing needs clearing).  Calls
+ *     that may run at the same time on the GPU -- on different streams, or
+ *     from different host threads -- race on it; serialise them.
+ */
+qlin_status w8a8_linear_noalloc(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const int8_t* w,
+                                const float* scale_w, int64_t N, const void* bias, void* y, void* stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the library's device
  * status word: QLIN_ERR_TIMEOUT if a bounded on-device wait in any kernel
  * gave up since the last call, QLIN_ERR_CUDA if the stream holds an error,
