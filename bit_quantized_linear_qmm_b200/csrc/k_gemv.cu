@@ -701,7 +701,268 @@ __global__ void __launch_bounds__(kThreads, 2) bitlinear_gemv_kernel(const __gri
     }
 }
 
+// ---------------------------------------------------------------- BitLinear decode
+
+// A CTA owns 8 packed rows (32 outputs) over the whole of K.  Its 8 warps
+// take 64-k chunks round robin; lane (g, t) of a warp handles, per chunk, the
+// 16 bytes k = 64c + 16t .. +15 of packed row g and the same 16 x values of
+// token g (and g + 8 when M > 8).  Each 32-bit weight word (4 consecutive k)
+// feeds two mma.m16n8k16: fields {0, 2} and {1, 3} as A rows g and g + 8.
+// Its bytes are first reordered (0, 2, 1, 3), so that the bf16 pairs the
+// LOP3 decode yields are consecutive k, like x in memory.
+//
+// Data movement (M <= 8): every thread copies its own 16-byte pieces with
+// cp.async into a private slot of shared memory -- the weights of its first
+// eight chunks before griddepcontrol.wait (under programmatic dependent
+// launch a layer's weight stream overlaps the previous kernel), the x pieces
+// right after it, one commit group per chunk -- and consumes them chunk by
+// chunk behind cp.async.wait_group.  Everything is in flight at once, no
+// block barrier is needed, and lanes touch consecutive 16-byte units (no
+// bank conflicts).  Chunks beyond the eighth are refilled into the slot just
+// consumed.  For 9..16 tokens, x goes through a ring of registers instead.
+//
+// The grid has at least one CTA per SM; the spare ones only pass the
+// dependency wait.  With every kernel holding one CTA on every SM, the next
+// layer's CTAs (two fit per SM) land one per SM as well.
+constexpr int kBlWarps = 8;
+constexpr int kBlThreads = kBlWarps * 32;
+constexpr int kBlRows = 8;     // packed rows per CTA (32 outputs)
+constexpr int kBlChunk = 64;   // k per chunk
+constexpr int kBlRound = 8;    // chunks in flight per warp
+// shared memory of the cp.async path: weights, then x, 16-byte units [slot][unit][thread]
+constexpr int kBlSmemW = kBlRound * kBlThreads * 16;       // 32 KB
+constexpr int kBlSmemX = kBlRound * 2 * kBlThreads * 16;   // 64 KB
+constexpr int kBlSmemAsync = kBlSmemW + kBlSmemX;
+
+struct BitRegParams {
+    const uint8_t* packed;   // [R][K]
+    const __nv_bfloat16* x;  // [M][K]
+    const float* weight_scale;
+    const __nv_bfloat16* bias;
+    __nv_bfloat16* y;  // [M][N]
+    int M, K, N, R;
+    int tiles;  // CTAs with rows to compute
+    int invert;
+    unsigned* status;
+};
+
+// ASYNC: the cp.async shared-memory path (NT == 1); else weights in
+// registers and x through an XD-deep register ring.
+template <int NT, int XD, bool ASYNC>
+__global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __grid_constant__ BitRegParams p)
+{
+    static_assert(kBlRound % XD == 0, "x ring depth must divide the register round");
+    static_assert(!ASYNC || NT == 1, "the shared-memory path holds 8 tokens");
+    __shared__ float red[kBlWarps * 8 * NT * 32];
+    extern __shared__ __align__(16) uint8_t dsm[];  // ASYNC: weight slots, then x slots
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+
+    pdl_launch_dependents();
+    if ((int)blockIdx.x >= p.tiles) {
+        // hold this SM's slot until the previous kernel is done, then leave
+        pdl_wait_prior_grids();
+        return;
+    }
+    const int p0 = blockIdx.x * kBlRows;
+    const int nch = (p.K + kBlChunk - 1) / kBlChunk;
+    const int my = nch > warp ? (nch - 1 - warp) / kBlWarps + 1 : 0;  // chunks of this warp
+    const bool row_ok = p0 + gid < p.R;
+    const uint8_t* wrow = p.packed + (size_t)(row_ok ? p0 + gid : 0) * p.K + 16 * tig;
+    const bool tok_ok = gid < p.M;  // token of this lane (first token tile)
+    const __nv_bfloat16* xrow = p.x + (size_t)(tok_ok ? gid : 0) * p.K + 16 * tig;
+    // ci-th chunk of this warp: c = warp + 8 ci, k = 64 c + 16 tig
+    auto chunk_k = [&](int ci) { return (warp + ci * kBlWarps) * kBlChunk; };
+    auto w_ok = [&](int ci) { return row_ok && ci < my && chunk_k(ci) + 16 * tig < p.K; };
+    auto x_ok = [&](int ci) { return tok_ok && ci < my && chunk_k(ci) + 16 * tig < p.K; };
+    uint4* wslot = reinterpret_cast<uint4*>(dsm) + threadIdx.x;             // + j * kBlThreads
+    uint4* xslot = reinterpret_cast<uint4*>(dsm + kBlSmemW) + threadIdx.x;  // + (2 j + h) * kBlThreads
+
+    auto load_w = [&](uint4& dst, int ci) {
+        if (w_ok(ci))
+            dst = ldg_stream_v4(wrow + chunk_k(ci));
+        else
+            dst = make_uint4(0u, 0u, 0u, 0u);
+    };
+    auto load_x = [&](uint4 (&dst)[NT][2], int ci) {
+        const int k = chunk_k(ci) + 16 * tig;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const int m = 8 * t + gid;
+            if (ci < my && m < p.M && k < p.K) {
+                const __nv_bfloat16* src = p.x + (size_t)m * p.K + k;
+                dst[t][0] = ldg_cg_v4(src);
+                dst[t][1] = ldg_cg_v4(src + 8);
+            } else {
+                dst[t][0] = dst[t][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+
+    uint4 wr[ASYNC ? 1 : kBlRound];
+    uint4 xb[XD][NT][2];
+    if constexpr (ASYNC) {
+#pragma unroll
+        for (int j = 0; j < kBlRound; ++j)
+            if (w_ok(j))
+                cp_async16(wslot + j * kBlThreads, wrow + chunk_k(j));
+        cp_async_commit();
+    } else {
+#pragma unroll
+        for (int j = 0; j < kBlRound; ++j)
+            load_w(wr[j], j);
+    }
+    pdl_wait_prior_grids();  // x, weight_scale and y may belong to the previous kernel
+    if constexpr (ASYNC) {
+#pragma unroll
+        for (int j = 0; j < kBlRound; ++j) {
+            if (x_ok(j)) {
+                cp_async16(xslot + (2 * j) * kBlThreads, xrow + chunk_k(j));
+                cp_async16(xslot + (2 * j + 1) * kBlThreads, xrow + chunk_k(j) + 8);
+            }
+            cp_async_commit();
+        }
+    } else {
+#pragma unroll
+        for (int d = 0; d < XD; ++d)
+            load_x(xb[d], d);
+    }
+    const float ws = *p.weight_scale;
+    const float scale = p.invert ? __fdiv_rn(1.0f, ws) : ws;
+
+    // per-field bf16x2 constants {4^-j, -(128 4^-j + 1)}: (128 + 4^j c) -> c - 1, exact
+    constexpr uint32_t kScale0 = 0x3F803F80u, kBias0 = 0xC301C301u;  // j=0: 1, -129
+    constexpr uint32_t kScale1 = 0x3E803E80u, kBias1 = 0xC204C204u;  // j=1: 1/4, -33
+    constexpr uint32_t kScale2 = 0x3D803D80u, kBias2 = 0xC110C110u;  // j=2: 1/16, -9
+    constexpr uint32_t kMagic = 0x43004300u;
+    // with one token tile, two accumulator sets (even / odd steps) keep four
+    // MMA chains in flight per warp
+    constexpr int AS = NT == 1 ? 2 : 1;
+    float a02[AS][NT][4], a13[AS][NT][4];
+#pragma unroll
+    for (int h = 0; h < AS; ++h)
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                a02[h][t][e] = a13[h][t][e] = 0.f;
+
+    auto chunk = [&](const uint4& w4, const uint4 (&xv)[NT][2]) {
+        const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // k = 64c + 16 tig + 4i .. +3
+            const uint32_t w = prmt(wv[i], 0u, 0x3120);  // bytes (k, k+2, k+1, k+3)
+            const uint32_t hw = w >> 8;                 // k+2, k+3 in the low byte of each half
+            uint32_t f02[4], f13[4];
+            f02[0] = bf16x2_fma(lop3_and_or(w, 0x00030003u, kMagic), kScale0, kBias0);        // f0 (k, k+1)
+            f02[1] = bf16x2_fma(lop3_and_or(w, 0x00300030u, kMagic), kScale2, kBias2);        // f2 (k, k+1)
+            f02[2] = bf16x2_fma(lop3_and_or(hw, 0x00030003u, kMagic), kScale0, kBias0);       // f0 (k+2, k+3)
+            f02[3] = bf16x2_fma(lop3_and_or(hw, 0x00300030u, kMagic), kScale2, kBias2);       // f2 (k+2, k+3)
+            f13[0] = bf16x2_fma(lop3_and_or(w, 0x000C000Cu, kMagic), kScale1, kBias1);        // f1 (k, k+1)
+            f13[1] = bf16x2_fma(lop3_and_or(w >> 6, 0x00030003u, kMagic), kScale0, kBias0);   // f3 (k, k+1)
+            f13[2] = bf16x2_fma(lop3_and_or(hw, 0x000C000Cu, kMagic), kScale1, kBias1);       // f1 (k+2, k+3)
+            f13[3] = bf16x2_fma(lop3_and_or(w >> 14, 0x00030003u, kMagic), kScale0, kBias0);  // f3 (k+2, k+3)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const uint4& xh = xv[t][i >> 1];
+                const uint32_t b0 = (i & 1) ? xh.z : xh.x;  // (x_k, x_k+1)
+                const uint32_t b1 = (i & 1) ? xh.w : xh.y;  // (x_k+2, x_k+3)
+                mma_bf16_16816(a02[i % AS][t], f02, b0, b1);
+                mma_bf16_16816(a13[i % AS][t], f13, b0, b1);
+            }
+        }
+    };
+
+    const int rounds = (my + kBlRound - 1) / kBlRound;
+    for (int rd = 0; rd < rounds; ++rd) {
+#pragma unroll
+        for (int j = 0; j < kBlRound; ++j) {
+            const int ci = rd * kBlRound + j;
+            if constexpr (ASYNC) {
+                // groups after this chunk's: the x of the later first-round chunks and one refill per
+                // chunk already done -- always kBlRound - 1
+                cp_async_wait_group<kBlRound - 1>();
+                if (ci < my) {
+                    const uint4 w4 = wslot[j * kBlThreads];
+                    uint4 xv[1][2];
+                    if (x_ok(ci)) {  // x past K (or past M) is zero
+                        xv[0][0] = xslot[(2 * j) * kBlThreads];
+                        xv[0][1] = xslot[(2 * j + 1) * kBlThreads];
+                    } else {
+                        xv[0][0] = xv[0][1] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    chunk(w4, xv);
+                }
+                // refill this slot with chunk ci + 8 (the values above are already in registers)
+                const int cn = ci + kBlRound;
+                if (w_ok(cn))
+                    cp_async16(wslot + j * kBlThreads, wrow + chunk_k(cn));
+                if (x_ok(cn)) {
+                    cp_async16(xslot + (2 * j) * kBlThreads, xrow + chunk_k(cn));
+                    cp_async16(xslot + (2 * j + 1) * kBlThreads, xrow + chunk_k(cn) + 8);
+                }
+                cp_async_commit();
+            } else {
+                if (ci < my)
+                    chunk(wr[j], xb[j % XD]);
+                load_x(xb[j % XD], ci + XD);
+                load_w(wr[j], ci + kBlRound);
+            }
+        }
+    }
+    if constexpr (ASYNC)
+        cp_async_wait_all();  // nothing may still be landing in shared memory at exit
+
+    // sum the 8 warps' partial tiles; v = t * 8 + a * 4 + e (a: fields {0,2} / {1,3})
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            red[((warp * NT + t) * 8 + e) * 32 + lane] = a02[0][t][e] + (AS > 1 ? a02[AS - 1][t][e] : 0.f);
+            red[((warp * NT + t) * 8 + 4 + e) * 32 + lane] = a13[0][t][e] + (AS > 1 ? a13[AS - 1][t][e] : 0.f);
+        }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < NT * 8 * 32; idx += kBlThreads) {
+        const int v = idx >> 5, ln = idx & 31;
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kBlWarps; ++w)
+            sum += red[(w * NT * 8 + v) * 32 + ln];
+        const int t = v >> 3, a = (v >> 2) & 1, e = v & 3;
+        const int pr = p0 + (ln >> 2);
+        const int m = 8 * t + 2 * (ln & 3) + (e & 1);
+        if (pr < p.R && m < p.M) {
+            const int n = pr + (a + 2 * (e >> 1)) * p.R;
+            float out = sum * scale;
+            if (p.bias)
+                out += __bfloat162float(p.bias[n]);
+            p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(out);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- launch helpers
+
+template <typename Kern, typename Params>
+cudaError_t launch_pdl_threads(Kern kern, dim3 grid, int threads, int smem, cudaStream_t st, const Params& prm)
+{
+    if (smem > 0) {  // static + dynamic above 48 KB needs the opt-in
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess)
+            return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, prm);
+}
 
 template <typename Kern, typename Params>
 cudaError_t launch_pdl(Kern kern, dim3 grid, int smem, cudaStream_t st, const Params& prm)
@@ -809,10 +1070,13 @@ cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const D
 cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
     const int R = (int)(a.N / 4);
+    const int tiles = (R + kBlRows - 1) / kBlRows;
+    const dim3 grid((unsigned)(tiles > dev.sm_count ? tiles : dev.sm_count), 1, 1);
     for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
         const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
-        BitParams prm;
-        const void* x = static_cast<const __nv_bfloat16*>(a.x) + m0 * a.K;
+        BitRegParams prm;
+        prm.packed = a.packed;
+        prm.x = static_cast<const __nv_bfloat16*>(a.x) + m0 * a.K;
         prm.weight_scale = a.weight_scale;
         prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
         prm.y = static_cast<__nv_bfloat16*>(a.y) + m0 * a.N;
@@ -820,16 +1084,14 @@ cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const
         prm.K = (int)a.K;
         prm.N = (int)a.N;
         prm.R = R;
+        prm.tiles = tiles;
         prm.invert = a.invert;
         prm.status = dev.status;
-        if (!encode_tmap_2d(&prm.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, (uint64_t)a.K, (uint64_t)R,
-                            (uint64_t)a.K, 128, BitCfg<1>::PROWS) ||
-            !encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)a.K, (uint64_t)mc,
-                            (uint64_t)a.K * 2, 64, (uint32_t)mc))
-            return cudaErrorInvalidValue;
-        const int ctas = (R + BitCfg<1>::PROWS - 1) / BitCfg<1>::PROWS;
-        cudaError_t e = mc <= 8 ? launch_pdl(bitlinear_gemv_kernel<1>, dim3(ctas, 1, 1), BitCfg<1>::SMEM, st, prm)
-                                : launch_pdl(bitlinear_gemv_kernel<2>, dim3(ctas, 1, 1), BitCfg<2>::SMEM, st, prm);
+        cudaError_t e;
+        if (mc <= 8)
+            e = launch_pdl_threads(bitlinear_reg_kernel<1, 1, true>, grid, kBlThreads, kBlSmemAsync, st, prm);
+        else
+            e = launch_pdl_threads(bitlinear_reg_kernel<2, 2, false>, grid, kBlThreads, 0, st, prm);
         if (e != cudaSuccess)
             return e;
     }

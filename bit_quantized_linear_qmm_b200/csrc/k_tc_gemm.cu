@@ -11,65 +11,87 @@
 //              [nuvec-nn QuantizedLinear, forward; cider/ops.py pergroup_linear
 //               docstring, dequantize]
 //
-// One CTA computes a 128 x 128 output tile:
-//   warp 0       TMA producer: A tiles (and B, or the packed B source) into a
-//                shared-memory ring, 128-byte swizzle, mbarrier completion.
-//   warp 1       allocates 128 TMEM columns; one thread issues tcgen05.mma
-//                (M = 128, N = 128, K = 32 int8 / 16 bf16 per instruction) and
-//                tcgen05.commit releases each stage when its MMAs are done.
-//   warps 2..5   epilogue: tcgen05.ld of the fp32/int32 accumulator (each warp
-//                owns 32 TMEM lanes = 32 output rows), scales, bias, stores.
-//   warps 6..13  (W4A8, affine) transform the packed B source into the
-//                K-major swizzled operand layout: nibbles -> int8 (c - 8), or
-//                codes -> bf16(fma(q, scale, bias)) in fp32 (the dequantized
-//                weight, rounded once to bf16), then fence.proxy.async.
+// Persistent, warp-specialised kernel: one CTA per SM walks 128 x BN output
+// tiles (BN = 256, or 128 when there are too few tiles to fill the GPU) in a
+// grouped order: kGroupM M-tiles walk the N-tiles together, so each weight
+// tile is fetched from HBM about once and reused from L2.
+//   warp 0       TMA producer: A tiles and the B source (int8 B, packed int4,
+//                or affine code bytes) into a shared-memory ring, mbarrier
+//                completion (expect-tx).
+//   warp 1       allocates 2 x BN TMEM columns (two accumulators); one thread
+//                issues tcgen05.mma (M = 128, N = BN, K = 32 int8 / 16 bf16 per
+//                instruction); tcgen05.commit frees ring slots and transformed
+//                B buffers when their MMAs are done, and publishes each
+//                finished accumulator to the epilogue.
+//   warps 2..5   epilogue: tcgen05.ld of one accumulator (warp q owns TMEM
+//                lanes 32q .. 32q+31 = 32 output rows) while the MMAs of the
+//                next tile fill the other one; scales, bias, 16-byte stores.
+//   warps 6..    (W4A8, affine) one thread per B row turns the packed source
+//                into the K-major 128-byte-swizzled operand in a 2-deep
+//                buffer: nibbles -> int8 16 (c - 8) (the epilogue shifts the
+//                exact int32 sum back by 4 bits), or codes -> bf16(fma(q,
+//                scale, bias)) computed in fp32 (the dequantized weight,
+//                rounded once to bf16); the group parameters of a stage are
+//                loaded two stages ahead.  fence.proxy.async publishes the
+//                operand to the tensor core.
 // Every mbarrier wait is bounded; on expiry the kernel records the timeout,
-// skips the remaining work, and always frees its TMEM.
+// every role stops, the MMA thread waits for its MMAs in flight, and TMEM is
+// always freed.
 #include "qlin_common.cuh"
 
 namespace qlin {
 namespace {
 
-constexpr int kBM = 128;      // output rows (tokens) per CTA
-constexpr int kBN = 128;      // output columns (features) per CTA
-constexpr int kTmemCols = 128;
+constexpr int kBM = 128;    // output rows (tokens) per tile
+constexpr int kGroupM = 8;  // M-tiles that walk the N dimension together
+constexpr int kEpiWarps = 4;
+constexpr int kSmemBudget = 200 * 1024;
 
 enum BSource { B_TMA_I8 = 0, B_W4 = 1, B_AFFINE4 = 2 };
 enum Epi { E_I32 = 0, E_SCALED = 1, E_BIAS = 2 };
 
 __host__ __device__ constexpr int rup(int a, int b) { return (a + b - 1) / b * b; }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
-template <int BSRC>
+template <int BSRC, int BN>
 struct TcCfg {
     static constexpr bool I8 = BSRC != B_AFFINE4;          // kind::i8 (s32) or kind::f16 (bf16 -> f32)
     static constexpr int KE = I8 ? 128 : 64;                // K elements per stage (128 bytes of A)
+    static constexpr int XW = BSRC == B_TMA_I8 ? 0 : BN / 32;  // transform warps: one B row per thread
     static constexpr int A_BYTES = kBM * 128;
-    static constexpr int B_BYTES = kBN * 128;
-    static constexpr int RAW_BYTES = BSRC == B_W4 ? (KE / 2) * kBN : (BSRC == B_AFFINE4 ? kBN * (KE / 2) : 0);
-    static constexpr int STAGE = rup(A_BYTES + B_BYTES + RAW_BYTES, 1024);
-    static constexpr int NS = BSRC == B_TMA_I8 ? 6 : 5;
-    static constexpr int XW = BSRC == B_TMA_I8 ? 0 : 8;     // transform warps
-    static constexpr int THREADS = (6 + XW) * 32;
+    static constexpr int B_BYTES = BN * 128;                // one K-major swizzled B operand
+    static constexpr int RAW_BYTES = BSRC == B_W4 ? (KE / 2) * BN : (BSRC == B_AFFINE4 ? BN * (KE / 2) : B_BYTES);
+    static constexpr int SLOT = rup(A_BYTES + RAW_BYTES, 1024);
+    static constexpr int BRING = XW > 0 ? 2 * B_BYTES : 0;  // transformed B, 2-deep
+    static constexpr int NS = cmin(8, (kSmemBudget - BRING) / SLOT);
+    static constexpr int THREADS = (2 + kEpiWarps + XW) * 32;
+    static constexpr int TMEM_COLS = 2 * BN;
     static constexpr uint32_t IDESC =
         (I8 ? (2u << 4) : (1u << 4)) |                      // D: s32 / f32
         (1u << 7) | (1u << 10) |                            // A, B: s8 / bf16 (signed)
-        ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);  // K-major A and B
+        ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);  // K-major A and B
     struct Bars {
         uint64_t full[NS];
-        uint64_t bready[NS];
         uint64_t empty[NS];
-        uint64_t accf;
+        uint64_t bfull[2];
+        uint64_t bempty[2];
+        uint64_t acc_full[2];
+        uint64_t acc_empty[2];
+        uint64_t mma_done;
         uint32_t tmem;
         int abort_flag;
     };
-    static constexpr int SMEM = NS * STAGE + (int)sizeof(Bars) + 1024;
+    static constexpr int SMEM = NS * SLOT + BRING + (int)sizeof(Bars) + 1024;
+    static_assert(NS >= 2, "ring too shallow");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 struct TcParams {
     CUtensorMap tm_a;  // A [M][K], box {128 B, 128 rows}, 128-byte swizzle
-    CUtensorMap tm_b;  // int8 B [N][K] (box {128 B, 128 rows}, swizzled) | packed int4 [K/2][N]
-                       // (box {128 B, 64 rows}) | affine code bytes [N][K/2] (box {32 B, 128 rows})
+    CUtensorMap tm_b;  // int8 B [N][K] (box {128 B, BN rows}, swizzled) | packed int4 [K/2][N]
+                       // (box {BN B, 64 rows}) | affine code bytes [N][K/2] (box {32 B, BN rows})
     int M, N, K;
+    int tiles_m, tiles_n;
     void* out;
     const float* s_x;
     const float* s_w;
@@ -77,6 +99,7 @@ struct TcParams {
     const __nv_bfloat16* scales;
     const __nv_bfloat16* biases;
     int g;
+    int vec_sw, vec_bias, vec_out;  // 16-byte alignment of s_w, bias and out
     unsigned* status;
 };
 
@@ -92,34 +115,56 @@ QLIN_DEV uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int BSRC, int EPI>
-__global__ void __launch_bounds__(TcCfg<BSRC>::THREADS, 1) tc_gemm_kernel(const __grid_constant__ TcParams p)
+// Grouped tile order: kGroupM consecutive M-tiles walk the N-tiles together.
+QLIN_DEV void tile_coords(int t, int tiles_m, int tiles_n, int& mt, int& nt)
 {
-    using Cfg = TcCfg<BSRC>;
+    const int per_group = kGroupM * tiles_n;
+    const int grp = t / per_group;
+    const int first_m = grp * kGroupM;
+    const int gm = min(kGroupM, tiles_m - first_m);
+    const int r = t - grp * per_group;
+    mt = first_m + r % gm;
+    nt = r / gm;
+}
+
+QLIN_DEV bool aborted(int* flag) { return *reinterpret_cast<volatile int*>(flag) != 0; }
+
+template <int BSRC, int EPI, int BN>
+__global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(const __grid_constant__ TcParams p)
+{
+    using Cfg = TcCfg<BSRC, BN>;
     using Bars = typename Cfg::Bars;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars& bars = *reinterpret_cast<Bars*>(smem + Cfg::NS * Cfg::STAGE);
-    auto A = [&](int s) { return smem + s * Cfg::STAGE; };
-    auto B = [&](int s) { return smem + s * Cfg::STAGE + Cfg::A_BYTES; };
-    auto RAW = [&](int s) { return smem + s * Cfg::STAGE + Cfg::A_BYTES + Cfg::B_BYTES; };
+    Bars& bars = *reinterpret_cast<Bars*>(smem + Cfg::NS * Cfg::SLOT + Cfg::BRING);
+    auto A = [&](int s) { return smem + s * Cfg::SLOT; };
+    auto RAW = [&](int s) { return smem + s * Cfg::SLOT + Cfg::A_BYTES; };  // B itself for int8 B
+    auto BT = [&](int b) { return smem + Cfg::NS * Cfg::SLOT + b * Cfg::B_BYTES; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
     const int nk = (p.K + Cfg::KE - 1) / Cfg::KE;
+    const int tiles = p.tiles_m * p.tiles_n;
+    // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
+    const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = my_tiles * nk;  // ring stages this CTA runs
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::NS; ++s) {
             mbar_init(&bars.full[s], 1);
-            mbar_init(&bars.bready[s], Cfg::XW > 0 ? Cfg::XW : 1);
             mbar_init(&bars.empty[s], 1);
         }
-        mbar_init(&bars.accf, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.bfull[b], Cfg::XW > 0 ? Cfg::XW : 1);
+            mbar_init(&bars.bempty[b], 1);
+            mbar_init(&bars.acc_full[b], 1);
+            mbar_init(&bars.acc_empty[b], kEpiWarps);
+        }
+        mbar_init(&bars.mma_done, 1);
         bars.abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1)
-        tmem_alloc(&bars.tmem, kTmemCols);
+        tmem_alloc(&bars.tmem, Cfg::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -130,187 +175,339 @@ __global__ void __launch_bounds__(TcCfg<BSRC>::THREADS, 1) tc_gemm_kernel(const 
         if (lane == 0) {
             pdl_launch_dependents();
             pdl_wait_prior_grids();  // A (activations) may come from the previous kernel
-            int issued = 0;
-            for (int it = 0; it < nk; ++it) {
-                const int slot = it % Cfg::NS;
-                if (it >= Cfg::NS &&
-                    (!mbar_wait_bounded(&bars.empty[slot], ((it / Cfg::NS) & 1) ^ 1, p.status) ||
-                     *reinterpret_cast<volatile int*>(&bars.abort_flag))) {
-                    bars.abort_flag = 1;
-                    break;
+            int it = 0;
+            for (int ti = 0; ti < my_tiles && !aborted(&bars.abort_flag); ++ti) {
+                int mt, nt;
+                tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
+                int kb = 0;
+                for (; kb < nk; ++kb, ++it) {
+                    const int slot = it % Cfg::NS;
+                    if (it >= Cfg::NS && !mbar_wait_bounded(&bars.empty[slot], ((it / Cfg::NS) & 1) ^ 1, p.status)) {
+                        bars.abort_flag = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars.full[slot], Cfg::A_BYTES + Cfg::RAW_BYTES);
+                    tma_load_2d(A(slot), &p.tm_a, kb * Cfg::KE, mt * kBM, &bars.full[slot]);
+                    if constexpr (BSRC == B_TMA_I8)
+                        tma_load_2d(RAW(slot), &p.tm_b, kb * 128, nt * BN, &bars.full[slot]);
+                    else if constexpr (BSRC == B_W4)
+                        tma_load_2d(RAW(slot), &p.tm_b, nt * BN, kb * (Cfg::KE / 2), &bars.full[slot]);
+                    else
+                        tma_load_2d(RAW(slot), &p.tm_b, kb * (Cfg::KE / 2), nt * BN, &bars.full[slot]);
                 }
-                mbar_arrive_expect_tx(&bars.full[slot],
-                                      Cfg::A_BYTES + (BSRC == B_TMA_I8 ? Cfg::B_BYTES : Cfg::RAW_BYTES));
-                tma_load_2d(A(slot), &p.tm_a, it * Cfg::KE, m0, &bars.full[slot]);
-                if constexpr (BSRC == B_TMA_I8)
-                    tma_load_2d(B(slot), &p.tm_b, it * 128, n0, &bars.full[slot]);
-                else if constexpr (BSRC == B_W4)
-                    tma_load_2d(RAW(slot), &p.tm_b, n0, it * (Cfg::KE / 2), &bars.full[slot]);
-                else
-                    tma_load_2d(RAW(slot), &p.tm_b, it * (Cfg::KE / 2), n0, &bars.full[slot]);
-                ++issued;
+                if (kb < nk)
+                    break;
             }
-            for (int it = issued - Cfg::NS < 0 ? 0 : issued - Cfg::NS; it < issued; ++it)
-                mbar_wait_bounded(&bars.full[it % Cfg::NS], (it / Cfg::NS) & 1, p.status);
+            // drain: no copy may still be landing in this CTA's shared memory at exit
+            for (int j = it - Cfg::NS < 0 ? 0 : it - Cfg::NS; j < it; ++j)
+                mbar_wait_bounded(&bars.full[j % Cfg::NS], (j / Cfg::NS) & 1, p.status);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            int it = 0;
             bool ok = true;
-            for (int it = 0; it < nk && ok; ++it) {
-                const int slot = it % Cfg::NS;
-                const unsigned par = (it / Cfg::NS) & 1;
-                ok = mbar_wait_bounded(&bars.full[slot], par, p.status);
-                if (ok && Cfg::XW > 0)
-                    ok = mbar_wait_bounded(&bars.bready[slot], par, p.status);
-                if (!ok) {
-                    bars.abort_flag = 1;
-                    break;
-                }
+            for (int ti = 0; ti < my_tiles && ok; ++ti) {
+                const int buf = ti & 1;
+                ok = mbar_wait_bounded(&bars.acc_empty[buf], ((ti >> 1) & 1) ^ 1, p.status);
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(A(slot)), b0 = smem_u32(B(slot));
+                const uint32_t acc = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < nk && ok; ++kb, ++it) {
+                    const int slot = it % Cfg::NS;
+                    ok = mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status);
+                    if (ok && Cfg::XW > 0)
+                        ok = mbar_wait_bounded(&bars.bfull[it & 1], (it >> 1) & 1, p.status);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(A(slot));
+                    const uint32_t b0 = smem_u32(Cfg::XW > 0 ? BT(it & 1) : RAW(slot));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc_mma<Cfg::I8>(tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), Cfg::IDESC,
-                                    (it | kk) != 0 ? 1u : 0u);
-                tc_commit(&bars.empty[slot]);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma<Cfg::I8>(acc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
+                                        Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit(&bars.empty[slot]);
+                    if (Cfg::XW > 0)
+                        tc_commit(&bars.bempty[it & 1]);
+                }
+                tc_commit(&bars.acc_full[buf]);  // fires when this tile's MMAs are done
             }
-            tc_commit(&bars.accf);  // also fires when nothing was issued
+            if (!ok)
+                bars.abort_flag = 1;
+            // every MMA issued has completed before TMEM is released
+            tc_commit(&bars.mma_done);
+            mbar_wait_bounded(&bars.mma_done, 0, p.status);
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp < 2 + kEpiWarps) {
         // ------------------------------------------------------------ epilogue
-        const bool ok = mbar_wait_bounded(&bars.accf, 0, p.status);
-        tc_fence_after();
-        pdl_wait_prior_grids();  // scales / bias / out may be touched by the previous kernel
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int row = m0 + 32 * q + lane;
-        float sx = 0.f;
-        if constexpr (EPI == E_SCALED)
-            sx = (row < p.M) ? p.s_x[row] : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * 16), r);
-            const int n = n0 + c * 16;
-            if (!ok || row >= p.M || n >= p.N)
-                continue;
-            // vector stores need the row pitch aligned: N % 4 (int32) / N % 8 (bf16)
-            const bool full16 = n + 16 <= p.N && (p.N % (EPI == E_I32 ? 4 : 8)) == 0;
-            if constexpr (EPI == E_I32) {
-                int32_t* o = static_cast<int32_t*>(p.out) + (size_t)row * p.N + n;
-                if (full16) {
-#pragma unroll
-                    for (int j = 0; j < 16; j += 4)
-                        *reinterpret_cast<uint4*>(o + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
-                } else {
-                    for (int j = 0; j < 16 && n + j < p.N; ++j)
-                        o[j] = (int32_t)r[j];
-                }
-            } else {
-                float v[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int nj = n + j < p.N ? n + j : p.N - 1;
-                    float a;
-                    if constexpr (EPI == E_SCALED)
-                        a = fmaf((float)(int32_t)r[j], sx * __ldg(p.s_w + nj), 0.f);
-                    else
-                        a = __uint_as_float(r[j]);
-                    if (p.bias)
-                        a += __bfloat162float(p.bias[nj]);
-                    v[j] = a;
-                }
-                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + n;
-                if (full16) {
-                    *reinterpret_cast<uint4*>(o) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-                    *reinterpret_cast<uint4*>(o + 8) =
-                        make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                   pack_bf16x2(v[14], v[15]));
-                } else {
-                    for (int j = 0; j < 16 && n + j < p.N; ++j)
-                        o[j] = __float2bfloat16_rn(v[j]);
-                }
-            }
-        }
-    } else if constexpr (Cfg::XW > 0) {
-        // ------------------------------------------------------------ B transform
-        const int tt = threadIdx.x - 6 * 32;  // 0 .. 255
-        const int r = tt & (kBN - 1);         // operand row (output column n0 + r)
-        const int half = tt >> 7;             // which 64 bytes of the 128-byte K slice
-        const int ng = p.K / (p.g > 0 ? p.g : 1);
-        const int nrow = min(n0 + r, p.N - 1);
-        pdl_wait_prior_grids();  // the packed weights' parameters may come from the previous kernel
-        for (int it = 0; it < nk; ++it) {
-            const int slot = it % Cfg::NS;
-            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status)) {
+        pdl_wait_prior_grids();  // scales / bias / out may be touched by the previous kernel
+        for (int ti = 0; ti < my_tiles; ++ti) {
+            const int buf = ti & 1;
+            if (!mbar_wait_bounded(&bars.acc_full[buf], (ti >> 1) & 1, p.status) || aborted(&bars.abort_flag)) {
                 bars.abort_flag = 1;
                 break;
             }
-            uint8_t* dst = B(slot);
-            if constexpr (BSRC == B_W4) {
-                // raw[i][n]: k-pair row i (k = 2i high nibble, 2i+1 low), column n; 64 rows x 128 bytes
-                const uint8_t* raw = RAW(slot);
+            tc_fence_after();
+            int mt, nt;
+            tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
+            const int row = mt * kBM + 32 * q + lane;
+            const bool row_ok = row < p.M;
+            float sx = 0.f;
+            if constexpr (EPI == E_SCALED)
+                sx = row_ok ? p.s_x[row] : 0.f;
+            const uint32_t acc = tmem + (uint32_t)(buf * BN) + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+            for (int c = 0; c < BN / 16; ++c) {
+                const int n = nt * BN + c * 16;
+                // 16 whole columns with 16-byte aligned rows: vector loads and stores
+                const bool full16 = n + 16 <= p.N && p.vec_out && (p.N % (EPI == E_I32 ? 4 : 8)) == 0;
+                float sw[16], bb[16];
+                if constexpr (EPI != E_I32) {
+                    // column constants first, so their latency overlaps the TMEM load
+                    if (n < p.N) {
+                        if (full16 && EPI == E_SCALED && p.vec_sw) {
+                            const float4* s4 = reinterpret_cast<const float4*>(p.s_w + n);
 #pragma unroll
-                for (int u = 4 * half; u < 4 * half + 4; ++u) {  // 16-byte unit: k = 16u .. 16u+15
-                    uint32_t wd[4];
+                            for (int j4 = 0; j4 < 4; ++j4) {
+                                const float4 v = __ldg(s4 + j4);
+                                sw[4 * j4] = v.x;
+                                sw[4 * j4 + 1] = v.y;
+                                sw[4 * j4 + 2] = v.z;
+                                sw[4 * j4 + 3] = v.w;
+                            }
+                        } else {
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const uint32_t b0 = raw[(8 * u + 2 * w) * kBN + r];
-                        const uint32_t b1 = raw[(8 * u + 2 * w + 1) * kBN + r];
-                        const uint32_t v = (b0 >> 4) | ((b0 & 15u) << 8) | ((b1 >> 4) << 16) | ((b1 & 15u) << 24);
-                        wd[w] = (v + 0x78787878u) ^ 0x80808080u;  // each nibble c -> int8 c - 8
+                            for (int j = 0; j < 16; ++j)
+                                sw[j] = EPI == E_SCALED ? __ldg(p.s_w + min(n + j, p.N - 1)) : 1.f;
+                        }
+                        if (p.bias && full16 && p.vec_bias) {
+                            const uint4* b4 = reinterpret_cast<const uint4*>(p.bias + n);
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint4 v = __ldg(b4 + h);
+                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    bb[8 * h + 2 * j] = __uint_as_float(w4[j] << 16);
+                                    bb[8 * h + 2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                bb[j] = p.bias ? __bfloat162float(p.bias[min(n + j, p.N - 1)]) : 0.f;
+                        }
                     }
-                    st_shared_v4(dst + swz128(r, u), wd[0], wd[1], wd[2], wd[3]);
+                }
+                uint32_t r[16];
+                tmem_ld16(acc + (uint32_t)(c * 16), r);
+                if (!row_ok || n >= p.N)
+                    continue;
+                if constexpr (EPI == E_I32) {
+                    int32_t* o = static_cast<int32_t*>(p.out) + (size_t)row * p.N + n;
+                    if (full16) {
+#pragma unroll
+                        for (int j = 0; j < 16; j += 4)
+                            *reinterpret_cast<uint4*>(o + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (n + j < p.N)
+                                o[j] = (int32_t)r[j];
+                    }
+                } else {
+                    float v[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        float a;
+                        if constexpr (EPI == E_SCALED)  // W4 operands are 16 (c - 8): exact shift back
+                            a = (float)((int32_t)r[j] >> (BSRC == B_W4 ? 4 : 0)) * (sx * sw[j]);
+                        else
+                            a = __uint_as_float(r[j]);
+                        v[j] = a + bb[j];
+                    }
+                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + n;
+                    if (full16) {
+                        *reinterpret_cast<uint4*>(o) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                                  pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                        *reinterpret_cast<uint4*>(o + 8) =
+                            make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                                       pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (n + j < p.N)
+                                o[j] = __float2bfloat16_rn(v[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars.acc_empty[buf]);
+        }
+    } else if constexpr (Cfg::XW > 0) {
+        // ------------------------------------------------------------ B transform
+        const int r = threadIdx.x - (2 + kEpiWarps) * 32;  // B operand row 0 .. BN-1
+        const int ng = p.g > 0 ? p.K / p.g : 1;
+        // W4: warp wt of the transform takes 128-column half wt % (BN/128) and units wt / (BN/128) (+4)
+        const int wt = r >> 5;
+        const int w4_q = 32 * (wt % (BN / 128)) + lane;  // column quad
+        const int w4_u0 = wt / (BN / 128);
+        const int w4_rot = (lane >> 1) & 3;
+        const uint32_t c0 = w4_rot, c1 = (w4_rot + 1) & 3, c2 = (w4_rot + 2) & 3, c3 = (w4_rot + 3) & 3;
+        const uint32_t w4_selA = c0 | ((4 + c0) << 4) | (c1 << 8) | ((4 + c1) << 12);
+        const uint32_t w4_selB = c2 | ((4 + c2) << 4) | (c3 << 8) | ((4 + c3) << 12);
+        pdl_wait_prior_grids();  // the weights' parameters may come from the previous kernel
+        // group (scale, bias) bf16 bits of this row for stage `it` (k0 .. k0+31 and k0+32 .. k0+63),
+        // loaded two stages before their use and converted only then
+        const unsigned short* sc16 = reinterpret_cast<const unsigned short*>(p.scales);
+        const unsigned short* bi16 = reinterpret_cast<const unsigned short*>(p.biases);
+        auto load_params = [&](int it, unsigned (&pr)[4]) {
+            if (it >= total)
+                return;
+            const int ti = it / nk, kb = it - (it / nk) * nk;
+            int mt, nt;
+            tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
+            const size_t base = (size_t)min(nt * BN + r, p.N - 1) * ng;
+            const int k0 = kb * Cfg::KE;
+            const int g0 = k0 / p.g;
+            const int g1 = min(k0 + 32, p.K - 1) / p.g;
+            pr[0] = __ldg(sc16 + base + g0);
+            pr[1] = __ldg(bi16 + base + g0);
+            pr[2] = __ldg(sc16 + base + g1);
+            pr[3] = __ldg(bi16 + base + g1);
+        };
+        // one stage: RAW(slot) -> BT(it & 1); pr = this stage's parameters
+        auto stage = [&](int it, const unsigned (&pr)[4]) -> bool {
+            const int slot = it % Cfg::NS;
+            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status) ||
+                !mbar_wait_bounded(&bars.bempty[it & 1], ((it >> 1) & 1) ^ 1, p.status) || aborted(&bars.abort_flag))
+                return false;
+            uint8_t* dst = BT(it & 1);
+            if constexpr (BSRC == B_W4) {
+                // raw[i][n]: k-pair row i (k = 2i high nibble, 2i+1 low) of column n; 64 rows x BN bytes.
+                // This thread: columns 4q .. 4q+3, 16-k units u0 and u0 + 4.  Eight 32-bit loads (k-pair
+                // rows of a unit; the warp's lanes hit 32 distinct banks) are byte-transposed by PRMT into
+                // per-column words; slot sl holds column (rot + sl) & 3 so that the 16-byte stores of
+                // each 8-lane phase land in 8 distinct swizzle chunks.
+                const uint32_t* raw32 = reinterpret_cast<const uint32_t*>(RAW(slot));
+#pragma unroll
+                for (int uu = 0; uu < 2; ++uu) {
+                    const int u = w4_u0 + 4 * uu;
+                    uint32_t W[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        W[i] = raw32[(8 * u + i) * (BN / 4) + w4_q];
+                    uint32_t Ar[4], Br[4];  // row pairs (0,1), (2,3), (4,5), (6,7)
+#pragma unroll
+                    for (int pr2 = 0; pr2 < 4; ++pr2) {
+                        Ar[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selA);
+                        Br[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selB);
+                    }
+#pragma unroll
+                    for (int sl = 0; sl < 4; ++sl) {
+                        const uint32_t* src = sl < 2 ? Ar : Br;
+                        const uint32_t sel2 = (sl & 1) ? 0x7632u : 0x5410u;
+                        const uint32_t t0 = prmt(src[0], src[1], sel2);  // k-pair rows 0..3 of the column
+                        const uint32_t t1 = prmt(src[2], src[3], sel2);  // rows 4..7
+                        uint32_t o[4];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            // each nibble c -> int8 16 (c - 8): flip bit 3, keep it in the high half of the byte
+                            const uint32_t x = (h ? t1 : t0) ^ 0x88888888u;
+                            const uint32_t hi = x & 0xF0F0F0F0u;         // k = 2i
+                            const uint32_t lo = (x << 4) & 0xF0F0F0F0u;  // k = 2i + 1
+                            o[2 * h] = prmt(hi, lo, 0x5140u);
+                            o[2 * h + 1] = prmt(hi, lo, 0x7362u);
+                        }
+                        const int n = 4 * w4_q + ((w4_rot + sl) & 3);
+                        st_shared_v4(dst + swz128(n, u), o[0], o[1], o[2], o[3]);
+                    }
                 }
             } else {
                 // raw[n][32 bytes]: 64 LSB-first 4-bit codes of row n, k = k0 .. k0+63
-                const int kbase = it * Cfg::KE + 32 * half;  // first k of this thread's 32 codes
-                const uint4 cw = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * half);
-                const int gi = min(kbase, p.K - 1) / p.g;
-                const float s = __bfloat162float(p.scales[(size_t)nrow * ng + gi]);
-                const float b = __bfloat162float(p.biases[(size_t)nrow * ng + gi]);
-                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                const int k0 = (it % nk) * Cfg::KE;
+                // the two 16-byte halves in an order that keeps each 8-lane phase on distinct banks
+                const int u0 = (r >> 2) & 1;
+                const uint4 first = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * u0);
+                const uint4 second = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * (u0 ^ 1));
+                const uint4 half[2] = {u0 ? second : first, u0 ? first : second};
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {  // word w: k = kbase + 8w .. +7 -> unit 4 half + w
-                    uint32_t o[4];
+                for (int h = 0; h < 2; ++h) {
+                    // group of k0 + 32h .. k0 + 32h + 31
+                    const float s = __uint_as_float(pr[2 * h] << 16), b = __uint_as_float(pr[2 * h + 1] << 16);
+                    const uint32_t words[4] = {half[h].x, half[h].y, half[h].z, half[h].w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t w0 = words[w] >> (8 * j);
-                        const float q0 = __uint_as_float(0x4B000000u | (w0 & 15u)) - 8388608.0f;
-                        const float q1 = __uint_as_float(0x4B000000u | ((w0 >> 4) & 15u)) - 8388608.0f;
-                        o[j] = pack_bf16x2(__fmaf_rn(q0, s, b), __fmaf_rn(q1, s, b));
+                    for (int w = 0; w < 4; ++w) {  // word w: k = k0 + 32h + 8w .. +7 -> unit 4h + w
+                        uint32_t o[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t w0 = words[w] >> (8 * j);
+                            const float q0 = __uint_as_float(0x4B000000u | (w0 & 15u)) - 8388608.0f;
+                            const float q1 = __uint_as_float(0x4B000000u | ((w0 >> 4) & 15u)) - 8388608.0f;
+                            o[j] = pack_bf16x2(__fmaf_rn(q0, s, b), __fmaf_rn(q1, s, b));
+                        }
+                        // k beyond K: zero weights (the activations there are zero too)
+                        if (k0 + 32 * h + 8 * w >= p.K)
+                            o[0] = o[1] = o[2] = o[3] = 0u;
+                        st_shared_v4(dst + swz128(r, 4 * h + w), o[0], o[1], o[2], o[3]);
                     }
-                    // k beyond K: zero weights (the activations there are zero too)
-                    if (kbase + 8 * w >= p.K)
-                        o[0] = o[1] = o[2] = o[3] = 0u;
-                    st_shared_v4(dst + swz128(r, 4 * half + w), o[0], o[1], o[2], o[3]);
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars.bready[slot]);
+                mbar_arrive(&bars.bfull[it & 1]);
+            return true;
+        };
+        // three parameter sets rotate so that each is loaded two stages before its use
+        unsigned P0[4] = {0u, 0u, 0u, 0u}, P1[4] = {0u, 0u, 0u, 0u}, P2[4] = {0u, 0u, 0u, 0u};
+        if constexpr (BSRC == B_AFFINE4) {
+            load_params(0, P0);
+            load_params(1, P1);
         }
+        bool ok = true;
+        for (int it = 0; it < total && ok; it += 3) {
+            if constexpr (BSRC == B_AFFINE4)
+                load_params(it + 2, P2);
+            ok = stage(it, P0);
+            if (!ok || it + 1 >= total)
+                break;
+            if constexpr (BSRC == B_AFFINE4)
+                load_params(it + 3, P0);
+            ok = stage(it + 1, P1);
+            if (!ok || it + 2 >= total)
+                break;
+            if constexpr (BSRC == B_AFFINE4)
+                load_params(it + 4, P1);
+            ok = stage(it + 2, P2);
+        }
+        if (!ok)
+            bars.abort_flag = 1;
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1)
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
 
-template <int BSRC, int EPI>
-cudaError_t launch_t(const TcParams& prm, int M, int N, cudaStream_t st)
+template <int BSRC, int EPI, int BN>
+cudaError_t launch_t(TcParams& prm, cudaStream_t st, const DeviceInfo& dev)
 {
-    using Cfg = TcCfg<BSRC>;
-    auto kern = tc_gemm_kernel<BSRC, EPI>;
+    using Cfg = TcCfg<BSRC, BN>;
+    auto kern = tc_gemm_kernel<BSRC, EPI, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess)
         return e;
+    prm.tiles_m = (prm.M + kBM - 1) / kBM;
+    prm.tiles_n = (prm.N + BN - 1) / BN;
+    const int tiles = prm.tiles_m * prm.tiles_n;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBM - 1) / kBM), 1);
+    cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count), 1, 1);
     cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
     cfg.dynamicSmemBytes = (size_t)Cfg::SMEM;
     cfg.stream = st;
@@ -321,6 +518,35 @@ cudaError_t launch_t(const TcParams& prm, int M, int N, cudaStream_t st)
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, prm);
 }
+
+bool encode_b(TcOp op, CUtensorMap* tm, const TcGemmArgs& a, int bn)
+{
+    switch (op) {
+    case TC_I8_RAW:
+    case TC_W8A8:
+        return encode_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K,
+                              128, (uint32_t)bn);
+    case TC_W4A8:
+        return encode_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)a.N, (uint64_t)(a.K / 2),
+                              (uint64_t)a.N, (uint32_t)bn, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+    default:
+        return encode_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                              (uint64_t)(a.K / 2), 32, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+}
+
+template <int BN>
+cudaError_t launch_bn(TcOp op, TcParams& prm, cudaStream_t st, const DeviceInfo& dev)
+{
+    switch (op) {
+    case TC_I8_RAW: return launch_t<B_TMA_I8, E_I32, BN>(prm, st, dev);
+    case TC_W8A8: return launch_t<B_TMA_I8, E_SCALED, BN>(prm, st, dev);
+    case TC_W4A8: return launch_t<B_W4, E_SCALED, BN>(prm, st, dev);
+    default: return launch_t<B_AFFINE4, E_BIAS, BN>(prm, st, dev);
+    }
+}
+
+bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -337,36 +563,21 @@ cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const 
     prm.scales = static_cast<const __nv_bfloat16*>(a.scales);
     prm.biases = static_cast<const __nv_bfloat16*>(a.biases);
     prm.g = a.g;
+    prm.vec_sw = aligned16p(a.s_w);
+    prm.vec_bias = aligned16p(a.bias);
+    prm.vec_out = aligned16p(a.out);
     prm.status = dev.status;
     const bool bf16_a = op == TC_AFFINE4;
     const uint64_t a_pitch = (uint64_t)a.K * (bf16_a ? 2 : 1);
     if (!encode_tmap_2d(&prm.tm_a, bf16_a ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a,
                         (uint64_t)a.K, (uint64_t)a.M, a_pitch, bf16_a ? 64 : 128, kBM))
         return cudaErrorInvalidValue;
-    bool ok;
-    switch (op) {
-    case TC_I8_RAW:
-    case TC_W8A8:
-        ok = encode_tmap_2d(&prm.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)a.K, (uint64_t)a.N,
-                            (uint64_t)a.K, 128, kBN);
-        break;
-    case TC_W4A8:
-        ok = encode_tmap_2d(&prm.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)a.N, (uint64_t)(a.K / 2),
-                            (uint64_t)a.N, kBN, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
-        break;
-    default:
-        ok = encode_tmap_2d(&prm.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)(a.K / 2), (uint64_t)a.N,
-                            (uint64_t)(a.K / 2), 32, kBN, CU_TENSOR_MAP_SWIZZLE_NONE);
-        break;
-    }
-    if (!ok)
+    // 256-column tiles when they still give every SM a tile, else 128
+    const int64_t tiles_m = (a.M + kBM - 1) / kBM;
+    const bool wide = tiles_m * ((a.N + 255) / 256) >= dev.sm_count;
+    if (!encode_b(op, &prm.tm_b, a, wide ? 256 : 128))
         return cudaErrorInvalidValue;
-    switch (op) {
-    case TC_I8_RAW: return launch_t<B_TMA_I8, E_I32>(prm, prm.M, prm.N, st);
-    case TC_W8A8: return launch_t<B_TMA_I8, E_SCALED>(prm, prm.M, prm.N, st);
-    case TC_W4A8: return launch_t<B_W4, E_SCALED>(prm, prm.M, prm.N, st);
-    default: return launch_t<B_AFFINE4, E_BIAS>(prm, prm.M, prm.N, st);
-    }
+    return wide ? launch_bn<256>(op, prm, st, dev) : launch_bn<128>(op, prm, st, dev);
 }
 
 }  // namespace qlin

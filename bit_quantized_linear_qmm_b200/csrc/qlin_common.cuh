@@ -72,13 +72,15 @@ QLIN_DEV void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes)
                  : "memory");
 }
 
+// Suspends the thread (up to a hint of 1 ms, or until the phase completes)
+// instead of spinning, so waiting warps leave the issue slots to the others.
 QLIN_DEV bool mbar_try_wait(uint64_t* bar, unsigned parity)
 {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
@@ -91,9 +93,8 @@ QLIN_DEV bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned* status
         return true;
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity))
-                return true;
+        if (mbar_try_wait(bar, parity))
+            return true;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             atomicOr(status, kStatusTimeout);
             return false;
@@ -125,6 +126,35 @@ QLIN_DEV void bulk_prefetch_l2(const void* gmem_src, unsigned bytes)
 QLIN_DEV void prefetch_l2(const void* p)
 {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// 16-byte global loads: read-only streaming data that is not kept in L1, and
+// data another kernel may have written (cached in L2 only).
+QLIN_DEV uint4 ldg_stream_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte global -> shared copy that bypasses registers and L1 (cp.async);
+// cp_async_wait_all() waits for this thread's copies.
+QLIN_DEV void cp_async16(void* smem_dst, const void* gmem_src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
+QLIN_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+QLIN_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> QLIN_DEV void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+QLIN_DEV uint4 ldg_cg_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
 }
 
 // ---------------------------------------------------------------- tensor-map TMA (2-D tiles)
