@@ -10,20 +10,23 @@
 //  * A CTA owns a block of output rows over the whole of K (about one CTA
 //    per SM), so the only reduction is inside the CTA: no clusters, no
 //    workspace, no global atomics.  A small footprint leaves room on each SM
-//    for the next kernel in the stream.
-//  * One producer thread streams the block through a shared-memory ring with
-//    2-D tensor-map TMA (cp.async.bulk.tensor, 128-byte swizzle, completion
-//    on mbarriers): one instruction moves a 128-byte column block of all the
-//    CTA's weight rows, one the same columns of the M token rows of x (the
-//    remaining token rows of the ring stay zero).  With programmatic
-//    dependent launch the next kernel is released at once, and each kernel
+//    for the next kernel in the stream, which programmatic dependent launch
+//    releases at once.
+//  * affine: one producer thread streams the block through a shared-memory
+//    ring with 2-D tensor-map TMA (cp.async.bulk.tensor, 128-byte swizzle,
+//    completion on mbarriers): one instruction moves a 128-byte column block
+//    of all the CTA's weight rows, one the same columns of the M token rows
+//    of x (the remaining token rows of the ring stay zero).  Each kernel
 //    prefetches its first stages into L2 before griddepcontrol.wait, so a
-//    layer's DRAM fetch overlaps the previous layer's tail.
-//  * Eight consumer warps split K (whole groups / k16 steps round robin);
-//    each covers all the CTA's 16-row tiles, so every x fragment serves them
-//    all.  They dequantise in registers and run the MACs on the tensor cores
-//    with the legacy mma.sync.m16n8k16 (weights as the 16-row A operand, x as
-//    the n=8 B operand, fp32 accumulation); partial tiles are summed through
+//    layer's DRAM fetch overlaps the previous layer's tail.  Eight consumer
+//    warps split K (whole groups round robin); each covers all the CTA's
+//    16-row tiles, so every x fragment serves them all.
+//  * bitlinear: a layer's packed weights are small enough (a few MB) for the
+//    CTAs to hold them in registers: they are loaded before
+//    griddepcontrol.wait, and only x is read after it.
+//  * Both dequantise in registers and run the MACs on the tensor cores with
+//    the legacy mma.sync.m16n8k16 (weights as the 16-row A operand, x as the
+//    n=8 B operand, fp32 accumulation); partial tiles are summed through
 //    shared memory.
 //  * affine: codes become bf16 with one LOP3 per pair: (w >> s) & 0x000F000F
 //    | 0x43004300 is the bf16 pair (128 + q_i, 128 + q_j), exact.  The 128
@@ -528,177 +531,13 @@ __global__ void __launch_bounds__(kThreads, 2) affine_gemv_kernel(const __grid_c
     }
 }
 
-// ---------------------------------------------------------------- BitLinear decode kernel
-
-template <int NT>
-struct BitCfg {
-    static constexpr int PROWS = 8;                 // packed rows per CTA -> 32 output rows
-    static constexpr int KST = 512;                 // k (bytes per packed row) per stage
-    static constexpr int NWB = KST / 128;           // 128-byte weight boxes per stage
-    static constexpr int NXB = KST * 2 / 128;       // 128-byte x boxes per stage
-    static constexpr int MMAX = 8 * NT;
-    static constexpr int W_STAGE = NWB * PROWS * 128;
-    static constexpr int X_STAGE = NXB * MMAX * 128;
-    static constexpr int STAGE = W_STAGE + X_STAGE;
-    static constexpr int NS = (64 * 1024 / STAGE) > kStages ? kStages : (64 * 1024 / STAGE);
-    static constexpr int SPW = KST / 16 / kConsumerWarps;  // k16 steps per warp in a full stage
-    static_assert(STAGE % 1024 == 0, "swizzled boxes need 1024-byte alignment");
-    static constexpr int RED = MMAX * kRedStride * 4;
-    static constexpr int SMEM = NS * STAGE + RED + (int)sizeof(Barriers) + 1024;
-};
-
-struct BitParams {
-    CUtensorMap tm_w;  // packed [N/4][K] bytes, box {128 B, 8 rows}
-    CUtensorMap tm_x;  // x [M][K] bf16, box {64 elements, M tokens}
-    const float* weight_scale;
-    const __nv_bfloat16* bias;
-    __nv_bfloat16* y;
-    int M, K, N, R;  // R = N / 4
-    int invert;
-    unsigned* status;
-};
+// ---------------------------------------------------------------- bf16x2 helper
 
 QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
 {
     uint32_t r;
     asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
     return r;
-}
-
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 2) bitlinear_gemv_kernel(const __grid_constant__ BitParams p)
-{
-    using Cfg = BitCfg<NT>;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* stages = smem;
-    float* red = reinterpret_cast<float*>(smem + Cfg::NS * Cfg::STAGE);
-    Barriers& bars = *reinterpret_cast<Barriers*>(reinterpret_cast<uint8_t*>(red) + Cfg::RED);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int p0 = blockIdx.x * Cfg::PROWS;
-    const int nst = (p.K + Cfg::KST - 1) / Cfg::KST;
-    const int M = p.M;
-
-    init_barriers(bars);
-
-    if (warp == kConsumerWarps) {
-        producer_loop<Cfg::NS>(
-            bars, nst, p.status,
-            [&](int it, int slot) {
-                const int k0 = it * Cfg::KST;
-                uint8_t* wst = stages + slot * Cfg::STAGE;
-                uint8_t* xst = wst + Cfg::W_STAGE;
-#pragma unroll
-                for (int b = 0; b < Cfg::NWB; ++b)
-                    tma_load_2d(wst + b * (Cfg::PROWS * 128), &p.tm_w, k0 + b * 128, p0, &bars.full[slot]);
-#pragma unroll
-                for (int b = 0; b < Cfg::NXB; ++b)
-                    tma_load_2d(xst + b * (Cfg::MMAX * 128), &p.tm_x, k0 + b * 64, 0, &bars.full[slot]);
-            },
-            [&](int it) {
-#pragma unroll
-                for (int b = 0; b < Cfg::NWB; ++b)
-                    tma_prefetch_2d(&p.tm_w, it * Cfg::KST + b * 128, p0);
-            },
-            [&](int) { return (unsigned)(Cfg::W_STAGE + Cfg::NXB * M * 128); });
-    } else {
-        zero_x_tail(stages, Cfg::NS, Cfg::STAGE, Cfg::W_STAGE, Cfg::NXB, Cfg::MMAX, M);
-        pdl_wait_prior_grids();  // weight_scale may come from an earlier kernel
-        const float ws = *p.weight_scale;
-        const float scale = p.invert ? __fdiv_rn(1.0f, ws) : ws;
-        consumer_bar();
-        // Warps take k16 steps round robin.  A lane's 32-bit word (4 consecutive
-        // k of packed row gid) feeds two MMAs: fields {0, 2} and {1, 3} of its
-        // bytes, as A rows gid / gid+8.  Field j is read in place with one LOP3,
-        // (w & (3 << 2j)) | 0x4300 = bf16 128 + 4^j c, and one bf16x2 FMA,
-        // times 4^-j minus (128 4^-j + 1), gives the exact weight c - 1.
-        const int gid = lane >> 2, tig = lane & 3;
-        // per-field bf16x2 constants: {4^-j, -(128 4^-j + 1)} for the rows of each MMA
-        constexpr uint32_t kScale0 = 0x3F803F80u, kBias0 = 0xC301C301u;  // j=0: 1, -129
-        constexpr uint32_t kScale1 = 0x3E803E80u, kBias1 = 0xC204C204u;  // j=1: 1/4, -33
-        constexpr uint32_t kScale2 = 0x3D803D80u, kBias2 = 0xC110C110u;  // j=2: 1/16, -9
-        float a02[NT][4], a13[NT][4];
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                a02[t][e] = a13[t][e] = 0.f;
-        auto step = [&](const uint8_t* wst, const uint8_t* xst, int s) {
-            const int wi = s * 4 + tig;  // word of 4 bytes (k = 4 wi .. 4 wi + 3)
-            const uint32_t w = w_word(wst, Cfg::PROWS, gid, wi);
-            const uint32_t hw = w >> 8;  // bytes k+1, k+3 in the low byte of each half
-            uint32_t f02[4], f13[4];
-            f02[0] = bf16x2_fma(lop3_and_or(w, 0x00030003u, 0x43004300u), kScale0, kBias0);         // f0 (k, k+2)
-            f02[1] = bf16x2_fma(lop3_and_or(w, 0x00300030u, 0x43004300u), kScale2, kBias2);         // f2 (k, k+2)
-            f02[2] = bf16x2_fma(lop3_and_or(hw, 0x00030003u, 0x43004300u), kScale0, kBias0);        // f0 (k+1, k+3)
-            f02[3] = bf16x2_fma(lop3_and_or(hw, 0x00300030u, 0x43004300u), kScale2, kBias2);        // f2 (k+1, k+3)
-            f13[0] = bf16x2_fma(lop3_and_or(w, 0x000C000Cu, 0x43004300u), kScale1, kBias1);         // f1 (k, k+2)
-            f13[1] = bf16x2_fma(lop3_and_or(w >> 6, 0x00030003u, 0x43004300u), kScale0, kBias0);    // f3 (k, k+2)
-            f13[2] = bf16x2_fma(lop3_and_or(hw, 0x000C000Cu, 0x43004300u), kScale1, kBias1);        // f1 (k+1, k+3)
-            f13[3] = bf16x2_fma(lop3_and_or(w >> 14, 0x00030003u, 0x43004300u), kScale0, kBias0);   // f3 (k+1, k+3)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                // tokens >= M read zeros
-                const uint2 v = *reinterpret_cast<const uint2*>(
-                    x_addr<__nv_bfloat16, Cfg::MMAX>(xst, t * 8 + gid, 4 * wi));
-                const uint32_t b0 = pair_lo(v.x, v.y);  // (x_k, x_{k+2})
-                const uint32_t b1 = pair_hi(v.x, v.y);  // (x_{k+1}, x_{k+3})
-                mma_bf16_16816(a02[t], f02, b0, b1);
-                mma_bf16_16816(a13[t], f13, b0, b1);
-            }
-        };
-        for (int it = 0; it < nst; ++it) {
-            const int slot = it % Cfg::NS;
-            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status)) {
-                bars.abort_flag = 1;
-                break;
-            }
-            const uint8_t* wst = stages + slot * Cfg::STAGE;
-            const uint8_t* xst = wst + Cfg::W_STAGE;
-            const int steps = min(Cfg::KST, p.K - it * Cfg::KST) / 16;
-            if (steps == Cfg::KST / 16) {
-#pragma unroll
-                for (int j = 0; j < Cfg::SPW; ++j)
-                    step(wst, xst, warp + j * kConsumerWarps);
-            } else {
-                for (int s2 = warp; s2 < steps; s2 += kConsumerWarps)
-                    step(wst, xst, s2);
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bars.empty[slot]);
-        }
-        // red row index = field * 8 + local packed row
-        cta_reduce<NT * 8, 1>(
-            reinterpret_cast<float*>(stages), red,
-            [&](int j) {
-                const int t = j / 8, e = (j / 4) % 2, f = j % 4;
-                switch (f) {
-                case 0: return a02[t][e];
-                case 1: return a13[t][e];
-                case 2: return a02[t][e + 2];
-                default: return a13[t][e + 2];
-                }
-            },
-            [&](int, int j, int ln, int& row, int& tok) {
-                const int t = j / 8, e = (j / 4) % 2, f = j % 4;
-                row = f * 8 + (ln >> 2);
-                tok = t * 8 + 2 * (ln & 3) + e;
-            });
-        consumer_bar();
-        for (int e = threadIdx.x; e < M * 32; e += kConsumerThreads) {
-            const int tok = e / 32, i = e % 32;
-            const int pr = p0 + (i & 7);
-            if (pr < p.R) {
-                const int n = pr + (i >> 3) * p.R;
-                float v = red[tok * kRedStride + i] * scale;
-                if (p.bias)
-                    v += __bfloat162float(p.bias[n]);
-                p.y[(size_t)tok * p.N + n] = __float2bfloat16_rn(v);
-            }
-        }
-    }
 }
 
 // ---------------------------------------------------------------- BitLinear decode
@@ -711,28 +550,21 @@ __global__ void __launch_bounds__(kThreads, 2) bitlinear_gemv_kernel(const __gri
 // Its bytes are first reordered (0, 2, 1, 3), so that the bf16 pairs the
 // LOP3 decode yields are consecutive k, like x in memory.
 //
-// Data movement (M <= 8): every thread copies its own 16-byte pieces with
-// cp.async into a private slot of shared memory -- the weights of its first
-// eight chunks before griddepcontrol.wait (under programmatic dependent
-// launch a layer's weight stream overlaps the previous kernel), the x pieces
-// right after it, one commit group per chunk -- and consumes them chunk by
-// chunk behind cp.async.wait_group.  Everything is in flight at once, no
-// block barrier is needed, and lanes touch consecutive 16-byte units (no
-// bank conflicts).  Chunks beyond the eighth are refilled into the slot just
-// consumed.  For 9..16 tokens, x goes through a ring of registers instead.
+// Data movement: the packed weights go straight from HBM into registers
+// before griddepcontrol.wait (under programmatic dependent launch a layer's
+// weight stream overlaps the previous kernel); after the wait each lane
+// streams its x through a small ring of registers.  With K % 64 == 0 and at
+// most eight chunks per warp (K <= 4096) a lean variant drops the per-chunk
+// bounds logic and the refill of later rounds.
 //
 // The grid has at least one CTA per SM; the spare ones only pass the
 // dependency wait.  With every kernel holding one CTA on every SM, the next
-// layer's CTAs (two fit per SM) land one per SM as well.
+// layer's CTAs (two fit per SM) tend to land one per SM as well.
 constexpr int kBlWarps = 8;
 constexpr int kBlThreads = kBlWarps * 32;
-constexpr int kBlRows = 8;     // packed rows per CTA (32 outputs)
-constexpr int kBlChunk = 64;   // k per chunk
-constexpr int kBlRound = 8;    // chunks in flight per warp
-// shared memory of the cp.async path: weights, then x, 16-byte units [slot][unit][thread]
-constexpr int kBlSmemW = kBlRound * kBlThreads * 16;       // 32 KB
-constexpr int kBlSmemX = kBlRound * 2 * kBlThreads * 16;   // 64 KB
-constexpr int kBlSmemAsync = kBlSmemW + kBlSmemX;
+constexpr int kBlRows = 8;    // packed rows per CTA (32 outputs)
+constexpr int kBlChunk = 64;  // k per chunk
+constexpr int kBlRound = 8;   // chunks a warp holds in registers at once
 
 struct BitRegParams {
     const uint8_t* packed;   // [R][K]
@@ -746,15 +578,12 @@ struct BitRegParams {
     unsigned* status;
 };
 
-// ASYNC: the cp.async shared-memory path (NT == 1); else weights in
-// registers and x through an XD-deep register ring.
-template <int NT, int XD, bool ASYNC>
+// NT token tiles of 8; XD-deep x ring; FAST: whole chunks and a single round.
+template <int NT, int XD, bool FAST>
 __global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __grid_constant__ BitRegParams p)
 {
     static_assert(kBlRound % XD == 0, "x ring depth must divide the register round");
-    static_assert(!ASYNC || NT == 1, "the shared-memory path holds 8 tokens");
     __shared__ float red[kBlWarps * 8 * NT * 32];
-    extern __shared__ __align__(16) uint8_t dsm[];  // ASYNC: weight slots, then x slots
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
 
@@ -769,17 +598,11 @@ __global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __gr
     const int my = nch > warp ? (nch - 1 - warp) / kBlWarps + 1 : 0;  // chunks of this warp
     const bool row_ok = p0 + gid < p.R;
     const uint8_t* wrow = p.packed + (size_t)(row_ok ? p0 + gid : 0) * p.K + 16 * tig;
-    const bool tok_ok = gid < p.M;  // token of this lane (first token tile)
-    const __nv_bfloat16* xrow = p.x + (size_t)(tok_ok ? gid : 0) * p.K + 16 * tig;
     // ci-th chunk of this warp: c = warp + 8 ci, k = 64 c + 16 tig
     auto chunk_k = [&](int ci) { return (warp + ci * kBlWarps) * kBlChunk; };
-    auto w_ok = [&](int ci) { return row_ok && ci < my && chunk_k(ci) + 16 * tig < p.K; };
-    auto x_ok = [&](int ci) { return tok_ok && ci < my && chunk_k(ci) + 16 * tig < p.K; };
-    uint4* wslot = reinterpret_cast<uint4*>(dsm) + threadIdx.x;             // + j * kBlThreads
-    uint4* xslot = reinterpret_cast<uint4*>(dsm + kBlSmemW) + threadIdx.x;  // + (2 j + h) * kBlThreads
 
     auto load_w = [&](uint4& dst, int ci) {
-        if (w_ok(ci))
+        if (row_ok && ci < my && (FAST || chunk_k(ci) + 16 * tig < p.K))
             dst = ldg_stream_v4(wrow + chunk_k(ci));
         else
             dst = make_uint4(0u, 0u, 0u, 0u);
@@ -789,7 +612,7 @@ __global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __gr
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             const int m = 8 * t + gid;
-            if (ci < my && m < p.M && k < p.K) {
+            if (ci < my && m < p.M && (FAST || k < p.K)) {
                 const __nv_bfloat16* src = p.x + (size_t)m * p.K + k;
                 dst[t][0] = ldg_cg_v4(src);
                 dst[t][1] = ldg_cg_v4(src + 8);
@@ -799,34 +622,15 @@ __global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __gr
         }
     };
 
-    uint4 wr[ASYNC ? 1 : kBlRound];
-    uint4 xb[XD][NT][2];
-    if constexpr (ASYNC) {
+    uint4 wr[kBlRound];
 #pragma unroll
-        for (int j = 0; j < kBlRound; ++j)
-            if (w_ok(j))
-                cp_async16(wslot + j * kBlThreads, wrow + chunk_k(j));
-        cp_async_commit();
-    } else {
-#pragma unroll
-        for (int j = 0; j < kBlRound; ++j)
-            load_w(wr[j], j);
-    }
+    for (int j = 0; j < kBlRound; ++j)
+        load_w(wr[j], j);
     pdl_wait_prior_grids();  // x, weight_scale and y may belong to the previous kernel
-    if constexpr (ASYNC) {
+    uint4 xb[XD][NT][2];
 #pragma unroll
-        for (int j = 0; j < kBlRound; ++j) {
-            if (x_ok(j)) {
-                cp_async16(xslot + (2 * j) * kBlThreads, xrow + chunk_k(j));
-                cp_async16(xslot + (2 * j + 1) * kBlThreads, xrow + chunk_k(j) + 8);
-            }
-            cp_async_commit();
-        }
-    } else {
-#pragma unroll
-        for (int d = 0; d < XD; ++d)
-            load_x(xb[d], d);
-    }
+    for (int d = 0; d < XD; ++d)
+        load_x(xb[d], d);
     const float ws = *p.weight_scale;
     const float scale = p.invert ? __fdiv_rn(1.0f, ws) : ws;
 
@@ -873,36 +677,20 @@ __global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __gr
         }
     };
 
-    const int rounds = (my + kBlRound - 1) / kBlRound;
-    for (int rd = 0; rd < rounds; ++rd) {
+    if constexpr (FAST) {
 #pragma unroll
         for (int j = 0; j < kBlRound; ++j) {
-            const int ci = rd * kBlRound + j;
-            if constexpr (ASYNC) {
-                // groups after this chunk's: the x of the later first-round chunks and one refill per
-                // chunk already done -- always kBlRound - 1
-                cp_async_wait_group<kBlRound - 1>();
-                if (ci < my) {
-                    const uint4 w4 = wslot[j * kBlThreads];
-                    uint4 xv[1][2];
-                    if (x_ok(ci)) {  // x past K (or past M) is zero
-                        xv[0][0] = xslot[(2 * j) * kBlThreads];
-                        xv[0][1] = xslot[(2 * j + 1) * kBlThreads];
-                    } else {
-                        xv[0][0] = xv[0][1] = make_uint4(0u, 0u, 0u, 0u);
-                    }
-                    chunk(w4, xv);
-                }
-                // refill this slot with chunk ci + 8 (the values above are already in registers)
-                const int cn = ci + kBlRound;
-                if (w_ok(cn))
-                    cp_async16(wslot + j * kBlThreads, wrow + chunk_k(cn));
-                if (x_ok(cn)) {
-                    cp_async16(xslot + (2 * j) * kBlThreads, xrow + chunk_k(cn));
-                    cp_async16(xslot + (2 * j + 1) * kBlThreads, xrow + chunk_k(cn) + 8);
-                }
-                cp_async_commit();
-            } else {
+            if (j < my)
+                chunk(wr[j], xb[j % XD]);
+            if (j + XD < kBlRound)
+                load_x(xb[j % XD], j + XD);
+        }
+    } else {
+        const int rounds = (my + kBlRound - 1) / kBlRound;
+        for (int rd = 0; rd < rounds; ++rd) {
+#pragma unroll
+            for (int j = 0; j < kBlRound; ++j) {
+                const int ci = rd * kBlRound + j;
                 if (ci < my)
                     chunk(wr[j], xb[j % XD]);
                 load_x(xb[j % XD], ci + XD);
@@ -910,8 +698,6 @@ __global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __gr
             }
         }
     }
-    if constexpr (ASYNC)
-        cp_async_wait_all();  // nothing may still be landing in shared memory at exit
 
     // sum the 8 warps' partial tiles; v = t * 8 + a * 4 + e (a: fields {0,2} / {1,3})
 #pragma unroll
@@ -1087,9 +873,12 @@ cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const
         prm.tiles = tiles;
         prm.invert = a.invert;
         prm.status = dev.status;
+        const bool fast = a.K % kBlChunk == 0 && a.K <= (int64_t)kBlChunk * kBlWarps * kBlRound;
         cudaError_t e;
-        if (mc <= 8)
-            e = launch_pdl_threads(bitlinear_reg_kernel<1, 1, true>, grid, kBlThreads, kBlSmemAsync, st, prm);
+        if (mc <= 8 && fast)
+            e = launch_pdl_threads(bitlinear_reg_kernel<1, 2, true>, grid, kBlThreads, 0, st, prm);
+        else if (mc <= 8)
+            e = launch_pdl_threads(bitlinear_reg_kernel<1, 4, false>, grid, kBlThreads, 0, st, prm);
         else
             e = launch_pdl_threads(bitlinear_reg_kernel<2, 2, false>, grid, kBlThreads, 0, st, prm);
         if (e != cudaSuccess)

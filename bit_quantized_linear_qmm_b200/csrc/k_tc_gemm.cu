@@ -7,7 +7,7 @@
 //              [cider/ops.py perchannel_linear]
 //   W4A8:      y[m,n] = acc * s_x[m] * s_w[n] (+ bias[n]),   acc = qx . (c - 8)
 //              [cider/ops.py w4a8_linear, pack_weight_int4]
-//   affine:    y[m,n] = sum_k x[m,k] * bf16(fma(q, s, b)) + bias[n]
+//   affine:    y[m,n] = sum_k x[m,k] * bf16(s q + b) + bias[n]   (s q + b rounded once)
 //              [nuvec-nn QuantizedLinear, forward; cider/ops.py pergroup_linear
 //               docstring, dequantize]
 //
@@ -26,14 +26,14 @@
 //   warps 2..5   epilogue: tcgen05.ld of one accumulator (warp q owns TMEM
 //                lanes 32q .. 32q+31 = 32 output rows) while the MMAs of the
 //                next tile fill the other one; scales, bias, 16-byte stores.
-//   warps 6..    (W4A8, affine) one thread per B row turns the packed source
-//                into the K-major 128-byte-swizzled operand in a 2-deep
-//                buffer: nibbles -> int8 16 (c - 8) (the epilogue shifts the
-//                exact int32 sum back by 4 bits), or codes -> bf16(fma(q,
-//                scale, bias)) computed in fp32 (the dequantized weight,
-//                rounded once to bf16); the group parameters of a stage are
-//                loaded two stages ahead.  fence.proxy.async publishes the
-//                operand to the tensor core.
+//   warps 6..    (W4A8, affine) 2 x BN transform threads turn the packed
+//                source into the K-major 128-byte-swizzled operand in a
+//                2-deep buffer: nibbles -> int8 16 (c - 8) (the epilogue
+//                shifts the exact int32 sum back by 4 bits), or codes ->
+//                bf16(s q + b), the exact value rounded once to bf16 (bf16x2
+//                FMA); the group parameters of a stage are loaded two stages
+//                ahead.  fence.proxy.async publishes the operand to the
+//                tensor core.
 // Every mbarrier wait is bounded; on expiry the kernel records the timeout,
 // every role stops, the MMA thread waits for its MMAs in flight, and TMEM is
 // always freed.
@@ -46,6 +46,10 @@ constexpr int kBM = 128;    // output rows (tokens) per tile
 constexpr int kGroupM = 8;  // M-tiles that walk the N dimension together
 constexpr int kEpiWarps = 4;
 constexpr int kSmemBudget = 200 * 1024;
+#ifndef QLIN_TC_BDEPTH
+#define QLIN_TC_BDEPTH 2
+#endif
+constexpr int kBDepth = QLIN_TC_BDEPTH;  // transformed-B buffers
 
 enum BSource { B_TMA_I8 = 0, B_W4 = 1, B_AFFINE4 = 2 };
 enum Epi { E_I32 = 0, E_SCALED = 1, E_BIAS = 2 };
@@ -57,12 +61,12 @@ template <int BSRC, int BN>
 struct TcCfg {
     static constexpr bool I8 = BSRC != B_AFFINE4;          // kind::i8 (s32) or kind::f16 (bf16 -> f32)
     static constexpr int KE = I8 ? 128 : 64;                // K elements per stage (128 bytes of A)
-    static constexpr int XW = BSRC == B_TMA_I8 ? 0 : BN / 32;  // transform warps: one B row per thread
+    static constexpr int XW = BSRC == B_TMA_I8 ? 0 : BN / 16;  // transform warps: two threads per B row
     static constexpr int A_BYTES = kBM * 128;
     static constexpr int B_BYTES = BN * 128;                // one K-major swizzled B operand
     static constexpr int RAW_BYTES = BSRC == B_W4 ? (KE / 2) * BN : (BSRC == B_AFFINE4 ? BN * (KE / 2) : B_BYTES);
     static constexpr int SLOT = rup(A_BYTES + RAW_BYTES, 1024);
-    static constexpr int BRING = XW > 0 ? 2 * B_BYTES : 0;  // transformed B, 2-deep
+    static constexpr int BRING = XW > 0 ? kBDepth * B_BYTES : 0;  // transformed B ring
     static constexpr int NS = cmin(8, (kSmemBudget - BRING) / SLOT);
     static constexpr int THREADS = (2 + kEpiWarps + XW) * 32;
     static constexpr int TMEM_COLS = 2 * BN;
@@ -73,8 +77,8 @@ struct TcCfg {
     struct Bars {
         uint64_t full[NS];
         uint64_t empty[NS];
-        uint64_t bfull[2];
-        uint64_t bempty[2];
+        uint64_t bfull[kBDepth];
+        uint64_t bempty[kBDepth];
         uint64_t acc_full[2];
         uint64_t acc_empty[2];
         uint64_t mma_done;
@@ -98,8 +102,9 @@ struct TcParams {
     const __nv_bfloat16* bias;
     const __nv_bfloat16* scales;
     const __nv_bfloat16* biases;
-    int g;
+    int g, g_shift;  // group size and its log2
     int vec_sw, vec_bias, vec_out;  // 16-byte alignment of s_w, bias and out
+    int vec_params;                 // scales / biases rows allow 16-byte loads of 8 groups
     unsigned* status;
 };
 
@@ -107,6 +112,13 @@ QLIN_DEV void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t
 {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
+}
+
+QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
 QLIN_DEV uint32_t pack_bf16x2(float lo, float hi)
@@ -153,9 +165,11 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             mbar_init(&bars.full[s], 1);
             mbar_init(&bars.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kBDepth; ++b) {
             mbar_init(&bars.bfull[b], Cfg::XW > 0 ? Cfg::XW : 1);
             mbar_init(&bars.bempty[b], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.acc_full[b], 1);
             mbar_init(&bars.acc_empty[b], kEpiWarps);
         }
@@ -217,19 +231,19 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                     const int slot = it % Cfg::NS;
                     ok = mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status);
                     if (ok && Cfg::XW > 0)
-                        ok = mbar_wait_bounded(&bars.bfull[it & 1], (it >> 1) & 1, p.status);
+                        ok = mbar_wait_bounded(&bars.bfull[it % kBDepth], (it / kBDepth) & 1, p.status);
                     if (!ok)
                         break;
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(A(slot));
-                    const uint32_t b0 = smem_u32(Cfg::XW > 0 ? BT(it & 1) : RAW(slot));
+                    const uint32_t b0 = smem_u32(Cfg::XW > 0 ? BT(it % kBDepth) : RAW(slot));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc_mma<Cfg::I8>(acc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
                                         Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
                     tc_commit(&bars.empty[slot]);
                     if (Cfg::XW > 0)
-                        tc_commit(&bars.bempty[it & 1]);
+                        tc_commit(&bars.bempty[it % kBDepth]);
                 }
                 tc_commit(&bars.acc_full[buf]);  // fires when this tile's MMAs are done
             }
@@ -351,140 +365,167 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         }
     } else if constexpr (Cfg::XW > 0) {
         // ------------------------------------------------------------ B transform
-        const int r = threadIdx.x - (2 + kEpiWarps) * 32;  // B operand row 0 .. BN-1
+        const int tt = threadIdx.x - (2 + kEpiWarps) * 32;  // 0 .. 2 BN - 1
+        const int wt = tt >> 5;                             // transform warp
+        // affine: thread = (B row r, 32-code half h); the half alternates every 8 rows so that the
+        // 16-byte stores of an 8-lane phase hit 8 distinct swizzle chunks
+        const int r = tt % BN;
+        const int h = ((r >> 3) & 1) ^ (tt / BN);
         const int ng = p.g > 0 ? p.K / p.g : 1;
-        // W4: warp wt of the transform takes 128-column half wt % (BN/128) and units wt / (BN/128) (+4)
-        const int wt = r >> 5;
+        // W4: warp wt takes 128-column half wt % (BN/128) and 16-k unit wt / (BN/128)
         const int w4_q = 32 * (wt % (BN / 128)) + lane;  // column quad
-        const int w4_u0 = wt / (BN / 128);
+        const int w4_u = wt / (BN / 128);
         const int w4_rot = (lane >> 1) & 3;
         const uint32_t c0 = w4_rot, c1 = (w4_rot + 1) & 3, c2 = (w4_rot + 2) & 3, c3 = (w4_rot + 3) & 3;
         const uint32_t w4_selA = c0 | ((4 + c0) << 4) | (c1 << 8) | ((4 + c1) << 12);
         const uint32_t w4_selB = c2 | ((4 + c2) << 4) | (c3 << 8) | ((4 + c3) << 12);
         pdl_wait_prior_grids();  // the weights' parameters may come from the previous kernel
-        // group (scale, bias) bf16 bits of this row for stage `it` (k0 .. k0+31 and k0+32 .. k0+63),
-        // loaded two stages before their use and converted only then
+        // affine: the group parameters of this thread's row come in windows of 8 groups (16 bytes of
+        // scales, 16 of biases: one vector load each when the row pitch allows); the window after the
+        // current one is always in flight.
         const unsigned short* sc16 = reinterpret_cast<const unsigned short*>(p.scales);
         const unsigned short* bi16 = reinterpret_cast<const unsigned short*>(p.biases);
-        auto load_params = [&](int it, unsigned (&pr)[4]) {
-            if (it >= total)
+        const int nwin = (ng + 7) / 8;
+        auto win_load = [&](int ti, int win, uint4& S, uint4& B) {
+            if (ti >= my_tiles)
                 return;
-            const int ti = it / nk, kb = it - (it / nk) * nk;
             int mt, nt;
             tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
-            const size_t base = (size_t)min(nt * BN + r, p.N - 1) * ng;
-            const int k0 = kb * Cfg::KE;
-            const int g0 = k0 / p.g;
-            const int g1 = min(k0 + 32, p.K - 1) / p.g;
-            pr[0] = __ldg(sc16 + base + g0);
-            pr[1] = __ldg(bi16 + base + g0);
-            pr[2] = __ldg(sc16 + base + g1);
-            pr[3] = __ldg(bi16 + base + g1);
+            const size_t off = (size_t)min(nt * BN + r, p.N - 1) * ng + 8 * win;
+            if (p.vec_params) {
+                S = __ldg(reinterpret_cast<const uint4*>(sc16 + off));
+                B = __ldg(reinterpret_cast<const uint4*>(bi16 + off));
+            } else {
+                uint32_t sv[4], bv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int g0 = 8 * win + 2 * e;
+                    const uint32_t slo = g0 < ng ? __ldg(sc16 + off + 2 * e) : 0u;
+                    const uint32_t shi = g0 + 1 < ng ? __ldg(sc16 + off + 2 * e + 1) : 0u;
+                    const uint32_t blo = g0 < ng ? __ldg(bi16 + off + 2 * e) : 0u;
+                    const uint32_t bhi = g0 + 1 < ng ? __ldg(bi16 + off + 2 * e + 1) : 0u;
+                    sv[e] = slo | (shi << 16);
+                    bv[e] = blo | (bhi << 16);
+                }
+                S = make_uint4(sv[0], sv[1], sv[2], sv[3]);
+                B = make_uint4(bv[0], bv[1], bv[2], bv[3]);
+            }
         };
-        // one stage: RAW(slot) -> BT(it & 1); pr = this stage's parameters
-        auto stage = [&](int it, const unsigned (&pr)[4]) -> bool {
+        uint4 curS = make_uint4(0u, 0u, 0u, 0u), curB = curS, nxtS = curS, nxtB = curS;
+        int cur_ti = 0, cur_win = -1;
+        // (scale, bias) bf16 bits for stage `it` (tile ti, k block kb)
+        auto params_for = [&](int ti, int kb, unsigned (&pr)[2]) {
+            const int gi = min(kb * Cfg::KE + 32 * h, p.K - 1) >> p.g_shift;
+            const int win = gi >> 3;
+            if (ti != cur_ti || win != cur_win) {
+                if (cur_win < 0) {  // first window of this CTA
+                    win_load(ti, win, curS, curB);
+                } else {
+                    curS = nxtS;
+                    curB = nxtB;
+                }
+                cur_ti = ti;
+                cur_win = win;
+                if (win + 1 < nwin)
+                    win_load(ti, win + 1, nxtS, nxtB);
+                else
+                    win_load(ti + 1, 0, nxtS, nxtB);
+            }
+            const int sub = gi & 7;
+            const uint32_t sw = (sub >> 1) == 0 ? curS.x : (sub >> 1) == 1 ? curS.y : (sub >> 1) == 2 ? curS.z : curS.w;
+            const uint32_t bw = (sub >> 1) == 0 ? curB.x : (sub >> 1) == 1 ? curB.y : (sub >> 1) == 2 ? curB.z : curB.w;
+            pr[0] = (sw >> (16 * (sub & 1))) & 0xFFFFu;
+            pr[1] = (bw >> (16 * (sub & 1))) & 0xFFFFu;
+        };
+        // one stage: RAW(slot) -> BT(it % kBDepth)
+        auto stage = [&](int it, int kb, const unsigned (&pr)[2]) -> bool {
             const int slot = it % Cfg::NS;
             if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status) ||
-                !mbar_wait_bounded(&bars.bempty[it & 1], ((it >> 1) & 1) ^ 1, p.status) || aborted(&bars.abort_flag))
+                !mbar_wait_bounded(&bars.bempty[it % kBDepth], ((it / kBDepth) & 1) ^ 1, p.status) ||
+                aborted(&bars.abort_flag))
                 return false;
-            uint8_t* dst = BT(it & 1);
+            uint8_t* dst = BT(it % kBDepth);
             if constexpr (BSRC == B_W4) {
                 // raw[i][n]: k-pair row i (k = 2i high nibble, 2i+1 low) of column n; 64 rows x BN bytes.
-                // This thread: columns 4q .. 4q+3, 16-k units u0 and u0 + 4.  Eight 32-bit loads (k-pair
-                // rows of a unit; the warp's lanes hit 32 distinct banks) are byte-transposed by PRMT into
-                // per-column words; slot sl holds column (rot + sl) & 3 so that the 16-byte stores of
-                // each 8-lane phase land in 8 distinct swizzle chunks.
+                // Eight 32-bit loads (the k-pair rows of unit u for columns 4q .. 4q+3; a warp's lanes
+                // hit 32 distinct banks) are byte-transposed by PRMT into per-column words; slot sl
+                // holds column (rot + sl) & 3 so that the 16-byte stores of each 8-lane phase land in 8
+                // distinct swizzle chunks.  Nibble c -> int8 16 (c - 8): bit 3 flipped, kept in the
+                // high half of the byte.
                 const uint32_t* raw32 = reinterpret_cast<const uint32_t*>(RAW(slot));
+                const int u = w4_u;
+                uint32_t W[8];
 #pragma unroll
-                for (int uu = 0; uu < 2; ++uu) {
-                    const int u = w4_u0 + 4 * uu;
-                    uint32_t W[8];
+                for (int i = 0; i < 8; ++i)
+                    W[i] = raw32[(8 * u + i) * (BN / 4) + w4_q];
+                uint32_t Ar[4], Br[4];  // row pairs (0,1), (2,3), (4,5), (6,7)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        W[i] = raw32[(8 * u + i) * (BN / 4) + w4_q];
-                    uint32_t Ar[4], Br[4];  // row pairs (0,1), (2,3), (4,5), (6,7)
+                for (int pr2 = 0; pr2 < 4; ++pr2) {
+                    Ar[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selA);
+                    Br[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selB);
+                }
 #pragma unroll
-                    for (int pr2 = 0; pr2 < 4; ++pr2) {
-                        Ar[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selA);
-                        Br[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selB);
+                for (int sl = 0; sl < 4; ++sl) {
+                    const uint32_t* src = sl < 2 ? Ar : Br;
+                    const uint32_t sel2 = (sl & 1) ? 0x7632u : 0x5410u;
+                    const uint32_t t0 = prmt(src[0], src[1], sel2);  // k-pair rows 0..3 of the column
+                    const uint32_t t1 = prmt(src[2], src[3], sel2);  // rows 4..7
+                    uint32_t o[4];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t x = (hh ? t1 : t0) ^ 0x88888888u;
+                        const uint32_t hi = x & 0xF0F0F0F0u;         // k = 2i
+                        const uint32_t lo = (x << 4) & 0xF0F0F0F0u;  // k = 2i + 1
+                        o[2 * hh] = prmt(hi, lo, 0x5140u);
+                        o[2 * hh + 1] = prmt(hi, lo, 0x7362u);
                     }
-#pragma unroll
-                    for (int sl = 0; sl < 4; ++sl) {
-                        const uint32_t* src = sl < 2 ? Ar : Br;
-                        const uint32_t sel2 = (sl & 1) ? 0x7632u : 0x5410u;
-                        const uint32_t t0 = prmt(src[0], src[1], sel2);  // k-pair rows 0..3 of the column
-                        const uint32_t t1 = prmt(src[2], src[3], sel2);  // rows 4..7
-                        uint32_t o[4];
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            // each nibble c -> int8 16 (c - 8): flip bit 3, keep it in the high half of the byte
-                            const uint32_t x = (h ? t1 : t0) ^ 0x88888888u;
-                            const uint32_t hi = x & 0xF0F0F0F0u;         // k = 2i
-                            const uint32_t lo = (x << 4) & 0xF0F0F0F0u;  // k = 2i + 1
-                            o[2 * h] = prmt(hi, lo, 0x5140u);
-                            o[2 * h + 1] = prmt(hi, lo, 0x7362u);
-                        }
-                        const int n = 4 * w4_q + ((w4_rot + sl) & 3);
-                        st_shared_v4(dst + swz128(n, u), o[0], o[1], o[2], o[3]);
-                    }
+                    const int n = 4 * w4_q + ((w4_rot + sl) & 3);
+                    st_shared_v4(dst + swz128(n, u), o[0], o[1], o[2], o[3]);
                 }
             } else {
-                // raw[n][32 bytes]: 64 LSB-first 4-bit codes of row n, k = k0 .. k0+63
-                const int k0 = (it % nk) * Cfg::KE;
-                // the two 16-byte halves in an order that keeps each 8-lane phase on distinct banks
-                const int u0 = (r >> 2) & 1;
-                const uint4 first = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * u0);
-                const uint4 second = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * (u0 ^ 1));
-                const uint4 half[2] = {u0 ? second : first, u0 ? first : second};
+                // raw[n][32 bytes]: 64 LSB-first 4-bit codes of row n; this thread: k0 + 32h .. +31.
+                // A pair of codes (q, q') of one byte becomes bf16x2 in four instructions: PRMT puts
+                // the byte (low half) and the byte of w >> 1 (high half) in place, one LOP3 makes the
+                // exact bf16 (128 + q, 128 + 8 q'), one bf16x2 FMA recovers (q, q') exactly, and one
+                // gives bf16(s q + b), the exact value rounded once.
+                const int k0 = kb * Cfg::KE + 32 * h;
+                const uint4 cw = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * h);
+                const uint32_t s2 = prmt(pr[0], pr[0], 0x1010u), b2 = prmt(pr[1], pr[1], 0x1010u);
+                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    // group of k0 + 32h .. k0 + 32h + 31
-                    const float s = __uint_as_float(pr[2 * h] << 16), b = __uint_as_float(pr[2 * h + 1] << 16);
-                    const uint32_t words[4] = {half[h].x, half[h].y, half[h].z, half[h].w};
+                for (int w = 0; w < 4; ++w) {  // word w: k = k0 + 8w .. +7 -> unit 4h + w
+                    const uint32_t w1 = words[w] >> 1;
+                    uint32_t o[4];
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {  // word w: k = k0 + 32h + 8w .. +7 -> unit 4h + w
-                        uint32_t o[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t w0 = words[w] >> (8 * j);
-                            const float q0 = __uint_as_float(0x4B000000u | (w0 & 15u)) - 8388608.0f;
-                            const float q1 = __uint_as_float(0x4B000000u | ((w0 >> 4) & 15u)) - 8388608.0f;
-                            o[j] = pack_bf16x2(__fmaf_rn(q0, s, b), __fmaf_rn(q1, s, b));
-                        }
-                        // k beyond K: zero weights (the activations there are zero too)
-                        if (k0 + 32 * h + 8 * w >= p.K)
-                            o[0] = o[1] = o[2] = o[3] = 0u;
-                        st_shared_v4(dst + swz128(r, 4 * h + w), o[0], o[1], o[2], o[3]);
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t sel = (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12));
+                        const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x43004300u);
+                        const uint32_t q = bf16x2_fma(v, 0x3E003F80u, 0xC180C300u);  // (1, 1/8), (-128, -16)
+                        o[j] = bf16x2_fma(q, s2, b2);
                     }
+                    // k beyond K: zero weights (the activations there are zero too)
+                    if (k0 + 8 * w >= p.K)
+                        o[0] = o[1] = o[2] = o[3] = 0u;
+                    st_shared_v4(dst + swz128(r, 4 * h + w), o[0], o[1], o[2], o[3]);
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars.bfull[it & 1]);
+                mbar_arrive(&bars.bfull[it % kBDepth]);
             return true;
         };
-        // three parameter sets rotate so that each is loaded two stages before its use
-        unsigned P0[4] = {0u, 0u, 0u, 0u}, P1[4] = {0u, 0u, 0u, 0u}, P2[4] = {0u, 0u, 0u, 0u};
-        if constexpr (BSRC == B_AFFINE4) {
-            load_params(0, P0);
-            load_params(1, P1);
-        }
         bool ok = true;
-        for (int it = 0; it < total && ok; it += 3) {
+        int ti = 0, kb = 0;  // tile and k block of stage it (no divisions in the loop)
+        for (int it = 0; it < total && ok; ++it) {
+            unsigned pr[2] = {0u, 0u};
             if constexpr (BSRC == B_AFFINE4)
-                load_params(it + 2, P2);
-            ok = stage(it, P0);
-            if (!ok || it + 1 >= total)
-                break;
-            if constexpr (BSRC == B_AFFINE4)
-                load_params(it + 3, P0);
-            ok = stage(it + 1, P1);
-            if (!ok || it + 2 >= total)
-                break;
-            if constexpr (BSRC == B_AFFINE4)
-                load_params(it + 4, P1);
-            ok = stage(it + 2, P2);
+                params_for(ti, kb, pr);
+            ok = stage(it, kb, pr);
+            if (++kb == nk) {
+                kb = 0;
+                ++ti;
+            }
         }
         if (!ok)
             bars.abort_flag = 1;
@@ -563,9 +604,13 @@ cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const 
     prm.scales = static_cast<const __nv_bfloat16*>(a.scales);
     prm.biases = static_cast<const __nv_bfloat16*>(a.biases);
     prm.g = a.g;
+    prm.g_shift = 0;
+    while (a.g > 0 && (1 << prm.g_shift) < a.g)
+        ++prm.g_shift;
     prm.vec_sw = aligned16p(a.s_w);
     prm.vec_bias = aligned16p(a.bias);
     prm.vec_out = aligned16p(a.out);
+    prm.vec_params = a.g > 0 && (a.K / a.g) % 8 == 0 && aligned16p(a.scales) && aligned16p(a.biases);
     prm.status = dev.status;
     const bool bf16_a = op == TC_AFFINE4;
     const uint64_t a_pitch = (uint64_t)a.K * (bf16_a ? 2 : 1);

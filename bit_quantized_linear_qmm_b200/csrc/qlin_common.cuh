@@ -72,6 +72,9 @@ QLIN_DEV void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes)
                  : "memory");
 }
 
+#ifndef QLIN_MBAR_SUSPEND_NS
+#define QLIN_MBAR_SUSPEND_NS 1000000u
+#endif
 // Suspends the thread (up to a hint of 1 ms, or until the phase completes)
 // instead of spinning, so waiting warps leave the issue slots to the others.
 QLIN_DEV bool mbar_try_wait(uint64_t* bar, unsigned parity)
@@ -80,7 +83,7 @@ QLIN_DEV bool mbar_try_wait(uint64_t* bar, unsigned parity)
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(QLIN_MBAR_SUSPEND_NS)
         : "memory");
     return ok != 0;
 }
