@@ -201,7 +201,7 @@ def _copies(bytes_per_copy: int, l2_bytes: int, minimum: int = 2) -> int:
 class BitlinearDecode:
     """BitLinear ternary decode GEMV: x bf16 [M, 4096], packed uint8 [1024, 4096],
     M in {1, 8}, weight_scale 0.5, multiply and divide modes; no bias."""
-    key = "bitlinear_gemv_kernel"
+    key = "bitlinear_reg_kernel"
     unit = "GB/s"
     bound = "hbm"
 
@@ -468,6 +468,7 @@ PROFILE_CASES = {
     "bitlinear_m1": lambda: _prof_bitlinear(1),
     "bitlinear_m8": lambda: _prof_bitlinear(8),
     "affine_decode_m1": lambda: _prof_affine(1, 4096, 4096),
+    "affine_decode_m1_k11008": lambda: _prof_affine(1, 11008, 4096),
     "affine_prefill_m512": lambda: _prof_affine(512, 4096, 14336),
     "w8a8_m4096": lambda: _prof_int("w8a8", 4096),
     "w4a8_m4096": lambda: _prof_int("w4a8", 4096),

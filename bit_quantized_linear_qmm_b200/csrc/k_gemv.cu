@@ -16,11 +16,12 @@
 //    ring with 2-D tensor-map TMA (cp.async.bulk.tensor, 128-byte swizzle,
 //    completion on mbarriers): one instruction moves a 128-byte column block
 //    of all the CTA's weight rows, one the same columns of the M token rows
-//    of x (the remaining token rows of the ring stay zero).  Each kernel
-//    prefetches its first stages into L2 before griddepcontrol.wait, so a
-//    layer's DRAM fetch overlaps the previous layer's tail.  Eight consumer
-//    warps split K (whole groups round robin); each covers all the CTA's
-//    16-row tiles, so every x fragment serves them all.
+//    of x (the remaining token rows of the ring stay zero).  The weights of
+//    the first stages (and the group parameters) are fetched before
+//    griddepcontrol.wait, the next stages prefetched into L2, so a layer's
+//    DRAM fetch overlaps the previous layer's tail.  Eight consumer warps
+//    take whole groups round robin; each covers all the CTA's 16-row tiles,
+//    so every x fragment serves them all.
 //  * bitlinear: a layer's packed weights are small enough (a few MB) for the
 //    CTAs to hold them in registers: they are loaded before
 //    griddepcontrol.wait, and only x is read after it.
@@ -54,7 +55,8 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;    // + one producer warp
 constexpr int kRowsPerCta = 16 * kRowTiles;
-constexpr int kStages = 6;                          // barrier slots; a kernel uses NS <= kStages
+constexpr int kStages = 12;                         // barrier slots; a kernel uses NS <= kStages
+constexpr int kRingBytes = 80 * 1024;               // stage ring budget: two CTAs still fit per SM
 constexpr int kRedStride = kRowsPerCta + 4;        // padded row of the partial tile (bank spread)
 
 __host__ __device__ constexpr int round_up(int a, int b) { return (a + b - 1) / b * b; }
@@ -93,30 +95,35 @@ QLIN_DEV void split_f32_pair(float a, float b, uint32_t& hi, uint32_t& lo)
 // griddepcontrol.wait only L2 prefetches of weights are issued (coherent
 // with any earlier kernel's writes); every load into shared memory follows
 // the wait.
-template <int NS, typename IssueFn, typename PFn, typename BytesFn>
-QLIN_DEV void producer_loop(Barriers& bars, int nst, unsigned* status, IssueFn issue, PFn prefetch,
+template <int NS, typename WFn, typename XFn, typename PFn, typename BytesFn>
+QLIN_DEV void producer_loop(Barriers& bars, int nst, unsigned* status, WFn issue_w, XFn issue_x, PFn prefetch,
                             BytesFn stage_bytes)
 {
     if ((threadIdx.x & 31) == 0) {
-        // let the next kernel in the stream start its own prologue and L2
-        // prefetch on whatever SM room is left
+        // let the next kernel in the stream start its own prologue on whatever
+        // SM room is left
         pdl_launch_dependents();
         const int pre = nst < NS ? nst : NS;
         const int npf = nst < 2 * NS ? nst : 2 * NS;
-        for (int it = 0; it < npf; ++it)
-            prefetch(it);
-        pdl_wait_prior_grids();
+        // the layer's constant weights: the first NS stages straight into the
+        // ring, the next NS into L2, all before the dependency wait
         for (int it = 0; it < pre; ++it) {
             mbar_arrive_expect_tx(&bars.full[it], stage_bytes(it));
-            issue(it, it);
+            issue_w(it, it);
         }
+        for (int it = pre; it < npf; ++it)
+            prefetch(it);
+        pdl_wait_prior_grids();
+        for (int it = 0; it < pre; ++it)
+            issue_x(it, it);
         int issued = pre;
         for (int it = pre; it < nst; ++it) {
             const int slot = it % NS;
             if (!mbar_wait_bounded(&bars.empty[slot], ((it / NS) & 1) ^ 1, status) || volatile_abort(bars))
                 break;
             mbar_arrive_expect_tx(&bars.full[slot], stage_bytes(it));
-            issue(it, slot);
+            issue_w(it, slot);
+            issue_x(it, slot);
             ++issued;
         }
         // Drain: no TMA load may still target this CTA's shared memory at exit.
@@ -194,7 +201,7 @@ struct AffineCfg {
     static constexpr int W_STAGE = NWB * ROWS * 128;
     static constexpr int X_STAGE = NXB * MMAX * 128;
     static constexpr int STAGE = W_STAGE + X_STAGE;       // multiple of 1024
-    static constexpr int NS = (64 * 1024 / STAGE) < 2 ? 2 : ((64 * 1024 / STAGE) > kStages ? kStages : (64 * 1024 / STAGE));
+    static constexpr int NS = (kRingBytes / STAGE) < 2 ? 2 : ((kRingBytes / STAGE) > kStages ? kStages : (kRingBytes / STAGE));
     static constexpr int CPW = 32 / BITS;                  // codes per 32-bit word
     static constexpr int WPG = G * BITS / 32;              // words per row per group
     static constexpr int WPL = WPG / 4;                    // words per lane per row per group
@@ -359,15 +366,17 @@ __global__ void __launch_bounds__(kThreads, 2) affine_gemv_kernel(const __grid_c
         producer_loop<Cfg::NS>(
             bars, nst, p.status,
             [&](int it, int slot) {
-                const int k0 = it * Cfg::KST;
                 uint8_t* wst = stages + slot * Cfg::STAGE;
-                uint8_t* xst = wst + Cfg::W_STAGE;
 #pragma unroll
                 for (int b = 0; b < Cfg::NWB; ++b)
-                    tma_load_2d(wst + b * (ROWS * 128), &p.tm_w, k0 * BITS / 8 + b * 128, n0, &bars.full[slot]);
+                    tma_load_2d(wst + b * (ROWS * 128), &p.tm_w, it * Cfg::KST * BITS / 8 + b * 128, n0,
+                                &bars.full[slot]);
+            },
+            [&](int it, int slot) {
+                uint8_t* xst = stages + slot * Cfg::STAGE + Cfg::W_STAGE;
 #pragma unroll
                 for (int b = 0; b < Cfg::NXB; ++b)
-                    tma_load_2d(xst + b * (Cfg::MMAX * 128), &p.tm_x, k0 + b * Cfg::XE, 0, &bars.full[slot]);
+                    tma_load_2d(xst + b * (Cfg::MMAX * 128), &p.tm_x, it * Cfg::KST + b * Cfg::XE, 0, &bars.full[slot]);
             },
             [&](int it) {
 #pragma unroll
@@ -378,42 +387,46 @@ __global__ void __launch_bounds__(kThreads, 2) affine_gemv_kernel(const __grid_c
     } else {
         // ------------------------------------------------ consumer warps
         zero_x_tail(stages, Cfg::NS, Cfg::STAGE, Cfg::W_STAGE, Cfg::NXB, Cfg::MMAX, M);
-        // group parameters of the CTA's rows -> smem as {s, b - OFFSET s}: all loads of a
-        // batch issued before its stores
+        // group parameters of the CTA's rows -> smem as {s, b - OFFSET s}.  They are constants of
+        // the layer, like the packed weights, so they are read before griddepcontrol.wait: one
+        // 16-byte vector per thread and batch (the CTA's parameters are contiguous).
         {
-            const PT* sc = static_cast<const PT*>(p.scales);
-            const PT* bi = static_cast<const PT*>(p.biases);
-            const int pbytes = rows_valid * ng * (int)sizeof(PT);  // the CTA's params are contiguous
-            for (int off = threadIdx.x * 128; off < pbytes; off += kConsumerThreads * 128) {
-                prefetch_l2(reinterpret_cast<const uint8_t*>(sc + (size_t)n0 * ng) + off);
-                prefetch_l2(reinterpret_cast<const uint8_t*>(bi + (size_t)n0 * ng) + off);
-            }
-            pdl_wait_prior_grids();
-            constexpr int B = 8;
-            for (int e0 = threadIdx.x; e0 < ROWS * ng; e0 += B * kConsumerThreads) {
-                PT sv[B], bv[B];
+            const PT* sc = static_cast<const PT*>(p.scales) + (size_t)n0 * ng;
+            const PT* bi = static_cast<const PT*>(p.biases) + (size_t)n0 * ng;
+            constexpr int VE = 16 / (int)sizeof(PT);
+            const int total = rows_valid * ng;
+            const bool vec = ((reinterpret_cast<uintptr_t>(sc) | reinterpret_cast<uintptr_t>(bi)) & 15u) == 0;
+#pragma unroll 4
+            for (int c = threadIdx.x; c * VE < ROWS * ng; c += kConsumerThreads) {
+                const int e0 = c * VE;
+                float sv[VE], bv[VE];
+                if (vec && e0 + VE <= total) {
+                    const uint4 s4 = ldg_stream_v4(sc + e0), b4 = ldg_stream_v4(bi + e0);
+                    const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w}, bw[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                for (int i = 0; i < B; ++i) {
-                    const int e = e0 + i * kConsumerThreads;
-                    if (e < rows_valid * ng) {
-                        sv[i] = sc[(size_t)n0 * ng + e];
-                        bv[i] = bi[(size_t)n0 * ng + e];
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < B; ++i) {
-                    const int e = e0 + i * kConsumerThreads;
-                    if (e < ROWS * ng) {
-                        float s = 0.f, b = 0.f;
-                        if (e < rows_valid * ng) {
-                            s = to_float(sv[i]);
-                            b = to_float(bv[i]);
+                    for (int e = 0; e < VE; ++e) {
+                        if constexpr (sizeof(PT) == 2) {  // bf16: two per word, low half first
+                            sv[e] = __uint_as_float((sw[e >> 1] >> (16 * (e & 1))) << 16);
+                            bv[e] = __uint_as_float((bw[e >> 1] >> (16 * (e & 1))) << 16);
+                        } else {
+                            sv[e] = __uint_as_float(sw[e]);
+                            bv[e] = __uint_as_float(bw[e]);
                         }
-                        params[e] = make_float2(s, fmaf(-Cfg::OFFSET, s, b));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) {
+                        sv[e] = e0 + e < total ? to_float(sc[e0 + e]) : 0.f;
+                        bv[e] = e0 + e < total ? to_float(bi[e0 + e]) : 0.f;
                     }
                 }
+#pragma unroll
+                for (int e = 0; e < VE; ++e)
+                    if (e0 + e < ROWS * ng)
+                        params[e0 + e] = make_float2(sv[e], fmaf(-Cfg::OFFSET, sv[e], bv[e]));
             }
         }
+        pdl_wait_prior_grids();  // x, y and the bias may belong to the previous kernel
         consumer_bar();
 
         // every warp covers all RT row tiles (sharing each x fragment and the
