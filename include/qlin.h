@@ -29,6 +29,17 @@
  *     qlin_workspace_size()).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and never synchronise, except qlin_get_device_status().
+ *   - Ordering on a stream: the GEMV / GEMM kernels (qlin_matmul,
+ *     bitlinear_matmul, w8a8_linear, w8a8_linear_noalloc, w4a8_linear,
+ *     qlin_int8_matmul_int32) use programmatic dependent launch: each releases
+ *     the next kernel of the stream when it starts, and that kernel fetches
+ *     its layer constants -- packed weights and group scales / biases --
+ *     before waiting for its predecessor (x, the BitLinear weight scale, the
+ *     layer bias and y only after).  So the packed weights and group
+ *     parameters of a call must not be written by the call immediately
+ *     before it on the same stream if that call is one of the above.  Any
+ *     other predecessor (a quantize or pack call, a copy, another library's
+ *     kernel) completes before the call starts.
  *   - Every call validates its arguments before launching anything and
  *     returns a qlin_status; nothing is launched when it is not QLIN_OK.
  *     No C++ exception crosses this interface.
@@ -116,8 +127,8 @@ qlin_status qlin_dequantize(const uint32_t* codes, const void* scales, const voi
  * computed from the packed weight, its scales and biases].
  * x: [M, K] of x_dt (which is also the dtype of bias and y).  bias: [N] or
  * NULL.  y: [M, N].  M <= 16 runs the decode kernel (bulk-copy streamed
- * codes, register dequantisation, tensor-core MACs, split-K reduced through
- * cluster shared memory); larger M runs the prefill GEMM (codes dequantised
+ * codes, register dequantisation, tensor-core MACs, partial sums reduced
+ * inside the CTA); larger M runs the prefill GEMM (codes dequantised
  * to bf16 in shared memory feeding tcgen05 MMA with fp32 accumulation in
  * tensor memory).  Requires (K*bits/8) % 16 == 0 and, for x, (K*sizeof(x_dt))
  * % 16 == 0.  `workspace` may be NULL when qlin_workspace_size() is 0.
