@@ -544,6 +544,161 @@ __global__ void __launch_bounds__(kThreads, 2) affine_gemv_kernel(const __grid_c
     }
 }
 
+// ---------------------------------------------------------------- W8A8 decode kernel
+
+// y[m,n] = (float)(sum_k qx[m,k] * w[n,k]) * s_x[m] * s_w[n] + bias[n]
+// [cider/ops.py perchannel_linear], M <= 16.  The same pipeline as the affine
+// decode kernel (TMA stage ring fed by one producer thread, the weights of the
+// first stages fetched before griddepcontrol.wait), with no dequantisation:
+// int8 weights and int8 activations go straight into mma.m16n8k32.s8 (int32
+// accumulation, exact).  Warps take k32 steps round robin; the partial int32
+// tiles are summed in any order (exact) through shared memory.
+template <int NT, int RT>
+struct W8Cfg {
+    static constexpr int ROWS = 16 * RT;
+    static constexpr int KST = RT == 4 ? 256 : 512;  // k per stage (a ring of at least 3 stages)
+    static constexpr int NWB = KST / 128;            // 128-byte weight boxes per stage
+    static constexpr int NXB = KST / 128;            // 128-byte x boxes per stage
+    static constexpr int MMAX = 8 * NT;
+    static constexpr int W_STAGE = NWB * ROWS * 128;
+    static constexpr int X_STAGE = NXB * MMAX * 128;
+    static constexpr int STAGE = W_STAGE + X_STAGE;  // multiple of 1024
+    static constexpr int NS = (kRingBytes / STAGE) < 2 ? 2 : ((kRingBytes / STAGE) > kStages ? kStages : (kRingBytes / STAGE));
+    static constexpr int SMEM = NS * STAGE + (int)sizeof(Barriers) + 1024;
+    static_assert(STAGE % 1024 == 0, "swizzled boxes need 1024-byte alignment");
+    static_assert(kConsumerWarps * RT * NT * 4 * 32 * 4 <= NS * STAGE, "reduction scratch fits the ring");
+};
+
+struct W8Params {
+    CUtensorMap tm_w;  // w [N][K] int8, box {128 B, ROWS rows}
+    CUtensorMap tm_x;  // qx [M][K] int8, box {128 B, M rows}
+    const float* s_x;
+    const float* s_w;
+    const __nv_bfloat16* bias;
+    __nv_bfloat16* y;
+    int M, K, N;
+    unsigned* status;
+};
+
+template <int NT, int RT>
+__global__ void __launch_bounds__(kThreads, 2) w8_gemv_kernel(const __grid_constant__ W8Params p)
+{
+    using Cfg = W8Cfg<NT, RT>;
+    constexpr int ROWS = Cfg::ROWS;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    Barriers& bars = *reinterpret_cast<Barriers*>(smem + Cfg::NS * Cfg::STAGE);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * ROWS;
+    const int nst = (p.K + Cfg::KST - 1) / Cfg::KST;
+    const int M = p.M;
+
+    init_barriers(bars);
+
+    if (warp == kConsumerWarps) {
+        producer_loop<Cfg::NS>(
+            bars, nst, p.status,
+            [&](int it, int slot) {
+                uint8_t* wst = stages + slot * Cfg::STAGE;
+#pragma unroll
+                for (int b = 0; b < Cfg::NWB; ++b)
+                    tma_load_2d(wst + b * (ROWS * 128), &p.tm_w, it * Cfg::KST + b * 128, n0, &bars.full[slot]);
+            },
+            [&](int it, int slot) {
+                uint8_t* xst = stages + slot * Cfg::STAGE + Cfg::W_STAGE;
+#pragma unroll
+                for (int b = 0; b < Cfg::NXB; ++b)
+                    tma_load_2d(xst + b * (Cfg::MMAX * 128), &p.tm_x, it * Cfg::KST + b * 128, 0, &bars.full[slot]);
+            },
+            [&](int it) {
+#pragma unroll
+                for (int b = 0; b < Cfg::NWB; ++b)
+                    tma_prefetch_2d(&p.tm_w, it * Cfg::KST + b * 128, n0);
+            },
+            [&](int) { return (unsigned)(Cfg::W_STAGE + Cfg::NXB * M * 128); });
+    } else {
+        // ------------------------------------------------ consumer warps
+        zero_x_tail(stages, Cfg::NS, Cfg::STAGE, Cfg::W_STAGE, Cfg::NXB, Cfg::MMAX, M);
+        consumer_bar();
+        const int gid = lane >> 2, tig = lane & 3;
+        int acc[RT][NT][4];
+#pragma unroll
+        for (int i = 0; i < RT; ++i)
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[i][t][e] = 0;
+        for (int it = 0; it < nst; ++it) {
+            const int slot = it % Cfg::NS;
+            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status)) {
+                bars.abort_flag = 1;
+                break;
+            }
+            const uint8_t* wst = stages + slot * Cfg::STAGE;
+            const uint8_t* xst = wst + Cfg::W_STAGE;
+            // k past K reads the zeros the TMA wrote, in both operands
+            const int steps = (min(Cfg::KST, p.K - it * Cfg::KST) + 31) / 32;
+            for (int st = warp; st < steps; st += kConsumerWarps) {
+                const int wi = st * 8;  // first 32-bit word of this k32 step in the stage row
+                uint32_t b0[NT], b1[NT];
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    b0[t] = *reinterpret_cast<const uint32_t*>(x_addr<int8_t, Cfg::MMAX>(xst, t * 8 + gid, 32 * st + 4 * tig));
+                    b1[t] = *reinterpret_cast<const uint32_t*>(
+                        x_addr<int8_t, Cfg::MMAX>(xst, t * 8 + gid, 32 * st + 16 + 4 * tig));
+                }
+#pragma unroll
+                for (int i = 0; i < RT; ++i) {
+                    uint32_t a[4];
+                    a[0] = w_word(wst, ROWS, i * 16 + gid, wi + tig);
+                    a[1] = w_word(wst, ROWS, i * 16 + gid + 8, wi + tig);
+                    a[2] = w_word(wst, ROWS, i * 16 + gid, wi + 4 + tig);
+                    a[3] = w_word(wst, ROWS, i * 16 + gid + 8, wi + 4 + tig);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t)
+                        mma_s8_16832(acc[i][t], a, b0[t], b1[t]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars.empty[slot]);
+        }
+        // sum the warps' partial tiles (int32: exact in any order); the idle stage ring is the scratch
+        consumer_bar();
+        int* scratch = reinterpret_cast<int*>(stages);
+        constexpr int V = RT * NT * 4;
+#pragma unroll
+        for (int i = 0; i < RT; ++i)
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    scratch[(warp * V + (i * NT + t) * 4 + e) * 32 + lane] = acc[i][t][e];
+        consumer_bar();
+        pdl_wait_prior_grids();  // s_x comes from the activation quantiser; y and bias after it too
+        for (int idx = threadIdx.x; idx < V * 32; idx += kConsumerThreads) {
+            const int v = idx >> 5, ln = idx & 31;
+            int sum = 0;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w)
+                sum += scratch[(w * V + v) * 32 + ln];
+            const int i = v / (NT * 4), t = (v / 4) % NT, e = v % 4;
+            const int row = i * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
+            const int tok = t * 8 + 2 * (ln & 3) + (e & 1);
+            const int n = n0 + row;
+            if (tok < M && n < p.N) {
+                float out = (float)sum * (p.s_x[tok] * p.s_w[n]);
+                if (p.bias)
+                    out += __bfloat162float(p.bias[n]);
+                p.y[(size_t)tok * p.N + n] = __float2bfloat16_rn(out);
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- bf16x2 helper
 
 QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
@@ -894,6 +1049,41 @@ cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const
             e = launch_pdl_threads(bitlinear_reg_kernel<1, 4, false>, grid, kBlThreads, 0, st, prm);
         else
             e = launch_pdl_threads(bitlinear_reg_kernel<2, 2, false>, grid, kBlThreads, 0, st, prm);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
+
+cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
+{
+    const bool wide = a.N / 64 >= dev.sm_count;  // 64-row CTAs when they still fill the GPU
+    for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
+        const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
+        W8Params prm;
+        prm.s_x = a.s_x + m0;
+        prm.s_w = a.s_w;
+        prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
+        prm.y = static_cast<__nv_bfloat16*>(a.y) + m0 * a.N;
+        prm.M = mc;
+        prm.K = (int)a.K;
+        prm.N = (int)a.N;
+        prm.status = dev.status;
+        const int rows = mc <= 8 && wide ? 64 : 32;
+        if (!encode_tmap_2d(&prm.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K,
+                            128, (uint32_t)rows) ||
+            !encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx + m0 * a.K, (uint64_t)a.K, (uint64_t)mc,
+                            (uint64_t)a.K, 128, (uint32_t)mc))
+            return cudaErrorInvalidValue;
+        const dim3 grid((unsigned)((a.N + rows - 1) / rows), 1, 1);
+        cudaError_t e;
+        if (mc <= 8 && wide)
+            e = launch_pdl(w8_gemv_kernel<1, 4>, grid, W8Cfg<1, 4>::SMEM, st, prm);
+        else if (mc <= 8)
+            e = launch_pdl(w8_gemv_kernel<1, 2>, grid, W8Cfg<1, 2>::SMEM, st, prm);
+        else
+            e = launch_pdl(w8_gemv_kernel<2, 2>, grid, W8Cfg<2, 2>::SMEM, st, prm);
         if (e != cudaSuccess)
             return e;
     }

@@ -125,8 +125,10 @@ __global__ void __launch_bounds__(256) affine_dequantize_kernel(const uint32_t* 
 template <typename TW>
 __global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __restrict__ w, int64_t C,
                                                                  int8_t* __restrict__ q, float* __restrict__ scale,
-                                                                 int32_t* __restrict__ rowsum)
+                                                                 int32_t* __restrict__ rowsum, int release)
 {
+    if (release)
+        pdl_launch_dependents();
     __shared__ float red[8];
     __shared__ int ired[8];
     const int64_t r = blockIdx.x;
@@ -177,8 +179,10 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __res
 __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __nv_bfloat16* __restrict__ w,
                                                                         int64_t C, int8_t* __restrict__ q,
                                                                         float* __restrict__ scale,
-                                                                        int32_t* __restrict__ rowsum)
+                                                                        int32_t* __restrict__ rowsum, int release)
 {
+    if (release)
+        pdl_launch_dependents();
     __shared__ float red[8];
     __shared__ int ired[8];
     const int64_t r = blockIdx.x;
@@ -354,18 +358,22 @@ cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, 
 }
 
 cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
-                                      int32_t* rowsum, cudaStream_t st, const DeviceInfo&)
+                                      int32_t* rowsum, cudaStream_t st, const DeviceInfo&, bool release_dependents)
 {
+    // The kernel itself starts only after its predecessor completes; with
+    // release_dependents it lets the next (programmatic-dependent) kernel start
+    // its prologue early -- that kernel waits before reading q and scale.
+    const int rel = release_dependents ? 1 : 0;
     if (w_dt == QLIN_BF16 && C % 8 == 0 && (reinterpret_cast<uintptr_t>(w) & 15) == 0 &&
         (reinterpret_cast<uintptr_t>(q) & 7) == 0)
         quantize_int8_rows_bf16x8_kernel<<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
-                                                                       scale, rowsum);
+                                                                       scale, rowsum, rel);
     else if (w_dt == QLIN_BF16)
         quantize_int8_rows_kernel<__nv_bfloat16>
-            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q, scale, rowsum);
+            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q, scale, rowsum, rel);
     else
         quantize_int8_rows_kernel<float><<<(unsigned)R, 256, 0, st>>>(static_cast<const float*>(w), C, q, scale,
-                                                                      rowsum);
+                                                                      rowsum, rel);
     return cudaGetLastError();
 }
 

@@ -323,9 +323,23 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
     int8_t* qx = static_cast<int8_t*>(workspace);
     float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)M * (size_t)K));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, nullptr, st, dev);
+    // the quantiser lets the next kernel start its prologue (fetching the layer's weights) early
+    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, nullptr, st, dev, true);
     if (e != cudaSuccess)
         return from_cuda(e);
+    if (op == TC_W8A8 && M <= 16) {  // decode: weight-streaming GEMV on int8 mma.sync
+        W8GemvArgs g;
+        g.qx = qx;
+        g.s_x = sx;
+        g.w = static_cast<const int8_t*>(w);
+        g.s_w = scale_w;
+        g.bias = bias;
+        g.y = y;
+        g.M = M;
+        g.K = K;
+        g.N = N;
+        return from_cuda(launch_w8_gemv(g, st, dev));
+    }
     TcGemmArgs t = {};
     t.M = M;
     t.N = N;

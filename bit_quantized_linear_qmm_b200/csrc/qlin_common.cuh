@@ -414,7 +414,7 @@ cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, 
                                      qlin_dtype p_dt, int64_t N, int64_t K, int bits, int g, void* out,
                                      qlin_dtype o_dt, cudaStream_t st, const DeviceInfo& dev);
 cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
-                                      float* scale, int32_t* rowsum, cudaStream_t st, const DeviceInfo& dev);
+                                      float* scale, int32_t* rowsum, cudaStream_t st, const DeviceInfo& dev, bool release_dependents = false);
 cudaError_t launch_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64_t N, uint8_t* packed,
                                   float* scale, cudaStream_t st, const DeviceInfo& dev);
 
@@ -431,6 +431,18 @@ struct AffineGemvArgs {
     void* y;
 };
 cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
+
+// int8 decode GEMV (M <= 16): y = (float)(qx . w) * s_x[m] * s_w[n] + bias[n], bf16 out
+struct W8GemvArgs {
+    const int8_t* qx;  // [M][K]
+    const float* s_x;  // [M]
+    const int8_t* w;   // [N][K]
+    const float* s_w;  // [N]
+    const void* bias;  // bf16 [N] or NULL
+    void* y;           // bf16 [M][N]
+    int64_t M, K, N;
+};
+cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
 
 struct BitlinearArgs {
     const void* x;

@@ -64,9 +64,13 @@ def _w4a8(ql, orc, case, cols=None):
 
 SMALL = [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
          [(1, 256, 128), (3, 512, 272), (17, 1024, 384), (200, 768, 144), (256, 4096, 256)]]
+# W8A8 decode GEMV edges (W4A8 needs K % 32 == 0 and N % 16 == 0): two token tiles,
+# a k32 step half past K, rows past N
+SMALL_W8 = SMALL + [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
+                    [(16, 272, 100), (9, 1040, 64), (8, 4096, 520)]]
 
 
-@pytest.mark.parametrize("case", SMALL, ids=[c.name for c in SMALL])
+@pytest.mark.parametrize("case", SMALL_W8, ids=[c.name for c in SMALL_W8])
 @pytest.mark.parametrize("bias", [False, True])
 def test_w8a8_small(ql, orc, case, bias):
     _w8a8(ql, orc, case, bias=bias)
