@@ -699,6 +699,165 @@ __global__ void __launch_bounds__(kThreads, 2) w8_gemv_kernel(const __grid_const
     }
 }
 
+// ---------------------------------------------------------------- W4A8 decode kernel
+
+// y[m,n] = (float)(sum_k qx[m,k] * (c[k,n] - 8)) * s_x[m] * s_w[n] (+ bias[n])
+// [cider/ops.py w4a8_linear, pack_weight_int4], M <= 16.  The packed weights
+// are [K/2][N] bytes (N contiguous, high nibble = even k); a CTA streams a
+// 64-column strip through the TMA stage ring (boxes of 64 bytes x 256 k-pair
+// rows).  Per k32 step a lane reads four 32-bit words -- columns 4g .. 4g+3 of
+// k-pair rows 4t .. 4t+3 -- and turns them with PRMT into the int8 A
+// fragments of two 16-row tiles (columns 4g, 4g+1 and 4g+2, 4g+3 as rows g,
+// g+8), each nibble c as 16 (c - 8) (bit 3 flipped, kept in the high half of
+// the byte); the MMA's k slots 4t .. 4t+3 / 16+4t .. 16+4t+3 stand for
+// k = 8t .. 8t+3 / 8t+4 .. 8t+7, so x is one 8-byte read.  The exact int32
+// sum is shifted back by 4 bits in the epilogue.
+template <int NT>
+struct W4Cfg {
+    static constexpr int COLS = 64;                   // output columns per CTA
+    static constexpr int KP = 256;                    // k-pair rows per stage (512 k)
+    static constexpr int KST = 2 * KP;
+    static constexpr int NXB = KST / 128;             // 128-byte x boxes per stage
+    static constexpr int MMAX = 8 * NT;
+    static constexpr int W_STAGE = KP * COLS;         // 16 KB
+    static constexpr int X_STAGE = NXB * MMAX * 128;
+    static constexpr int STAGE = W_STAGE + X_STAGE;   // multiple of 1024
+    static constexpr int NS = (kRingBytes / STAGE) < 2 ? 2 : ((kRingBytes / STAGE) > kStages ? kStages : (kRingBytes / STAGE));
+    static constexpr int V = 2 * NT * 4;              // accumulators per lane
+    static constexpr int SMEM = NS * STAGE + (int)sizeof(Barriers) + 1024;
+    static_assert(STAGE % 1024 == 0, "swizzled x boxes need 1024-byte alignment");
+    static_assert(kConsumerWarps * V * 32 * 4 <= NS * STAGE, "reduction scratch fits the ring");
+};
+
+struct W4Params {
+    CUtensorMap tm_w;  // packed [K/2][N] bytes, box {64 B, 256 rows}, no swizzle
+    CUtensorMap tm_x;  // qx [M][K] int8, box {128 B, M rows}
+    const float* s_x;
+    const float* s_w;
+    const __nv_bfloat16* bias;
+    __nv_bfloat16* y;
+    int M, K, N;
+    unsigned* status;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 2) w4_gemv_kernel(const __grid_constant__ W4Params p)
+{
+    using Cfg = W4Cfg<NT>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    Barriers& bars = *reinterpret_cast<Barriers*>(smem + Cfg::NS * Cfg::STAGE);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c0 = blockIdx.x * Cfg::COLS;
+    const int nst = (p.K + Cfg::KST - 1) / Cfg::KST;
+    const int M = p.M;
+
+    init_barriers(bars);
+
+    if (warp == kConsumerWarps) {
+        producer_loop<Cfg::NS>(
+            bars, nst, p.status,
+            [&](int it, int slot) {
+                tma_load_2d(stages + slot * Cfg::STAGE, &p.tm_w, c0, it * Cfg::KP, &bars.full[slot]);
+            },
+            [&](int it, int slot) {
+                uint8_t* xst = stages + slot * Cfg::STAGE + Cfg::W_STAGE;
+#pragma unroll
+                for (int b = 0; b < Cfg::NXB; ++b)
+                    tma_load_2d(xst + b * (Cfg::MMAX * 128), &p.tm_x, it * Cfg::KST + b * 128, 0, &bars.full[slot]);
+            },
+            [&](int it) { tma_prefetch_2d(&p.tm_w, c0, it * Cfg::KP); },
+            [&](int) { return (unsigned)(Cfg::W_STAGE + Cfg::NXB * M * 128); });
+    } else {
+        // ------------------------------------------------ consumer warps
+        zero_x_tail(stages, Cfg::NS, Cfg::STAGE, Cfg::W_STAGE, Cfg::NXB, Cfg::MMAX, M);
+        consumer_bar();
+        const int gid = lane >> 2, tig = lane & 3;
+        const int cg = warp & 1;   // 32-column group of the strip
+        const int kw = warp >> 1;  // k32 steps kw, kw + 4, ... of every stage
+        int acc[2][NT][4];
+#pragma unroll
+        for (int t2 = 0; t2 < 2; ++t2)
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[t2][t][e] = 0;
+        for (int it = 0; it < nst; ++it) {
+            const int slot = it % Cfg::NS;
+            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status)) {
+                bars.abort_flag = 1;
+                break;
+            }
+            const uint32_t* raw32 = reinterpret_cast<const uint32_t*>(stages + slot * Cfg::STAGE);
+            const uint8_t* xst = stages + slot * Cfg::STAGE + Cfg::W_STAGE;
+            // k past K: the TMA wrote zero codes and zero activations
+            const int steps = (min(Cfg::KST, p.K - it * Cfg::KST) + 31) / 32;
+            for (int st = kw; st < steps; st += 4) {
+                uint32_t W[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    W[j] = raw32[(16 * st + 4 * tig + j) * (Cfg::COLS / 4) + 8 * cg + gid];
+                uint32_t a[2][4];  // [tile][fragment register]
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // k-pair rows (0,1) -> slots 4t.., rows (2,3) -> slots 16+4t..
+#pragma unroll
+                    for (int t2 = 0; t2 < 2; ++t2) {  // tile: columns (4g, 4g+1) or (4g+2, 4g+3)
+                        const uint32_t x = prmt(W[2 * h], W[2 * h + 1], t2 ? 0x7362u : 0x5140u) ^ 0x88888888u;
+                        const uint32_t hi = x & 0xF0F0F0F0u;         // even k
+                        const uint32_t lo = (x << 4) & 0xF0F0F0F0u;  // odd k
+                        a[t2][2 * h] = prmt(hi, lo, 0x5140u);        // row g
+                        a[t2][2 * h + 1] = prmt(hi, lo, 0x7362u);    // row g + 8
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const uint2 xb = *reinterpret_cast<const uint2*>(x_addr<int8_t, Cfg::MMAX>(xst, t * 8 + gid, 32 * st + 8 * tig));
+#pragma unroll
+                    for (int t2 = 0; t2 < 2; ++t2) {
+                        const uint32_t fa[4] = {a[t2][0], a[t2][1], a[t2][2], a[t2][3]};
+                        mma_s8_16832(acc[t2][t], fa, xb.x, xb.y);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars.empty[slot]);
+        }
+        // sum the partial tiles of the four k warps of each column group (int32, exact)
+        consumer_bar();
+        int* scratch = reinterpret_cast<int*>(stages);
+        constexpr int V = Cfg::V;
+#pragma unroll
+        for (int t2 = 0; t2 < 2; ++t2)
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    scratch[(warp * V + (t2 * NT + t) * 4 + e) * 32 + lane] = acc[t2][t][e];
+        consumer_bar();
+        pdl_wait_prior_grids();  // s_x comes from the activation quantiser; y and bias after it too
+        for (int idx = threadIdx.x; idx < 2 * V * 32; idx += kConsumerThreads) {
+            const int g2 = idx / (V * 32), v = (idx / 32) % V, ln = idx & 31;
+            int sum = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                sum += scratch[((2 * q + g2) * V + v) * 32 + ln];
+            const int t2 = v / (NT * 4), t = (v / 4) % NT, e = v % 4;
+            const int col = c0 + 32 * g2 + 4 * (ln >> 2) + 2 * t2 + (e >= 2 ? 1 : 0);
+            const int tok = t * 8 + 2 * (ln & 3) + (e & 1);
+            if (tok < M && col < p.N) {
+                float out = (float)(sum >> 4) * (p.s_x[tok] * p.s_w[col]);
+                if (p.bias)
+                    out += __bfloat162float(p.bias[col]);
+                p.y[(size_t)tok * p.N + col] = __float2bfloat16_rn(out);
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- bf16x2 helper
 
 QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
@@ -1084,6 +1243,34 @@ cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInf
             e = launch_pdl(w8_gemv_kernel<1, 2>, grid, W8Cfg<1, 2>::SMEM, st, prm);
         else
             e = launch_pdl(w8_gemv_kernel<2, 2>, grid, W8Cfg<2, 2>::SMEM, st, prm);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
+
+cudaError_t launch_w4_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
+{
+    for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
+        const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
+        W4Params prm;
+        prm.s_x = a.s_x + m0;
+        prm.s_w = a.s_w;
+        prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
+        prm.y = static_cast<__nv_bfloat16*>(a.y) + m0 * a.N;
+        prm.M = mc;
+        prm.K = (int)a.K;
+        prm.N = (int)a.N;
+        prm.status = dev.status;
+        if (!encode_tmap_2d(&prm.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, (uint64_t)a.N, (uint64_t)(a.K / 2),
+                            (uint64_t)a.N, W4Cfg<1>::COLS, W4Cfg<1>::KP, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.qx + m0 * a.K, (uint64_t)a.K, (uint64_t)mc,
+                            (uint64_t)a.K, 128, (uint32_t)mc))
+            return cudaErrorInvalidValue;
+        const dim3 grid((unsigned)((a.N + W4Cfg<1>::COLS - 1) / W4Cfg<1>::COLS), 1, 1);
+        const cudaError_t e = mc <= 8 ? launch_pdl(w4_gemv_kernel<1>, grid, W4Cfg<1>::SMEM, st, prm)
+                                      : launch_pdl(w4_gemv_kernel<2>, grid, W4Cfg<2>::SMEM, st, prm);
         if (e != cudaSuccess)
             return e;
     }

@@ -327,7 +327,7 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
     cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, nullptr, st, dev, true);
     if (e != cudaSuccess)
         return from_cuda(e);
-    if (op == TC_W8A8 && M <= 16) {  // decode: weight-streaming GEMV on int8 mma.sync
+    if (M <= 16) {  // decode: weight-streaming GEMV on int8 mma.sync
         W8GemvArgs g;
         g.qx = qx;
         g.s_x = sx;
@@ -338,7 +338,7 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
         g.M = M;
         g.K = K;
         g.N = N;
-        return from_cuda(launch_w8_gemv(g, st, dev));
+        return from_cuda(op == TC_W8A8 ? launch_w8_gemv(g, st, dev) : launch_w4_gemv(g, st, dev));
     }
     TcGemmArgs t = {};
     t.M = M;

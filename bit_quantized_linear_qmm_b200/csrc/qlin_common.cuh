@@ -436,13 +436,15 @@ cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const D
 struct W8GemvArgs {
     const int8_t* qx;  // [M][K]
     const float* s_x;  // [M]
-    const int8_t* w;   // [N][K]
+    const int8_t* w;   // [N][K] int8 (W8), or packed [K/2][N] bytes (W4)
     const float* s_w;  // [N]
     const void* bias;  // bf16 [N] or NULL
     void* y;           // bf16 [M][N]
     int64_t M, K, N;
 };
 cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
+// int4 decode GEMV (M <= 16): the same arguments, w = packed [K/2][N] bytes
+cudaError_t launch_w4_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
 
 struct BitlinearArgs {
     const void* x;

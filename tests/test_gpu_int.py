@@ -76,7 +76,12 @@ def test_w8a8_small(ql, orc, case, bias):
     _w8a8(ql, orc, case, bias=bias)
 
 
-@pytest.mark.parametrize("case", SMALL, ids=[c.name for c in SMALL])
+# W4A8 decode GEMV edges: two token tiles with a partial 64-column strip, a partial last stage
+SMALL_W4 = SMALL + [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
+                    [(16, 1024, 112), (9, 544, 48), (1, 8192, 80)]]
+
+
+@pytest.mark.parametrize("case", SMALL_W4, ids=[c.name for c in SMALL_W4])
 def test_w4a8_small(ql, orc, case):
     _w4a8(ql, orc, case)
 
