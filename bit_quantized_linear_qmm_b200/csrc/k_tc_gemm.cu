@@ -438,13 +438,19 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             pr[1] = (bw >> (16 * (sub & 1))) & 0xFFFFu;
         };
         // one stage: RAW(slot) -> BT(it % kBDepth)
-        auto stage = [&](int it, int kb, const unsigned (&pr)[2]) -> bool {
-            const int slot = it % Cfg::NS;
-            if (!mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status) ||
-                !mbar_wait_bounded(&bars.bempty[it % kBDepth], ((it / kBDepth) & 1) ^ 1, p.status) ||
-                aborted(&bars.abort_flag))
+        // affine: the four 16-byte store offsets of this thread's half row in the swizzled operand
+        int st_off[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            st_off[w] = swz128(r, 4 * h + w);
+        // ring positions of stage it: slot / phase of the code ring, buffer / phase of the operand ring
+        int slot = 0, bslot = 0;
+        unsigned fph = 0u, bph = 0u;
+        auto stage = [&](const unsigned (&pr)[2]) -> bool {
+            if (!mbar_wait_bounded(&bars.full[slot], fph, p.status) ||
+                !mbar_wait_bounded(&bars.bempty[bslot], bph ^ 1u, p.status) || aborted(&bars.abort_flag))
                 return false;
-            uint8_t* dst = BT(it % kBDepth);
+            uint8_t* dst = BT(bslot);
             if constexpr (BSRC == B_W4) {
                 // raw[i][n]: k-pair row i (k = 2i high nibble, 2i+1 low) of column n; 64 rows x BN bytes.
                 // Eight 32-bit loads (the k-pair rows of unit u for columns 4q .. 4q+3; a warp's lanes
@@ -488,7 +494,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                 // the byte (low half) and the byte of w >> 1 (high half) in place, one LOP3 makes the
                 // exact bf16 (128 + q, 128 + 8 q'), one bf16x2 FMA recovers (q, q') exactly, and one
                 // gives bf16(s q + b), the exact value rounded once.
-                const int k0 = kb * Cfg::KE + 32 * h;
+                // codes past K are zero-filled by the copy and meet zero activations: no masking needed
                 const uint4 cw = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * h);
                 const uint32_t s2 = prmt(pr[0], pr[0], 0x1010u), b2 = prmt(pr[1], pr[1], 0x1010u);
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
@@ -503,16 +509,21 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                         const uint32_t q = bf16x2_fma(v, 0x3E003F80u, 0xC180C300u);  // (1, 1/8), (-128, -16)
                         o[j] = bf16x2_fma(q, s2, b2);
                     }
-                    // k beyond K: zero weights (the activations there are zero too)
-                    if (k0 + 8 * w >= p.K)
-                        o[0] = o[1] = o[2] = o[3] = 0u;
-                    st_shared_v4(dst + swz128(r, 4 * h + w), o[0], o[1], o[2], o[3]);
+                    st_shared_v4(dst + st_off[w], o[0], o[1], o[2], o[3]);
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars.bfull[it % kBDepth]);
+                mbar_arrive(&bars.bfull[bslot]);
+            if (++slot == Cfg::NS) {
+                slot = 0;
+                fph ^= 1u;
+            }
+            if (++bslot == kBDepth) {
+                bslot = 0;
+                bph ^= 1u;
+            }
             return true;
         };
         bool ok = true;
@@ -521,7 +532,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             unsigned pr[2] = {0u, 0u};
             if constexpr (BSRC == B_AFFINE4)
                 params_for(ti, kb, pr);
-            ok = stage(it, kb, pr);
+            ok = stage(pr);
             if (++kb == nk) {
                 kb = 0;
                 ++ti;
