@@ -1127,16 +1127,21 @@ cudaError_t affine_launch_t(const AffineGemvArgs& a, int m0, int mcount, cudaStr
 template <int BITS, int G, typename XT, typename PT>
 cudaError_t affine_launch_nt(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
-    // 64-row CTAs when that still gives about one CTA per SM, else 32-row CTAs
+    // 64-row CTAs when that still gives about one CTA per SM, 32-row CTAs, or 16-row CTAs (two
+    // working CTAs per SM) when even 32-row CTAs would leave SMs idle
     const bool wide = a.N / 64 >= dev.sm_count;
+    const bool narrow = a.N / 32 < dev.sm_count;
     for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
         const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
         cudaError_t e;
         if (mc <= 8 && sizeof(XT) == 2)
-            e = wide ? affine_launch_t<BITS, G, XT, PT, 1, 4>(a, (int)m0, mc, st, dev)
-                     : affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev);
+            e = wide     ? affine_launch_t<BITS, G, XT, PT, 1, 4>(a, (int)m0, mc, st, dev)
+                : narrow ? affine_launch_t<BITS, G, XT, PT, 1, 1>(a, (int)m0, mc, st, dev)
+                         : affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev);
         else if (mc <= 8)
             e = affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev);
+        else if (narrow && sizeof(XT) == 2)
+            e = affine_launch_t<BITS, G, XT, PT, 2, 1>(a, (int)m0, mc, st, dev);
         else
             e = affine_launch_t<BITS, G, XT, PT, 2, 2>(a, (int)m0, mc, st, dev);
         if (e != cudaSuccess)
