@@ -175,6 +175,86 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __res
     }
 }
 
+// Single-pass variant for bf16 rows with C % 8 == 0 and C <= 256 * 8 * VPT: each
+// thread keeps its VPT 16-byte pieces of the row in registers between the
+// absmax reduction and the quantisation, so the row is read from memory once.
+template <int VPT>
+__global__ void __launch_bounds__(256) quantize_int8_rows_bf16_reg_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                         int64_t C, int8_t* __restrict__ q,
+                                                                         float* __restrict__ scale,
+                                                                         int32_t* __restrict__ rowsum, int release)
+{
+    if (release)
+        pdl_launch_dependents();
+    __shared__ float red[8];
+    __shared__ int ired[8];
+    const int64_t r = blockIdx.x;
+    const uint4* row = reinterpret_cast<const uint4*>(w + r * C);
+    const int C8 = (int)(C / 8);
+    uint4 v[VPT];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int c = (int)threadIdx.x + j * 256;
+        v[j] = c < C8 ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] << 16)));
+            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] & 0xffff0000u)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x / 32] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i)
+        amax = fmaxf(amax, red[i]);
+    float s = __fdiv_rn(amax, 127.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    if (threadIdx.x == 0)
+        scale[r] = s;
+    int sum = 0;
+    uint2* qrow = reinterpret_cast<uint2*>(q + r * C);
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int c = (int)threadIdx.x + j * 256;
+        if (c < C8) {
+            const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bits = (i & 1) ? (u[i / 2] & 0xffff0000u) : (u[i / 2] << 16);
+                float t = rintf(__fdiv_rn(__uint_as_float(bits), s));
+                t = fminf(fmaxf(t, -128.0f), 127.0f);
+                const int qi = static_cast<int>(t);
+                sum += qi;
+                packed[i / 4] |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * (i % 4));
+            }
+            qrow[c] = make_uint2(packed[0], packed[1]);
+        }
+    }
+    if (rowsum) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if ((threadIdx.x & 31) == 0)
+            ired[threadIdx.x / 32] = sum;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int t = 0;
+            for (int i = 0; i < 8; ++i)
+                t += ired[i];
+            rowsum[r] = t;
+        }
+    }
+}
+
 // Vectorised variant for bf16 rows with C % 8 == 0 (16-byte loads, 8-byte stores).
 __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __nv_bfloat16* __restrict__ w,
                                                                         int64_t C, int8_t* __restrict__ q,
@@ -364,8 +444,15 @@ cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R,
     // release_dependents it lets the next (programmatic-dependent) kernel start
     // its prologue early -- that kernel waits before reading q and scale.
     const int rel = release_dependents ? 1 : 0;
-    if (w_dt == QLIN_BF16 && C % 8 == 0 && (reinterpret_cast<uintptr_t>(w) & 15) == 0 &&
-        (reinterpret_cast<uintptr_t>(q) & 7) == 0)
+    const bool vec = w_dt == QLIN_BF16 && C % 8 == 0 && (reinterpret_cast<uintptr_t>(w) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(q) & 7) == 0;
+    if (vec && C <= 256 * 8 * 4)
+        quantize_int8_rows_bf16_reg_kernel<4><<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
+                                                                          scale, rowsum, rel);
+    else if (vec && C <= 256 * 8 * 8)
+        quantize_int8_rows_bf16_reg_kernel<8><<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
+                                                                          scale, rowsum, rel);
+    else if (vec)
         quantize_int8_rows_bf16x8_kernel<<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
                                                                        scale, rowsum, rel);
     else if (w_dt == QLIN_BF16)
