@@ -473,6 +473,7 @@ PROFILE_CASES = {
     "w8a8_m4096": lambda: _prof_int("w8a8", 4096),
     "w4a8_m4096": lambda: _prof_int("w4a8", 4096),
     "w8a8_m1": lambda: _prof_int("w8a8", 1),
+    "w4a8_m1": lambda: _prof_int("w4a8", 1),
     "w8a8_m256": lambda: _prof_int("w8a8", 256),
     "w4a8_m256": lambda: _prof_int("w4a8", 256),
 }
