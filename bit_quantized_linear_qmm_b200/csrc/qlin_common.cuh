@@ -1,5 +1,5 @@
 // qlin_common.cuh -- shared device helpers of the sm_100a kernels (inline PTX
-// for mbarriers, bulk copies and the legacy warp MMA) and the internal launch
+// for mbarriers, tensor-map TMA, tcgen05 and the legacy warp MMA) and the internal launch
 // interface between the C ABI (qlin_abi.cu) and the kernel files.
 #pragma once
 
@@ -31,11 +31,6 @@ QLIN_DEV unsigned long long globaltimer_ns()
 QLIN_DEV uint32_t smem_u32(const void* p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-QLIN_DEV float bf16_bits_to_float(uint16_t h)
-{
-    return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
 
 template <typename T> QLIN_DEV float to_float(T v);
@@ -105,33 +100,9 @@ QLIN_DEV bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned* status
     }
 }
 
-// ---------------------------------------------------------------- bulk copies (1-D TMA)
+// ---------------------------------------------------------------- 16-byte global loads
 
-// Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte
-// aligned) completing as transaction bytes on `bar`.
-QLIN_DEV void bulk_g2s(void* smem_dst, const void* gmem_src, unsigned bytes, uint64_t* bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(smem_dst)),
-        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Hint: bring `bytes` (multiple of 16, 16-byte aligned) of global memory into
-// L2.  Safe before griddepcontrol.wait: L2 is the coherence point, so a later
-// load still sees any write an earlier kernel makes to these bytes.
-QLIN_DEV void bulk_prefetch_l2(const void* gmem_src, unsigned bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes) : "memory");
-}
-
-QLIN_DEV void prefetch_l2(const void* p)
-{
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
-// 16-byte global loads: read-only streaming data that is not kept in L1, and
+// Read-only streaming data that is not kept in L1, and
 // data another kernel may have written (cached in L2 only).
 QLIN_DEV uint4 ldg_stream_v4(const void* p)
 {
@@ -141,17 +112,6 @@ QLIN_DEV uint4 ldg_stream_v4(const void* p)
                  : "l"(p));
     return v;
 }
-
-// 16-byte global -> shared copy that bypasses registers and L1 (cp.async);
-// cp_async_wait_all() waits for this thread's copies.
-QLIN_DEV void cp_async16(void* smem_dst, const void* gmem_src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
-}
-
-QLIN_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-QLIN_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N> QLIN_DEV void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 QLIN_DEV uint4 ldg_cg_v4(const void* p)
 {
@@ -258,88 +218,6 @@ QLIN_DEV uint64_t umma_desc_sw128(uint32_t smem_addr)
 // Make this thread's generic-proxy shared-memory writes visible to the
 // async proxy (TMA, tensor cores).
 QLIN_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// ---------------------------------------------------------------- cluster helpers
-
-QLIN_DEV unsigned cluster_ctarank()
-{
-    unsigned r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-QLIN_DEV void cluster_sync()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-QLIN_DEV void cluster_arrive_relaxed()
-{
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-
-QLIN_DEV void cluster_wait()
-{
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-}
-
-QLIN_DEV void st_shared_cluster_v4(uint32_t addr, float4 v)
-{
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
-                 "f"(v.w)
-                 : "memory");
-}
-
-// Arrive on an mbarrier of another CTA of the cluster (remote address from
-// map_shared_rank), releasing this thread's prior writes at cluster scope.
-QLIN_DEV void mbar_remote_arrive_cluster(uint32_t remote_bar)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
-}
-
-QLIN_DEV bool mbar_try_wait_cluster(uint64_t* bar, unsigned parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// As mbar_wait_bounded, with acquire at cluster scope (for arrivals from other CTAs).
-QLIN_DEV bool mbar_wait_cluster_bounded(uint64_t* bar, unsigned parity, unsigned* status)
-{
-    if (mbar_try_wait_cluster(bar, parity))
-        return true;
-    const unsigned long long t0 = globaltimer_ns();
-    while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait_cluster(bar, parity))
-                return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(status, kStatusTimeout);
-            return false;
-        }
-    }
-}
-
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-QLIN_DEV uint32_t map_shared_rank(uint32_t local_addr, unsigned rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
-    return r;
-}
-
-QLIN_DEV float ld_shared_cluster_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
 
 // ---------------------------------------------------------------- programmatic dependent launch
 

@@ -188,6 +188,8 @@ qlin_status qlin_int8_matmul_int32(const int8_t* a, const int8_t* b, int64_t M, 
  * in fp32 and one rounding to x_dt.  x: [M, K] of x_dt; w: int8 [N, K];
  * scale_w: fp32 [N]; bias: [N] of x_dt or NULL; y: [M, N] of x_dt.
  * K % 16 == 0.  workspace >= qlin_workspace_size(QLIN_OP_W8A8, M, N, K, 0, 0).
+ * M <= 16 runs a weight-streaming GEMV (int8 mma.sync), larger M the tcgen05
+ * GEMM (int32 accumulation in tensor memory).
  */
 qlin_status w8a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const int8_t* w,
                         const float* scale_w, int64_t N, const void* bias, void* y,
@@ -199,7 +201,8 @@ qlin_status w8a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
  * nibble for even k) with weight c - 8; int32 accumulation; y = acc *
  * s_x[m] * scale_w[n] (+ bias, an extension: the page has none) rounded to
  * x_dt.  packed: uint8 [K/2, N]; other arguments as w8a8_linear.
- * K % 32 == 0, N % 16 == 0.
+ * K % 32 == 0, N % 16 == 0.  M <= 16 runs a weight-streaming GEMV, larger M
+ * the tcgen05 GEMM (the nibbles are converted to int8 in shared memory).
  */
 qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
                         const uint8_t* packed_w, const float* scale_w, int64_t N,
