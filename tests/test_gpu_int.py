@@ -15,6 +15,7 @@ def ql():
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (130, 200, 272), (256, 384, 512), (5, 1000, 4096),
+                                   (1280, 4096, 256),  # 160 tiles of 128 x 256: the wide tile path
                                    (128, 128, 16), (333, 129, 1040)])
 def test_int8_matmul_int32_bit_exact(ql, orc, M, N, K):
     rng = np.random.default_rng(M * 7 + N)
@@ -67,7 +68,8 @@ SMALL = [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
 # W8A8 decode GEMV edges (W4A8 needs K % 32 == 0 and N % 16 == 0): two token tiles,
 # a k32 step half past K, rows past N
 SMALL_W8 = SMALL + [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
-                    [(16, 272, 100), (9, 1040, 64), (8, 4096, 520)]]
+                    [(16, 272, 100), (9, 1040, 64), (8, 4096, 520),
+                     (1280, 256, 4096)]]  # the wide (128 x 256) tile path
 
 
 @pytest.mark.parametrize("case", SMALL_W8, ids=[c.name for c in SMALL_W8])
@@ -78,7 +80,8 @@ def test_w8a8_small(ql, orc, case, bias):
 
 # W4A8 decode GEMV edges: two token tiles with a partial 64-column strip, a partial last stage
 SMALL_W4 = SMALL + [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
-                    [(16, 1024, 112), (9, 544, 48), (1, 8192, 80)]]
+                    [(16, 1024, 112), (9, 544, 48), (1, 8192, 80),
+                     (1280, 256, 4096)]]  # the wide (128 x 256) tile path
 
 
 @pytest.mark.parametrize("case", SMALL_W4, ids=[c.name for c in SMALL_W4])
