@@ -4,19 +4,10 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-# Floating-point bar: |y - y_ref| <= rel * (sum_k |x_k w_k| + |bias_n|) + ABS, with
+# Floating-point bar: |y - y_ref| <= REL * (sum_k |x_k w_k| + |bias_n|) + ABS, with
 # y_ref the oracle's unrounded double result.  The |bias| term covers the
 # final rounding of a bias-dominated output.
-#
-# REL: paths whose products are exact (ternary or integer weights times bf16 or
-# int8 activations): the one rounding of the output to bf16 costs at most
-# 2^-9 |y| <= 2^-9 (sum |x w| + |b|), and fp32 accumulation a few 2^-24 more.
-#
-# REL_BF16W: the affine paths, which round each dequantised weight s*q + b to
-# bf16 before the product: that adds at most 2^-9 |x_k w_k| per term, so the
-# bound is 2 * 2^-9 = 2^-8 of the same scale, plus the fp32 accumulation slack.
 REL = 2e-3
-REL_BF16W = 4e-3
 ABS = 1e-5
 
 
@@ -58,13 +49,13 @@ def host_bits16(t: torch.Tensor) -> np.ndarray:
     return t.cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-def assert_fp_close(y_gpu: torch.Tensor, y_ref: np.ndarray, absdot: np.ndarray, bias=None, what="", rel=REL):
+def assert_fp_close(y_gpu: torch.Tensor, y_ref: np.ndarray, absdot: np.ndarray, bias=None, what=""):
     y = y_gpu.double().cpu().numpy()
     assert y.shape == y_ref.shape, (y.shape, y_ref.shape)
     scale = absdot.copy()
     if bias is not None:
         scale = scale + np.abs(np.asarray(bias, np.float64))[None, :]
-    tol = rel * scale + ABS
+    tol = REL * scale + ABS
     err = np.abs(y - y_ref)
     bad = err > tol
     if bad.any():

@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import synth
-from helpers import REL_BF16W, assert_fp_close, build_lib, params_dev, u32_dev
+from helpers import assert_fp_close, build_lib, params_dev, u32_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,7 @@ def _run_case(ql, orc, case: synth.AffineCase, rows=None):
         y = y[:, torch.as_tensor(rows, device=y.device)]
     bias_v = None if lb is None else lb.vals if rows is None else lb.vals[rows]
     yr, mag = orc.affine_matmul(x.vals, codes, s, b, case.bits, case.group_size, bias_v)
-    return assert_fp_close(y, yr, mag, bias_v, case.name, rel=REL_BF16W)
+    return assert_fp_close(y, yr, mag, bias_v, case.name)
 
 
 SMALL = [
@@ -84,7 +84,7 @@ PREFILL_SMALL = [
                          # K % 64 == 32 (half of the last stage past K) and K/g % 8 != 0 (scalar parameter windows)
                          (40, 1056, 200, 32),
                          # enough 128 x 256 tiles to fill the GPU: the wide tile path
-                         (1280, 128, 4096, 32)]
+                         (1280, 512, 4096, 32)]
 ]
 
 
@@ -109,4 +109,4 @@ def test_affine_prefill_config_sampled(ql, orc):
     feats[-1] = case.N - 1
     yr, mag = orc.affine_matmul(x.vals[toks], codes[feats], s[feats], b[feats], 4, 64, lb.vals[feats])
     ys = y[torch.as_tensor(toks, device="cuda")][:, torch.as_tensor(feats, device="cuda")]
-    assert_fp_close(ys, yr, mag, lb.vals[feats], case.name, rel=REL_BF16W)
+    assert_fp_close(ys, yr, mag, lb.vals[feats], case.name)
