@@ -1,0 +1,487 @@
+// k_tc_affine.cu -- affine-format prefill GEMM on the 5th-generation tensor
+// cores with the dequantised weights as the tensor-memory A operand, sm_100a.
+//
+//   y[m,n] = sum_k x[m,k] * bf16(s[n,k/g] q[n,k] + b[n,k/g]) + bias[n]   (s q + b rounded once)
+//   [nuvec-nn QuantizedLinear, forward; cider/ops.py pergroup_linear docstring, dequantize]
+//
+// Each tile computes the transposed product  yT[128 weight rows][256 tokens] =
+// W^ . xT  as one M = 128, N = 256 MMA per 16-wide k step.  The dequantised
+// weights never touch shared memory: transform threads (two per weight row,
+// 32 k each per stage) read the 4-bit codes straight from global memory, turn
+// a code pair into bf16x2 in registers and write 16 columns each into tensor
+// memory with tcgen05.st; the tensor core reads them there (tcgen05.mma with
+// A in TMEM).  Shared memory carries only the x tile (TMA, 128-byte swizzle):
+// a stage moves 32 KB in and 32 KB out of it for 128 x 256 x 64 MACs, and
+// each dequantised weight serves 256 tokens.
+//
+// Warp roles (persistent: one CTA per SM walks tiles in a grouped order):
+//   warp 0       TMA producer of the x ring (32 KB stages, expect-tx mbarriers)
+//   warp 1       allocates 512 TMEM columns: the accumulator (256 columns) at
+//                0, the A ring (8 stages x 32 columns) at 256; one thread
+//                issues the MMAs and commits ring releases
+//   warps 2..9   transform: warp w writes TMEM lanes 32 (w % 4) .. +31, k half
+//                (w - 2) / 4 of each stage; the codes of a stage are loaded
+//                four stages ahead, the group parameters in 8-group windows
+//                with the next window in flight; a stage's tensor-memory store
+//                completes while the next stage is decoded
+//   warps 10..17 epilogue: warp w reads token half (w - 10) / 4 of lanes
+//                32 (w % 4) .. +31: tcgen05.ld, + bias[n], bf16 stores
+// Every mbarrier wait is bounded; on expiry the kernel records the timeout,
+// every role stops, the MMA thread waits for its MMAs in flight, and TMEM is
+// always freed.
+#include "qlin_common.cuh"
+
+namespace qlin {
+namespace {
+
+constexpr int kTW = 128;            // weight rows (outputs n) per tile: MMA M
+constexpr int kTT = 256;            // tokens per tile: MMA N
+constexpr int kKE = 64;             // k per stage (128 bytes of bf16 x)
+constexpr int kXStages = 6;         // x ring depth
+constexpr int kAStages = 8;         // TMEM A ring depth
+constexpr int kACols = kKE / 2;     // TMEM columns of one A stage (two bf16 per column)
+constexpr int kXBytes = kTT * 128;  // one x stage
+constexpr int kXformWarps = 8;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (2 + kXformWarps + kEpiWarps) * 32;
+constexpr int kTmemCols = 512;
+constexpr int kAccCols = kTT;       // A ring starts here
+constexpr int kCodePF = 4;          // stages of codes in flight per transform thread
+constexpr int kGroupT = 4;          // token tiles that walk the weight tiles together
+// kind::f16: D f32, A and B bf16, both K-major, N = 256, M = 128
+constexpr uint32_t kIdesc =
+    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+struct Bars {
+    uint64_t xfull[kXStages];
+    uint64_t xempty[kXStages];
+    uint64_t afull[kAStages];
+    uint64_t aempty[kAStages];
+    uint64_t acc_full;
+    uint64_t acc_empty;
+    uint64_t mma_done;
+    uint32_t tmem;
+    int abort_flag;
+};
+constexpr int kSmem = kXStages * kXBytes + (int)sizeof(Bars) + 1024;
+static_assert(kSmem <= 227 * 1024, "shared memory");
+static_assert(kAccCols + kAStages * kACols <= kTmemCols, "tensor memory");
+
+struct TsParams {
+    CUtensorMap tm_x;                 // x [M][K] bf16, box {64, 256}, 128-byte swizzle
+    const uint8_t* codes;             // [N][K/2]: LSB-first 4-bit codes
+    const unsigned short* scales;     // bf16 bits [N][K/g]
+    const unsigned short* biases;
+    const __nv_bfloat16* bias;        // [N] or null
+    __nv_bfloat16* out;               // [M][N]
+    int M, N, K;
+    int g_shift, ng;                  // log2 g, K / g
+    int tiles_t, tiles_w;
+    int vec_params;                   // parameter rows allow 16-byte loads of 8 groups
+    unsigned* status;
+};
+
+QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// 16 bytes of read-only global memory, not kept in L1 (each line is read once per CTA).
+QLIN_DEV uint4 ldg_nc_na_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T (kind::f16), one thread.
+QLIN_DEV void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+
+// 16 registers per thread -> this warp's 32 TMEM lanes, 16 consecutive columns.
+QLIN_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+QLIN_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+QLIN_DEV bool aborted(int* flag) { return *reinterpret_cast<volatile int*>(flag) != 0; }
+
+// Grouped tile order: kGroupT consecutive token tiles walk the weight tiles together.
+QLIN_DEV void tile_coords(int t, int tiles_t, int tiles_w, int& tt, int& wt)
+{
+    const int per_group = kGroupT * tiles_w;
+    const int grp = t / per_group;
+    const int first = grp * kGroupT;
+    const int gt = min(kGroupT, tiles_t - first);
+    const int r = t - grp * per_group;
+    tt = first + r % gt;
+    wt = r / gt;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_constant__ TsParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars& bars = *reinterpret_cast<Bars*>(smem + kXStages * kXBytes);
+    auto X = [&](int s) { return smem + s * kXBytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nk = (p.K + kKE - 1) / kKE;
+    const int tiles = p.tiles_t * p.tiles_w;
+    const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = my_tiles * nk;  // stages this CTA runs
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kXStages; ++s) {
+            mbar_init(&bars.xfull[s], 1);
+            mbar_init(&bars.xempty[s], 1);
+        }
+        for (int a = 0; a < kAStages; ++a) {
+            mbar_init(&bars.afull[a], kXformWarps);
+            mbar_init(&bars.aempty[a], 1);
+        }
+        mbar_init(&bars.acc_full, 1);
+        mbar_init(&bars.acc_empty, kEpiWarps);
+        mbar_init(&bars.mma_done, 1);
+        bars.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1)
+        tmem_alloc(&bars.tmem, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ x producer
+        if (lane == 0) {
+            pdl_launch_dependents();
+            pdl_wait_prior_grids();  // x may come from the previous kernel
+            int it = 0, slot = 0;
+            unsigned ph = 0u;
+            bool ok = true;
+            for (int ti = 0; ti < my_tiles && ok; ++ti) {
+                int tt, wt;
+                tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    if ((it >= kXStages && !mbar_wait_bounded(&bars.xempty[slot], ph ^ 1u, p.status)) ||
+                        aborted(&bars.abort_flag)) {
+                        bars.abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars.xfull[slot], kXBytes);
+                    tma_load_2d(X(slot), &p.tm_x, kb * kKE, tt * kTT, &bars.xfull[slot]);
+                    if (++slot == kXStages) {
+                        slot = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // drain: no copy may still be landing in this CTA's shared memory at exit
+            for (int j = it - kXStages < 0 ? 0 : it - kXStages; j < it; ++j)
+                mbar_wait_bounded(&bars.xfull[j % kXStages], (j / kXStages) & 1, p.status);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int xs = 0, as = 0;
+            unsigned xph = 0u, aph = 0u;
+            bool ok = true;
+            for (int ti = 0; ti < my_tiles && ok; ++ti) {
+                // the epilogue has read the previous tile's accumulators
+                ok = mbar_wait_bounded(&bars.acc_empty, (unsigned)(ti & 1) ^ 1u, p.status);
+                tc_fence_after();
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    ok = mbar_wait_bounded(&bars.xfull[xs], xph, p.status) &&
+                         mbar_wait_bounded(&bars.afull[as], aph, p.status);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    const uint32_t b0 = smem_u32(X(xs));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_ts(tmem, tmem + (uint32_t)(kAccCols + as * kACols + kk * 8), umma_desc_sw128(b0 + kk * 32),
+                                  kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit(&bars.xempty[xs]);
+                    tc_commit(&bars.aempty[as]);
+                    if (++xs == kXStages) {
+                        xs = 0;
+                        xph ^= 1u;
+                    }
+                    if (++as == kAStages) {
+                        as = 0;
+                        aph ^= 1u;
+                    }
+                }
+                if (ok)
+                    tc_commit(&bars.acc_full);  // fires when this tile's MMAs are done
+            }
+            if (!ok)
+                bars.abort_flag = 1;
+            // every MMA issued has completed before TMEM is released
+            tc_commit(&bars.mma_done);
+            mbar_wait_bounded(&bars.mma_done, 0, p.status);
+        }
+        __syncwarp();
+    } else if (warp < 2 + kXformWarps) {
+        // ------------------------------------------------------------ weight transform
+        const int q = warp & 3;             // TMEM lane quarter this warp may access
+        const int kh = (warp - 2) >> 2;     // 32-k half of each stage
+        const int r = 32 * q + lane;        // weight row within the tile
+        const size_t pitch = (size_t)p.K / 2;
+        pdl_wait_prior_grids();  // the weights' parameters may come from the previous kernel
+
+        auto row_of = [&](int ti) {
+            int tt, wt;
+            tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
+            return min(wt * kTW + r, p.N - 1);
+        };
+        // codes of stage (ti, kb) for this thread: 16 bytes (32 k) of row n; a half stage past K
+        // reads nothing (zero codes meet the zero-filled x columns there)
+        int lti = 0, lkb = 0;
+        const uint8_t* lrow = my_tiles > 0 ? p.codes + (size_t)row_of(0) * pitch + 16 * kh : p.codes;
+        auto load_next = [&](uint4& c) {
+            if (lti < my_tiles) {
+                c = lkb * kKE + 32 * kh < p.K ? ldg_nc_na_v4(lrow + (size_t)lkb * (kKE / 2))
+                                              : make_uint4(0u, 0u, 0u, 0u);
+                if (++lkb == nk) {
+                    lkb = 0;
+                    if (++lti < my_tiles)
+                        lrow = p.codes + (size_t)row_of(lti) * pitch + 16 * kh;
+                }
+            } else {
+                c = make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+
+        // group parameters of this thread's row in windows of 8 groups (16 bytes of scales, 16 of
+        // biases); the window after the current one is always in flight
+        const int nwin = (p.ng + 7) / 8;
+        auto win_load = [&](int ti, int win, uint4& S, uint4& B) {
+            if (ti >= my_tiles)
+                return;
+            const size_t off = (size_t)row_of(ti) * p.ng + 8 * win;
+            if (p.vec_params) {
+                S = __ldg(reinterpret_cast<const uint4*>(p.scales + off));
+                B = __ldg(reinterpret_cast<const uint4*>(p.biases + off));
+            } else {
+                uint32_t sv[4], bv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int g0 = 8 * win + 2 * e;
+                    const uint32_t slo = g0 < p.ng ? __ldg(p.scales + off + 2 * e) : 0u;
+                    const uint32_t shi = g0 + 1 < p.ng ? __ldg(p.scales + off + 2 * e + 1) : 0u;
+                    const uint32_t blo = g0 < p.ng ? __ldg(p.biases + off + 2 * e) : 0u;
+                    const uint32_t bhi = g0 + 1 < p.ng ? __ldg(p.biases + off + 2 * e + 1) : 0u;
+                    sv[e] = slo | (shi << 16);
+                    bv[e] = blo | (bhi << 16);
+                }
+                S = make_uint4(sv[0], sv[1], sv[2], sv[3]);
+                B = make_uint4(bv[0], bv[1], bv[2], bv[3]);
+            }
+        };
+        uint4 curS = make_uint4(0u, 0u, 0u, 0u), curB = curS, nxtS = curS, nxtB = curS;
+        int cur_ti = 0, cur_win = -1;
+        // bf16x2 (s, s) and (b, b) of this thread's 32 k of stage (ti, kb)
+        auto params_for = [&](int ti, int kb, uint32_t& s2, uint32_t& b2) {
+            const int gi = min(kb * kKE + 32 * kh, p.K - 1) >> p.g_shift;
+            const int win = gi >> 3;
+            if (ti != cur_ti || win != cur_win) {
+                if (cur_win < 0) {
+                    win_load(ti, win, curS, curB);
+                } else {
+                    curS = nxtS;
+                    curB = nxtB;
+                }
+                cur_ti = ti;
+                cur_win = win;
+                if (win + 1 < nwin)
+                    win_load(ti, win + 1, nxtS, nxtB);
+                else
+                    win_load(ti + 1, 0, nxtS, nxtB);
+            }
+            const int sub = gi & 7;
+            const uint32_t sw = (sub >> 1) == 0 ? curS.x : (sub >> 1) == 1 ? curS.y : (sub >> 1) == 2 ? curS.z : curS.w;
+            const uint32_t bw = (sub >> 1) == 0 ? curB.x : (sub >> 1) == 1 ? curB.y : (sub >> 1) == 2 ? curB.z : curB.w;
+            const uint32_t sv = (sw >> (16 * (sub & 1))) & 0xFFFFu, bv = (bw >> (16 * (sub & 1))) & 0xFFFFu;
+            s2 = sv | (sv << 16);
+            b2 = bv | (bv << 16);
+        };
+
+        uint4 cb[kCodePF];
+#pragma unroll
+        for (int j = 0; j < kCodePF; ++j)
+            load_next(cb[j]);
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols + 16 * kh);
+        int ti = 0, kb = 0, as = 0, pend_as = -1;
+        unsigned aph = 0u;
+        bool ok = true;
+        // the tensor-memory store of a stage is published (wait, fence, arrive) after the next stage
+        // has been decoded, so its latency overlaps that work
+        auto publish = [&]() {
+            if (pend_as >= 0) {
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars.afull[pend_as]);
+                pend_as = -1;
+            }
+        };
+        for (int base = 0; base < total && ok; base += kCodePF) {
+#pragma unroll
+            for (int j = 0; j < kCodePF; ++j) {
+                if (base + j >= total || !ok)
+                    break;
+                uint32_t s2, b2;
+                params_for(ti, kb, s2, b2);
+                // a pair of codes (q, q') of one byte becomes bf16x2 in four instructions: PRMT puts
+                // the byte (low half) and the byte of w >> 1 (high half) in place, one LOP3 makes the
+                // exact bf16 (128 + q, 128 + 8 q'), one bf16x2 FMA recovers (q, q') exactly, and one
+                // gives bf16(s q + b), the exact value rounded once.  Column c holds k = 2c, 2c + 1.
+                const uint32_t words[4] = {cb[j].x, cb[j].y, cb[j].z, cb[j].w};
+                uint32_t o[16];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const uint32_t w1 = words[w] >> 1;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t sel = (uint32_t)(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12));
+                        const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x43004300u);
+                        const uint32_t qq = bf16x2_fma(v, 0x3E003F80u, 0xC180C300u);  // (1, 1/8), (-128, -16)
+                        o[4 * w + e] = bf16x2_fma(qq, s2, b2);
+                    }
+                }
+                load_next(cb[j]);  // the stage kCodePF ahead
+                publish();
+                if (!mbar_wait_bounded(&bars.aempty[as], aph ^ 1u, p.status) || aborted(&bars.abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                tmem_st16(lane_base + (uint32_t)(as * kACols), o);
+                pend_as = as;
+                if (++as == kAStages) {
+                    as = 0;
+                    aph ^= 1u;
+                }
+                if (++kb == nk) {
+                    kb = 0;
+                    ++ti;
+                }
+            }
+        }
+        if (ok)
+            publish();
+        tmem_wait_st();  // no store may be in flight when TMEM is released
+        if (!ok)
+            bars.abort_flag = 1;
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                        // TMEM lane quarter this warp may access
+        const int th = (warp - 2 - kXformWarps) >> 2;  // token half
+        pdl_wait_prior_grids();  // bias / out may be touched by the previous kernel
+        for (int ti = 0; ti < my_tiles; ++ti) {
+            if (!mbar_wait_bounded(&bars.acc_full, (unsigned)(ti & 1), p.status) || aborted(&bars.abort_flag)) {
+                bars.abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            int tt, wt;
+            tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
+            const int m0 = tt * kTT + th * (kTT / 2);
+            const int n = wt * kTW + 32 * q + lane;
+            const bool n_ok = n < p.N;
+            const float bn = (p.bias && n_ok) ? __bfloat162float(p.bias[n]) : 0.f;
+            const uint32_t acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(th * (kTT / 2));
+            __nv_bfloat16* o = p.out + (size_t)m0 * p.N + n;
+#pragma unroll 1
+            for (int c = 0; c < kTT / 32; ++c) {
+                uint32_t v[16];
+                tmem_ld16(acc + (uint32_t)(c * 16), v);
+                if (!n_ok)
+                    continue;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int m = m0 + c * 16 + j;
+                    if (m < p.M)
+                        o[(size_t)(c * 16 + j) * p.N] = __float2bfloat16_rn(__uint_as_float(v[j]) + bn);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars.acc_empty);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1)
+        tmem_dealloc(tmem, kTmemCols);
+}
+
+bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev)
+{
+    TsParams prm;
+    prm.codes = static_cast<const uint8_t*>(a.b);
+    prm.scales = static_cast<const unsigned short*>(a.scales);
+    prm.biases = static_cast<const unsigned short*>(a.biases);
+    prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
+    prm.out = static_cast<__nv_bfloat16*>(a.out);
+    prm.M = (int)a.M;
+    prm.N = (int)a.N;
+    prm.K = (int)a.K;
+    prm.g_shift = 0;
+    while ((1 << prm.g_shift) < a.g)
+        ++prm.g_shift;
+    prm.ng = (int)(a.K / a.g);
+    prm.tiles_t = (int)((a.M + kTT - 1) / kTT);
+    prm.tiles_w = (int)((a.N + kTW - 1) / kTW);
+    prm.vec_params = prm.ng % 8 == 0 && aligned16p(a.scales) && aligned16p(a.biases);
+    prm.status = dev.status;
+    if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.a, (uint64_t)a.K, (uint64_t)a.M,
+                        (uint64_t)a.K * 2, kKE, kTT))
+        return cudaErrorInvalidValue;
+    auto kern = tc_affine_ts_kernel;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess)
+        return e;
+    const int tiles = prm.tiles_t * prm.tiles_w;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+}  // namespace qlin

@@ -194,7 +194,7 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
         t.scales = scales;
         t.biases = biases;
         t.g = group_size;
-        return from_cuda(launch_tc_gemm(TC_AFFINE4, t, static_cast<cudaStream_t>(stream), dev));
+        return from_cuda(launch_tc_affine(t, static_cast<cudaStream_t>(stream), dev));
     }
     AffineGemvArgs a;
     a.x = x;

@@ -356,5 +356,8 @@ struct TcGemmArgs {
 };
 enum TcOp { TC_I8_RAW = 0, TC_W8A8 = 1, TC_W4A8 = 2, TC_AFFINE4 = 3 };
 cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev);
+// affine 4-bit prefill with the dequantised weights as the TMEM A operand (k_tc_affine.cu):
+// x bf16 [M][K], codes [N][K/2], bf16 scales / biases [N][K/g], out bf16 [M][N].
+cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev);
 
 }  // namespace qlin
