@@ -7,33 +7,27 @@
 //              [cider/ops.py perchannel_linear]
 //   W4A8:      y[m,n] = acc * s_x[m] * s_w[n] (+ bias[n]),   acc = qx . (c - 8)
 //              [cider/ops.py w4a8_linear, pack_weight_int4]
-//   affine:    y[m,n] = sum_k x[m,k] * bf16(s q + b) + bias[n]   (s q + b rounded once)
-//              [nuvec-nn QuantizedLinear, forward; cider/ops.py pergroup_linear
-//               docstring, dequantize]
 //
 // Persistent, warp-specialised kernel: one CTA per SM walks 128 x BN output
 // tiles (BN = 256, or 128 when there are too few tiles to fill the GPU) in a
 // grouped order: kGroupM M-tiles walk the N-tiles together, so each weight
 // tile is fetched from HBM about once and reused from L2.
-//   warp 0       TMA producer: A tiles and the B source (int8 B, packed int4,
-//                or affine code bytes) into a shared-memory ring, mbarrier
-//                completion (expect-tx).
+//   warp 0       TMA producer: A tiles and the B source (int8 B or packed
+//                int4) into a shared-memory ring, mbarrier completion
+//                (expect-tx).
 //   warp 1       allocates 2 x BN TMEM columns (two accumulators); one thread
-//                issues tcgen05.mma (M = 128, N = BN, K = 32 int8 / 16 bf16 per
+//                issues tcgen05.mma (kind::i8, M = 128, N = BN, K = 32 per
 //                instruction); tcgen05.commit frees ring slots and transformed
 //                B buffers when their MMAs are done, and publishes each
 //                finished accumulator to the epilogue.
 //   warps 2..5   epilogue: tcgen05.ld of one accumulator (warp q owns TMEM
 //                lanes 32q .. 32q+31 = 32 output rows) while the MMAs of the
 //                next tile fill the other one; scales, bias, 16-byte stores.
-//   warps 6..    (W4A8, affine) 2 x BN transform threads turn the packed
-//                source into the K-major 128-byte-swizzled operand in a
-//                2-deep buffer: nibbles -> int8 16 (c - 8) (the epilogue
-//                shifts the exact int32 sum back by 4 bits), or codes ->
-//                bf16(s q + b), the exact value rounded once to bf16 (bf16x2
-//                FMA); the group parameters of a stage are loaded two stages
-//                ahead.  fence.proxy.async publishes the operand to the
-//                tensor core.
+//   warps 6..    (W4A8) 2 x BN transform threads turn the packed source into
+//                the K-major 128-byte-swizzled operand in a 2-deep buffer:
+//                nibbles -> int8 16 (c - 8) (the epilogue shifts the exact
+//                int32 sum back by 4 bits).  fence.proxy.async publishes the
+//                operand to the tensor core.
 // Every mbarrier wait is bounded; on expiry the kernel records the timeout,
 // every role stops, the MMA thread waits for its MMAs in flight, and TMEM is
 // always freed.
@@ -51,28 +45,27 @@ constexpr int kSmemBudget = 200 * 1024;
 #endif
 constexpr int kBDepth = QLIN_TC_BDEPTH;  // transformed-B buffers
 
-enum BSource { B_TMA_I8 = 0, B_W4 = 1, B_AFFINE4 = 2 };
-enum Epi { E_I32 = 0, E_SCALED = 1, E_BIAS = 2 };
+enum BSource { B_TMA_I8 = 0, B_W4 = 1 };
+enum Epi { E_I32 = 0, E_SCALED = 1 };
 
 __host__ __device__ constexpr int rup(int a, int b) { return (a + b - 1) / b * b; }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 template <int BSRC, int BN>
 struct TcCfg {
-    static constexpr bool I8 = BSRC != B_AFFINE4;          // kind::i8 (s32) or kind::f16 (bf16 -> f32)
-    static constexpr int KE = I8 ? 128 : 64;                // K elements per stage (128 bytes of A)
+    static constexpr int KE = 128;                          // K elements per stage (128 bytes of A)
     static constexpr int XW = BSRC == B_TMA_I8 ? 0 : BN / 16;  // transform warps: two threads per B row
     static constexpr int A_BYTES = kBM * 128;
     static constexpr int B_BYTES = BN * 128;                // one K-major swizzled B operand
-    static constexpr int RAW_BYTES = BSRC == B_W4 ? (KE / 2) * BN : (BSRC == B_AFFINE4 ? BN * (KE / 2) : B_BYTES);
+    static constexpr int RAW_BYTES = BSRC == B_W4 ? (KE / 2) * BN : B_BYTES;
     static constexpr int SLOT = rup(A_BYTES + RAW_BYTES, 1024);
     static constexpr int BRING = XW > 0 ? kBDepth * B_BYTES : 0;  // transformed B ring
     static constexpr int NS = cmin(8, (kSmemBudget - BRING) / SLOT);
     static constexpr int THREADS = (2 + kEpiWarps + XW) * 32;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr uint32_t IDESC =
-        (I8 ? (2u << 4) : (1u << 4)) |                      // D: s32 / f32
-        (1u << 7) | (1u << 10) |                            // A, B: s8 / bf16 (signed)
+        (2u << 4) |                                         // D: s32
+        (1u << 7) | (1u << 10) |                            // A, B: s8 (signed)
         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);  // K-major A and B
     struct Bars {
         uint64_t full[NS];
@@ -91,20 +84,16 @@ struct TcCfg {
 };
 
 struct TcParams {
-    CUtensorMap tm_a;  // A [M][K], box {128 B, 128 rows}, 128-byte swizzle
+    CUtensorMap tm_a;  // A [M][K] int8, box {128 B, 128 rows}, 128-byte swizzle
     CUtensorMap tm_b;  // int8 B [N][K] (box {128 B, BN rows}, swizzled) | packed int4 [K/2][N]
-                       // (box {BN B, 64 rows}) | affine code bytes [N][K/2] (box {32 B, BN rows})
+                       // (box {BN B, 64 rows})
     int M, N, K;
     int tiles_m, tiles_n;
     void* out;
     const float* s_x;
     const float* s_w;
     const __nv_bfloat16* bias;
-    const __nv_bfloat16* scales;
-    const __nv_bfloat16* biases;
-    int g, g_shift;  // group size and its log2
     int vec_sw, vec_bias, vec_out;  // 16-byte alignment of s_w, bias and out
-    int vec_params;                 // scales / biases rows allow 16-byte loads of 8 groups
     unsigned* status;
 };
 
@@ -112,13 +101,6 @@ QLIN_DEV void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t
 {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
-}
-
-QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
-{
-    uint32_t d;
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
 }
 
 QLIN_DEV uint32_t pack_bf16x2(float lo, float hi)
@@ -204,10 +186,8 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                     tma_load_2d(A(slot), &p.tm_a, kb * Cfg::KE, mt * kBM, &bars.full[slot]);
                     if constexpr (BSRC == B_TMA_I8)
                         tma_load_2d(RAW(slot), &p.tm_b, kb * 128, nt * BN, &bars.full[slot]);
-                    else if constexpr (BSRC == B_W4)
-                        tma_load_2d(RAW(slot), &p.tm_b, nt * BN, kb * (Cfg::KE / 2), &bars.full[slot]);
                     else
-                        tma_load_2d(RAW(slot), &p.tm_b, kb * (Cfg::KE / 2), nt * BN, &bars.full[slot]);
+                        tma_load_2d(RAW(slot), &p.tm_b, nt * BN, kb * (Cfg::KE / 2), &bars.full[slot]);
                 }
                 if (kb < nk)
                     break;
@@ -239,7 +219,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                     const uint32_t b0 = smem_u32(Cfg::XW > 0 ? BT(it % kBDepth) : RAW(slot));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc_mma<Cfg::I8>(acc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
+                        tc_mma<true>(acc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
                                         Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
                     tc_commit(&bars.empty[slot]);
                     if (Cfg::XW > 0)
@@ -367,11 +347,6 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         // ------------------------------------------------------------ B transform
         const int tt = threadIdx.x - (2 + kEpiWarps) * 32;  // 0 .. 2 BN - 1
         const int wt = tt >> 5;                             // transform warp
-        // affine: thread = (B row r, 32-code half h); the half alternates every 8 rows so that the
-        // 16-byte stores of an 8-lane phase hit 8 distinct swizzle chunks
-        const int r = tt % BN;
-        const int h = ((r >> 3) & 1) ^ (tt / BN);
-        const int ng = p.g > 0 ? p.K / p.g : 1;
         // W4: warp wt takes 128-column half wt % (BN/128) and 16-k unit wt / (BN/128)
         const int w4_q = 32 * (wt % (BN / 128)) + lane;  // column quad
         const int w4_u = wt / (BN / 128);
@@ -379,79 +354,17 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         const uint32_t c0 = w4_rot, c1 = (w4_rot + 1) & 3, c2 = (w4_rot + 2) & 3, c3 = (w4_rot + 3) & 3;
         const uint32_t w4_selA = c0 | ((4 + c0) << 4) | (c1 << 8) | ((4 + c1) << 12);
         const uint32_t w4_selB = c2 | ((4 + c2) << 4) | (c3 << 8) | ((4 + c3) << 12);
-        pdl_wait_prior_grids();  // the weights' parameters may come from the previous kernel
-        // affine: the group parameters of this thread's row come in windows of 8 groups (16 bytes of
-        // scales, 16 of biases: one vector load each when the row pitch allows); the window after the
-        // current one is always in flight.
-        const unsigned short* sc16 = reinterpret_cast<const unsigned short*>(p.scales);
-        const unsigned short* bi16 = reinterpret_cast<const unsigned short*>(p.biases);
-        const int nwin = (ng + 7) / 8;
-        auto win_load = [&](int ti, int win, uint4& S, uint4& B) {
-            if (ti >= my_tiles)
-                return;
-            int mt, nt;
-            tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
-            const size_t off = (size_t)min(nt * BN + r, p.N - 1) * ng + 8 * win;
-            if (p.vec_params) {
-                S = __ldg(reinterpret_cast<const uint4*>(sc16 + off));
-                B = __ldg(reinterpret_cast<const uint4*>(bi16 + off));
-            } else {
-                uint32_t sv[4], bv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int g0 = 8 * win + 2 * e;
-                    const uint32_t slo = g0 < ng ? __ldg(sc16 + off + 2 * e) : 0u;
-                    const uint32_t shi = g0 + 1 < ng ? __ldg(sc16 + off + 2 * e + 1) : 0u;
-                    const uint32_t blo = g0 < ng ? __ldg(bi16 + off + 2 * e) : 0u;
-                    const uint32_t bhi = g0 + 1 < ng ? __ldg(bi16 + off + 2 * e + 1) : 0u;
-                    sv[e] = slo | (shi << 16);
-                    bv[e] = blo | (bhi << 16);
-                }
-                S = make_uint4(sv[0], sv[1], sv[2], sv[3]);
-                B = make_uint4(bv[0], bv[1], bv[2], bv[3]);
-            }
-        };
-        uint4 curS = make_uint4(0u, 0u, 0u, 0u), curB = curS, nxtS = curS, nxtB = curS;
-        int cur_ti = 0, cur_win = -1;
-        // (scale, bias) bf16 bits for stage `it` (tile ti, k block kb)
-        auto params_for = [&](int ti, int kb, unsigned (&pr)[2]) {
-            const int gi = min(kb * Cfg::KE + 32 * h, p.K - 1) >> p.g_shift;
-            const int win = gi >> 3;
-            if (ti != cur_ti || win != cur_win) {
-                if (cur_win < 0) {  // first window of this CTA
-                    win_load(ti, win, curS, curB);
-                } else {
-                    curS = nxtS;
-                    curB = nxtB;
-                }
-                cur_ti = ti;
-                cur_win = win;
-                if (win + 1 < nwin)
-                    win_load(ti, win + 1, nxtS, nxtB);
-                else
-                    win_load(ti + 1, 0, nxtS, nxtB);
-            }
-            const int sub = gi & 7;
-            const uint32_t sw = (sub >> 1) == 0 ? curS.x : (sub >> 1) == 1 ? curS.y : (sub >> 1) == 2 ? curS.z : curS.w;
-            const uint32_t bw = (sub >> 1) == 0 ? curB.x : (sub >> 1) == 1 ? curB.y : (sub >> 1) == 2 ? curB.z : curB.w;
-            pr[0] = (sw >> (16 * (sub & 1))) & 0xFFFFu;
-            pr[1] = (bw >> (16 * (sub & 1))) & 0xFFFFu;
-        };
+        pdl_wait_prior_grids();  // the packed weights may come from the previous kernel
         // one stage: RAW(slot) -> BT(it % kBDepth)
-        // affine: the four 16-byte store offsets of this thread's half row in the swizzled operand
-        int st_off[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-            st_off[w] = swz128(r, 4 * h + w);
         // ring positions of stage it: slot / phase of the code ring, buffer / phase of the operand ring
         int slot = 0, bslot = 0;
         unsigned fph = 0u, bph = 0u;
-        auto stage = [&](const unsigned (&pr)[2]) -> bool {
+        auto stage = [&]() -> bool {
             if (!mbar_wait_bounded(&bars.full[slot], fph, p.status) ||
                 !mbar_wait_bounded(&bars.bempty[bslot], bph ^ 1u, p.status) || aborted(&bars.abort_flag))
                 return false;
             uint8_t* dst = BT(bslot);
-            if constexpr (BSRC == B_W4) {
+            {
                 // raw[i][n]: k-pair row i (k = 2i high nibble, 2i+1 low) of column n; 64 rows x BN bytes.
                 // Eight 32-bit loads (the k-pair rows of unit u for columns 4q .. 4q+3; a warp's lanes
                 // hit 32 distinct banks) are byte-transposed by PRMT into per-column words; slot sl
@@ -488,29 +401,6 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                     const int n = 4 * w4_q + ((w4_rot + sl) & 3);
                     st_shared_v4(dst + swz128(n, u), o[0], o[1], o[2], o[3]);
                 }
-            } else {
-                // raw[n][32 bytes]: 64 LSB-first 4-bit codes of row n; this thread: k0 + 32h .. +31.
-                // A pair of codes (q, q') of one byte becomes bf16x2 in four instructions: PRMT puts
-                // the byte (low half) and the byte of w >> 1 (high half) in place, one LOP3 makes the
-                // exact bf16 (128 + q, 128 + 8 q'), one bf16x2 FMA recovers (q, q') exactly, and one
-                // gives bf16(s q + b), the exact value rounded once.
-                // codes past K are zero-filled by the copy and meet zero activations: no masking needed
-                const uint4 cw = *reinterpret_cast<const uint4*>(RAW(slot) + r * 32 + 16 * h);
-                const uint32_t s2 = prmt(pr[0], pr[0], 0x1010u), b2 = prmt(pr[1], pr[1], 0x1010u);
-                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {  // word w: k = k0 + 8w .. +7 -> unit 4h + w
-                    const uint32_t w1 = words[w] >> 1;
-                    uint32_t o[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t sel = (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12));
-                        const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x43004300u);
-                        const uint32_t q = bf16x2_fma(v, 0x3E003F80u, 0xC180C300u);  // (1, 1/8), (-128, -16)
-                        o[j] = bf16x2_fma(q, s2, b2);
-                    }
-                    st_shared_v4(dst + st_off[w], o[0], o[1], o[2], o[3]);
-                }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -527,17 +417,8 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             return true;
         };
         bool ok = true;
-        int ti = 0, kb = 0;  // tile and k block of stage it (no divisions in the loop)
-        for (int it = 0; it < total && ok; ++it) {
-            unsigned pr[2] = {0u, 0u};
-            if constexpr (BSRC == B_AFFINE4)
-                params_for(ti, kb, pr);
-            ok = stage(pr);
-            if (++kb == nk) {
-                kb = 0;
-                ++ti;
-            }
-        }
+        for (int it = 0; it < total && ok; ++it)
+            ok = stage();
         if (!ok)
             bars.abort_flag = 1;
     }
@@ -578,12 +459,9 @@ bool encode_b(TcOp op, CUtensorMap* tm, const TcGemmArgs& a, int bn)
     case TC_W8A8:
         return encode_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K,
                               128, (uint32_t)bn);
-    case TC_W4A8:
+    default:  // TC_W4A8
         return encode_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)a.N, (uint64_t)(a.K / 2),
                               (uint64_t)a.N, (uint32_t)bn, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
-    default:
-        return encode_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b, (uint64_t)(a.K / 2), (uint64_t)a.N,
-                              (uint64_t)(a.K / 2), 32, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_NONE);
     }
 }
 
@@ -593,8 +471,7 @@ cudaError_t launch_bn(TcOp op, TcParams& prm, cudaStream_t st, const DeviceInfo&
     switch (op) {
     case TC_I8_RAW: return launch_t<B_TMA_I8, E_I32, BN>(prm, st, dev);
     case TC_W8A8: return launch_t<B_TMA_I8, E_SCALED, BN>(prm, st, dev);
-    case TC_W4A8: return launch_t<B_W4, E_SCALED, BN>(prm, st, dev);
-    default: return launch_t<B_AFFINE4, E_BIAS, BN>(prm, st, dev);
+    default: return launch_t<B_W4, E_SCALED, BN>(prm, st, dev);  // TC_W4A8
     }
 }
 
@@ -612,21 +489,12 @@ cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const 
     prm.s_x = a.s_x;
     prm.s_w = a.s_w;
     prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
-    prm.scales = static_cast<const __nv_bfloat16*>(a.scales);
-    prm.biases = static_cast<const __nv_bfloat16*>(a.biases);
-    prm.g = a.g;
-    prm.g_shift = 0;
-    while (a.g > 0 && (1 << prm.g_shift) < a.g)
-        ++prm.g_shift;
     prm.vec_sw = aligned16p(a.s_w);
     prm.vec_bias = aligned16p(a.bias);
     prm.vec_out = aligned16p(a.out);
-    prm.vec_params = a.g > 0 && (a.K / a.g) % 8 == 0 && aligned16p(a.scales) && aligned16p(a.biases);
     prm.status = dev.status;
-    const bool bf16_a = op == TC_AFFINE4;
-    const uint64_t a_pitch = (uint64_t)a.K * (bf16_a ? 2 : 1);
-    if (!encode_tmap_2d(&prm.tm_a, bf16_a ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a,
-                        (uint64_t)a.K, (uint64_t)a.M, a_pitch, bf16_a ? 64 : 128, kBM))
+    if (!encode_tmap_2d(&prm.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K,
+                        128, kBM))
         return cudaErrorInvalidValue;
     // 256-column tiles when they still give every SM a tile, else 128
     const int64_t tiles_m = (a.M + kBM - 1) / kBM;

@@ -340,8 +340,9 @@ cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const
 
 namespace qlin {
 
-// tcgen05 GEMM launches (k_tc_gemm.cu).  A is [M][K] row-major (int8 or
-// bf16), the output [M][N] row-major.
+// tcgen05 GEMM launches: int8 (k_tc_gemm.cu) and affine 4-bit (k_tc_affine.cu).
+// A is [M][K] row-major (int8, or bf16 x for the affine GEMM), the output [M][N]
+// row-major.
 struct TcGemmArgs {
     int64_t M, N, K;
     const void* a;            // int8 (qx / raw a) or bf16 (x)
@@ -354,7 +355,7 @@ struct TcGemmArgs {
     const void* biases;
     int g;
 };
-enum TcOp { TC_I8_RAW = 0, TC_W8A8 = 1, TC_W4A8 = 2, TC_AFFINE4 = 3 };
+enum TcOp { TC_I8_RAW = 0, TC_W8A8 = 1, TC_W4A8 = 2 };
 cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev);
 // affine 4-bit prefill with the dequantised weights as the TMEM A operand (k_tc_affine.cu):
 // x bf16 [M][K], codes [N][K/2], bf16 scales / biases [N][K/g], out bf16 [M][N].

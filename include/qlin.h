@@ -128,10 +128,12 @@ qlin_status qlin_dequantize(const uint32_t* codes, const void* scales, const voi
  * x: [M, K] of x_dt (which is also the dtype of bias and y).  bias: [N] or
  * NULL.  y: [M, N].  M <= 16 runs the decode kernel (bulk-copy streamed
  * codes, register dequantisation, tensor-core MACs, partial sums reduced
- * inside the CTA); larger M runs the prefill GEMM (codes dequantised
- * to bf16 in shared memory feeding tcgen05 MMA with fp32 accumulation in
- * tensor memory).  Requires (K*bits/8) % 16 == 0 and, for x, (K*sizeof(x_dt))
- * % 16 == 0.  `workspace` may be NULL when qlin_workspace_size() is 0.
+ * inside the CTA); larger M with 4-bit codes and bf16 x and parameters runs
+ * the prefill GEMM (codes dequantised to bf16 in registers and written to
+ * tensor memory as the A operand of tcgen05 MMA, fp32 accumulation in tensor
+ * memory).  Requires (K*bits/8) % 16 == 0 and, for x, (K*sizeof(x_dt)) % 16
+ * == 0.  `workspace` may be NULL when qlin_workspace_size() is 0 (it is for
+ * this operation).
  */
 qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
                         const uint32_t* codes, const void* scales, const void* biases,
