@@ -59,10 +59,18 @@ def load_peaks():
     return d
 
 
-def kernel_source_hash() -> str:
+# The source files each recorded kernel is compiled from (its own .cu and the
+# shared header of device helpers): its ncu counters stay valid while these hash
+# the same.
+KERNEL_SOURCES = {
+    "bitlinear_reg_kernel": ("k_gemv.cu", "qlin_common.cuh"),
+}
+
+
+def kernel_source_hash(kernel_key: str = "bitlinear_reg_kernel") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_quantized_linear_qmm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel_key]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -71,11 +79,11 @@ def kernel_source_hash() -> str:
 
 def recorded_traffic(kernel_key: str):
     """DRAM bytes per launch from a committed ncu summary, if taken on the
-    current kernel sources (else None)."""
+    kernel's current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kernel_key not in KERNEL_SOURCES:
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash(kernel_key)
     with open(path) as f:
         for line in f:
             parts = line.split()

@@ -91,6 +91,11 @@ qlin_status check_affine(int64_t N, int64_t K, int bits, int g, qlin_dtype p_dt)
 
 using namespace qlin;
 
+namespace qlin {
+// self-test of the bounded-wait path (k_selftest.cu): one wait that runs out after limit_ns.
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t st, const DeviceInfo& dev);
+}  // namespace qlin
+
 extern "C" {
 
 const char* qlin_status_string(qlin_status s)
@@ -366,6 +371,18 @@ qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
                         void* stream)
 {
     return int_linear(TC_W4A8, x, x_dt, M, K, packed_w, scale_w, N, bias, y, workspace, ws_bytes, stream);
+}
+
+qlin_status qlin_selftest_wait_timeout(unsigned limit_us, void* stream)
+{
+    if (limit_us == 0 || limit_us > 2000000u)
+        return QLIN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    qlin_status s = current_device(dev);
+    if (s != QLIN_OK)
+        return s;
+    return from_cuda(launch_wait_timeout_selftest((unsigned long long)limit_us * 1000ull,
+                                                  static_cast<cudaStream_t>(stream), dev));
 }
 
 qlin_status qlin_get_device_status(void* stream)

@@ -75,6 +75,7 @@ def lib():
         "w4a8_linear": ([P, I, I64, I64, P, P, I64, P, P, P, SZ, P], I),
         "w8a8_linear_noalloc": ([P, I, I64, I64, P, P, I64, P, P, P], I),
         "qlin_get_device_status": ([P], I),
+        "qlin_selftest_wait_timeout": ([C.c_uint, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -242,6 +243,11 @@ def w8a8_linear_noalloc(x, w, scale_w, bias=None, out=None):
     _check(lib().w8a8_linear_noalloc(_ptr(x), _dt(x), M, K, _ptr(w), _ptr(scale_w), N, _ptr(bias), _ptr(out),
                                      _stream(x.device)), "w8a8_linear_noalloc")
     return out
+
+
+def selftest_wait_timeout(limit_us: int = 1000, device=None):
+    """Queues a kernel whose bounded wait runs out after limit_us (see qlin.h)."""
+    _check(lib().qlin_selftest_wait_timeout(int(limit_us), _stream(device)), "qlin_selftest_wait_timeout")
 
 
 def device_status(device=None) -> int:

@@ -242,6 +242,16 @@ qlin_status w8a8_linear_noalloc(const void* x, qlin_dtype x_dt, int64_t M, int64
  */
 qlin_status qlin_get_device_status(void* stream);
 
+/*
+ * Self-test of the bounded-wait path: launches one kernel on `stream` that
+ * waits on an on-chip barrier nothing completes, gives up after `limit_us`
+ * microseconds (1 .. 2,000,000, else QLIN_ERR_INVALID_ARG), sets the timeout
+ * bit of the device status word and returns; the next
+ * qlin_get_device_status() then reports QLIN_ERR_TIMEOUT, and the library
+ * stays usable.  Nothing faults, nothing is left running.
+ */
+qlin_status qlin_selftest_wait_timeout(unsigned limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
