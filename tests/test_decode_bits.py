@@ -1,0 +1,172 @@
+"""CPU checks of the bit-level decode steps the kernels use, against plain unpacking.
+
+The GPU kernels turn packed codes into MMA operands with byte permutes (PRMT),
+masked ORs into a bf16 exponent pattern (LOP3) and one exact bf16x2 FMA.  These
+tests emulate those instructions bit for bit and check, for every code value,
+that the result equals what a plain unpacking of the formats gives:
+
+- affine 4-bit, a code pair of one byte -> bf16x2 (q, q'), exactly
+  [MLX affine format: LSB-first codes in uint32 words];
+- BitLinear 2-bit fields of one byte -> code - 1 for output rows r + j N/4
+  [BitLinear packing: code j of byte P[r, k] at bits 2j];
+- W4 nibbles -> int8 16 (c - 8), even k from the high nibble
+  [packed per-column INT4: zero point 8, high nibble = even k].
+
+The constants are read from the kernel sources, so a change there that these
+tests do not follow fails here.
+"""
+from __future__ import annotations
+
+import os
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+CSRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "bit_quantized_linear_qmm_b200",
+                    "csrc")
+
+
+def _src(name: str) -> str:
+    with open(os.path.join(CSRC, name)) as f:
+        return f.read()
+
+
+def prmt(a: int, b: int, sel: int) -> int:
+    """PRMT default mode: byte i of the result is byte (sel >> 4i) & 7 of {b, a} (a = bytes 0-3)."""
+    bs = [(a >> (8 * i)) & 0xFF for i in range(4)] + [(b >> (8 * i)) & 0xFF for i in range(4)]
+    return sum(bs[(sel >> (4 * i)) & 7] << (8 * i) for i in range(4))
+
+
+def lop3_and_or(a: int, mask: int, orv: int) -> int:
+    return ((a & mask) | orv) & 0xFFFFFFFF
+
+
+def bf16(h: int) -> Fraction:
+    """Exact value of a bf16 bit pattern (finite values only)."""
+    f = struct.unpack("<f", struct.pack("<I", (h & 0xFFFF) << 16))[0]
+    assert np.isfinite(f)
+    return Fraction(f)
+
+
+def halves(w: int):
+    return bf16(w & 0xFFFF), bf16(w >> 16)
+
+
+def fma_exact_pair(v: int, scale: int, bias: int):
+    """bf16x2 FMA v * scale + bias, per half, as exact rationals (the kernels rely on the result
+    being exactly representable, so the single rounding of fma.rn leaves it unchanged)."""
+    (v0, v1), (s0, s1), (b0, b1) = halves(v), halves(scale), halves(bias)
+    return v0 * s0 + b0, v1 * s1 + b1
+
+
+def exact_in_bf16(x: Fraction) -> bool:
+    if x == 0:
+        return True
+    f = float(x)
+    h = struct.unpack("<I", struct.pack("<f", f))[0]
+    return Fraction(f) == x and (h & 0xFFFF) == 0
+
+
+# ---------------------------------------------------------------- affine 4-bit pair -> bf16x2
+
+def test_affine_pair_decode_constants_in_source():
+    s = _src("k_tc_affine.cu")
+    assert "lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x43004300u)" in s
+    assert "bf16x2_fma(v, 0x3E003F80u, 0xC180C300u)" in s
+    assert "const uint32_t w1 = words[w] >> 1;" in s
+    assert "(uint32_t)(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12))" in s
+
+
+@pytest.mark.parametrize("pos", range(4))
+def test_affine_pair_decode_every_byte(pos):
+    rng = np.random.default_rng(pos)
+    for byte in range(256):
+        others = int(rng.integers(0, 2**32))
+        w = (others & ~(0xFF << (8 * pos)) | (byte << (8 * pos))) & 0xFFFFFFFF
+        q = [(w >> (4 * i)) & 15 for i in range(8)]  # LSB-first codes k = 0..7
+        sel = pos | (pos << 4) | ((4 + pos) << 8) | ((4 + pos) << 12)
+        v = lop3_and_or(prmt(w, w >> 1, sel), 0x0078000F, 0x43004300)
+        lo, hi = halves(v)
+        assert (lo, hi) == (128 + q[2 * pos], 128 + 8 * q[2 * pos + 1])
+        a, b = fma_exact_pair(v, 0x3E003F80, 0xC180C300)
+        assert (a, b) == (q[2 * pos], q[2 * pos + 1])  # column pos holds k = 2 pos, 2 pos + 1
+        assert exact_in_bf16(a) and exact_in_bf16(b)
+
+
+# ---------------------------------------------------------------- BitLinear 2-bit fields
+
+def test_bitlinear_decode_constants_in_source():
+    s = _src("k_gemv.cu")
+    for c in ("kScale0 = 0x3F803F80u, kBias0 = 0xC301C301u", "kScale1 = 0x3E803E80u, kBias1 = 0xC204C204u",
+              "kScale2 = 0x3D803D80u, kBias2 = 0xC110C110u", "kMagic = 0x43004300u",
+              "prmt(wv[i], 0u, 0x3120)", "lop3_and_or(w, 0x00030003u, kMagic), kScale0, kBias0",
+              "lop3_and_or(w, 0x00300030u, kMagic), kScale2, kBias2",
+              "lop3_and_or(w, 0x000C000Cu, kMagic), kScale1, kBias1",
+              "lop3_and_or(w >> 6, 0x00030003u, kMagic), kScale0, kBias0",
+              "lop3_and_or(w >> 14, 0x00030003u, kMagic), kScale0, kBias0"):
+        assert c in s, c
+
+
+def _bitlinear_chunk(word: int):
+    """The kernel's decode of one 32-bit word (bytes k .. k+3 of one packed row): field j of byte k
+    -> (k, value) pairs, as the four f02 / f13 registers produce them."""
+    MAGIC = 0x43004300
+    S0, B0, S1, B1, S2, B2 = 0x3F803F80, 0xC301C301, 0x3E803E80, 0xC204C204, 0x3D803D80, 0xC110C110
+    w = prmt(word, 0, 0x3120)  # bytes (k, k+2, k+1, k+3)
+    hw = w >> 8
+    out = {}
+    out[(0, 0)], out[(0, 1)] = fma_exact_pair(lop3_and_or(w, 0x00030003, MAGIC), S0, B0)
+    out[(2, 0)], out[(2, 1)] = fma_exact_pair(lop3_and_or(w, 0x00300030, MAGIC), S2, B2)
+    out[(0, 2)], out[(0, 3)] = fma_exact_pair(lop3_and_or(hw, 0x00030003, MAGIC), S0, B0)
+    out[(2, 2)], out[(2, 3)] = fma_exact_pair(lop3_and_or(hw, 0x00300030, MAGIC), S2, B2)
+    out[(1, 0)], out[(1, 1)] = fma_exact_pair(lop3_and_or(w, 0x000C000C, MAGIC), S1, B1)
+    out[(3, 0)], out[(3, 1)] = fma_exact_pair(lop3_and_or(w >> 6, 0x00030003, MAGIC), S0, B0)
+    out[(1, 2)], out[(1, 3)] = fma_exact_pair(lop3_and_or(hw, 0x000C000C, MAGIC), S1, B1)
+    out[(3, 2)], out[(3, 3)] = fma_exact_pair(lop3_and_or(w >> 14, 0x00030003, MAGIC), S0, B0)
+    return out  # (field j, k offset) -> value
+
+
+def test_bitlinear_fields_every_byte():
+    rng = np.random.default_rng(3)
+    for byte in range(256):
+        for pos in range(4):
+            word = int(rng.integers(0, 2**32))
+            word = (word & ~(0xFF << (8 * pos)) | (byte << (8 * pos))) & 0xFFFFFFFF
+            got = _bitlinear_chunk(word)
+            for kk in range(4):
+                b = (word >> (8 * kk)) & 0xFF
+                for j in range(4):
+                    code = (b >> (2 * j)) & 3  # output row r + j N/4
+                    assert got[(j, kk)] == code - 1, (hex(word), j, kk)
+                    assert exact_in_bf16(got[(j, kk)])
+
+
+# ---------------------------------------------------------------- W4 nibbles -> int8 16 (c - 8)
+
+def test_w4_decode_constants_in_source():
+    for name in ("k_tc_gemm.cu", "k_gemv.cu"):
+        s = _src(name)
+        assert "^ 0x88888888u" in s and "& 0xF0F0F0F0u" in s and "(x << 4) & 0xF0F0F0F0u" in s, name
+        assert "prmt(hi, lo, 0x5140u)" in s and "prmt(hi, lo, 0x7362u)" in s, name
+
+
+def test_w4_nibbles_every_byte():
+    """A word of four packed bytes (k-pair rows i = 0..3 of one column; high nibble = k = 2i) ->
+    two words of int8 16 (c - 8) in k order 0..3 and 4..7."""
+    rng = np.random.default_rng(5)
+    for byte in range(256):
+        for pos in range(4):
+            t = int(rng.integers(0, 2**32))
+            t = (t & ~(0xFF << (8 * pos)) | (byte << (8 * pos))) & 0xFFFFFFFF
+            x = t ^ 0x88888888
+            hi = x & 0xF0F0F0F0
+            lo = (x << 4) & 0xF0F0F0F0
+            o = [prmt(hi, lo, 0x5140), prmt(hi, lo, 0x7362)]
+            got = [int(np.int8(np.uint8((o[k // 4] >> (8 * (k % 4))) & 0xFF))) for k in range(8)]
+            want = []
+            for i in range(4):
+                b = (t >> (8 * i)) & 0xFF
+                want += [16 * ((b >> 4) - 8), 16 * ((b & 15) - 8)]
+            assert got == want, (hex(t), got, want)
