@@ -83,7 +83,7 @@ PREFILL_SMALL = [
     for (M, K, N, g) in [(17, 256, 128, 64), (128, 512, 256, 128), (200, 1024, 300, 32), (300, 2048, 640, 64),
                          # K % 64 == 32 (half of the last stage past K) and K/g % 8 != 0 (scalar parameter windows)
                          (40, 1056, 200, 32),
-                         # enough 128 x 256 tiles to fill the GPU: the wide tile path
+                         # more 128 x 256 tiles (160) than SMs: a persistent CTA takes a second tile
                          (1280, 512, 4096, 32)]
 ]
 
