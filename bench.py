@@ -63,11 +63,11 @@ def load_peaks():
 # shared header of device helpers): its ncu counters stay valid while these hash
 # the same.
 KERNEL_SOURCES = {
-    "bitlinear_reg_kernel": ("k_gemv.cu", "qlin_common.cuh"),
+    "bitlinear_kernel": ("k_bitlinear.cu", "qlin_common.cuh"),
 }
 
 
-def kernel_source_hash(kernel_key: str = "bitlinear_reg_kernel") -> str:
+def kernel_source_hash(kernel_key: str = "bitlinear_kernel") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_quantized_linear_qmm_b200", "csrc")
     for name in KERNEL_SOURCES[kernel_key]:
@@ -209,7 +209,7 @@ def _copies(bytes_per_copy: int, l2_bytes: int, minimum: int = 2) -> int:
 class BitlinearDecode:
     """BitLinear ternary decode GEMV: x bf16 [M, 4096], packed uint8 [1024, 4096],
     M in {1, 8}, weight_scale 0.5, multiply and divide modes; no bias."""
-    key = "bitlinear_reg_kernel"
+    key = "bitlinear_kernel"
     unit = "GB/s"
     bound = "hbm"
 

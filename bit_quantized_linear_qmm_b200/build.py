@@ -38,17 +38,27 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ and link libqlin.so beside this file."""
-    os.makedirs(OBJDIR, exist_ok=True)
+TRACE_LIB = os.path.join(PKG, "libqlin_trace.so")
+
+
+def build(force: bool = False, verbose: bool = False, trace: bool = False) -> str:
+    """Compile every .cu under csrc/ and link libqlin.so beside this file.
+
+    trace=True builds the same sources with QLIN_TRACE into libqlin_trace.so instead: the
+    decode kernels then record %globaltimer stamps per CTA (read with qlin_trace_read); the
+    product library is never built that way."""
+    objdir = os.path.join(OBJDIR, "trace") if trace else OBJDIR
+    lib = TRACE_LIB if trace else LIB
+    extra = ["-DQLIN_TRACE"] if trace else []
+    os.makedirs(objdir, exist_ok=True)
     headers = sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "qlin.h")]
     jobs = []
     objs = []
     for src in _sources():
-        obj = os.path.join(OBJDIR, os.path.basename(src).replace(".cu", ".o"))
+        obj = os.path.join(objdir, os.path.basename(src).replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            jobs.append([NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj])
+            jobs.append([NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj])
 
     def run(cmd):
         if verbose:
@@ -62,13 +72,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
         for err in ex.map(run, jobs):
             if verbose and err:
                 print(err, file=sys.stderr)
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         run([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-lrt", "-lpthread", "-ldl"])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv))

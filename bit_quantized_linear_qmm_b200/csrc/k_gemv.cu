@@ -1,10 +1,10 @@
-// k_gemv.cu -- decode-regime (M <= 16) quantized GEMV kernels for sm_100a.
+// k_gemv.cu -- decode-regime (M <= 16) quantized GEMV kernels for sm_100a:
+// the MLX-affine layer and the weight-streaming halves of W8A8 / W4A8.
+// (BitLinear's decode kernel is in k_bitlinear.cu.)
 //
 //   affine:    y[m,n] = sum_k x[m,k] * (q[n,k]*s[n,k/g] + b[n,k/g]) + bias[n]
 //              [nuvec-nn QuantizedLinear, forward / fields weight, scales,
 //               biases; cider/ops.py pergroup_linear docstring, dequantize]
-//   bitlinear: y[m, r + j*N/4] = scale * sum_k x[m,k] * (((P[r,k] >> 2j) & 3) - 1) + bias
-//              [mlx_lm bitlinear_layers.py, make_bitlinear_kernel, BitLinear.__call__]
 //
 // Design (B200, HBM- and latency-bound):
 //  * A CTA owns a block of output rows over the whole of K (about one CTA
@@ -22,13 +22,9 @@
 //    DRAM fetch overlaps the previous layer's tail.  Eight consumer warps
 //    take whole groups round robin; each covers all the CTA's 16-row tiles,
 //    so every x fragment serves them all.
-//  * bitlinear: a layer's packed weights are small enough (a few MB) for the
-//    CTAs to hold them in registers: they are loaded before
-//    griddepcontrol.wait, and only x is read after it.
-//  * Both dequantise in registers and run the MACs on the tensor cores with
-//    the legacy mma.sync.m16n8k16 (weights as the 16-row A operand, x as the
-//    n=8 B operand, fp32 accumulation); partial tiles are summed through
-//    shared memory.
+//  * The MACs run on the tensor cores with the legacy mma.sync (weights as
+//    the 16-row A operand, x as the n=8 B operand, fp32 accumulation);
+//    partial tiles are summed through shared memory.
 //  * affine: codes become bf16 with one LOP3 per pair: (w >> s) & 0x000F000F
 //    | 0x43004300 is the bf16 pair (128 + q_i, 128 + q_j), exact.  The 128
 //    offset and the group bias fold out per group with the group sums of x,
@@ -38,10 +34,6 @@
 //    (8-bit codes use no offset: bf16 holds 0..255 exactly.)  Because a dot
 //    product over a group does not depend on the order of k, each lane pairs
 //    codes in the order the LOP3 yields them and permutes x to match (PRMT).
-//  * bitlinear: each 2-bit field is read in place by one LOP3 as the bf16
-//    128 + 4^j c and turned into the exact weight c - 1 by one bf16x2 FMA
-//    (times 4^-j, minus 128 4^-j + 1), so a code-1 weight contributes an
-//    exact zero.
 //  * Every mbarrier wait is bounded (qlin::kWaitLimitNs); on expiry the
 //    kernel records the timeout in the status word, stops issuing copies,
 //    waits (bounded) for its copies in flight and runs to completion.
@@ -858,224 +850,7 @@ __global__ void __launch_bounds__(kThreads, 2) w4_gemv_kernel(const __grid_const
     }
 }
 
-// ---------------------------------------------------------------- bf16x2 helper
-
-QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
-{
-    uint32_t r;
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-    return r;
-}
-
-// ---------------------------------------------------------------- BitLinear decode
-
-// A CTA owns 8 packed rows (32 outputs) over the whole of K.  Its 8 warps
-// take 64-k chunks round robin; lane (g, t) of a warp handles, per chunk, the
-// 16 bytes k = 64c + 16t .. +15 of packed row g and the same 16 x values of
-// token g (and g + 8 when M > 8).  Each 32-bit weight word (4 consecutive k)
-// feeds two mma.m16n8k16: fields {0, 2} and {1, 3} as A rows g and g + 8.
-// Its bytes are first reordered (0, 2, 1, 3), so that the bf16 pairs the
-// LOP3 decode yields are consecutive k, like x in memory.
-//
-// Data movement: the packed weights go straight from HBM into registers
-// before griddepcontrol.wait (under programmatic dependent launch a layer's
-// weight stream overlaps the previous kernel); after the wait each lane
-// streams its x through a small ring of registers.  With K % 64 == 0 and at
-// most eight chunks per warp (K <= 4096) a lean variant drops the per-chunk
-// bounds logic and the refill of later rounds.
-//
-// The grid has at least one CTA per SM; the spare ones only pass the
-// dependency wait.  With every kernel holding one CTA on every SM, the next
-// layer's CTAs (two fit per SM) tend to land one per SM as well.
-constexpr int kBlWarps = 8;
-constexpr int kBlThreads = kBlWarps * 32;
-constexpr int kBlRows = 8;    // packed rows per CTA (32 outputs)
-constexpr int kBlChunk = 64;  // k per chunk
-constexpr int kBlRound = 8;   // chunks a warp holds in registers at once
-
-struct BitRegParams {
-    const uint8_t* packed;   // [R][K]
-    const __nv_bfloat16* x;  // [M][K]
-    const float* weight_scale;
-    const __nv_bfloat16* bias;
-    __nv_bfloat16* y;  // [M][N]
-    int M, K, N, R;
-    int tiles;  // CTAs with rows to compute
-    int invert;
-    unsigned* status;
-};
-
-// NT token tiles of 8; XD-deep x ring; FAST: whole chunks and a single round.
-template <int NT, int XD, bool FAST>
-__global__ void __launch_bounds__(kBlThreads, 2) bitlinear_reg_kernel(const __grid_constant__ BitRegParams p)
-{
-    static_assert(kBlRound % XD == 0, "x ring depth must divide the register round");
-    __shared__ float red[kBlWarps * 8 * NT * 32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gid = lane >> 2, tig = lane & 3;
-
-    pdl_launch_dependents();
-    if ((int)blockIdx.x >= p.tiles) {
-        // hold this SM's slot until the previous kernel is done, then leave
-        pdl_wait_prior_grids();
-        return;
-    }
-    const int p0 = blockIdx.x * kBlRows;
-    const int nch = (p.K + kBlChunk - 1) / kBlChunk;
-    const int my = nch > warp ? (nch - 1 - warp) / kBlWarps + 1 : 0;  // chunks of this warp
-    const bool row_ok = p0 + gid < p.R;
-    const uint8_t* wrow = p.packed + (size_t)(row_ok ? p0 + gid : 0) * p.K + 16 * tig;
-    // ci-th chunk of this warp: c = warp + 8 ci, k = 64 c + 16 tig
-    auto chunk_k = [&](int ci) { return (warp + ci * kBlWarps) * kBlChunk; };
-
-    auto load_w = [&](uint4& dst, int ci) {
-        if (row_ok && ci < my && (FAST || chunk_k(ci) + 16 * tig < p.K))
-            dst = ldg_stream_v4(wrow + chunk_k(ci));
-        else
-            dst = make_uint4(0u, 0u, 0u, 0u);
-    };
-    auto load_x = [&](uint4 (&dst)[NT][2], int ci) {
-        const int k = chunk_k(ci) + 16 * tig;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const int m = 8 * t + gid;
-            if (ci < my && m < p.M && (FAST || k < p.K)) {
-                const __nv_bfloat16* src = p.x + (size_t)m * p.K + k;
-                dst[t][0] = ldg_cg_v4(src);
-                dst[t][1] = ldg_cg_v4(src + 8);
-            } else {
-                dst[t][0] = dst[t][1] = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-    };
-
-    uint4 wr[kBlRound];
-#pragma unroll
-    for (int j = 0; j < kBlRound; ++j)
-        load_w(wr[j], j);
-    pdl_wait_prior_grids();  // x, weight_scale and y may belong to the previous kernel
-    uint4 xb[XD][NT][2];
-#pragma unroll
-    for (int d = 0; d < XD; ++d)
-        load_x(xb[d], d);
-    const float ws = *p.weight_scale;
-    const float scale = p.invert ? __fdiv_rn(1.0f, ws) : ws;
-
-    // per-field bf16x2 constants {4^-j, -(128 4^-j + 1)}: (128 + 4^j c) -> c - 1, exact
-    constexpr uint32_t kScale0 = 0x3F803F80u, kBias0 = 0xC301C301u;  // j=0: 1, -129
-    constexpr uint32_t kScale1 = 0x3E803E80u, kBias1 = 0xC204C204u;  // j=1: 1/4, -33
-    constexpr uint32_t kScale2 = 0x3D803D80u, kBias2 = 0xC110C110u;  // j=2: 1/16, -9
-    constexpr uint32_t kMagic = 0x43004300u;
-    // with one token tile, two accumulator sets (even / odd steps) keep four
-    // MMA chains in flight per warp
-    constexpr int AS = NT == 1 ? 2 : 1;
-    float a02[AS][NT][4], a13[AS][NT][4];
-#pragma unroll
-    for (int h = 0; h < AS; ++h)
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                a02[h][t][e] = a13[h][t][e] = 0.f;
-
-    auto chunk = [&](const uint4& w4, const uint4 (&xv)[NT][2]) {
-        const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {  // k = 64c + 16 tig + 4i .. +3
-            const uint32_t w = prmt(wv[i], 0u, 0x3120);  // bytes (k, k+2, k+1, k+3)
-            const uint32_t hw = w >> 8;                 // k+2, k+3 in the low byte of each half
-            uint32_t f02[4], f13[4];
-            f02[0] = bf16x2_fma(lop3_and_or(w, 0x00030003u, kMagic), kScale0, kBias0);        // f0 (k, k+1)
-            f02[1] = bf16x2_fma(lop3_and_or(w, 0x00300030u, kMagic), kScale2, kBias2);        // f2 (k, k+1)
-            f02[2] = bf16x2_fma(lop3_and_or(hw, 0x00030003u, kMagic), kScale0, kBias0);       // f0 (k+2, k+3)
-            f02[3] = bf16x2_fma(lop3_and_or(hw, 0x00300030u, kMagic), kScale2, kBias2);       // f2 (k+2, k+3)
-            f13[0] = bf16x2_fma(lop3_and_or(w, 0x000C000Cu, kMagic), kScale1, kBias1);        // f1 (k, k+1)
-            f13[1] = bf16x2_fma(lop3_and_or(w >> 6, 0x00030003u, kMagic), kScale0, kBias0);   // f3 (k, k+1)
-            f13[2] = bf16x2_fma(lop3_and_or(hw, 0x000C000Cu, kMagic), kScale1, kBias1);       // f1 (k+2, k+3)
-            f13[3] = bf16x2_fma(lop3_and_or(w >> 14, 0x00030003u, kMagic), kScale0, kBias0);  // f3 (k+2, k+3)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const uint4& xh = xv[t][i >> 1];
-                const uint32_t b0 = (i & 1) ? xh.z : xh.x;  // (x_k, x_k+1)
-                const uint32_t b1 = (i & 1) ? xh.w : xh.y;  // (x_k+2, x_k+3)
-                mma_bf16_16816(a02[i % AS][t], f02, b0, b1);
-                mma_bf16_16816(a13[i % AS][t], f13, b0, b1);
-            }
-        }
-    };
-
-    if constexpr (FAST) {
-#pragma unroll
-        for (int j = 0; j < kBlRound; ++j) {
-            if (j < my)
-                chunk(wr[j], xb[j % XD]);
-            if (j + XD < kBlRound)
-                load_x(xb[j % XD], j + XD);
-        }
-    } else {
-        const int rounds = (my + kBlRound - 1) / kBlRound;
-        for (int rd = 0; rd < rounds; ++rd) {
-#pragma unroll
-            for (int j = 0; j < kBlRound; ++j) {
-                const int ci = rd * kBlRound + j;
-                if (ci < my)
-                    chunk(wr[j], xb[j % XD]);
-                load_x(xb[j % XD], ci + XD);
-                load_w(wr[j], ci + kBlRound);
-            }
-        }
-    }
-
-    // sum the 8 warps' partial tiles; v = t * 8 + a * 4 + e (a: fields {0,2} / {1,3})
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            red[((warp * NT + t) * 8 + e) * 32 + lane] = a02[0][t][e] + (AS > 1 ? a02[AS - 1][t][e] : 0.f);
-            red[((warp * NT + t) * 8 + 4 + e) * 32 + lane] = a13[0][t][e] + (AS > 1 ? a13[AS - 1][t][e] : 0.f);
-        }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < NT * 8 * 32; idx += kBlThreads) {
-        const int v = idx >> 5, ln = idx & 31;
-        float sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < kBlWarps; ++w)
-            sum += red[(w * NT * 8 + v) * 32 + ln];
-        const int t = v >> 3, a = (v >> 2) & 1, e = v & 3;
-        const int pr = p0 + (ln >> 2);
-        const int m = 8 * t + 2 * (ln & 3) + (e & 1);
-        if (pr < p.R && m < p.M) {
-            const int n = pr + (a + 2 * (e >> 1)) * p.R;
-            float out = sum * scale;
-            if (p.bias)
-                out += __bfloat162float(p.bias[n]);
-            p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(out);
-        }
-    }
-}
-
 // ---------------------------------------------------------------- launch helpers
-
-template <typename Kern, typename Params>
-cudaError_t launch_pdl_threads(Kern kern, dim3 grid, int threads, int smem, cudaStream_t st, const Params& prm)
-{
-    if (smem > 0) {  // static + dynamic above 48 KB needs the opt-in
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3((unsigned)threads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, prm);
-}
 
 template <typename Kern, typename Params>
 cudaError_t launch_pdl(Kern kern, dim3 grid, int smem, cudaStream_t st, const Params& prm)
@@ -1184,41 +959,6 @@ cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const D
     return a.p_dt == QLIN_BF16 ? affine_launch_b<float, __nv_bfloat16>(a, st, dev)
                                : affine_launch_b<float, float>(a, st, dev);
 }
-
-cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const DeviceInfo& dev)
-{
-    const int R = (int)(a.N / 4);
-    const int tiles = (R + kBlRows - 1) / kBlRows;
-    const dim3 grid((unsigned)(tiles > dev.sm_count ? tiles : dev.sm_count), 1, 1);
-    for (int64_t m0 = 0; m0 < a.M; m0 += 16) {
-        const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
-        BitRegParams prm;
-        prm.packed = a.packed;
-        prm.x = static_cast<const __nv_bfloat16*>(a.x) + m0 * a.K;
-        prm.weight_scale = a.weight_scale;
-        prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
-        prm.y = static_cast<__nv_bfloat16*>(a.y) + m0 * a.N;
-        prm.M = mc;
-        prm.K = (int)a.K;
-        prm.N = (int)a.N;
-        prm.R = R;
-        prm.tiles = tiles;
-        prm.invert = a.invert;
-        prm.status = dev.status;
-        const bool fast = a.K % kBlChunk == 0 && a.K <= (int64_t)kBlChunk * kBlWarps * kBlRound;
-        cudaError_t e;
-        if (mc <= 8 && fast)
-            e = launch_pdl_threads(bitlinear_reg_kernel<1, 2, true>, grid, kBlThreads, 0, st, prm);
-        else if (mc <= 8)
-            e = launch_pdl_threads(bitlinear_reg_kernel<1, 4, false>, grid, kBlThreads, 0, st, prm);
-        else
-            e = launch_pdl_threads(bitlinear_reg_kernel<2, 2, false>, grid, kBlThreads, 0, st, prm);
-        if (e != cudaSuccess)
-            return e;
-    }
-    return cudaSuccess;
-}
-
 
 cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {

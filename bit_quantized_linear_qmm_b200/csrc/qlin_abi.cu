@@ -23,6 +23,8 @@ struct DeviceSlot {
 
 DeviceSlot g_slots[kMaxDevices];
 
+}  // namespace
+
 // Checks (once per device) that the current device is an sm_100 part, and
 // records its SM count and the address of the status word.  Must run with
 // that device current, outside stream capture (the first call per device).
@@ -58,6 +60,8 @@ qlin_status current_device(DeviceInfo& out)
     out = slot.info;
     return slot.state;
 }
+
+namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool dtype_ok(qlin_dtype d) { return d == QLIN_F32 || d == QLIN_BF16; }

@@ -277,6 +277,10 @@ struct DeviceInfo {
     unsigned* status;  // device status word
 };
 
+// The current device's DeviceInfo after a one-time check that it is an sm_100
+// part (QLIN_ERR_DEVICE otherwise); defined in qlin_abi.cu.
+qlin_status current_device(DeviceInfo& out);
+
 // Host: encodes a 2-D tiled tensor map (row-major [dim1][dim0] elements,
 // row pitch `pitch_bytes`) with box {box0, box1}, 128-byte swizzle, zero
 // fill (or the given swizzle).  Returns false if the driver entry point is unavailable or rejects

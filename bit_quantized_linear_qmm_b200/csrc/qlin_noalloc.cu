@@ -24,29 +24,34 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
+std::mutex g_mu;
 void* g_ptr[kMaxDevices];
-cudaError_t g_err[kMaxDevices];
 
-// Device address of the scratch array on the current device.  Looked up once
-// per device, on the first call made with that device current; the host-side
-// symbol itself is only a stand-in and must never reach a kernel.
+// Device address of the scratch array on the current device, after the same
+// sm_100 check every entry point makes.  Looked up on the first call made with
+// that device current (kept only once the lookup succeeded, so a failed first
+// attempt is retried on the next call); the host-side symbol itself is only a
+// stand-in and must never reach a kernel.
 qlin_status scratch_address(void** out)
 {
+    DeviceInfo info;
+    const qlin_status s = current_device(info);
+    if (s != QLIN_OK)
+        return s;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
         return QLIN_ERR_DEVICE;
     }
-    std::call_once(g_once[dev], [dev]() {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_ptr[dev] == nullptr) {
         void* p = nullptr;
-        g_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (g_err[dev] != cudaSuccess)
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
             cudaGetLastError();
+            return QLIN_ERR_CUDA;
+        }
         g_ptr[dev] = p;
-    });
-    if (g_err[dev] != cudaSuccess || g_ptr[dev] == nullptr)
-        return QLIN_ERR_CUDA;
+    }
     *out = g_ptr[dev];
     return QLIN_OK;
 }

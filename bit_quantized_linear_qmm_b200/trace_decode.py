@@ -1,0 +1,107 @@
+"""Time breakdown of the BitLinear decode kernel inside a chain of dependent layers.
+
+    python -m bit_quantized_linear_qmm_b200.trace_decode [--layers L] [--copies C]
+
+Builds the trace variant of the library (libqlin_trace.so: the same sources
+compiled with QLIN_TRACE, whose decode kernel records %globaltimer stamps per
+CTA), runs L BitLinear layers (K = N = 4096; M = 1, 1, 8, 8 repeating, the
+multiply and divide modes alternating) back to back in one CUDA graph with the
+weights rotating over C device copies (so each layer streams its weights from
+HBM), and prints, averaged over the layers:
+
+  period        graph time / L (the time per layer)
+  release       first CTA's griddepcontrol.wait return minus the previous
+                layer's last CTA end
+  x+chunk0      wait return -> first 64-k chunk done (x arrival + one chunk)
+  loop          rest of the main loop
+  reduce        CTA reduction, scaling, bias and y stores
+  critical      last CTA end minus first wait return
+  end spread    last CTA end minus first CTA end
+  doubled       SMs that ran two CTAs of the same layer (summed over layers)
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import os
+import sys
+
+import numpy as np
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from bit_quantized_linear_qmm_b200 import build, qlin  # noqa: E402
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--copies", type=int, default=64)
+    args = ap.parse_args()
+    path = build.build(trace=True)
+    qlin.LIB_PATH = path  # the binding loads the trace build instead of libqlin.so
+    L = qlin.lib()
+    L.qlin_trace_read.argtypes = [C.c_void_p, C.c_size_t]
+    L.qlin_trace_read.restype = C.c_int
+    ctas_max = int(L.qlin_trace_ctas())
+
+    torch.cuda.set_device(0)
+    cases = synth.BITLINEAR_DECODE  # M = 1, 1, 8, 8; multiply / divide
+    K, N = cases[0].K, cases[0].N
+    packed = torch.from_numpy(cases[0].packed()).cuda()
+    pool = [packed.clone() for _ in range(args.copies)]
+    xs = [c.x().torch("cuda") for c in cases]
+    ys = [torch.empty((c.M, N), dtype=torch.bfloat16, device="cuda") for c in cases]
+    ws = torch.tensor([cases[0].weight_scale], dtype=torch.float32, device="cuda")
+
+    def chain():
+        for i in range(args.layers):
+            c = i % len(cases)
+            qlin.bitlinear_matmul(xs[c], pool[i % len(pool)], N, ws, cases[c].invert, out=ys[c])
+
+    chain()  # first calls outside capture
+    torch.cuda.synchronize()
+    L.qlin_trace_read(None, 0)  # reset the slot counter; the graph's launches take slots 0 .. L-1
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        chain()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    period_us = e0.elapsed_time(e1) * 1e3 / args.layers
+
+    buf = np.zeros((args.layers, ctas_max, 8), np.uint64)
+    used = L.qlin_trace_read(buf.ctypes.data, buf.nbytes)
+    assert used == args.layers, (used, args.layers)
+    grid = int(np.count_nonzero(buf[0, :, 0]))
+    t = buf[:, :grid, :].astype(np.int64)
+    rel, x0, loop, red, crit, spread, dbl = [], [], [], [], [], [], 0
+    for i in range(1, args.layers):
+        rel.append(t[i, :, 2].min() - t[i - 1, :, 5].max())
+        x0.append((t[i, :, 3] - t[i, :, 2]).mean())
+        loop.append((t[i, :, 4] - t[i, :, 3]).mean())
+        red.append((t[i, :, 5] - t[i, :, 4]).mean())
+        crit.append(t[i, :, 5].max() - t[i, :, 2].min())
+        spread.append(t[i, :, 5].max() - t[i, :, 5].min())
+        sm = t[i, :, 7]
+        dbl += int(np.sum(np.bincount(sm) > 1))
+    out = {"layers": args.layers, "ctas": grid, "period_us": round(period_us, 3),
+           "release_ns": round(float(np.mean(rel))), "x_chunk0_ns": round(float(np.mean(x0))),
+           "loop_ns": round(float(np.mean(loop))), "reduce_ns": round(float(np.mean(red))),
+           "critical_ns": round(float(np.mean(crit))), "end_spread_ns": round(float(np.mean(spread))),
+           "doubled_sms": dbl}
+    print(out, flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -29,17 +29,22 @@
  *     qlin_workspace_size()).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and never synchronise, except qlin_get_device_status().
- *   - Ordering on a stream: the GEMV / GEMM kernels (qlin_matmul,
- *     bitlinear_matmul, w8a8_linear, w8a8_linear_noalloc, w4a8_linear,
- *     qlin_int8_matmul_int32) use programmatic dependent launch: each releases
- *     the next kernel of the stream when it starts, and that kernel fetches
- *     its layer constants -- packed weights and group scales / biases --
- *     before waiting for its predecessor (x, the BitLinear weight scale, the
- *     layer bias and y only after).  So the packed weights and group
- *     parameters of a call must not be written by the call immediately
- *     before it on the same stream if that call is one of the above.  Any
- *     other predecessor (a quantize or pack call, a copy, another library's
- *     kernel) completes before the call starts.
+ *   - Ordering on a stream: the GEMV / GEMM kernels of qlin_matmul,
+ *     bitlinear_matmul and qlin_int8_matmul_int32, and the second kernel of
+ *     w8a8_linear, w8a8_linear_noalloc and w4a8_linear, use programmatic
+ *     dependent launch: each releases the next kernel of the stream as soon
+ *     as it starts, so in an unbroken run of such calls several kernels can
+ *     be resident at once.  Each fetches its layer constants -- packed
+ *     weights and group scales / biases -- BEFORE waiting for its
+ *     predecessors (x, the BitLinear weight scale, the layer bias and y only
+ *     after the wait, by which time every earlier kernel of the stream has
+ *     completed).  Rule: the packed weights and group parameters of a call
+ *     must not be written by ANY earlier call of the same run.  A run ends at
+ *     every other operation on the stream -- a quantize, dequantize or pack
+ *     call, the activation quantiser that opens each w8a8 / w4a8 call, a
+ *     copy, an event wait, another library's kernel -- because such an
+ *     operation starts only after everything before it has completed and
+ *     releases nothing early.
  *   - Every call validates its arguments before launching anything and
  *     returns a qlin_status; nothing is launched when it is not QLIN_OK.
  *     No C++ exception crosses this interface.
@@ -224,8 +229,9 @@ qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
  *     8 MiB (M*K rounded up to 256 bytes, plus 4*M rounded up to 256);
  *     larger problems return QLIN_ERR_WORKSPACE and launch nothing.
  *   - The buffer's device address is looked up on the first call made with
- *     a given device current; make that first call before any stream
- *     capture on that device.
+ *     a given device current (after the same sm_100 check as every other
+ *     call; a lookup that fails is retried on the next call); make that
+ *     first call before any stream capture on that device.
  *   - All calls share the one buffer and it keeps the last call's contents
  *     (every call rewrites what it reads, so nothing needs clearing).  Calls
  *     that may run at the same time on the GPU -- on different streams, or

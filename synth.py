@@ -62,6 +62,12 @@ def ternary_bytes(seed: int, rows: int, K: int) -> np.ndarray:
     return _TERNARY_BYTES[idx]
 
 
+def any_bytes(seed: int, rows: int, K: int) -> np.ndarray:
+    """uint8 [rows, K] uniform over all 256 values (2-bit fields 0..3, code 3 included)."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 256, size=(rows, K)).astype(np.uint8)
+
+
 def ternary_codes(seed: int, N: int, K: int) -> np.ndarray:
     """uint8 [N, K] codes uniform in {0, 1, 2} (unpacked form)."""
     rng = np.random.default_rng(seed)
@@ -134,8 +140,11 @@ class BitLinearCase:
     bias: bool = False
     x_dtype: str = "bf16"
     seed: int = 0
+    all_bytes: bool = False  # fields uniform in 0..3 (code 3 included) instead of {0, 1, 2}
 
     def packed(self) -> np.ndarray:
+        if self.all_bytes:
+            return any_bytes(self.seed, self.N // 4, self.K)
         return ternary_bytes(self.seed, self.N // 4, self.K)
 
     def x(self) -> Activations:

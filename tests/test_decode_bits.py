@@ -98,34 +98,56 @@ def test_affine_pair_decode_every_byte(pos):
 # ---------------------------------------------------------------- BitLinear 2-bit fields
 
 def test_bitlinear_decode_constants_in_source():
-    s = _src("k_gemv.cu")
-    for c in ("kScale0 = 0x3F803F80u, kBias0 = 0xC301C301u", "kScale1 = 0x3E803E80u, kBias1 = 0xC204C204u",
-              "kScale2 = 0x3D803D80u, kBias2 = 0xC110C110u", "kMagic = 0x43004300u",
-              "prmt(wv[i], 0u, 0x3120)", "lop3_and_or(w, 0x00030003u, kMagic), kScale0, kBias0",
-              "lop3_and_or(w, 0x00300030u, kMagic), kScale2, kBias2",
-              "lop3_and_or(w, 0x000C000Cu, kMagic), kScale1, kBias1",
-              "lop3_and_or(w >> 6, 0x00030003u, kMagic), kScale0, kBias0",
-              "lop3_and_or(w >> 14, 0x00030003u, kMagic), kScale0, kBias0"):
+    s = _src("k_bitlinear.cu")
+    for c in ("kMagic = 0x43004300u", "kScale0 = 0x3F803F80u, kBias0 = 0xC301C301u",
+              "kScale1 = 0x3E803E80u, kBias1 = 0xC204C204u", "kScale2 = 0x3D803D80u, kBias2 = 0xC110C110u",
+              "kScale3 = 0x3C803C80u, kBias3 = 0xC040C040u", "kTwo = 0x40004000u",
+              "prmt(raw, 0u, 0x0100u)", "prmt(raw, 0u, 0x0302u)",
+              "f[0] = bf16x2_fma(lop3_and_or(lo, 0x00030003u, kMagic), kScale0, kBias0)",
+              "f[1] = bf16x2_fma(lop3_and_or(lo, 0x00300030u, kMagic), kScale2, kBias2)",
+              "f[2] = bf16x2_fma(lop3_and_or(hi, 0x00030003u, kMagic), kScale0, kBias0)",
+              "f[3] = bf16x2_fma(lop3_and_or(hi, 0x00300030u, kMagic), kScale2, kBias2)",
+              "f[4] = bf16x2_fma(lop3_and_or(lo, 0x000C000Cu, kMagic), kScale1, kBias1)",
+              "f[5] = bf16x2_min(bf16x2_fma(lop3_and_or(lo, 0x00C000C0u, kMagic), kScale3, kBias3), kTwo)",
+              "f[6] = bf16x2_fma(lop3_and_or(hi, 0x000C000Cu, kMagic), kScale1, kBias1)",
+              "f[7] = bf16x2_min(bf16x2_fma(lop3_and_or(hi, 0x00C000C0u, kMagic), kScale3, kBias3), kTwo)"):
         assert c in s, c
+
+
+def _min2(pair, two=0x40004000):
+    t0, t1 = halves(two)
+    return min(pair[0], t0), min(pair[1], t1)
 
 
 def _bitlinear_chunk(word: int):
     """The kernel's decode of one 32-bit word (bytes k .. k+3 of one packed row): field j of byte k
-    -> (k, value) pairs, as the four f02 / f13 registers produce them."""
+    -> value, as the eight A registers f[0..7] produce them."""
     MAGIC = 0x43004300
     S0, B0, S1, B1, S2, B2 = 0x3F803F80, 0xC301C301, 0x3E803E80, 0xC204C204, 0x3D803D80, 0xC110C110
-    w = prmt(word, 0, 0x3120)  # bytes (k, k+2, k+1, k+3)
-    hw = w >> 8
+    S3, B3 = 0x3C803C80, 0xC040C040
+    lo = prmt(word, 0, 0x0100)  # bytes k, k+1 in the low byte of each half
+    hi = prmt(word, 0, 0x0302)  # bytes k+2, k+3
     out = {}
-    out[(0, 0)], out[(0, 1)] = fma_exact_pair(lop3_and_or(w, 0x00030003, MAGIC), S0, B0)
-    out[(2, 0)], out[(2, 1)] = fma_exact_pair(lop3_and_or(w, 0x00300030, MAGIC), S2, B2)
-    out[(0, 2)], out[(0, 3)] = fma_exact_pair(lop3_and_or(hw, 0x00030003, MAGIC), S0, B0)
-    out[(2, 2)], out[(2, 3)] = fma_exact_pair(lop3_and_or(hw, 0x00300030, MAGIC), S2, B2)
-    out[(1, 0)], out[(1, 1)] = fma_exact_pair(lop3_and_or(w, 0x000C000C, MAGIC), S1, B1)
-    out[(3, 0)], out[(3, 1)] = fma_exact_pair(lop3_and_or(w >> 6, 0x00030003, MAGIC), S0, B0)
-    out[(1, 2)], out[(1, 3)] = fma_exact_pair(lop3_and_or(hw, 0x000C000C, MAGIC), S1, B1)
-    out[(3, 2)], out[(3, 3)] = fma_exact_pair(lop3_and_or(w >> 14, 0x00030003, MAGIC), S0, B0)
+    out[(0, 0)], out[(0, 1)] = fma_exact_pair(lop3_and_or(lo, 0x00030003, MAGIC), S0, B0)
+    out[(2, 0)], out[(2, 1)] = fma_exact_pair(lop3_and_or(lo, 0x00300030, MAGIC), S2, B2)
+    out[(0, 2)], out[(0, 3)] = fma_exact_pair(lop3_and_or(hi, 0x00030003, MAGIC), S0, B0)
+    out[(2, 2)], out[(2, 3)] = fma_exact_pair(lop3_and_or(hi, 0x00300030, MAGIC), S2, B2)
+    out[(1, 0)], out[(1, 1)] = fma_exact_pair(lop3_and_or(lo, 0x000C000C, MAGIC), S1, B1)
+    out[(3, 0)], out[(3, 1)] = _min2(fma_exact_pair(lop3_and_or(lo, 0x00C000C0, MAGIC), S3, B3))
+    out[(1, 2)], out[(1, 3)] = fma_exact_pair(lop3_and_or(hi, 0x000C000C, MAGIC), S1, B1)
+    out[(3, 2)], out[(3, 3)] = _min2(fma_exact_pair(lop3_and_or(hi, 0x00C000C0, MAGIC), S3, B3))
     return out  # (field j, k offset) -> value
+
+
+def test_bitlinear_field3_pattern():
+    """Field 3 sits on the exponent's low bit: codes 0..3 read 128, 192, 256, 384 (not affine),
+    the FMA gives -1, 0, 1, 3 and the min with 2 gives code 3 its weight 2."""
+    for c in range(4):
+        v = lop3_and_or(c << 6, 0x00C000C0, 0x43004300)
+        assert halves(v)[0] == [128, 192, 256, 384][c]
+        raw = fma_exact_pair(v, 0x3C803C80, 0xC040C040)[0]
+        assert raw == [-1, 0, 1, 3][c]
+        assert _min2((raw, raw))[0] == (c - 1 if c < 3 else 2)
 
 
 def test_bitlinear_fields_every_byte():

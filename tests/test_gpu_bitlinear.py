@@ -38,6 +38,33 @@ def test_bitlinear_small(ql, orc, case):
     _run(ql, orc, case)
 
 
+# every byte value (code 3 -> weight 2), the one-CTA-per-SM split (N = 4096), 8-row CTAs in waves
+# (N > 4736 on 148 SMs), K beyond one register round (K > 4096) and a partial last chunk
+# (K % 64 != 0), fewer packed rows than SMs, and M > 16 (16-token slices)
+WIDE = [synth.BitLinearCase(f"all_bytes_M{M}_K{K}_N{N}_{'div' if inv else 'mul'}{'_bias' if b else ''}", M, K, N,
+                            0.5, inv, b, seed=21, all_bytes=True)
+        for (M, K, N, inv, b) in [(1, 4096, 4096, False, False), (8, 4096, 4096, True, False),
+                                  (16, 4096, 4096, False, True), (3, 1040, 6000, False, True),
+                                  (8, 4112, 1024, True, False), (1, 8192, 512, False, False),
+                                  (12, 2064, 64, True, True), (17, 512, 520, False, True),
+                                  (40, 1024, 1024, True, False)]]
+
+
+@pytest.mark.parametrize("case", WIDE, ids=[c.name for c in WIDE])
+def test_bitlinear_all_bytes_and_paths(ql, orc, case):
+    _run(ql, orc, case)
+
+
+def test_bitlinear_code3_is_two(ql):
+    """All codes 3 (weight 2): y = 2 rowsum(x) * scale, exact for small-integer x."""
+    x = torch.randint(-4, 5, (5, 1024), device="cuda").to(torch.bfloat16)
+    P = torch.full((16, 1024), 0xFF, dtype=torch.uint8, device="cuda")
+    ws = torch.tensor([0.5], device="cuda")
+    y = ql.bitlinear_matmul(x, P, 64, ws, False).float()
+    expect = x.float().sum(dim=1, keepdim=True).expand(5, 64) * 2 * 0.5
+    assert torch.equal(y, expect)
+
+
 @pytest.mark.parametrize("case", synth.BITLINEAR_DECODE, ids=[c.name for c in synth.BITLINEAR_DECODE])
 def test_bitlinear_decode_config_full(ql, orc, case):
     _run(ql, orc, case)

@@ -1,7 +1,8 @@
 """w8a8_linear_noalloc: the W8A8 layer for callers that cannot give the
 library device memory (its scratch is a buffer inside libqlin.so).  Checked
-through the C ABI against w8a8_linear, within the suite's tolerance, on two
-calls in a row.  This file is collected last on purpose."""
+through the C ABI against w8a8_linear (bit-equal) and the oracle (fp bar) on
+three calls in a row that cover both kernel paths.  This file is collected
+last on purpose."""
 import ctypes as C
 
 import numpy as np
@@ -24,6 +25,10 @@ def _call_noalloc(ql, x, w, s, bias, y):
 
 
 def test_noalloc_matches_w8a8_linear_twice(orc):
+    """Three calls in a row on the built-in scratch: the tcgen05 GEMM (M = 300), the
+    weight-streaming GEMV (M = 8) and the GEMM again with a ragged M.  Each is bit-equal
+    to w8a8_linear with a caller workspace (the same deterministic kernels) and within
+    the fp bar of the oracle."""
     ql = build_lib()
     N, K = 384, 2048
     w = synth.normal(61, (N, K), 0.02)
@@ -31,16 +36,18 @@ def test_noalloc_matches_w8a8_linear_twice(orc):
     wd, sd = to_dev(qw), to_dev(sw)
     lb = synth.activations(62, (N,), "bf16", 0.01)
     bias = lb.torch("cuda")
-    for call, (M, seed) in enumerate([(300, 63), (17, 64)]):
+    for call, (M, seed) in enumerate([(300, 63), (8, 65), (17, 64)]):
         xa = synth.activations(seed, (M, K), "bf16")
         x = xa.torch("cuda")
-        y_ref = ql.w8a8_linear(x, wd, sd, bias)
+        ws = torch.empty(ql.workspace_size(ql.QLIN_OP_W8A8, M, N, K), dtype=torch.uint8, device="cuda")
+        y_ref = ql.w8a8_linear(x, wd, sd, bias, workspace=ws)
         y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         assert _call_noalloc(ql, x, wd, sd, bias, y) == ql.QLIN_OK, f"call {call}"
         torch.cuda.synchronize()
-        _, mag, _, _ = orc.w8a8_linear(xa.vals, qw, sw, lb.vals)
+        assert torch.equal(y, y_ref), f"call {call} (M = {M}): differs from w8a8_linear"
+        yr, mag, _, _ = orc.w8a8_linear(xa.vals, qw, sw, lb.vals)
         tol = REL * (mag + np.abs(lb.vals)[None, :]) + ABS
-        err = np.abs(y.double().cpu().numpy() - y_ref.double().cpu().numpy())
+        err = np.abs(y.double().cpu().numpy() - yr)
         assert (err <= tol).all(), (call, float((err / tol).max()))
     assert ql.device_status() == ql.QLIN_OK
 
