@@ -362,10 +362,11 @@ def suite(l2: int, peaks: dict, int8_peak: float):
     bias = c.layer_bias().torch(dev)
     y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
     pool = [(codes.clone(), s.clone(), b.clone()) for _ in range(3)]
+    wsp = torch.empty(ql.workspace_size(ql.QLIN_OP_MATMUL, c.M, c.N, c.K, 4, 64), dtype=torch.uint8, device=dev)
 
     def stp(i):
         cc, ss, bb = pool[i % 3]
-        ql.matmul(x, cc, ss, bb, 4, 64, bias, out=y)
+        ql.matmul(x, cc, ss, bb, 4, 64, bias, out=y, workspace=wsp)
     us = time_steps(stp, 20, 3) * 1e3
     flops = 2.0 * c.M * c.N * c.K
     out.append(_entry(c.name, us, flops, "TFLOP/s", "tensor", bf16, "bf16 tcgen05, fp32 accumulate; dequant fused"))
@@ -478,6 +479,7 @@ PROFILE_CASES = {
     "affine_decode_m1": lambda: _prof_affine(1, 4096, 4096),
     "affine_decode_m1_k11008": lambda: _prof_affine(1, 11008, 4096),
     "affine_prefill_m512": lambda: _prof_affine(512, 4096, 14336),
+    "affine_prefill_m2048": lambda: _prof_affine(2048, 4096, 14336),
     "w8a8_m4096": lambda: _prof_int("w8a8", 4096),
     "w4a8_m4096": lambda: _prof_int("w4a8", 4096),
     "w8a8_m1": lambda: _prof_int("w8a8", 1),

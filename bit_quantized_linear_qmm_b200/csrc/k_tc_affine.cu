@@ -1,14 +1,24 @@
 // k_tc_affine.cu -- affine-format prefill GEMM on the 5th-generation tensor
 // cores with the dequantised weights as the tensor-memory A operand, sm_100a.
 //
-//   y[m,n] = sum_k x[m,k] * bf16(s[n,k/g] q[n,k] + b[n,k/g]) + bias[n]   (s q + b rounded once)
+//   y[m,n] = sum_k x[m,k] * (s[n,k/g] q[n,k] + b[n,k/g]) + bias[n]
 //   [nuvec-nn QuantizedLinear, forward; cider/ops.py pergroup_linear docstring, dequantize]
+//
+// Operands are fp16, so that every product is within 2^-11 of the exact one
+// (a bf16 operand would allow 2^-8): a preparation kernel writes, into the
+// caller's workspace,
+//   x16[m,k] = fp16(x[m,k] 2^-E_m)          E_m: max_k |x[m,k]| 2^-E_m in [2^14, 2^15)
+//   s16, b16 = fp16(s 2^-F_n), fp16(b 2^-F_n)  F_n: max_g (|b| + (2^bits-1)|s|) 2^-F_n in [2^14, 2^15)
+// (exact for bf16 inputs in fp16's normal range: the power-of-two factors keep
+// them there and rule out overflow), and the GEMM forms each weight as
+// fp16(s16 q + b16) -- the exact value, rounded once -- and scales the fp32
+// accumulator by 2^(E_m + F_n) in the epilogue.
 //
 // Each tile computes the transposed product  yT[128 weight rows][256 tokens] =
 // W^ . xT  as one M = 128, N = 256 MMA per 16-wide k step.  The dequantised
 // weights never touch shared memory: transform threads (two per weight row,
 // 32 k each per stage) read the 4-bit codes straight from global memory, turn
-// a code pair into bf16x2 in registers and write 16 columns each into tensor
+// a code pair into f16x2 in registers and write 16 columns each into tensor
 // memory with tcgen05.st; the tensor core reads them there (tcgen05.mma with
 // A in TMEM).  Shared memory carries only the x tile (TMA, 128-byte swizzle):
 // a stage moves 32 KB in and 32 KB out of it for 128 x 256 x 64 MACs, and
@@ -25,7 +35,7 @@
 //                with the next window in flight; a stage's tensor-memory store
 //                completes while the next stage is decoded
 //   warps 10..17 epilogue: warp w reads token half (w - 10) / 4 of lanes
-//                32 (w % 4) .. +31: tcgen05.ld, + bias[n], bf16 stores
+//                32 (w % 4) .. +31: tcgen05.ld, * 2^(E_m + F_n) + bias[n], bf16 stores
 // Every mbarrier wait is bounded; on expiry the kernel records the timeout,
 // every role stops, the MMA thread waits for its MMAs in flight, and TMEM is
 // always freed.
@@ -46,11 +56,13 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kXformWarps + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = kTT;       // A ring starts here
-constexpr int kCodePF = 4;          // stages of codes in flight per transform thread
+constexpr int kCodePF = 6;          // stages of codes in flight per transform thread (cp.async ring)
 constexpr int kGroupT = 4;          // token tiles that walk the weight tiles together
-// kind::f16: D f32, A and B bf16, both K-major, N = 256, M = 128
-constexpr uint32_t kIdesc =
-    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+// kind::f16: D f32, A and B f16 (format 0), both K-major, N = 256, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+// per transform thread, kCodePF stages of its 16 bytes of codes: [stage][transform thread]
+constexpr int kCodeRing = kCodePF * kXformWarps * 32 * 16;
 
 struct Bars {
     uint64_t xfull[kXStages];
@@ -63,17 +75,20 @@ struct Bars {
     uint32_t tmem;
     int abort_flag;
 };
-constexpr int kSmem = kXStages * kXBytes + (int)sizeof(Bars) + 1024;
+constexpr int kSmem = kXStages * kXBytes + kCodeRing + (int)sizeof(Bars) + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(kAccCols + kAStages * kACols <= kTmemCols, "tensor memory");
 
 struct TsParams {
-    CUtensorMap tm_x;                 // x [M][K] bf16, box {64, 256}, 128-byte swizzle
+    CUtensorMap tm_x;                 // x16 [M][K] fp16 (workspace), box {64, 256}, 128-byte swizzle
     const uint8_t* codes;             // [N][K/2]: LSB-first 4-bit codes
-    const unsigned short* scales;     // bf16 bits [N][K/g]
-    const unsigned short* biases;
-    const __nv_bfloat16* bias;        // [N] or null
-    __nv_bfloat16* out;               // [M][N]
+    const unsigned short* scales;     // fp16 bits [N][K/g]: s 2^-F_n (workspace)
+    const unsigned short* biases;     //                      b 2^-F_n
+    const float* tok_scale;           // [M] 2^E_m
+    const float* row_scale;           // [N] 2^F_n
+    const void* bias;                 // [N] or null, the output dtype
+    void* out;                        // [M][N] bf16, or fp32 when out_f32
+    int out_f32;
     int M, N, K;
     int g_shift, ng;                  // log2 g, K / g
     int tiles_t, tiles_w;
@@ -81,21 +96,11 @@ struct TsParams {
     unsigned* status;
 };
 
-QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
+QLIN_DEV uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c)
 {
     uint32_t d;
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
-}
-
-// 16 bytes of read-only global memory, not kept in L1 (each line is read once per CTA).
-QLIN_DEV uint4 ldg_nc_na_v4(const void* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]^T (kind::f16), one thread.
@@ -121,6 +126,17 @@ QLIN_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 
 QLIN_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 16-byte asynchronous global -> shared copy (L2 only); src_bytes = 0 writes zeros.
+QLIN_DEV void cp_async16(void* smem_dst, const void* src, int src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+QLIN_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's committed copy groups are still in flight.
+template <int N>
+QLIN_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 QLIN_DEV bool aborted(int* flag) { return *reinterpret_cast<volatile int*>(flag) != 0; }
 
 // Grouped tile order: kGroupT consecutive token tiles walk the weight tiles together.
@@ -139,7 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars& bars = *reinterpret_cast<Bars*>(smem + kXStages * kXBytes);
+    uint4* code_ring = reinterpret_cast<uint4*>(smem + kXStages * kXBytes);
+    Bars& bars = *reinterpret_cast<Bars*>(smem + kXStages * kXBytes + kCodeRing);
     auto X = [&](int s) { return smem + s * kXBytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -256,21 +273,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
             return min(wt * kTW + r, p.N - 1);
         };
-        // codes of stage (ti, kb) for this thread: 16 bytes (32 k) of row n; a half stage past K
-        // reads nothing (zero codes meet the zero-filled x columns there)
+        // codes of stage (ti, kb) for this thread: 16 bytes (32 k) of row n, copied kCodePF stages
+        // ahead into this thread's slots of the shared-memory ring with cp.async (one commit group
+        // per stage, so the wait before a stage's decode is explicit); a half stage past K or a
+        // stage past the last tile is written as zeros (zero codes meet the zero-filled x columns)
         int lti = 0, lkb = 0;
         const uint8_t* lrow = my_tiles > 0 ? p.codes + (size_t)row_of(0) * pitch + 16 * kh : p.codes;
-        auto load_next = [&](uint4& c) {
-            if (lti < my_tiles) {
-                c = lkb * kKE + 32 * kh < p.K ? ldg_nc_na_v4(lrow + (size_t)lkb * (kKE / 2))
-                                              : make_uint4(0u, 0u, 0u, 0u);
-                if (++lkb == nk) {
-                    lkb = 0;
-                    if (++lti < my_tiles)
-                        lrow = p.codes + (size_t)row_of(lti) * pitch + 16 * kh;
-                }
-            } else {
-                c = make_uint4(0u, 0u, 0u, 0u);
+        uint4* my_ring = code_ring + (warp - 2) * 32 + lane;  // slot j at my_ring[j * kXformWarps * 32]
+        auto load_next = [&](int slot) {
+            const bool in = lti < my_tiles && lkb * kKE + 32 * kh < p.K;
+            cp_async16(my_ring + slot * kXformWarps * 32, in ? lrow + (size_t)lkb * (kKE / 2) : p.codes, in ? 16 : 0);
+            cp_async_commit();
+            if (lti < my_tiles && ++lkb == nk) {
+                lkb = 0;
+                if (++lti < my_tiles)
+                    lrow = p.codes + (size_t)row_of(lti) * pitch + 16 * kh;
             }
         };
 
@@ -302,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         };
         uint4 curS = make_uint4(0u, 0u, 0u, 0u), curB = curS, nxtS = curS, nxtB = curS;
         int cur_ti = 0, cur_win = -1;
-        // bf16x2 (s, s) and (b, b) of this thread's 32 k of stage (ti, kb)
+        // f16x2 (s, s) and (b, b) of this thread's 32 k of stage (ti, kb)
         auto params_for = [&](int ti, int kb, uint32_t& s2, uint32_t& b2) {
             const int gi = min(kb * kKE + 32 * kh, p.K - 1) >> p.g_shift;
             const int win = gi >> 3;
@@ -328,10 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             b2 = bv | (bv << 16);
         };
 
-        uint4 cb[kCodePF];
 #pragma unroll
         for (int j = 0; j < kCodePF; ++j)
-            load_next(cb[j]);
+            load_next(j);
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols + 16 * kh);
         int ti = 0, kb = 0, as = 0, pend_as = -1;
         unsigned aph = 0u;
@@ -355,11 +371,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                     break;
                 uint32_t s2, b2;
                 params_for(ti, kb, s2, b2);
-                // a pair of codes (q, q') of one byte becomes bf16x2 in four instructions: PRMT puts
+                // a pair of codes (q, q') of one byte becomes f16x2 in four instructions: PRMT puts
                 // the byte (low half) and the byte of w >> 1 (high half) in place, one LOP3 makes the
-                // exact bf16 (128 + q, 128 + 8 q'), one bf16x2 FMA recovers (q, q') exactly, and one
-                // gives bf16(s q + b), the exact value rounded once.  Column c holds k = 2c, 2c + 1.
-                const uint32_t words[4] = {cb[j].x, cb[j].y, cb[j].z, cb[j].w};
+                // exact fp16 (1024 + q, 1024 + 8 q'), one f16x2 FMA recovers (q, q') exactly, and one
+                // gives fp16(s q + b), the exact value rounded once.  Column c holds k = 2c, 2c + 1.
+                cp_async_wait<kCodePF - 1>();  // this stage's copy (the oldest in flight) has landed
+                const uint4 cbj = my_ring[j * kXformWarps * 32];
+                const uint32_t words[4] = {cbj.x, cbj.y, cbj.z, cbj.w};
                 uint32_t o[16];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
@@ -367,12 +385,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const uint32_t sel = (uint32_t)(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12));
-                        const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x43004300u);
-                        const uint32_t qq = bf16x2_fma(v, 0x3E003F80u, 0xC180C300u);  // (1, 1/8), (-128, -16)
-                        o[4 * w + e] = bf16x2_fma(qq, s2, b2);
+                        const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x64006400u);
+                        const uint32_t qq = f16x2_fma(v, 0x30003C00u, 0xD800E400u);  // (1, 1/8), (-1024, -128)
+                        o[4 * w + e] = f16x2_fma(qq, s2, b2);
                     }
                 }
-                load_next(cb[j]);  // the stage kCodePF ahead
+                load_next(j);  // the stage kCodePF ahead, into the slot just read
                 publish();
                 if (!mbar_wait_bounded(&bars.aempty[as], aph ^ 1u, p.status) || aborted(&bars.abort_flag)) {
                     ok = false;
@@ -393,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         }
         if (ok)
             publish();
+        cp_async_wait<0>();  // no copy may still be landing in shared memory at exit
         tmem_wait_st();  // no store may be in flight when TMEM is released
         if (!ok)
             bars.abort_flag = 1;
@@ -412,20 +431,40 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             const int m0 = tt * kTT + th * (kTT / 2);
             const int n = wt * kTW + 32 * q + lane;
             const bool n_ok = n < p.N;
-            const float bn = (p.bias && n_ok) ? __bfloat162float(p.bias[n]) : 0.f;
+            const float bn = (p.bias && n_ok) ? (p.out_f32 ? static_cast<const float*>(p.bias)[n]
+                                                           : __bfloat162float(static_cast<const __nv_bfloat16*>(p.bias)[n]))
+                                              : 0.f;
+            const float rs = n_ok ? p.row_scale[n] : 0.f;
             const uint32_t acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(th * (kTT / 2));
-            __nv_bfloat16* o = p.out + (size_t)m0 * p.N + n;
+            const size_t o0 = (size_t)m0 * p.N + n;
 #pragma unroll 1
             for (int c = 0; c < kTT / 32; ++c) {
                 uint32_t v[16];
                 tmem_ld16(acc + (uint32_t)(c * 16), v);
                 if (!n_ok)
                     continue;
+                // token scales of the chunk (the workspace holds them for whole 256-token tiles)
+                float ts[16];
+                const float4* tsp = reinterpret_cast<const float4*>(p.tok_scale + m0 + c * 16);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 t4 = __ldg(tsp + u);
+                    ts[4 * u] = t4.x * rs;
+                    ts[4 * u + 1] = t4.y * rs;
+                    ts[4 * u + 2] = t4.z * rs;
+                    ts[4 * u + 3] = t4.w * rs;
+                }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int m = m0 + c * 16 + j;
-                    if (m < p.M)
-                        o[(size_t)(c * 16 + j) * p.N] = __float2bfloat16_rn(__uint_as_float(v[j]) + bn);
+                    if (m < p.M) {  // 2^E_m 2^F_n is an exact power of two: one rounding in the fma
+                        const float out = fmaf(__uint_as_float(v[j]), ts[j], bn);
+                        const size_t oi = o0 + (size_t)(c * 16 + j) * p.N;
+                        if (p.out_f32)
+                            static_cast<float*>(p.out)[oi] = out;
+                        else
+                            static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(out);
+                    }
                 }
             }
             tc_fence_before();
@@ -442,16 +481,179 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
 
 bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Power-of-two exponent that brings a magnitude bound v (> 0) into [2^14, 2^15).
+QLIN_DEV int prep_shift(float v)
+{
+    if (!(v > 0.f) || !isfinite(v))
+        return 0;
+    const int e = ilogbf(v) - 14;
+    return e < -120 ? -120 : e > 120 ? 120 : e;
+}
+
+QLIN_DEV float block_max(float v, float* red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0)
+        red[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = red[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+            m = fmaxf(m, red[w]);
+        red[32] = m;
+    }
+    __syncthreads();
+    return red[32];
+}
+
+// 8 consecutive x values (16-byte aligned) as fp32.
+QLIN_DEV void load8(const __nv_bfloat16* p, float (&v)[8])
+{
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+QLIN_DEV void load8(const float* p, float (&v)[8])
+{
+    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Blocks [0, M): token rows of x -> x16 and tok_scale (16-byte loads and stores; a row of up to
+// 256 * 8 * VPT values is held in registers between the max and the conversion).  Blocks
+// [M, M + ceil(N / 8)): one warp per weight row -> fp16 group parameters and row_scale.
+// qmax = 2^bits - 1.  K % 8 == 0.
+template <typename XT, int VPT>
+__global__ void __launch_bounds__(256) affine_prefill_prep_kernel(
+    const XT* __restrict__ x, int M, int K, const __nv_bfloat16* __restrict__ scales,
+    const __nv_bfloat16* __restrict__ biases, int N, int ng, float qmax, __half* __restrict__ x16,
+    __half* __restrict__ s16, __half* __restrict__ b16, float* __restrict__ tok_scale, float* __restrict__ row_scale)
+{
+    pdl_launch_dependents();  // the GEMM waits for this kernel before reading anything it writes
+    __shared__ float red[33];
+    if ((int)blockIdx.x < M) {
+        const int m = blockIdx.x;
+        const XT* row = x + (size_t)m * K;
+        const int n8 = K / 8;
+        float v[VPT][8];
+        float mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int c = (int)threadIdx.x + i * 256;
+            if (c < n8) {
+                load8(row + 8 * c, v[i]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    mx = fmaxf(mx, fabsf(v[i][e]));
+            }
+        }
+        for (int c = (int)threadIdx.x + VPT * 256; c < n8; c += 256) {  // rows longer than the registers hold
+            float t[8];
+            load8(row + 8 * c, t);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                mx = fmaxf(mx, fabsf(t[e]));
+        }
+        const int e = prep_shift(block_max(mx, red));
+        auto store8 = [&](int c, const float (&t)[8]) {
+            uint32_t h[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const __half2 p2 = __floats2half2_rn(ldexpf(t[2 * i], -e), ldexpf(t[2 * i + 1], -e));
+                h[i] = *reinterpret_cast<const uint32_t*>(&p2);
+            }
+            *reinterpret_cast<uint4*>(x16 + (size_t)m * K + 8 * c) = make_uint4(h[0], h[1], h[2], h[3]);
+        };
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int c = (int)threadIdx.x + i * 256;
+            if (c < n8)
+                store8(c, v[i]);
+        }
+        for (int c = (int)threadIdx.x + VPT * 256; c < n8; c += 256) {
+            float t[8];
+            load8(row + 8 * c, t);
+            store8(c, t);
+        }
+        if (threadIdx.x == 0)
+            tok_scale[m] = ldexpf(1.f, e);
+        return;
+    }
+    const int n = ((int)blockIdx.x - M) * 8 + (int)(threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (n >= N)
+        return;
+    const __nv_bfloat16* sr = scales + (size_t)n * ng;
+    const __nv_bfloat16* br = biases + (size_t)n * ng;
+    float bound = 0.f;
+    for (int gi = lane; gi < ng; gi += 32)
+        bound = fmaxf(bound, fabsf(__bfloat162float(br[gi])) + qmax * fabsf(__bfloat162float(sr[gi])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        bound = fmaxf(bound, __shfl_xor_sync(0xffffffffu, bound, o));
+    const int f = prep_shift(bound);
+    for (int gi = lane; gi < ng; gi += 32) {
+        s16[(size_t)n * ng + gi] = __float2half_rn(ldexpf(__bfloat162float(sr[gi]), -f));
+        b16[(size_t)n * ng + gi] = __float2half_rn(ldexpf(__bfloat162float(br[gi]), -f));
+    }
+    if (lane == 0)
+        row_scale[n] = ldexpf(1.f, f);
+}
+
 }  // namespace
+
+size_t tc_affine_workspace(int64_t M, int64_t N, int64_t K, int g)
+{
+    auto a256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+    const size_t ng = (size_t)(K / g);
+    const size_t mt = (size_t)(M + kTT - 1) / kTT * kTT;  // token scales of whole tiles (read in 16s)
+    return a256((size_t)M * K * 2) + 2 * a256((size_t)N * ng * 2) + a256(mt * 4) + a256((size_t)N * 4);
+}
 
 cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
+    // workspace: x16 [M][K], s16 / b16 [N][ng] (fp16), tok_scale [M rounded up to 256 tokens],
+    // row_scale [N] (fp32)
+    auto a256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+    const int ng = (int)(a.K / a.g);
+    uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+    __half* x16 = reinterpret_cast<__half*>(ws);
+    __half* s16 = reinterpret_cast<__half*>(ws + a256((size_t)a.M * a.K * 2));
+    __half* b16 = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(s16) + a256((size_t)a.N * ng * 2));
+    float* tok_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(b16) + a256((size_t)a.N * ng * 2));
+    const size_t mt = (size_t)(a.M + kTT - 1) / kTT * kTT;
+    float* row_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(tok_scale) + a256(mt * 4));
+    {
+        const unsigned blocks = (unsigned)(a.M + (a.N + 7) / 8);
+        const float qmax = (float)((1 << a.bits) - 1);
+        if (a.x_f32)
+            affine_prefill_prep_kernel<float, 2><<<blocks, 256, 0, st>>>(
+                static_cast<const float*>(a.a), (int)a.M, (int)a.K, static_cast<const __nv_bfloat16*>(a.scales),
+                static_cast<const __nv_bfloat16*>(a.biases), (int)a.N, ng, qmax, x16, s16, b16, tok_scale, row_scale);
+        else
+            affine_prefill_prep_kernel<__nv_bfloat16, 2><<<blocks, 256, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(a.a), (int)a.M, (int)a.K,
+                static_cast<const __nv_bfloat16*>(a.scales), static_cast<const __nv_bfloat16*>(a.biases), (int)a.N,
+                ng, qmax, x16, s16, b16, tok_scale, row_scale);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
     TsParams prm;
     prm.codes = static_cast<const uint8_t*>(a.b);
-    prm.scales = static_cast<const unsigned short*>(a.scales);
-    prm.biases = static_cast<const unsigned short*>(a.biases);
-    prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
-    prm.out = static_cast<__nv_bfloat16*>(a.out);
+    prm.scales = reinterpret_cast<const unsigned short*>(s16);
+    prm.biases = reinterpret_cast<const unsigned short*>(b16);
+    prm.tok_scale = tok_scale;
+    prm.row_scale = row_scale;
+    prm.bias = a.bias;
+    prm.out = a.out;
+    prm.out_f32 = a.x_f32;
     prm.M = (int)a.M;
     prm.N = (int)a.N;
     prm.K = (int)a.K;
@@ -461,9 +663,9 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     prm.ng = (int)(a.K / a.g);
     prm.tiles_t = (int)((a.M + kTT - 1) / kTT);
     prm.tiles_w = (int)((a.N + kTW - 1) / kTW);
-    prm.vec_params = prm.ng % 8 == 0 && aligned16p(a.scales) && aligned16p(a.biases);
+    prm.vec_params = prm.ng % 8 == 0;  // workspace rows are then 16-byte aligned
     prm.status = dev.status;
-    if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.a, (uint64_t)a.K, (uint64_t)a.M,
+    if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)a.K, (uint64_t)a.M,
                         (uint64_t)a.K * 2, kKE, kTT))
         return cudaErrorInvalidValue;
     auto kern = tc_affine_ts_kernel;

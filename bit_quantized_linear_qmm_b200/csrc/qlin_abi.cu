@@ -121,14 +121,16 @@ int qlin_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 
 size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size)
 {
-    (void)N;
-    (void)bits;
-    (void)group_size;
     if (M <= 0 || K <= 0)
         return 0;
     switch (op) {
     case QLIN_OP_W8A8:
     case QLIN_OP_W4A8: return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
+    case QLIN_OP_MATMUL:
+        // the tensor-core prefill (M > 16, 4-bit codes): fp16 x and group parameters, scales
+        return (M > 16 && bits == 4 && N > 0 && group_size > 0 && K % group_size == 0)
+                   ? tc_affine_workspace(M, N, K, group_size)
+                   : 0;
     default: return 0;
     }
 }
@@ -175,8 +177,6 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
                         const void* scales, const void* biases, qlin_dtype param_dt, int64_t N, int bits,
                         int group_size, const void* bias, void* y, void* workspace, size_t ws_bytes, void* stream)
 {
-    (void)workspace;
-    (void)ws_bytes;
     if (!x || !codes || !scales || !biases || !y || M <= 0 || M > INT32_MAX)
         return QLIN_ERR_INVALID_ARG;
     if (!dtype_ok(x_dt))
@@ -191,7 +191,10 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
     DeviceInfo dev;
     if ((s = current_device(dev)) != QLIN_OK)
         return s;
-    if (M > 16 && bits == 4 && x_dt == QLIN_BF16 && param_dt == QLIN_BF16) {
+    if (M > 16 && bits == 4 && param_dt == QLIN_BF16) {
+        const size_t need = qlin_workspace_size(QLIN_OP_MATMUL, M, N, K, bits, group_size);
+        if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return QLIN_ERR_WORKSPACE;
         TcGemmArgs t = {};
         t.M = M;
         t.N = N;
@@ -203,6 +206,9 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
         t.scales = scales;
         t.biases = biases;
         t.g = group_size;
+        t.bits = bits;
+        t.x_f32 = x_dt == QLIN_F32 ? 1 : 0;
+        t.workspace = workspace;
         return from_cuda(launch_tc_affine(t, static_cast<cudaStream_t>(stream), dev));
     }
     AffineGemvArgs a;

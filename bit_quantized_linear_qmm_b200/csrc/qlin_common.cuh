@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "qlin.h"
@@ -358,11 +359,16 @@ struct TcGemmArgs {
     const void* scales;       // affine: bf16 [N][K/g]
     const void* biases;
     int g;
+    int bits;                 // affine code width
+    int x_f32;                // affine: x is fp32 (else bf16)
+    void* workspace;          // affine prefill: tc_affine_workspace() bytes, 256-byte aligned
 };
 enum TcOp { TC_I8_RAW = 0, TC_W8A8 = 1, TC_W4A8 = 2 };
 cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev);
 // affine 4-bit prefill with the dequantised weights as the TMEM A operand (k_tc_affine.cu):
 // x bf16 [M][K], codes [N][K/2], bf16 scales / biases [N][K/g], out bf16 [M][N].
 cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev);
+// bytes of workspace launch_tc_affine needs (fp16 x and group parameters, token and row scales)
+size_t tc_affine_workspace(int64_t M, int64_t N, int64_t K, int g);
 
 }  // namespace qlin

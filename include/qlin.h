@@ -31,7 +31,8 @@
  *     default stream) and never synchronise, except qlin_get_device_status().
  *   - Ordering on a stream: the GEMV / GEMM kernels of qlin_matmul,
  *     bitlinear_matmul and qlin_int8_matmul_int32, and the second kernel of
- *     w8a8_linear, w8a8_linear_noalloc and w4a8_linear, use programmatic
+ *     w8a8_linear, w8a8_linear_noalloc, w4a8_linear and of qlin_matmul's
+ *     prefill path (after its preparation kernel), use programmatic
  *     dependent launch: each releases the next kernel of the stream as soon
  *     as it starts, so in an unbroken run of such calls several kernels can
  *     be resident at once.  Each fetches its layer constants -- packed
@@ -41,7 +42,8 @@
  *     completed).  Rule: the packed weights and group parameters of a call
  *     must not be written by ANY earlier call of the same run.  A run ends at
  *     every other operation on the stream -- a quantize, dequantize or pack
- *     call, the activation quantiser that opens each w8a8 / w4a8 call, a
+ *     call, the activation quantiser that opens each w8a8 / w4a8 call or
+ *     the preparation kernel that opens a qlin_matmul prefill, a
  *     copy, an event wait, another library's kernel -- because such an
  *     operation starts only after everything before it has completed and
  *     releases nothing early.
@@ -133,12 +135,18 @@ qlin_status qlin_dequantize(const uint32_t* codes, const void* scales, const voi
  * x: [M, K] of x_dt (which is also the dtype of bias and y).  bias: [N] or
  * NULL.  y: [M, N].  M <= 16 runs the decode kernel (bulk-copy streamed
  * codes, register dequantisation, tensor-core MACs, partial sums reduced
- * inside the CTA); larger M with 4-bit codes and bf16 x and parameters runs
- * the prefill GEMM (codes dequantised to bf16 in registers and written to
- * tensor memory as the A operand of tcgen05 MMA, fp32 accumulation in tensor
- * memory).  Requires (K*bits/8) % 16 == 0 and, for x, (K*sizeof(x_dt)) % 16
- * == 0.  `workspace` may be NULL when qlin_workspace_size() is 0 (it is for
- * this operation).
+ * inside the CTA).  M > 16 with 4-bit codes and bf16 parameters (x bf16 or
+ * fp32) runs the prefill GEMM: a preparation kernel writes x and the group
+ * parameters as fp16 into `workspace`, each token row and each weight row
+ * scaled by a power of two that keeps it in fp16's range (undone exactly in
+ * the epilogue), and the GEMM dequantises the codes to fp16(s q + b) in
+ * registers, writes them to tensor memory as the A operand of tcgen05 MMA
+ * and accumulates in fp32 in tensor memory -- every product within 2^-11 of
+ * the exact one.  Other M > 16 calls run the decode kernel on 16-token
+ * slices.  Requires (K*bits/8) % 16 == 0 and, for x, (K*sizeof(x_dt)) % 16
+ * == 0.  workspace: at least qlin_workspace_size(QLIN_OP_MATMUL, M, N, K,
+ * bits, group_size) bytes, 256-byte aligned (QLIN_ERR_WORKSPACE otherwise);
+ * NULL is accepted when that size is 0 (M <= 16, or bits != 4).
  */
 qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
                         const uint32_t* codes, const void* scales, const void* biases,

@@ -29,6 +29,12 @@ def test_status_strings(ql):
 
 def test_workspace_sizes(ql):
     assert ql.workspace_size(ql.QLIN_OP_MATMUL, 16, 4096, 4096, 4, 128) == 0
+    # tensor-core prefill: fp16 x [M, K] and group parameters [N, K/g] x 2, token and row scales
+    M, N, K, g = 2048, 14336, 4096, 64
+    a = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    assert ql.workspace_size(ql.QLIN_OP_MATMUL, M, N, K, 4, g) == \
+        a(M * K * 2) + 2 * a(N * (K // g) * 2) + a(-(-M // 256) * 256 * 4) + a(N * 4)
+    assert ql.workspace_size(ql.QLIN_OP_MATMUL, M, N, K, 2, g) == 0  # 2-bit codes: no prefill GEMM
     assert ql.workspace_size(ql.QLIN_OP_BITLINEAR, 8, 4096, 4096) == 0
     assert ql.workspace_size(ql.QLIN_OP_W8A8, 4096, 8192, 8192) == 4096 * 8192 + 4096 * 4
     assert ql.workspace_size(ql.QLIN_OP_W8A8, 1, 8192, 8192) == 8192 + 256

@@ -71,28 +71,40 @@ def exact_in_bf16(x: Fraction) -> bool:
 
 # ---------------------------------------------------------------- affine 4-bit pair -> bf16x2
 
+def f16(h: int) -> Fraction:
+    """Exact value of an fp16 bit pattern (finite values only)."""
+    f = float(np.frombuffer(struct.pack("<H", h & 0xFFFF), dtype=np.float16)[0])
+    assert np.isfinite(f)
+    return Fraction(f)
+
+
+def f16_halves(w: int):
+    return f16(w & 0xFFFF), f16(w >> 16)
+
+
 def test_affine_pair_decode_constants_in_source():
     s = _src("k_tc_affine.cu")
-    assert "lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x43004300u)" in s
-    assert "bf16x2_fma(v, 0x3E003F80u, 0xC180C300u)" in s
+    assert "lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x64006400u)" in s
+    assert "f16x2_fma(v, 0x30003C00u, 0xD800E400u)" in s
     assert "const uint32_t w1 = words[w] >> 1;" in s
     assert "(uint32_t)(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12))" in s
 
 
 @pytest.mark.parametrize("pos", range(4))
 def test_affine_pair_decode_every_byte(pos):
+    """One byte of a word of 4-bit codes -> the fp16 pair (1024 + q, 1024 + 8 q') -> (q, q') exactly."""
     rng = np.random.default_rng(pos)
     for byte in range(256):
         others = int(rng.integers(0, 2**32))
         w = (others & ~(0xFF << (8 * pos)) | (byte << (8 * pos))) & 0xFFFFFFFF
         q = [(w >> (4 * i)) & 15 for i in range(8)]  # LSB-first codes k = 0..7
         sel = pos | (pos << 4) | ((4 + pos) << 8) | ((4 + pos) << 12)
-        v = lop3_and_or(prmt(w, w >> 1, sel), 0x0078000F, 0x43004300)
-        lo, hi = halves(v)
-        assert (lo, hi) == (128 + q[2 * pos], 128 + 8 * q[2 * pos + 1])
-        a, b = fma_exact_pair(v, 0x3E003F80, 0xC180C300)
+        v = lop3_and_or(prmt(w, w >> 1, sel), 0x0078000F, 0x64006400)
+        lo, hi = f16_halves(v)
+        assert (lo, hi) == (1024 + q[2 * pos], 1024 + 8 * q[2 * pos + 1])
+        (s0, s1), (b0, b1) = f16_halves(0x30003C00), f16_halves(0xD800E400)
+        a, b = lo * s0 + b0, hi * s1 + b1
         assert (a, b) == (q[2 * pos], q[2 * pos + 1])  # column pos holds k = 2 pos, 2 pos + 1
-        assert exact_in_bf16(a) and exact_in_bf16(b)
 
 
 # ---------------------------------------------------------------- BitLinear 2-bit fields

@@ -65,6 +65,19 @@ def test_affine_m_above_16(ql, orc):
     _run_case(ql, orc, case)
 
 
+# M > 16 outside the tensor-core prefill (2- and 8-bit codes, fp32 group parameters): the decode
+# kernel over 16-token slices
+SLICED = [synth.AffineCase(f"sliced_b{b}_g{g}_M{M}_{xd}_{pd}", M, K, N, b, g, xd, pd, True, seed=23)
+          for (M, K, N, b, g, xd, pd) in [(17, 512, 200, 2, 64, "bf16", "bf16"), (40, 1024, 130, 8, 64, "bf16", "bf16"),
+                                          (33, 640, 96, 4, 32, "bf16", "f32"), (20, 512, 64, 4, 128, "f32", "f32"),
+                                          (48, 768, 72, 8, 128, "f32", "bf16")]]
+
+
+@pytest.mark.parametrize("case", SLICED, ids=[c.name for c in SLICED])
+def test_affine_m_above_16_sliced(ql, orc, case):
+    _run_case(ql, orc, case)
+
+
 def test_affine_rejects_bad_args(ql):
     x = torch.zeros((1, 96), dtype=torch.bfloat16, device="cuda")
     codes = torch.zeros((4, 12), dtype=torch.int32, device="cuda")
@@ -79,15 +92,18 @@ def test_affine_rejects_bad_args(ql):
 
 
 PREFILL_SMALL = [
-    synth.AffineCase(f"prefill_b4_g{g}_M{M}_K{K}_N{N}", M, K, N, 4, g, "bf16", "bf16", True, seed=17)
-    for (M, K, N, g) in [(17, 256, 128, 64), (128, 512, 256, 128), (200, 1024, 300, 32), (300, 2048, 640, 64),
-                         # K % 64 == 32 (half of the last stage past K) and K/g % 8 != 0 (scalar parameter windows)
-                         (40, 1056, 200, 32),
-                         # more 128 x 256 tiles (160) than SMs: a persistent CTA takes a second tile
-                         (1280, 512, 4096, 32)]
+    synth.AffineCase(f"prefill_b4_g{g}_M{M}_K{K}_N{N}_{xd}", M, K, N, 4, g, xd, "bf16", True, seed=17)
+    for (M, K, N, g, xd) in [(17, 256, 128, 64, "bf16"), (128, 512, 256, 128, "bf16"), (200, 1024, 300, 32, "bf16"),
+                             (300, 2048, 640, 64, "bf16"),
+                             # K % 64 == 32 (half of the last stage past K) and K/g % 8 != 0 (scalar parameter windows)
+                             (40, 1056, 200, 32, "bf16"),
+                             # more 128 x 256 tiles (160) than SMs: a persistent CTA takes a second tile
+                             (1280, 512, 4096, 32, "bf16"),
+                             # short K: few terms, little cancellation -- the products' own error must meet the bar
+                             (1280, 128, 4096, 32, "bf16"), (300, 64, 520, 32, "bf16"), (64, 128, 128, 64, "bf16"),
+                             # fp32 x (and output, bias) through the same fp16 tensor-core path
+                             (100, 512, 384, 64, "f32"), (33, 128, 64, 128, "f32")]
 ]
-
-
 @pytest.mark.parametrize("case", PREFILL_SMALL, ids=[c.name for c in PREFILL_SMALL])
 def test_affine_prefill_small(ql, orc, case):
     _run_case(ql, orc, case)
