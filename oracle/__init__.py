@@ -57,6 +57,8 @@ def _load():
         lib.orc_int8_matmul.argtypes = [P, P, I64, I64, I64, P]
         lib.orc_w8a8_linear.argtypes = [P, I64, I64, P, P, I64, P, P, P, P, P]
         lib.orc_w4a8_linear.argtypes = [P, I64, I64, P, P, I64, P, P, P, P, P]
+        lib.orc_quantize_int8_groups.argtypes = [P, I64, I64, C.c_int, P, P]
+        lib.orc_pergroup_linear.argtypes = [P, I64, I64, P, P, I64, C.c_int, P, P, P, P, P]
         lib.orc_f32_to_bf16.argtypes = [P, I64, P]
         lib.orc_bf16_to_f32.argtypes = [P, I64, P]
         for name in ("orc_pack", "orc_unpack", "orc_affine_quantize", "orc_affine_dequantize",
@@ -251,4 +253,32 @@ def w4a8_linear(x, P, scale_w, bias=None):
     mag = np.empty((M, N), np.float64)
     _check(_load().orc_w4a8_linear(_p(x), M, K, _p(P), _p(scale_w), N, _p(bias), _p(qx), _p(sx),
                                    _p(y), _p(mag)), "w4a8_linear")
+    return y, mag, qx, sx
+
+
+def quantize_int8_groups(w, g: int):
+    """Per-group symmetric int8 weights: returns (q int8 [N, K], scale_w fp32 [K/g, N])."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    q = np.empty((N, K), np.int8)
+    scale_w = np.empty((K // g, N), np.float32)
+    _check(_load().orc_quantize_int8_groups(_p(w), N, K, g, _p(q), _p(scale_w)), "quantize_int8_groups")
+    return q, scale_w
+
+
+def pergroup_linear(x, w, scale_w, g: int, bias=None):
+    """Per-group INT8 linear with the page's M == 1 / M > 1 dispatch.
+    Returns (y, absdot, qx, s_x) (qx, s_x meaningful for M > 1 only)."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    w = _c(w, np.int8)
+    N = w.shape[0]
+    scale_w = _c(scale_w, np.float32)
+    bias = None if bias is None else _c(bias, np.float32)
+    qx = np.zeros((M, K), np.int8)
+    sx = np.zeros((M,), np.float32)
+    y = np.empty((M, N), np.float64)
+    mag = np.empty((M, N), np.float64)
+    _check(_load().orc_pergroup_linear(_p(x), M, K, _p(w), _p(scale_w), N, g, _p(bias), _p(qx), _p(sx),
+                                       _p(y), _p(mag)), "pergroup_linear")
     return y, mag, qx, sx

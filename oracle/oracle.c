@@ -24,6 +24,11 @@
  *   [PC]  cider/ops.py, perchannel_linear (W8A8).
  *   [W4]  cider/ops.py, w4a8_linear (W4A8).
  *   [I8]  cider/ops.py, int8_matmul_int32.
+ *   [PG]  also: cider/ops.py, pergroup_linear (Args and Dispatches
+ *         paragraphs) -- per-group symmetric INT8 weights w [N, K], scales
+ *         scale_w [num_groups, N] indexed scale_w[g * N + n], group size 64 /
+ *         128 / 256, and the dispatch M > 1 -> activation quantize + INT8
+ *         GEMM, M == 1 -> FP activation with the weights dequantised.
  *
  * Readings taken where the pages are silent (each also listed in the design
  * notes): round() is round-half-to-even (numpy's rule, and rintf under the
@@ -493,4 +498,106 @@ int orc_w4a8_linear(const float* x, int64_t M, int64_t K, const uint8_t* P, cons
             absdot[m * N + n] = (double)mag * sc;
         }
     return overflow ? ORC_EOVERFLOW : 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* [PG] per-group symmetric INT8 linear (pergroup_linear).              */
+/* ------------------------------------------------------------------ */
+
+static int orc_pg_group_ok(int g) { return g == 64 || g == 128 || g == 256; }
+
+/*
+ * The weight quantiser of the per-group format (the page prints none; its
+ * Args say "per-group symmetric quantized"): the rule of [Q8] applied to each
+ * group of g consecutive inputs of a row -- scale = max |w| / 127 (fp32), zero
+ * -> 1, q = clip(round(w / scale), -128, 127).  w: [N, K]; q: [N, K] int8;
+ * scale_w: [K/g, N], stored transposed as the page's Args give it (group grp,
+ * output n at scale_w[grp * N + n]).
+ */
+int orc_quantize_int8_groups(const float* w, int64_t N, int64_t K, int g, int8_t* q, float* scale_w)
+{
+    if (N <= 0 || K <= 0 || !orc_pg_group_ok(g) || K % g != 0)
+        return ORC_EINVAL;
+    const int64_t G = K / g;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t grp = 0; grp < G; ++grp) {
+            const float* wg = w + n * K + grp * g;
+            float amax = 0.0f;
+            for (int k = 0; k < g; ++k) {
+                float a = fabsf(wg[k]);
+                if (a > amax) amax = a;
+            }
+            float s = amax / 127.0f;
+            if (s == 0.0f)
+                s = 1.0f;
+            scale_w[grp * N + n] = s;
+            for (int k = 0; k < g; ++k) {
+                float t = rintf(wg[k] / s);
+                if (t < -128.0f) t = -128.0f;
+                if (t > 127.0f) t = 127.0f;
+                q[n * K + grp * g + k] = (int8_t)t;
+            }
+        }
+    return 0;
+}
+
+/*
+ * [PG] y = pergroup_linear(x, w, scale_w, g, bias), with the page's dispatch:
+ *   M == 1: FP activation, weights dequantised per group:
+ *       y[n] = sum_grp scale_w[grp, n] * sum_{k in grp} x[k] * w[n, k] + bias[n]
+ *   M > 1:  quant_a(x) (the per-token int8 rule of [PC]), exact integer sums
+ *       per group, then y[m, n] = s_x[m] * sum_grp scale_w[grp, n] * acc_grp + bias[n]
+ *       with acc_grp = sum_{k in grp} qx[m, k] * w[n, k].
+ * Double accumulation.  x: [M, K]; w: [N, K] int8; scale_w: [K/g, N]; bias: [N]
+ * or NULL.  qx, s_x (outputs, M > 1 only): [M, K], [M].  y, absdot: [M, N],
+ * absdot = the same sums over |products|.
+ */
+int orc_pergroup_linear(const float* x, int64_t M, int64_t K, const int8_t* w, const float* scale_w,
+                        int64_t N, int g, const float* bias, int8_t* qx, float* s_x, double* y, double* absdot)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || !orc_pg_group_ok(g) || K % g != 0)
+        return ORC_EINVAL;
+    const int64_t G = K / g;
+    const int fp_act = M == 1;  /* the page's dispatch: FP activation only for a single token */
+    if (!fp_act) {
+        int rc = orc_quantize_int8_rows(x, M, K, qx, s_x);
+        if (rc != 0)
+            return rc;
+    }
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double out = 0.0, mag = 0.0;
+            for (int64_t grp = 0; grp < G; ++grp) {
+                const double sw = (double)scale_w[grp * N + n];
+                if (fp_act) {
+                    double acc = 0.0, am = 0.0;
+                    for (int k = 0; k < g; ++k) {
+                        const double p = (double)x[grp * g + k] * (double)w[n * K + grp * g + k];
+                        acc += p;
+                        am += fabs(p);
+                    }
+                    out += sw * acc;
+                    mag += sw * am;
+                } else {
+                    int64_t acc = 0, am = 0;
+                    for (int k = 0; k < g; ++k) {
+                        const int64_t p = (int64_t)qx[m * K + grp * g + k] * (int64_t)w[n * K + grp * g + k];
+                        acc += p;
+                        am += p < 0 ? -p : p;
+                    }
+                    out += sw * (double)acc;
+                    mag += sw * (double)am;
+                }
+            }
+            if (!fp_act) {
+                out *= (double)s_x[m];
+                mag *= (double)s_x[m];
+            }
+            if (bias)
+                out += (double)bias[n];
+            y[m * N + n] = out;
+            absdot[m * N + n] = mag;
+        }
+    return 0;
 }

@@ -34,7 +34,14 @@ MUTATIONS = [
      "int64_t p = (int64_t)qx[m * K + k] * (int64_t)(c - 7);"),
     ("w4a8_nibble_read", "int c = (k % 2 == 0) ? (byte >> 4) : (byte & 15);",
      "int c = (k % 2 == 0) ? (byte & 15) : (byte >> 4);"),
-    ("int8_absmax_scale", "float s = amax / 127.0f;", "float s = amax / 128.0f;"),
+    ("int8_absmax_scale", "float s = amax / 127.0f;\n        if (s == 0.0f)\n            s = 1.0f;\n        scale[r] = s;",
+     "float s = amax / 128.0f;\n        if (s == 0.0f)\n            s = 1.0f;\n        scale[r] = s;"),
+    ("groups_scale_row_major", "scale_w[grp * N + n] = s;", "scale_w[n * G + grp] = s;"),
+    ("pergroup_scale_index", "const double sw = (double)scale_w[grp * N + n];", "const double sw = (double)scale_w[n * G + grp];"),
+    ("pergroup_m1_quantizes_x", "const int fp_act = M == 1;", "const int fp_act = 0;"),
+    ("pergroup_drops_s_x", "                out *= (double)s_x[m];", "                out *= 1.0;"),
+    ("groups_absmax_scale", "            float s = amax / 127.0f;\n            if (s == 0.0f)\n                s = 1.0f;\n            scale_w[grp * N + n] = s;",
+     "            float s = amax / 128.0f;\n            if (s == 0.0f)\n                s = 1.0f;\n            scale_w[grp * N + n] = s;"),
     ("w8a8_scale_drop", "double sc = (double)s_x[m] * (double)scale_w[n];\n            double out = (double)acc * sc;\n            if (bias)\n                out += (double)bias[n];\n            y[m * N + n] = out;\n            absdot[m * N + n] = (double)mag * sc;\n        }\n    return overflow ? ORC_EOVERFLOW : 0;\n}\n\n/*\n * [W4]",
      "double sc = (double)scale_w[n];\n            double out = (double)acc * sc;\n            if (bias)\n                out += (double)bias[n];\n            y[m * N + n] = out;\n            absdot[m * N + n] = (double)mag * sc;\n        }\n    return overflow ? ORC_EOVERFLOW : 0;\n}\n\n/*\n * [W4]"),
 ]

@@ -393,3 +393,95 @@ def test_quantize_golden_ties(orc):
         c, s, b = orc.affine_quantize(w, bits, g, bf16)
         assert s[0, 0] == 1.0 and b[0, 0] == 0.0
         assert np.array_equal(orc.unpack(c, g, bits), want)
+
+
+# ------------------------------------------------------------------ per-group INT8 (pergroup_linear)
+
+def test_int8_groups_properties(orc):
+    """Per-group symmetric int8 (the [Q8] rule per group): every group's absmax element maps to
+    +-127, a zero group gets scale 1 and zero codes, |w - q s| <= s/2, and the scales sit
+    transposed, group-major, as the page's Args give them (scale_w[grp, n])."""
+    rng = np.random.default_rng(5)
+    N, K, g = 6, 256, 64
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    w[2, 64:128] = 0.0                                    # a zero group: row 2, group 1
+    w[4, 130] = 0.5                                       # group 2 of row 4 dominated by one element
+    q, s = orc.quantize_int8_groups(w, g)
+    assert s.shape == (K // g, N)
+    assert s[1, 2] == 1.0 and not np.any(q[2, 64:128])
+    assert s[2, 4] == np.float32(np.float32(0.5) / np.float32(127.0)) and q[4, 130] == 127
+    for n in range(N):
+        for grp in range(K // g):
+            blk = w[n, grp * g:(grp + 1) * g]
+            if not np.any(blk):
+                continue
+            i = int(np.argmax(np.abs(blk)))
+            assert abs(int(q[n, grp * g + i])) == 127
+            err = np.abs(blk - q[n, grp * g:(grp + 1) * g].astype(np.float64) * s[grp, n])
+            assert np.all(err <= s[grp, n] / 2 * (1 + 1e-6))
+
+
+def test_pergroup_m1_brute_force_exact(orc):
+    """M == 1 (FP activation): y[n] = sum_grp s[grp, n] sum_{k in grp} x_k w[n, k] + bias, checked
+    exactly with Fractions on dyadic inputs (every product and sum exact in double)."""
+    rng = np.random.default_rng(6)
+    N, K, g = 5, 128, 64
+    w = rng.integers(-128, 128, (N, K)).astype(np.int8)
+    s = (2.0 ** rng.integers(-9, -3, (K // g, N))).astype(np.float32)
+    x = (rng.integers(-8, 9, (1, K)) / 4.0).astype(np.float32)
+    bias = (rng.integers(-4, 5, N) / 8.0).astype(np.float32)
+    y, mag, _, _ = orc.pergroup_linear(x, w, s, g, bias)
+    for n in range(N):
+        want = Fraction(float(bias[n]))
+        for grp in range(K // g):
+            want += Fraction(float(s[grp, n])) * sum(Fraction(float(x[0, k])) * int(w[n, k])
+                                                     for k in range(grp * g, (grp + 1) * g))
+        assert Fraction(y[0, n]) == want
+
+
+def test_pergroup_single_group_equals_w8a8(orc):
+    """With one group spanning K, the per-group layer is the per-channel W8A8 layer: M > 1 must give
+    exactly the W8A8 result (same quant_a, same scale per output)."""
+    rng = np.random.default_rng(7)
+    M, N, K = 3, 7, 256
+    wf = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    q, s = orc.quantize_int8_groups(wf, 256)
+    y, mag, qx, sx = orc.pergroup_linear(x, q, s, 256)
+    y8, mag8, qx8, sx8 = orc.w8a8_linear(x, q, s[0], None)
+    assert np.array_equal(qx, qx8) and np.array_equal(sx, sx8)
+    assert np.allclose(y, y8, rtol=1e-15, atol=0) and np.allclose(mag, mag8, rtol=1e-15, atol=0)
+
+
+def test_pergroup_m1_vs_float64_library(orc):
+    """M == 1 with several groups equals x @ (w * s)^T by torch float64 (the dequantised weight
+    built from the transposed scales)."""
+    rng = np.random.default_rng(8)
+    N, K, g = 33, 512, 128
+    wf = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    q, s = orc.quantize_int8_groups(wf, g)
+    x = rng.standard_normal((1, K)).astype(np.float32)
+    y, _, _, _ = orc.pergroup_linear(x, q, s, g)
+    wd = torch.from_numpy(q.astype(np.float64)) * torch.from_numpy(np.repeat(s.T.astype(np.float64), g, axis=1))
+    ref = (torch.from_numpy(x.astype(np.float64)) @ wd.T).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_pergroup_dispatch_m1_vs_m2(orc):
+    """The page's dispatch: M == 1 uses x as it is, M > 1 its int8 quantisation.  On activations that
+    are already on the int8 grid of their row (x = c * amax/127 with integer c) both branches agree;
+    on generic activations they differ."""
+    rng = np.random.default_rng(9)
+    N, K, g = 9, 256, 64
+    q, s = orc.quantize_int8_groups((rng.standard_normal((N, K)) * 0.02).astype(np.float32), g)
+    c = rng.integers(-127, 128, (1, K)).astype(np.float32)
+    c[0, 0] = 127.0
+    grid = (c * np.float32(2.0 ** -6)).astype(np.float32)  # amax = 127 / 64, s_x = 1/64 exactly
+    y1, _, _, _ = orc.pergroup_linear(grid, q, s, g)
+    y2, _, qx, sx = orc.pergroup_linear(np.vstack([grid, grid]), q, s, g)
+    assert sx[0] == np.float32(2.0 ** -6) and np.array_equal(qx[0], c[0].astype(np.int8))
+    assert np.allclose(y2[0], y1[0], rtol=1e-13, atol=1e-13) and np.allclose(y2[1], y1[0], rtol=1e-13, atol=1e-13)
+    xr = rng.standard_normal((1, K)).astype(np.float32)
+    r1, _, _, _ = orc.pergroup_linear(xr, q, s, g)
+    r2, _, _, _ = orc.pergroup_linear(np.vstack([xr, xr]), q, s, g)
+    assert not np.allclose(r1[0], r2[0], rtol=1e-6, atol=0)
