@@ -327,6 +327,42 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __
 
 // ---------------------------------------------------------------- per-column int4
 // Block = 32 columns x 8 row slices.
+// ---------------------------------------------------------------- per-group int8 (pergroup_linear's format)
+// One warp per (row n, group): the int8 rule per group of g inputs -- scale = max |w| / 127 (zero
+// -> 1), q = clip(round(w / scale), -128, 127), IEEE divisions -- with the scales stored
+// group-major, scale_w[grp * N + n] [cider/ops.py pergroup_linear, Args].
+template <typename TW, int G>
+__global__ void __launch_bounds__(256) quantize_int8_groups_kernel(const TW* __restrict__ w, int64_t N, int64_t K,
+                                                                  int8_t* __restrict__ q, float* __restrict__ scale_w)
+{
+    constexpr int PER = G / 32;
+    const int64_t item = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int64_t ng = K / G;
+    if (item >= N * ng)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int64_t n = item / ng, grp = item % ng;
+    const TW* src = w + n * K + grp * G;
+    float v[PER];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        v[i] = to_float(src[i * 32 + lane]);
+        amax = fmaxf(amax, fabsf(v[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float sc = __fdiv_rn(amax, 127.0f);
+    if (sc == 0.f)
+        sc = 1.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        q[n * K + grp * G + i * 32 + lane] = (int8_t)fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -128.f), 127.f);
+    if (lane == 0)
+        scale_w[grp * N + n] = sc;
+}
+
 template <typename TW>
 __global__ void __launch_bounds__(256) pack_int4_cols_kernel(const TW* __restrict__ w, int64_t K, int64_t N,
                                                              uint8_t* __restrict__ packed, float* __restrict__ scale)
@@ -461,6 +497,21 @@ cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R,
     else
         quantize_int8_rows_kernel<float><<<(unsigned)R, 256, 0, st>>>(static_cast<const float*>(w), C, q, scale,
                                                                       rowsum, rel);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int g, int8_t* q,
+                                        float* scale_w, cudaStream_t st, const DeviceInfo&)
+{
+    const unsigned blocks = (unsigned)((N * (K / g) + 7) / 8);
+#define QLIN_QG(TW, G) \
+    quantize_int8_groups_kernel<TW, G><<<blocks, 256, 0, st>>>(static_cast<const TW*>(w), N, K, q, scale_w)
+    if (w_dt == QLIN_BF16) {
+        if (g == 64) QLIN_QG(__nv_bfloat16, 64); else if (g == 128) QLIN_QG(__nv_bfloat16, 128); else QLIN_QG(__nv_bfloat16, 256);
+    } else {
+        if (g == 64) QLIN_QG(float, 64); else if (g == 128) QLIN_QG(float, 128); else QLIN_QG(float, 256);
+    }
+#undef QLIN_QG
     return cudaGetLastError();
 }
 

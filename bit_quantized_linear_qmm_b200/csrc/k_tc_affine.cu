@@ -56,13 +56,22 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kXformWarps + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = kTT;       // A ring starts here
-constexpr int kCodePF = 6;          // stages of codes in flight per transform thread (cp.async ring)
+// Code formats of the A operand: CB = 4, the MLX affine 4-bit codes with a group scale and bias;
+// CB = 8, signed int8 weights with a group scale (the per-group INT8 format).  A transform thread
+// covers 32 k of one weight row per stage: 4 * CB bytes of codes, kept kCodePF(CB) stages ahead in
+// its slots of a cp.async ring of 24 KB.
+template <int CB> struct CodeFmt {
+    static constexpr int kBytes = 4 * CB;                    // code bytes per thread per stage
+    static constexpr int kCopies = kBytes / 16;              // 16-byte copies per stage
+    static constexpr int kPF = CB == 4 ? 6 : 3;              // stages in flight
+};
 constexpr int kGroupT = 4;          // token tiles that walk the weight tiles together
 // kind::f16: D f32, A and B f16 (format 0), both K-major, N = 256, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 
-// per transform thread, kCodePF stages of its 16 bytes of codes: [stage][transform thread]
-constexpr int kCodeRing = kCodePF * kXformWarps * 32 * 16;
+// per transform thread, kPF stages of its code bytes: [stage][copy][transform thread] x 16 bytes
+constexpr int kCodeRing = 6 * kXformWarps * 32 * 16;
+static_assert(CodeFmt<4>::kPF * CodeFmt<4>::kCopies <= 6 && CodeFmt<8>::kPF * CodeFmt<8>::kCopies <= 6, "ring");
 
 struct Bars {
     uint64_t xfull[kXStages];
@@ -151,8 +160,11 @@ QLIN_DEV void tile_coords(int t, int tiles_t, int tiles_w, int& tt, int& wt)
     wt = r / gt;
 }
 
+template <int CB>
 __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_constant__ TsParams p)
 {
+    using F = CodeFmt<CB>;
+    constexpr int kCodePF = F::kPF;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint4* code_ring = reinterpret_cast<uint4*>(smem + kXStages * kXBytes);
@@ -265,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         const int q = warp & 3;             // TMEM lane quarter this warp may access
         const int kh = (warp - 2) >> 2;     // 32-k half of each stage
         const int r = 32 * q + lane;        // weight row within the tile
-        const size_t pitch = (size_t)p.K / 2;
+        const size_t pitch = (size_t)p.K * CB / 8;
         pdl_wait_prior_grids();  // the weights' parameters may come from the previous kernel
 
         auto row_of = [&](int ti) {
@@ -273,21 +285,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
             return min(wt * kTW + r, p.N - 1);
         };
-        // codes of stage (ti, kb) for this thread: 16 bytes (32 k) of row n, copied kCodePF stages
-        // ahead into this thread's slots of the shared-memory ring with cp.async (one commit group
-        // per stage, so the wait before a stage's decode is explicit); a half stage past K or a
-        // stage past the last tile is written as zeros (zero codes meet the zero-filled x columns)
+        // codes of stage (ti, kb) for this thread: F::kBytes bytes (32 k) of row n, copied kCodePF
+        // stages ahead into this thread's slots of the shared-memory ring with cp.async (one commit
+        // group per stage, so the wait before a stage's decode is explicit); a half stage past K or
+        // a stage past the last tile is written as zeros (zero codes meet the zero-filled x columns)
         int lti = 0, lkb = 0;
-        const uint8_t* lrow = my_tiles > 0 ? p.codes + (size_t)row_of(0) * pitch + 16 * kh : p.codes;
-        uint4* my_ring = code_ring + (warp - 2) * 32 + lane;  // slot j at my_ring[j * kXformWarps * 32]
+        const uint8_t* lrow = my_tiles > 0 ? p.codes + (size_t)row_of(0) * pitch + F::kBytes * kh : p.codes;
+        uint4* my_ring = code_ring + (warp - 2) * 32 + lane;  // copy c of slot j: my_ring[(j * kCopies + c) * 256]
         auto load_next = [&](int slot) {
             const bool in = lti < my_tiles && lkb * kKE + 32 * kh < p.K;
-            cp_async16(my_ring + slot * kXformWarps * 32, in ? lrow + (size_t)lkb * (kKE / 2) : p.codes, in ? 16 : 0);
+#pragma unroll
+            for (int c = 0; c < F::kCopies; ++c)
+                cp_async16(my_ring + (slot * F::kCopies + c) * kXformWarps * 32,
+                           in ? lrow + (size_t)lkb * (kKE * CB / 8) + 16 * c : p.codes, in ? 16 : 0);
             cp_async_commit();
             if (lti < my_tiles && ++lkb == nk) {
                 lkb = 0;
                 if (++lti < my_tiles)
-                    lrow = p.codes + (size_t)row_of(lti) * pitch + 16 * kh;
+                    lrow = p.codes + (size_t)row_of(lti) * pitch + F::kBytes * kh;
             }
         };
 
@@ -376,18 +391,37 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                 // exact fp16 (1024 + q, 1024 + 8 q'), one f16x2 FMA recovers (q, q') exactly, and one
                 // gives fp16(s q + b), the exact value rounded once.  Column c holds k = 2c, 2c + 1.
                 cp_async_wait<kCodePF - 1>();  // this stage's copy (the oldest in flight) has landed
-                const uint4 cbj = my_ring[j * kXformWarps * 32];
-                const uint32_t words[4] = {cbj.x, cbj.y, cbj.z, cbj.w};
                 uint32_t o[16];
+                if constexpr (CB == 4) {
+                    const uint4 cbj = my_ring[j * kXformWarps * 32];
+                    const uint32_t words[4] = {cbj.x, cbj.y, cbj.z, cbj.w};
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const uint32_t w1 = words[w] >> 1;
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t w1 = words[w] >> 1;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t sel = (uint32_t)(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12));
-                        const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x64006400u);
-                        const uint32_t qq = f16x2_fma(v, 0x30003C00u, 0xD800E400u);  // (1, 1/8), (-1024, -128)
-                        o[4 * w + e] = f16x2_fma(qq, s2, b2);
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t sel = (uint32_t)(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12));
+                            const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x64006400u);
+                            const uint32_t qq = f16x2_fma(v, 0x30003C00u, 0xD800E400u);  // (1, 1/8), (-1024, -128)
+                            o[4 * w + e] = f16x2_fma(qq, s2, b2);
+                        }
+                    }
+                } else {
+                    // int8 weights, k in order: the pair (k, k+1) of a byte pair becomes the exact fp16
+                    // (1024 + (b ^ 0x80)) per half with one PRMT; one FMA subtracts 1152, leaving the
+                    // signed byte exactly, and one multiply gives fp16(s w), rounded once
+                    const uint4 c0 = my_ring[(2 * j) * kXformWarps * 32];
+                    const uint4 c1 = my_ring[(2 * j + 1) * kXformWarps * 32];
+                    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        const uint32_t u = words[w] ^ 0x80808080u;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t v = prmt(u, 0x64646464u, h ? 0x4342u : 0x4140u);
+                            const uint32_t qq = f16x2_fma(v, 0x3C003C00u, 0xE480E480u);  // 1, -1152
+                            o[2 * w + h] = f16x2_fma(qq, s2, 0u);
+                        }
                     }
                 }
                 load_next(j);  // the stage kCodePF ahead, into the slot just read
@@ -527,12 +561,18 @@ QLIN_DEV void load8(const float* p, float (&v)[8])
 }
 
 // Blocks [0, M): token rows of x -> x16 and tok_scale (16-byte loads and stores; a row of up to
-// 256 * 8 * VPT values is held in registers between the max and the conversion).  Blocks
-// [M, M + ceil(N / 8)): one warp per weight row -> fp16 group parameters and row_scale.
-// qmax = 2^bits - 1.  K % 8 == 0.
-template <typename XT, int VPT>
+// 256 * 8 * VPT values is held in registers between the max and the conversion).
+//   QX = 0: x16 = fp16(x 2^-E_m), tok_scale = 2^E_m (the activations as they are);
+//   QX = 1: the per-token int8 quantiser -- s = max|x| / 127 (zero -> 1), q = clip(round(x / s),
+//           -128, 127) with an IEEE division -- stored as exact fp16 integers, tok_scale = s.
+// Blocks [M, M + ceil(N / 8)): one warp per weight row -> fp16 group scales (and biases) scaled by
+// 2^-F_n, row_scale = 2^F_n:
+//   PG = 0: affine bf16 scales / biases [N][ng], bound max_g |b| + qmax |s|;
+//   PG = 1: per-group int8 scales, fp32 [ng][N] (group-major), bound 128 max_g |s|; no biases.
+// K % 8 == 0.
+template <typename XT, int VPT, int QX, int PG>
 __global__ void __launch_bounds__(256) affine_prefill_prep_kernel(
-    const XT* __restrict__ x, int M, int K, const __nv_bfloat16* __restrict__ scales,
+    const XT* __restrict__ x, int M, int K, const void* __restrict__ scales,
     const __nv_bfloat16* __restrict__ biases, int N, int ng, float qmax, __half* __restrict__ x16,
     __half* __restrict__ s16, __half* __restrict__ b16, float* __restrict__ tok_scale, float* __restrict__ row_scale)
 {
@@ -561,12 +601,27 @@ __global__ void __launch_bounds__(256) affine_prefill_prep_kernel(
             for (int e = 0; e < 8; ++e)
                 mx = fmaxf(mx, fabsf(t[e]));
         }
-        const int e = prep_shift(block_max(mx, red));
+        const float amax = block_max(mx, red);
+        int e = 0;
+        float sq = 1.f;
+        if constexpr (QX) {
+            sq = __fdiv_rn(amax, 127.0f);
+            if (sq == 0.f)
+                sq = 1.f;
+        } else {
+            e = prep_shift(amax);
+        }
+        auto conv = [&](float t) {
+            if constexpr (QX)
+                return fminf(fmaxf(rintf(__fdiv_rn(t, sq)), -128.f), 127.f);
+            else
+                return ldexpf(t, -e);
+        };
         auto store8 = [&](int c, const float (&t)[8]) {
             uint32_t h[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const __half2 p2 = __floats2half2_rn(ldexpf(t[2 * i], -e), ldexpf(t[2 * i + 1], -e));
+                const __half2 p2 = __floats2half2_rn(conv(t[2 * i]), conv(t[2 * i + 1]));
                 h[i] = *reinterpret_cast<const uint32_t*>(&p2);
             }
             *reinterpret_cast<uint4*>(x16 + (size_t)m * K + 8 * c) = make_uint4(h[0], h[1], h[2], h[3]);
@@ -583,24 +638,33 @@ __global__ void __launch_bounds__(256) affine_prefill_prep_kernel(
             store8(c, t);
         }
         if (threadIdx.x == 0)
-            tok_scale[m] = ldexpf(1.f, e);
+            tok_scale[m] = QX ? sq : ldexpf(1.f, e);
         return;
     }
     const int n = ((int)blockIdx.x - M) * 8 + (int)(threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (n >= N)
         return;
-    const __nv_bfloat16* sr = scales + (size_t)n * ng;
-    const __nv_bfloat16* br = biases + (size_t)n * ng;
+    auto scale_at = [&](int gi) {
+        if constexpr (PG)
+            return static_cast<const float*>(scales)[(size_t)gi * N + n];
+        else
+            return __bfloat162float(static_cast<const __nv_bfloat16*>(scales)[(size_t)n * ng + gi]);
+    };
     float bound = 0.f;
-    for (int gi = lane; gi < ng; gi += 32)
-        bound = fmaxf(bound, fabsf(__bfloat162float(br[gi])) + qmax * fabsf(__bfloat162float(sr[gi])));
+    for (int gi = lane; gi < ng; gi += 32) {
+        if constexpr (PG)
+            bound = fmaxf(bound, 128.f * fabsf(scale_at(gi)));
+        else
+            bound = fmaxf(bound, fabsf(__bfloat162float(biases[(size_t)n * ng + gi])) + qmax * fabsf(scale_at(gi)));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         bound = fmaxf(bound, __shfl_xor_sync(0xffffffffu, bound, o));
     const int f = prep_shift(bound);
     for (int gi = lane; gi < ng; gi += 32) {
-        s16[(size_t)n * ng + gi] = __float2half_rn(ldexpf(__bfloat162float(sr[gi]), -f));
-        b16[(size_t)n * ng + gi] = __float2half_rn(ldexpf(__bfloat162float(br[gi]), -f));
+        s16[(size_t)n * ng + gi] = __float2half_rn(ldexpf(scale_at(gi), -f));
+        if constexpr (!PG)
+            b16[(size_t)n * ng + gi] = __float2half_rn(ldexpf(__bfloat162float(biases[(size_t)n * ng + gi]), -f));
     }
     if (lane == 0)
         row_scale[n] = ldexpf(1.f, f);
@@ -632,15 +696,22 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     {
         const unsigned blocks = (unsigned)(a.M + (a.N + 7) / 8);
         const float qmax = (float)((1 << a.bits) - 1);
-        if (a.x_f32)
-            affine_prefill_prep_kernel<float, 2><<<blocks, 256, 0, st>>>(
-                static_cast<const float*>(a.a), (int)a.M, (int)a.K, static_cast<const __nv_bfloat16*>(a.scales),
-                static_cast<const __nv_bfloat16*>(a.biases), (int)a.N, ng, qmax, x16, s16, b16, tok_scale, row_scale);
-        else
-            affine_prefill_prep_kernel<__nv_bfloat16, 2><<<blocks, 256, 0, st>>>(
-                static_cast<const __nv_bfloat16*>(a.a), (int)a.M, (int)a.K,
-                static_cast<const __nv_bfloat16*>(a.scales), static_cast<const __nv_bfloat16*>(a.biases), (int)a.N,
-                ng, qmax, x16, s16, b16, tok_scale, row_scale);
+        const __nv_bfloat16* bb = static_cast<const __nv_bfloat16*>(a.biases);
+        // (x dtype, activation handling, parameter format)
+        const int form = (a.x_f32 ? 1 : 0) | (a.pergroup && a.M > 1 ? 2 : 0) | (a.pergroup ? 4 : 0);
+        switch (form) {
+#define QLIN_PREP(XT, QX, PG)                                                                                   \
+    affine_prefill_prep_kernel<XT, 2, QX, PG><<<blocks, 256, 0, st>>>(static_cast<const XT*>(a.a), (int)a.M,    \
+                                                                      (int)a.K, a.scales, bb, (int)a.N, ng, qmax, \
+                                                                      x16, s16, b16, tok_scale, row_scale)
+        case 0: QLIN_PREP(__nv_bfloat16, 0, 0); break;
+        case 1: QLIN_PREP(float, 0, 0); break;
+        case 4: QLIN_PREP(__nv_bfloat16, 0, 1); break;
+        case 5: QLIN_PREP(float, 0, 1); break;
+        case 6: QLIN_PREP(__nv_bfloat16, 1, 1); break;
+        default: QLIN_PREP(float, 1, 1); break;
+#undef QLIN_PREP
+        }
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
@@ -648,7 +719,7 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     TsParams prm;
     prm.codes = static_cast<const uint8_t*>(a.b);
     prm.scales = reinterpret_cast<const unsigned short*>(s16);
-    prm.biases = reinterpret_cast<const unsigned short*>(b16);
+    prm.biases = reinterpret_cast<const unsigned short*>(a.pergroup ? s16 : b16);  // read, unused, for int8
     prm.tok_scale = tok_scale;
     prm.row_scale = row_scale;
     prm.bias = a.bias;
@@ -668,7 +739,7 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)a.K, (uint64_t)a.M,
                         (uint64_t)a.K * 2, kKE, kTT))
         return cudaErrorInvalidValue;
-    auto kern = tc_affine_ts_kernel;
+    auto kern = a.bits == 8 ? tc_affine_ts_kernel<8> : tc_affine_ts_kernel<4>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess)
         return e;

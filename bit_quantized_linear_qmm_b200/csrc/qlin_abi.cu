@@ -126,6 +126,10 @@ size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits
     switch (op) {
     case QLIN_OP_W8A8:
     case QLIN_OP_W4A8: return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
+    case QLIN_OP_PERGROUP:
+        return (N > 0 && (group_size == 64 || group_size == 128 || group_size == 256) && K % group_size == 0)
+                   ? tc_affine_workspace(M, N, K, group_size)
+                   : 0;
     case QLIN_OP_MATMUL:
         // the tensor-core prefill (M > 16, 4-bit codes): fp16 x and group parameters, scales
         return (M > 16 && bits == 4 && N > 0 && group_size > 0 && K % group_size == 0)
@@ -286,6 +290,61 @@ qlin_status qlin_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64
     if ((s = current_device(dev)) != QLIN_OK)
         return s;
     return from_cuda(launch_pack_int4_cols(w, w_dt, K, N, packed, scale, static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status qlin_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int group_size,
+                                     int8_t* q, float* scale_w, void* stream)
+{
+    if (!w || !q || !scale_w || N <= 0 || K <= 0 || N > INT32_MAX || K > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(w_dt) || !(group_size == 64 || group_size == 128 || group_size == 256))
+        return QLIN_ERR_UNSUPPORTED;
+    if (K % group_size != 0)
+        return QLIN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    return from_cuda(
+        launch_quantize_int8_groups(w, w_dt, N, K, group_size, q, scale_w, static_cast<cudaStream_t>(stream), dev));
+}
+
+qlin_status pergroup_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const int8_t* w,
+                            const float* scale_w, int64_t N, int group_size, const void* bias, void* y,
+                            void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!x || !w || !scale_w || !y || M <= 0 || N <= 0 || K <= 0 || M > INT32_MAX || N > INT32_MAX ||
+        K > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(x_dt) || !(group_size == 64 || group_size == 128 || group_size == 256))
+        return QLIN_ERR_UNSUPPORTED;
+    if (K % group_size != 0)
+        return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || K % 16 != 0)
+        return QLIN_ERR_MISALIGNED;
+    const size_t need = qlin_workspace_size(QLIN_OP_PERGROUP, M, N, K, 8, group_size);
+    if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return QLIN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    TcGemmArgs t = {};
+    t.M = M;
+    t.N = N;
+    t.K = K;
+    t.a = x;
+    t.b = w;
+    t.out = y;
+    t.bias = bias;
+    t.scales = scale_w;
+    t.biases = nullptr;
+    t.g = group_size;
+    t.bits = 8;
+    t.x_f32 = x_dt == QLIN_F32 ? 1 : 0;
+    t.pergroup = 1;
+    t.workspace = workspace;
+    return from_cuda(launch_tc_affine(t, static_cast<cudaStream_t>(stream), dev));
 }
 
 qlin_status qlin_int8_matmul_int32(const int8_t* a, const int8_t* b, int64_t M, int64_t N, int64_t K, int32_t* c,

@@ -298,6 +298,8 @@ cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, 
                                      qlin_dtype o_dt, cudaStream_t st, const DeviceInfo& dev);
 cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
                                       float* scale, int32_t* rowsum, cudaStream_t st, const DeviceInfo& dev, bool release_dependents = false);
+cudaError_t launch_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int g, int8_t* q,
+                                        float* scale_w, cudaStream_t st, const DeviceInfo& dev);
 cudaError_t launch_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64_t N, uint8_t* packed,
                                   float* scale, cudaStream_t st, const DeviceInfo& dev);
 
@@ -359,8 +361,9 @@ struct TcGemmArgs {
     const void* scales;       // affine: bf16 [N][K/g]
     const void* biases;
     int g;
-    int bits;                 // affine code width
+    int bits;                 // affine code width (8 with pergroup)
     int x_f32;                // affine: x is fp32 (else bf16)
+    int pergroup;             // per-group int8 weights [N][K], fp32 scales [K/g][N] (group-major), no biases
     void* workspace;          // affine prefill: tc_affine_workspace() bytes, 256-byte aligned
 };
 enum TcOp { TC_I8_RAW = 0, TC_W8A8 = 1, TC_W4A8 = 2 };

@@ -34,6 +34,7 @@ QLIN_OP_MATMUL = 0
 QLIN_OP_BITLINEAR = 1
 QLIN_OP_W8A8 = 2
 QLIN_OP_W4A8 = 3
+QLIN_OP_PERGROUP = 4
 
 _lib = None
 
@@ -47,7 +48,7 @@ class QlinError(RuntimeError):
 def header_functions() -> list[str]:
     """Names of the functions include/qlin.h declares."""
     text = open(HEADER).read()
-    return re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\*?\s+\*?(qlin_\w+|bitlinear_\w+|w8a8_\w+|w4a8_\w+)\s*\(",
+    return re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\*?\s+\*?(qlin_\w+|bitlinear_\w+|w8a8_\w+|w4a8_\w+|pergroup_\w+)\s*\(",
                       text, re.M)
 
 
@@ -74,6 +75,8 @@ def lib():
         "w8a8_linear": ([P, I, I64, I64, P, P, I64, P, P, P, SZ, P], I),
         "w4a8_linear": ([P, I, I64, I64, P, P, I64, P, P, P, SZ, P], I),
         "w8a8_linear_noalloc": ([P, I, I64, I64, P, P, I64, P, P, P], I),
+        "qlin_quantize_int8_groups": ([P, I, I64, I64, I, P, P, P], I),
+        "pergroup_linear": ([P, I, I64, I64, P, P, I64, I, P, P, P, SZ, P], I),
         "qlin_get_device_status": ([P], I),
         "qlin_selftest_wait_timeout": ([C.c_uint, P], I),
     }
@@ -253,3 +256,29 @@ def selftest_wait_timeout(limit_us: int = 1000, device=None):
 def device_status(device=None) -> int:
     """Synchronises the current stream and returns (and clears) the device status."""
     return int(lib().qlin_get_device_status(_stream(device)))
+
+
+def quantize_int8_groups(w, group_size: int):
+    """Per-group symmetric int8 weights: (q int8 [N, K], scale_w fp32 [K/group_size, N])."""
+    _cuda(w)
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    s = torch.empty((K // group_size, N), dtype=torch.float32, device=w.device)
+    _check(lib().qlin_quantize_int8_groups(_ptr(w), _dt(w), N, K, group_size, _ptr(q), _ptr(s), _stream(w.device)),
+           "qlin_quantize_int8_groups")
+    return q, s
+
+
+def pergroup_linear(x, w, scale_w, group_size: int, bias=None, out=None, workspace=None):
+    """Per-group INT8 linear (M == 1: FP activation; M > 1: int8 activation quantisation)."""
+    _cuda(x, w, scale_w, bias)
+    M, K = x.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(QLIN_OP_PERGROUP, M, N, K, 8, group_size), dtype=torch.uint8,
+                                device=x.device)
+    _check(lib().pergroup_linear(_ptr(x), _dt(x), M, K, _ptr(w), _ptr(scale_w), N, group_size, _ptr(bias), _ptr(out),
+                                 _ptr(workspace), workspace.numel(), _stream(x.device)), "pergroup_linear")
+    return out

@@ -31,8 +31,8 @@
  *     default stream) and never synchronise, except qlin_get_device_status().
  *   - Ordering on a stream: the GEMV / GEMM kernels of qlin_matmul,
  *     bitlinear_matmul and qlin_int8_matmul_int32, and the second kernel of
- *     w8a8_linear, w8a8_linear_noalloc, w4a8_linear and of qlin_matmul's
- *     prefill path (after its preparation kernel), use programmatic
+ *     w8a8_linear, w8a8_linear_noalloc, w4a8_linear, pergroup_linear and of
+ *     qlin_matmul's prefill path (after its preparation kernel), use programmatic
  *     dependent launch: each releases the next kernel of the stream as soon
  *     as it starts, so in an unbroken run of such calls several kernels can
  *     be resident at once.  Each fetches its layer constants -- packed
@@ -88,7 +88,8 @@ typedef enum {
     QLIN_OP_MATMUL = 0,     /* qlin_matmul */
     QLIN_OP_BITLINEAR = 1,  /* bitlinear_matmul */
     QLIN_OP_W8A8 = 2,       /* w8a8_linear */
-    QLIN_OP_W4A8 = 3        /* w4a8_linear */
+    QLIN_OP_W4A8 = 3,       /* w4a8_linear */
+    QLIN_OP_PERGROUP = 4    /* pergroup_linear */
 } qlin_op;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -223,6 +224,40 @@ qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
                         const uint8_t* packed_w, const float* scale_w, int64_t N,
                         const void* bias, void* y, void* workspace, size_t ws_bytes,
                         void* stream);
+
+/*
+ * Per-group symmetric INT8 weight quantisation, the weight format of
+ * pergroup_linear [cider/ops.py pergroup_linear, Args: "INT8 weights [N, K]
+ * int8 (per-group symmetric quantized)", scales [num_groups, N]]: per group of
+ * group_size consecutive inputs of a row, scale = max |w| / 127 (fp32, zero ->
+ * 1) and q = clip(round_half_even(w / scale), -128, 127) -- the rule of
+ * qlin_quantize_int8_rows per group.  w: [N, K] of w_dt; q: int8 [N, K];
+ * scale_w: fp32 [K/group_size, N], group-major (scale_w[g * N + n]).
+ * group_size in {64, 128, 256}; K % group_size == 0.  Bit-exact.
+ */
+qlin_status qlin_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int group_size,
+                                     int8_t* q, float* scale_w, void* stream);
+
+/*
+ * Per-group INT8 linear [cider/ops.py pergroup_linear: Args, and "Dispatches
+ * internally: M > 1 -> per-group GEMM (activation quantize + INT8 TensorOps),
+ * M == 1 -> per-group MV (FP activation, weight dequant on-the-fly)"]:
+ *   M == 1: y[n] = sum_g scale_w[g, n] * sum_{k in g} x[k] * w[n, k] + bias[n]
+ *   M > 1:  y[m, n] = s_x[m] * sum_g scale_w[g, n] * sum_{k in g} qx[m, k] * w[n, k] + bias[n],
+ *           qx, s_x = the per-token int8 quantisation of x (the qlin_quantize_int8_rows rule)
+ * x: [M, K] of x_dt (also the dtype of bias and y); w: int8 [N, K];
+ * scale_w: fp32 [K/group_size, N] (group-major); bias: [N] or NULL; y: [M, N].
+ * group_size in {64, 128, 256}; K % 16 == 0.  Both branches run the tcgen05
+ * GEMM of the affine prefill: a preparation kernel writes x (M == 1, scaled
+ * by a power of two) or its int8 quantisation (M > 1) and the group scales as
+ * fp16 into `workspace`, and the GEMM forms each weight as fp16(scale w),
+ * rounded once (every product within 2^-11 of the exact one).  workspace: at
+ * least qlin_workspace_size(QLIN_OP_PERGROUP, M, N, K, 8, group_size) bytes,
+ * 256-byte aligned.
+ */
+qlin_status pergroup_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const int8_t* w,
+                            const float* scale_w, int64_t N, int group_size, const void* bias, void* y,
+                            void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * W8A8 linear without caller memory (no counterpart on the source pages).
