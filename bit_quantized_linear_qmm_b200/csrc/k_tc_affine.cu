@@ -60,14 +60,23 @@ constexpr int kAccCols = kTT;       // A ring starts here
 // CB = 8, signed int8 weights with a group scale (the per-group INT8 format).  A transform thread
 // covers 32 k of one weight row per stage: 4 * CB bytes of codes, kept kCodePF(CB) stages ahead in
 // its slots of a cp.async ring of 24 KB.
+// CB = 2 is the BitLinear ternary format: packed bytes [N/4, K], field j of byte [r, k] the code
+// of output r + j N/4; a tile's 128 A rows are 32 packed rows x 4 fields (TMEM lane quarter q =
+// field q), each transform thread reads 32 bytes of its packed row per stage and keeps its field.
+// Its weights {-1, 0, 1, 2} are exact in bf16, so that format runs bf16 A and B straight from the
+// caller's x (no preparation kernel, no workspace) and scales by the weight scale in the epilogue.
 template <int CB> struct CodeFmt {
-    static constexpr int kBytes = 4 * CB;                    // code bytes per thread per stage
+    static constexpr int kBytes = CB == 2 ? 32 : 4 * CB;     // code bytes per thread per stage
     static constexpr int kCopies = kBytes / 16;              // 16-byte copies per stage
     static constexpr int kPF = CB == 4 ? 6 : 3;              // stages in flight
+    static constexpr bool kTernary = CB == 2;
+    static constexpr int kKPerCopy = CB == 4 ? 32 : 16;      // k covered by one 16-byte copy
 };
 constexpr int kGroupT = 4;          // token tiles that walk the weight tiles together
-// kind::f16: D f32, A and B f16 (format 0), both K-major, N = 256, M = 128
+// kind::f16: D f32, A and B f16 (format 0; bf16 = format 1 for the ternary format), both K-major,
+// N = 256, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t kIdescBf16 = kIdesc | (1u << 7) | (1u << 10);
 
 // per transform thread, kPF stages of its code bytes: [stage][copy][transform thread] x 16 bytes
 constexpr int kCodeRing = 6 * kXformWarps * 32 * 16;
@@ -101,9 +110,26 @@ struct TsParams {
     int M, N, K;
     int g_shift, ng;                  // log2 g, K / g
     int tiles_t, tiles_w;
+    const float* weight_scale;        // ternary format: device scalar (multiplied, or its reciprocal)
+    int invert;
+    int R;                            // ternary format: packed rows N / 4
     int vec_params;                   // parameter rows allow 16-byte loads of 8 groups
     unsigned* status;
 };
+
+QLIN_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+QLIN_DEV uint32_t bf16x2_min(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 
 QLIN_DEV uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c)
 {
@@ -250,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc_mma_ts(tmem, tmem + (uint32_t)(kAccCols + as * kACols + kk * 8), umma_desc_sw128(b0 + kk * 32),
-                                  kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                                  CodeFmt<CB>::kTernary ? kIdescBf16 : kIdesc, (kb | kk) != 0 ? 1u : 0u);
                     tc_commit(&bars.xempty[xs]);
                     tc_commit(&bars.aempty[as]);
                     if (++xs == kXStages) {
@@ -277,13 +303,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         const int q = warp & 3;             // TMEM lane quarter this warp may access
         const int kh = (warp - 2) >> 2;     // 32-k half of each stage
         const int r = 32 * q + lane;        // weight row within the tile
-        const size_t pitch = (size_t)p.K * CB / 8;
+        const size_t pitch = (size_t)p.K * F::kBytes / 32;  // bytes per code row (kBytes per 32 k)
         pdl_wait_prior_grids();  // the weights' parameters may come from the previous kernel
 
-        auto row_of = [&](int ti) {
+        auto row_of = [&](int ti) {  // the code row this thread reads in tile ti
             int tt, wt;
             tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
-            return min(wt * kTW + r, p.N - 1);
+            if constexpr (F::kTernary)
+                return min(wt * 32 + lane, p.R - 1);
+            else
+                return min(wt * kTW + r, p.N - 1);
         };
         // codes of stage (ti, kb) for this thread: F::kBytes bytes (32 k) of row n, copied kCodePF
         // stages ahead into this thread's slots of the shared-memory ring with cp.async (one commit
@@ -293,11 +322,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         const uint8_t* lrow = my_tiles > 0 ? p.codes + (size_t)row_of(0) * pitch + F::kBytes * kh : p.codes;
         uint4* my_ring = code_ring + (warp - 2) * 32 + lane;  // copy c of slot j: my_ring[(j * kCopies + c) * 256]
         auto load_next = [&](int slot) {
-            const bool in = lti < my_tiles && lkb * kKE + 32 * kh < p.K;
 #pragma unroll
-            for (int c = 0; c < F::kCopies; ++c)
+            for (int c = 0; c < F::kCopies; ++c) {  // each copy is in range or zero-filled on its own
+                const bool in = lti < my_tiles && lkb * kKE + 32 * kh + c * F::kKPerCopy < p.K;
                 cp_async16(my_ring + (slot * F::kCopies + c) * kXformWarps * 32,
-                           in ? lrow + (size_t)lkb * (kKE * CB / 8) + 16 * c : p.codes, in ? 16 : 0);
+                           in ? lrow + (size_t)lkb * (F::kBytes * 2) + 16 * c : p.codes, in ? 16 : 0);
+            }
             cp_async_commit();
             if (lti < my_tiles && ++lkb == nk) {
                 lkb = 0;
@@ -364,6 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         for (int j = 0; j < kCodePF; ++j)
             load_next(j);
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols + 16 * kh);
+        // ternary format: this warp keeps field q (mask, and the bf16x2 scale / bias that map
+        // 128 + 4^q c to c - 1)
+        const uint32_t tmask = 0x00030003u << (2 * q);
+        const uint32_t tscale = q == 0 ? 0x3F803F80u : q == 1 ? 0x3E803E80u : q == 2 ? 0x3D803D80u : 0x3C803C80u;
+        const uint32_t tbias = q == 0 ? 0xC301C301u : q == 1 ? 0xC204C204u : q == 2 ? 0xC110C110u : 0xC040C040u;
         int ti = 0, kb = 0, as = 0, pend_as = -1;
         unsigned aph = 0u;
         bool ok = true;
@@ -384,8 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             for (int j = 0; j < kCodePF; ++j) {
                 if (base + j >= total || !ok)
                     break;
-                uint32_t s2, b2;
-                params_for(ti, kb, s2, b2);
+                uint32_t s2 = 0u, b2 = 0u;
+                if constexpr (!F::kTernary)
+                    params_for(ti, kb, s2, b2);
                 // a pair of codes (q, q') of one byte becomes f16x2 in four instructions: PRMT puts
                 // the byte (low half) and the byte of w >> 1 (high half) in place, one LOP3 makes the
                 // exact fp16 (1024 + q, 1024 + 8 q'), one f16x2 FMA recovers (q, q') exactly, and one
@@ -404,6 +440,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                             const uint32_t v = lop3_and_or(prmt(words[w], w1, sel), 0x0078000Fu, 0x64006400u);
                             const uint32_t qq = f16x2_fma(v, 0x30003C00u, 0xD800E400u);  // (1, 1/8), (-1024, -128)
                             o[4 * w + e] = f16x2_fma(qq, s2, b2);
+                        }
+                    }
+                } else if constexpr (F::kTernary) {
+                    // field q of each byte, k in order: PRMT puts bytes (k, k+1) in the low byte of each
+                    // bf16 half, one LOP3 masks the field into the mantissa of 128 (0x4300) -- 128 + 4^q c,
+                    // exact -- one bf16x2 FMA gives c - 1 exactly, and a min with 2 keeps code 3 at weight
+                    // 2 (field 3 lands on the exponent's low bit: 128, 192, 256, 384 -> -1, 0, 1, 3)
+                    const uint4 c0 = my_ring[(2 * j) * kXformWarps * 32];
+                    const uint4 c1 = my_ring[(2 * j + 1) * kXformWarps * 32];
+                    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t v = lop3_and_or(prmt(words[w], 0u, h ? 0x0302u : 0x0100u), tmask, 0x43004300u);
+                            o[2 * w + h] = bf16x2_min(bf16x2_fma(v, tscale, tbias), 0x40004000u);
                         }
                     }
                 } else {
@@ -463,12 +515,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             int tt, wt;
             tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
             const int m0 = tt * kTT + th * (kTT / 2);
-            const int n = wt * kTW + 32 * q + lane;
-            const bool n_ok = n < p.N;
+            // output row of TMEM lane 32 q + lane: ternary -> packed row 32 wt + lane, field q
+            const int n = F::kTernary ? wt * 32 + lane + q * p.R : wt * kTW + 32 * q + lane;
+            const bool n_ok = F::kTernary ? wt * 32 + lane < p.R : n < p.N;
             const float bn = (p.bias && n_ok) ? (p.out_f32 ? static_cast<const float*>(p.bias)[n]
                                                            : __bfloat162float(static_cast<const __nv_bfloat16*>(p.bias)[n]))
                                               : 0.f;
-            const float rs = n_ok ? p.row_scale[n] : 0.f;
+            float rs = 0.f;
+            if (n_ok) {
+                if constexpr (F::kTernary) {
+                    const float ws = *p.weight_scale;
+                    rs = p.invert ? __frcp_rn(ws) : ws;  // 1/ws rounded once, as a division would
+                } else {
+                    rs = p.row_scale[n];
+                }
+            }
             const uint32_t acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(th * (kTT / 2));
             const size_t o0 = (size_t)m0 * p.N + n;
 #pragma unroll 1
@@ -479,14 +540,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                     continue;
                 // token scales of the chunk (the workspace holds them for whole 256-token tiles)
                 float ts[16];
-                const float4* tsp = reinterpret_cast<const float4*>(p.tok_scale + m0 + c * 16);
+                if constexpr (F::kTernary) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float4 t4 = __ldg(tsp + u);
-                    ts[4 * u] = t4.x * rs;
-                    ts[4 * u + 1] = t4.y * rs;
-                    ts[4 * u + 2] = t4.z * rs;
-                    ts[4 * u + 3] = t4.w * rs;
+                    for (int u = 0; u < 16; ++u)
+                        ts[u] = rs;
+                } else {
+                    const float4* tsp = reinterpret_cast<const float4*>(p.tok_scale + m0 + c * 16);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4 t4 = __ldg(tsp + u);
+                        ts[4 * u] = t4.x * rs;
+                        ts[4 * u + 1] = t4.y * rs;
+                        ts[4 * u + 2] = t4.z * rs;
+                        ts[4 * u + 3] = t4.w * rs;
+                    }
                 }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -513,7 +580,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         tmem_dealloc(tmem, kTmemCols);
 }
 
-bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Power-of-two exponent that brings a magnitude bound v (> 0) into [2^14, 2^15).
 QLIN_DEV int prep_shift(float v)
@@ -680,6 +746,58 @@ size_t tc_affine_workspace(int64_t M, int64_t N, int64_t K, int g)
     return a256((size_t)M * K * 2) + 2 * a256((size_t)N * ng * 2) + a256(mt * 4) + a256((size_t)N * 4);
 }
 
+namespace {
+
+cudaError_t launch_ts(void (*kern)(TsParams), const TsParams& prm, cudaStream_t st, const DeviceInfo& dev)
+{
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess)
+        return e;
+    const int tiles = prm.tiles_t * prm.tiles_w;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+}  // namespace
+
+cudaError_t launch_tc_bitlinear(const BitlinearArgs& a, cudaStream_t st, const DeviceInfo& dev)
+{
+    TsParams prm = {};
+    prm.codes = a.packed;
+    prm.scales = nullptr;
+    prm.biases = nullptr;
+    prm.tok_scale = nullptr;
+    prm.row_scale = nullptr;
+    prm.bias = a.bias;
+    prm.out = a.y;
+    prm.out_f32 = 0;
+    prm.M = (int)a.M;
+    prm.N = (int)a.N;
+    prm.K = (int)a.K;
+    prm.R = (int)(a.N / 4);
+    prm.g_shift = 0;
+    prm.ng = 1;
+    prm.tiles_t = (int)((a.M + kTT - 1) / kTT);
+    prm.tiles_w = (prm.R + 31) / 32;
+    prm.vec_params = 0;
+    prm.weight_scale = a.weight_scale;
+    prm.invert = a.invert;
+    prm.status = dev.status;
+    if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
+                        (uint64_t)a.K * 2, kKE, kTT))
+        return cudaErrorInvalidValue;
+    return launch_ts(tc_affine_ts_kernel<2>, prm, st, dev);
+}
+
 cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
     // workspace: x16 [M][K], s16 / b16 [N][ng] (fp16), tok_scale [M rounded up to 256 tokens],
@@ -739,22 +857,10 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)a.K, (uint64_t)a.M,
                         (uint64_t)a.K * 2, kKE, kTT))
         return cudaErrorInvalidValue;
-    auto kern = a.bits == 8 ? tc_affine_ts_kernel<8> : tc_affine_ts_kernel<4>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess)
-        return e;
-    const int tiles = prm.tiles_t * prm.tiles_w;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)kSmem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, prm);
+    prm.weight_scale = nullptr;
+    prm.invert = 0;
+    prm.R = 0;
+    return launch_ts(a.bits == 8 ? tc_affine_ts_kernel<8> : tc_affine_ts_kernel<4>, prm, st, dev);
 }
 
 }  // namespace qlin

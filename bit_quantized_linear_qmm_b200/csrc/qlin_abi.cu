@@ -260,6 +260,8 @@ qlin_status bitlinear_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t 
     a.invert = invert_weight_scale ? 1 : 0;
     a.bias = bias;
     a.y = y;
+    if (M > 16)  // prefill: the tcgen05 GEMM reads the packed weights once per 256-token tile
+        return from_cuda(launch_tc_bitlinear(a, static_cast<cudaStream_t>(stream), dev));
     return from_cuda(launch_bitlinear_gemv(a, static_cast<cudaStream_t>(stream), dev));
 }
 

@@ -342,6 +342,8 @@ struct BitlinearArgs {
     void* y;
 };
 cudaError_t launch_bitlinear_gemv(const BitlinearArgs& a, cudaStream_t st, const DeviceInfo& dev);
+// BitLinear with M > 16 on the tcgen05 GEMM (k_tc_affine.cu; bf16 x, bf16 weights exact)
+cudaError_t launch_tc_bitlinear(const BitlinearArgs& a, cudaStream_t st, const DeviceInfo& dev);
 
 }  // namespace qlin
 

@@ -96,3 +96,36 @@ def test_bitlinear_rejects_ragged(ql):
     with pytest.raises(ql.QlinError) as e:
         ql.bitlinear_matmul(x, P, 6, ws, False)
     assert e.value.status == ql.QLIN_ERR_INVALID_ARG
+
+
+# M > 16: the tcgen05 GEMM (bf16 x, exact bf16 ternary weights, 32 packed rows x 4 fields per tile)
+PREFILL = [synth.BitLinearCase(f"prefill_M{M}_K{K}_N{N}_{'div' if inv else 'mul'}{'_bias' if b else ''}", M, K, N,
+                               0.5, inv, b, seed=25, all_bytes=ab)
+           for (M, K, N, inv, b, ab) in [(300, 1040, 600, False, True, True),   # K % 32 == 16, ragged tiles
+                                         (256, 512, 4096, True, False, False),
+                                         (33, 2048, 136, False, False, True),
+                                         (512, 4096, 512, False, True, False)]]
+
+
+@pytest.mark.parametrize("case", PREFILL, ids=[c.name for c in PREFILL])
+def test_bitlinear_prefill(ql, orc, case):
+    _run(ql, orc, case)
+
+
+def test_bitlinear_prefill_llm_sampled(ql, orc):
+    """M = 2048, K = N = 4096 in one call; 48 sampled tokens x all outputs of 64 sampled packed rows."""
+    case = synth.BitLinearCase("prefill_2048", 2048, 4096, 4096, 0.5, True, False, seed=27)
+    P = case.packed()
+    x = case.x()
+    ws = torch.tensor([0.5], dtype=torch.float32, device="cuda")
+    y = ql.bitlinear_matmul(x.torch("cuda"), to_dev(P), 4096, ws, True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(4)
+    toks = np.sort(rng.choice(2048, size=48, replace=False))
+    prow = np.sort(rng.choice(1024, size=64, replace=False))
+    prow[-1] = 1023
+    R = 1024
+    cols = np.concatenate([prow + j * R for j in range(4)])  # output n = r + j N/4
+    yr, mag = orc.bitlinear(x.vals[toks], P[prow], 4 * len(prow), 0.5, True)
+    ys = y[torch.as_tensor(toks, device="cuda")][:, torch.as_tensor(cols, device="cuda")]
+    assert_fp_close(ys, yr, mag, None, "prefill_2048 sampled")
