@@ -58,6 +58,9 @@ def _load():
         lib.orc_w8a8_linear.argtypes = [P, I64, I64, P, P, I64, P, P, P, P, P]
         lib.orc_w4a8_linear.argtypes = [P, I64, I64, P, P, I64, P, P, P, P, P]
         lib.orc_quantize_int8_groups.argtypes = [P, I64, I64, C.c_int, P, P]
+        lib.orc_percentile_linear.argtypes = [P, I64, C.c_double]
+        lib.orc_percentile_linear.restype = C.c_float
+        lib.orc_quantize_weight_int8_clip.argtypes = [P, I64, I64, C.c_double, P, P]
         lib.orc_pergroup_linear.argtypes = [P, I64, I64, P, P, I64, C.c_int, P, P, P, P, P]
         lib.orc_f32_to_bf16.argtypes = [P, I64, P]
         lib.orc_bf16_to_f32.argtypes = [P, I64, P]
@@ -282,3 +285,20 @@ def pergroup_linear(x, w, scale_w, g: int, bias=None):
     _check(_load().orc_pergroup_linear(_p(x), M, K, _p(w), _p(scale_w), N, g, _p(bias), _p(qx), _p(sx),
                                        _p(y), _p(mag)), "pergroup_linear")
     return y, mag, qx, sx
+
+
+def percentile_linear(v, p: float) -> float:
+    """The p-th percentile of a float32 vector, linear interpolation in float32 arithmetic."""
+    v = _c(v, np.float32).ravel()
+    return float(np.float32(_load().orc_percentile_linear(_p(v), v.size, float(p))))
+
+
+def quantize_weight_int8_clip(w, clip_percentile: float):
+    """Per-row int8 with a percentile clip: returns (q int8 [R, C], scale fp32 [R])."""
+    w = _c(w, np.float32)
+    R, Cc = w.shape
+    q = np.empty((R, Cc), np.int8)
+    s = np.empty((R,), np.float32)
+    _check(_load().orc_quantize_weight_int8_clip(_p(w), R, Cc, float(clip_percentile), _p(q), _p(s)),
+           "quantize_weight_int8_clip")
+    return q, s

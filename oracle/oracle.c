@@ -359,6 +359,90 @@ int orc_quantize_int8_rows(const float* w, int64_t R, int64_t C, int8_t* q, floa
 }
 
 /* ------------------------------------------------------------------ */
+/* [Q8] with clip_percentile: a per-row percentile of |w| as the clip.   */
+/* ------------------------------------------------------------------ */
+
+static int orc_cmp_f32(const void* a, const void* b)
+{
+    const float x = *(const float*)a, y = *(const float*)b;
+    return (x > y) - (x < y);
+}
+
+/*
+ * The p-th percentile of v[0..n) (0 <= p <= 100) by linear interpolation
+ * between the order statistics around (n - 1) p / 100 -- numpy's default
+ * ("linear", Hyndman and Fan's type 7), which [Q8] calls through
+ * np.percentile -- with numpy's float32 arithmetic for a float32 row:
+ * q = f32(p) / 100, h = (n - 1) q, j = floor(h), t = h - j, a = v_(j),
+ * b = v_(j+1), and  a + (b - a) t  when t < 1/2, else  b - (b - a)(1 - t);
+ * h >= n - 1 gives the largest value.  Each step rounded to float32.
+ */
+float orc_percentile_linear(const float* v, int64_t n, double p)
+{
+    float* s = (float*)malloc((size_t)n * sizeof(float));
+    if (!s)
+        return NAN;
+    memcpy(s, v, (size_t)n * sizeof(float));
+    qsort(s, (size_t)n, sizeof(float), orc_cmp_f32);
+    const float q = (float)p / 100.0f;
+    const float h = (float)(n - 1) * q;
+    float r;
+    if (h >= (float)(n - 1)) {
+        r = s[n - 1];
+    } else {
+        const float j = floorf(h);
+        const float t = h - j;
+        const float a = s[(int64_t)j], b = s[(int64_t)j + 1];
+        const float d = b - a;
+        r = t < 0.5f ? a + d * t : b - d * (1.0f - t);
+    }
+    free(s);
+    return r;
+}
+
+/*
+ * [Q8] quantize_weight_int8 with clip_percentile set: per row, row_clip =
+ * percentile(|w_row|, clip_percentile) (above), replaced by max |w_row| when
+ * it is 0; scale = row_clip / 127 (fp32), zero -> 1; w clipped to
+ * [-row_clip, row_clip]; q = clip(round(w / scale), -128, 127).
+ * w: [R, C]; q: [R, C] int8; scale: [R] fp32.
+ */
+int orc_quantize_weight_int8_clip(const float* w, int64_t R, int64_t C, double clip_percentile, int8_t* q,
+                                  float* scale)
+{
+    if (R <= 0 || C <= 0 || !(clip_percentile >= 0.0 && clip_percentile <= 100.0))
+        return ORC_EINVAL;
+    float* a = (float*)malloc((size_t)C * sizeof(float));
+    if (!a)
+        return ORC_EINVAL;
+    for (int64_t r = 0; r < R; ++r) {
+        float amax = 0.0f;
+        for (int64_t c = 0; c < C; ++c) {
+            a[c] = fabsf(w[r * C + c]);
+            if (a[c] > amax) amax = a[c];
+        }
+        float row_clip = orc_percentile_linear(a, C, clip_percentile);
+        if (row_clip == 0.0f)
+            row_clip = amax;
+        float s = row_clip / 127.0f;
+        if (s == 0.0f)
+            s = 1.0f;
+        scale[r] = s;
+        for (int64_t c = 0; c < C; ++c) {
+            float v = w[r * C + c];
+            if (v < -row_clip) v = -row_clip;
+            if (v > row_clip) v = row_clip;
+            float t = rintf(v / s);
+            if (t < -128.0f) t = -128.0f;
+            if (t > 127.0f) t = 127.0f;
+            q[r * C + c] = (int8_t)t;
+        }
+    }
+    free(a);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* [P4] per-column int4, zero point 8, two codes per byte.               */
 /* ------------------------------------------------------------------ */
 

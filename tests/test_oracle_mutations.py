@@ -36,6 +36,10 @@ MUTATIONS = [
      "int c = (k % 2 == 0) ? (byte & 15) : (byte >> 4);"),
     ("int8_absmax_scale", "float s = amax / 127.0f;\n        if (s == 0.0f)\n            s = 1.0f;\n        scale[r] = s;",
      "float s = amax / 128.0f;\n        if (s == 0.0f)\n            s = 1.0f;\n        scale[r] = s;"),
+    ("percentile_index_n", "const float h = (float)(n - 1) * q;", "const float h = (float)n * q;"),
+    ("percentile_lerp_side", "r = t < 0.5f ? a + d * t : b - d * (1.0f - t);", "r = t < 0.5f ? a + d * t : b - d * t;"),
+    ("percentile_no_zero_fallback", "        if (row_clip == 0.0f)\n            row_clip = amax;", "        if (row_clip < 0.0f)\n            row_clip = amax;"),
+    ("percentile_no_clip", "            if (v < -row_clip) v = -row_clip;\n            if (v > row_clip) v = row_clip;", "            (void)row_clip;"),
     ("groups_scale_row_major", "scale_w[grp * N + n] = s;", "scale_w[n * G + grp] = s;"),
     ("pergroup_scale_index", "const double sw = (double)scale_w[grp * N + n];", "const double sw = (double)scale_w[n * G + grp];"),
     ("pergroup_m1_quantizes_x", "const int fp_act = M == 1;", "const int fp_act = 0;"),

@@ -485,3 +485,51 @@ def test_pergroup_dispatch_m1_vs_m2(orc):
     r1, _, _, _ = orc.pergroup_linear(xr, q, s, g)
     r2, _, _, _ = orc.pergroup_linear(np.vstack([xr, xr]), q, s, g)
     assert not np.allclose(r1[0], r2[0], rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------------------------ clip_percentile (quantize_weight_int8)
+
+def test_percentile_linear_equals_numpy(orc):
+    """The oracle's percentile (sorting and interpolating in float32) is bit-equal to numpy's
+    np.percentile, an independent implementation of the same definition, on random rows of many
+    lengths and percentiles, the end points 0 and 100 and the median included."""
+    rng = np.random.default_rng(11)
+    for trial in range(600):
+        n = int(rng.integers(1, 400))
+        p = float(rng.choice([0.0, 50.0, 99.0, 99.9, 99.99, 100.0, rng.uniform(0, 100)]))
+        v = np.abs(rng.standard_normal(n).astype(np.float32) * np.float32(rng.uniform(1e-3, 1e3)))
+        assert orc.percentile_linear(v, p) == float(np.percentile(v, p)), (n, p)
+
+
+def test_percentile_end_points(orc):
+    v = np.array([3.0, 1.0, 2.0, 5.0, 4.0], np.float32)
+    assert orc.percentile_linear(v, 0.0) == 1.0 and orc.percentile_linear(v, 100.0) == 5.0
+    assert orc.percentile_linear(v, 50.0) == 3.0
+    assert orc.percentile_linear(v, 12.5) == 1.5  # h = 4 * 0.125 = 0.5: halfway between 1 and 2
+
+
+def test_quantize_clip_properties(orc):
+    """With a percentile clip: the scale is the clip / 127, elements past the clip saturate at
+    +-127, the others follow the absmax rule with that scale; p = 100 is the absmax quantiser
+    exactly; a row whose percentile is 0 falls back to its max; an all-zero row gets scale 1."""
+    rng = np.random.default_rng(12)
+    R, C = 8, 1000
+    w = (rng.standard_normal((R, C)) * 0.02).astype(np.float32)
+    w[0, :5] = [1.0, -2.0, 1.5, -0.9, 3.0]              # outliers
+    w[1, :] = 0.0
+    w[1, 7] = 0.25                                      # percentile 0 for p < 99.9 -> max
+    w[2, :] = 0.0                                       # all zero
+    q, s = orc.quantize_weight_int8_clip(w, 99.0)
+    clip = np.array([np.percentile(np.abs(w[r]), 99.0) for r in range(R)], np.float32)
+    assert s[1] == np.float32(np.float32(0.25) / np.float32(127.0)) and q[1, 7] == 127
+    assert s[2] == 1.0 and not np.any(q[2])
+    for r in (0, 3, 4, 5, 6, 7):
+        assert s[r] == np.float32(clip[r] / np.float32(127.0))
+        over = np.abs(w[r]) >= clip[r]
+        assert np.all(np.abs(q[r][over]) == 127)
+        inside = ~over
+        err = np.abs(w[r][inside] - q[r][inside].astype(np.float64) * s[r])
+        assert np.all(err <= s[r] / 2 * (1 + 1e-6))
+    q100, s100 = orc.quantize_weight_int8_clip(w, 100.0)
+    qa, sa = orc.quantize_int8_rows(w)
+    assert np.array_equal(q100, qa) and np.array_equal(s100, sa)
