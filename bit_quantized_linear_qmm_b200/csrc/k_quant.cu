@@ -327,6 +327,69 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __
 
 // ---------------------------------------------------------------- per-column int4
 // Block = 32 columns x 8 row slices.
+// ---------------------------------------------------------------- per-row int8 with a percentile clip
+// One CTA per row [cider/ops.py quantize_weight_int8, clip_percentile]: |w| of the row is sorted in
+// shared memory (bitonic, as uint32 bit patterns: non-negative floats order like their bits; the
+// pad is +inf), the clip is the linear-interpolated percentile at (C - 1) p / 100 in float32 with
+// every operation rounded separately (as numpy does it for a float32 row), 0 -> max |w|; then
+// scale = clip / 127 (zero -> 1), w clipped to [-clip, clip], q = clip(round(w / scale), -128,
+// 127) with IEEE divisions.  P2 = the power of two >= C that the sort runs over.
+template <typename TW>
+__global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW* __restrict__ w, int64_t C, int P2,
+                                                                       float pct, int8_t* __restrict__ q,
+                                                                       float* __restrict__ scale)
+{
+    extern __shared__ uint32_t sv[];
+    __shared__ float row_clip_s, scale_s;
+    const TW* row = w + (int64_t)blockIdx.x * C;
+    for (int i = threadIdx.x; i < P2; i += blockDim.x)
+        sv[i] = i < C ? __float_as_uint(fabsf(to_float(row[i]))) : 0x7F800000u;
+    __syncthreads();
+    for (int k = 2; k <= P2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < P2; i += blockDim.x) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const uint32_t a = sv[i], b = sv[l];
+                    if (((i & k) == 0) == (a > b)) {
+                        sv[i] = b;
+                        sv[l] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (threadIdx.x == 0) {
+        const float qq = __fdiv_rn(pct, 100.0f);
+        const float h = __fmul_rn((float)(C - 1), qq);
+        float r;
+        if (h >= (float)(C - 1)) {
+            r = __uint_as_float(sv[C - 1]);
+        } else {
+            const float j = floorf(h);
+            const float t = __fsub_rn(h, j);
+            const float a = __uint_as_float(sv[(int64_t)j]), b = __uint_as_float(sv[(int64_t)j + 1]);
+            const float d = __fsub_rn(b, a);
+            r = t < 0.5f ? __fadd_rn(a, __fmul_rn(d, t)) : __fsub_rn(b, __fmul_rn(d, __fsub_rn(1.0f, t)));
+        }
+        if (r == 0.0f)
+            r = __uint_as_float(sv[C - 1]);  // max |w|
+        float sc = __fdiv_rn(r, 127.0f);
+        if (sc == 0.0f)
+            sc = 1.0f;
+        row_clip_s = r;
+        scale_s = sc;
+        scale[blockIdx.x] = sc;
+    }
+    __syncthreads();
+    const float rc = row_clip_s, sc = scale_s;
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
+        const float v = fminf(fmaxf(to_float(row[c]), -rc), rc);
+        q[(int64_t)blockIdx.x * C + c] = (int8_t)fminf(fmaxf(rintf(__fdiv_rn(v, sc)), -128.f), 127.f);
+    }
+}
+
 // ---------------------------------------------------------------- per-group int8 (pergroup_linear's format)
 // One warp per (row n, group): the int8 rule per group of g inputs -- scale = max |w| / 127 (zero
 // -> 1), q = clip(round(w / scale), -128, 127), IEEE divisions -- with the scales stored
@@ -497,6 +560,31 @@ cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R,
     else
         quantize_int8_rows_kernel<float><<<(unsigned)R, 256, 0, st>>>(static_cast<const float*>(w), C, q, scale,
                                                                       rowsum, rel);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weight_int8_clip(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, float pct,
+                                             int8_t* q, float* scale, cudaStream_t st, const DeviceInfo&)
+{
+    int p2 = 1;
+    while (p2 < C)
+        p2 <<= 1;
+    const size_t smem = (size_t)p2 * 4;
+    if (w_dt == QLIN_BF16) {
+        cudaError_t e = cudaFuncSetAttribute(quantize_weight_int8_clip_kernel<__nv_bfloat16>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        quantize_weight_int8_clip_kernel<__nv_bfloat16><<<(unsigned)R, 256, smem, st>>>(
+            static_cast<const __nv_bfloat16*>(w), C, p2, pct, q, scale);
+    } else {
+        cudaError_t e = cudaFuncSetAttribute(quantize_weight_int8_clip_kernel<float>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        quantize_weight_int8_clip_kernel<float><<<(unsigned)R, 256, smem, st>>>(static_cast<const float*>(w), C, p2,
+                                                                              pct, q, scale);
+    }
     return cudaGetLastError();
 }
 

@@ -294,6 +294,29 @@ qlin_status qlin_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64
     return from_cuda(launch_pack_int4_cols(w, w_dt, K, N, packed, scale, static_cast<cudaStream_t>(stream), dev));
 }
 
+qlin_status qlin_quantize_weight_int8(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, double clip_percentile,
+                                     int8_t* q, float* scale, void* stream)
+{
+    if (!w || !q || !scale || R <= 0 || C <= 0 || R > INT32_MAX || C > INT32_MAX)
+        return QLIN_ERR_INVALID_ARG;
+    if (!dtype_ok(w_dt))
+        return QLIN_ERR_UNSUPPORTED;
+    if (clip_percentile > 100.0 || clip_percentile != clip_percentile)
+        return QLIN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    qlin_status s;
+    if ((s = current_device(dev)) != QLIN_OK)
+        return s;
+    if (clip_percentile < 0.0)  // no clip: the absmax rule
+        return from_cuda(
+            launch_quantize_int8_rows(w, w_dt, R, C, q, scale, nullptr, static_cast<cudaStream_t>(stream), dev));
+    if (C > 32768)  // the row is sorted in shared memory
+        return QLIN_ERR_UNSUPPORTED;
+    // numpy converts the percentile to the row's float32 before dividing by 100
+    return from_cuda(launch_quantize_weight_int8_clip(w, w_dt, R, C, (float)clip_percentile, q, scale,
+                                                      static_cast<cudaStream_t>(stream), dev));
+}
+
 qlin_status qlin_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int group_size,
                                      int8_t* q, float* scale_w, void* stream)
 {

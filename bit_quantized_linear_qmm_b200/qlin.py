@@ -76,6 +76,7 @@ def lib():
         "w4a8_linear": ([P, I, I64, I64, P, P, I64, P, P, P, SZ, P], I),
         "w8a8_linear_noalloc": ([P, I, I64, I64, P, P, I64, P, P, P], I),
         "qlin_quantize_int8_groups": ([P, I, I64, I64, I, P, P, P], I),
+        "qlin_quantize_weight_int8": ([P, I, I64, I64, C.c_double, P, P, P], I),
         "pergroup_linear": ([P, I, I64, I64, P, P, I64, I, P, P, P, SZ, P], I),
         "qlin_get_device_status": ([P], I),
         "qlin_selftest_wait_timeout": ([C.c_uint, P], I),
@@ -282,3 +283,15 @@ def pergroup_linear(x, w, scale_w, group_size: int, bias=None, out=None, workspa
     _check(lib().pergroup_linear(_ptr(x), _dt(x), M, K, _ptr(w), _ptr(scale_w), N, group_size, _ptr(bias), _ptr(out),
                                  _ptr(workspace), workspace.numel(), _stream(x.device)), "pergroup_linear")
     return out
+
+
+def quantize_weight_int8(w, clip_percentile=None):
+    """Per-row int8 weights, optionally clipped at a per-row percentile of |w|: (q [R, C], scale [R])."""
+    _cuda(w)
+    R, Cc = w.shape
+    q = torch.empty((R, Cc), dtype=torch.int8, device=w.device)
+    s = torch.empty((R,), dtype=torch.float32, device=w.device)
+    p = -1.0 if clip_percentile is None else float(clip_percentile)
+    _check(lib().qlin_quantize_weight_int8(_ptr(w), _dt(w), R, Cc, p, _ptr(q), _ptr(s), _stream(w.device)),
+           "qlin_quantize_weight_int8")
+    return q, s

@@ -226,6 +226,21 @@ qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
                         void* stream);
 
 /*
+ * Per-row symmetric INT8 weight quantisation with an optional percentile clip
+ * [cider/ops.py quantize_weight_int8, clip_percentile]: clip_percentile < 0
+ * (the page's None) is the absmax rule of qlin_quantize_int8_rows; 0 <= p <=
+ * 100 sets clip = the linear-interpolated p-th percentile of |w| over the row
+ * (numpy's default percentile method, in float32 as numpy computes it on a
+ * float32 row), replaced by max |w| when 0; scale = clip / 127 (zero -> 1);
+ * w clipped to [-clip, clip]; q = clip(round_half_even(w / scale), -128, 127).
+ * w: [R, C] of w_dt; q: int8 [R, C]; scale: fp32 [R].  The clip path sorts a
+ * row in shared memory: C <= 32768 (QLIN_ERR_UNSUPPORTED otherwise);
+ * p > 100 or NaN -> QLIN_ERR_INVALID_ARG.  Bit-exact.
+ */
+qlin_status qlin_quantize_weight_int8(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, double clip_percentile,
+                                     int8_t* q, float* scale, void* stream);
+
+/*
  * Per-group symmetric INT8 weight quantisation, the weight format of
  * pergroup_linear [cider/ops.py pergroup_linear, Args: "INT8 weights [N, K]
  * int8 (per-group symmetric quantized)", scales [num_groups, N]]: per group of

@@ -97,3 +97,35 @@ def test_quantize_full_prefill_weight_bit_exact(ql, orc):
     assert np.array_equal(codes.cpu().numpy().view(np.uint32), rc)
     assert np.array_equal(host_f32(s), rs)
     assert np.array_equal(host_f32(b), rb)
+
+
+CLIP_CASES = [(R, C, p, wdt) for (R, C) in [(7, 1000), (64, 4096), (3, 1), (5, 33), (2, 32768)]
+              for p in (99.9, 50.0, 0.0, 100.0, 97.25) for wdt in ("f32", "bf16")]
+
+
+@pytest.mark.parametrize("R,C,p,wdt", CLIP_CASES, ids=[f"R{c[0]}_C{c[1]}_p{c[2]}_{c[3]}" for c in CLIP_CASES])
+def test_quantize_weight_int8_clip_bit_exact(ql, orc, R, C, p, wdt):
+    """quantize_weight_int8 with clip_percentile [cider/ops.py]: codes and scales bit-equal to the
+    oracle (which is itself pinned to np.percentile)."""
+    import synth
+    w = synth.normal(71 + C, (R, C), 0.02)
+    w[0, : min(C, 3)] = [4.0, -3.0, 2.5][: min(C, 3)]  # outliers the clip cuts
+    if R > 1:
+        w[1, :] = 0.0                                    # zero row
+    if wdt == "bf16":
+        w = torch.from_numpy(w).to(torch.bfloat16).float().numpy()
+    q_ref, s_ref = orc.quantize_weight_int8_clip(w, p)
+    wt = torch.from_numpy(w).to(torch.bfloat16 if wdt == "bf16" else torch.float32).cuda()
+    q, s = ql.quantize_weight_int8(wt, p)
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_quantize_weight_int8_no_clip_is_absmax(ql, orc):
+    import synth
+    w = synth.normal(72, (16, 512), 0.02)
+    q_ref, s_ref = orc.quantize_int8_rows(w)
+    q, s = ql.quantize_weight_int8(torch.from_numpy(w).cuda(), None)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_ref) and np.array_equal(s.cpu().numpy(), s_ref)
