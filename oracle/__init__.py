@@ -63,6 +63,7 @@ def _load():
         lib.orc_quantize_weight_int8_clip.argtypes = [P, I64, I64, C.c_double, P, P]
         lib.orc_pergroup_linear.argtypes = [P, I64, I64, P, P, I64, C.c_int, P, P, P, P, P]
         lib.orc_f32_to_bf16.argtypes = [P, I64, P]
+        lib.orc_round_f16_array.argtypes = [P, I64, P]
         lib.orc_bf16_to_f32.argtypes = [P, I64, P]
         for name in ("orc_pack", "orc_unpack", "orc_affine_quantize", "orc_affine_dequantize",
                      "orc_affine_matmul", "orc_pack_ternary", "orc_bitlinear",
@@ -128,11 +129,14 @@ def unpack(packed, K: int, bits: int) -> np.ndarray:
     return q
 
 
-def affine_quantize(w, bits: int, group_size: int, bf16_params: bool):
+def affine_quantize(w, bits: int, group_size: int, bf16_params):
     """Returns (codes uint32 [N,K*b/32], scales f32 [N,K/g], biases f32 [N,K/g]).
 
-    With ``bf16_params`` the scales/biases are bf16 values (held exactly in f32).
+    ``bf16_params``: False / "f32" stores fp32 scales/biases; True / "bf16" bf16 values, "f16"
+    fp16 values (both held exactly in f32).
     """
+    if isinstance(bf16_params, str):
+        bf16_params = {"f32": 0, "bf16": 1, "f16": 2}[bf16_params]
     w = _c(w, np.float32)
     N, K = w.shape
     if K % group_size:
@@ -302,3 +306,11 @@ def quantize_weight_int8_clip(w, clip_percentile: float):
     _check(_load().orc_quantize_weight_int8_clip(_p(w), R, Cc, float(clip_percentile), _p(q), _p(s)),
            "quantize_weight_int8_clip")
     return q, s
+
+
+def round_f16(v) -> np.ndarray:
+    """Values rounded to the nearest binary16 (ties to even), as fp32."""
+    v = _c(v, np.float32)
+    out = np.empty_like(v)
+    _load().orc_round_f16_array(_p(v), v.size, _p(out))
+    return out

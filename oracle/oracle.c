@@ -96,15 +96,56 @@ void orc_bf16_to_f32(const uint16_t* in, int64_t n, float* out)
 }
 
 /* ------------------------------------------------------------------ */
+/* fp16: IEEE binary16, rounded to nearest even from binary32.           */
+/* ------------------------------------------------------------------ */
+
+/* Nearest binary16 value (ties to even) of a finite float, returned as a
+ * float; overflow past the largest binary16 gives +-inf, and values below the
+ * smallest normal round on the subnormal grid (multiples of 2^-24). */
+static float orc_round_f16(float f)
+{
+    if (f != f)
+        return f;
+    const double a = fabs((double)f);
+    if (a >= 65520.0)  /* rounds past 65504 (the tie at 65520 goes to the even, infinite side) */
+        return copysignf(INFINITY, f);
+    int e;
+    frexp(a, &e);             /* a = m 2^e, m in [0.5, 1) */
+    int q = e - 11;           /* spacing 2^q for 11 significant bits */
+    if (q < -24)
+        q = -24;              /* subnormal spacing */
+    const double step = ldexp(1.0, q);
+    double r = a / step;      /* exact: a has at most 24 bits */
+    double fl = floor(r);
+    const double frac = r - fl;
+    if (frac > 0.5 || (frac == 0.5 && fmod(fl, 2.0) != 0.0))
+        fl += 1.0;
+    return (float)copysign(fl * step, (double)f);  /* keeps the sign of a zero result */
+}
+
+void orc_round_f16_array(const float* in, int64_t n, float* out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = orc_round_f16(in[i]);
+}
+
+/* ------------------------------------------------------------------ */
 /* [QL] weight field: b-bit codes packed into uint32, shape [N, K*b/32].  */
 /* ------------------------------------------------------------------ */
 
+/* [QL] from_linear: 1 to 6 or 8 bits per weight. */
 static int orc_bits_ok(int bits)
 {
-    return bits == 2 || bits == 4 || bits == 8;
+    return (bits >= 1 && bits <= 6) || bits == 8;
 }
 
-/* q: one code per byte, [N, K], each < 2^bits.  out: [N, K*bits/32]. */
+/*
+ * q: one code per byte, [N, K], each < 2^bits.  out: [N, K*bits/32].  A row
+ * is one LSB-first bitstream: code k occupies bits k*bits .. k*bits+bits-1 of
+ * the row read as a little-endian integer of 32-bit words, so for 3, 5 and 6
+ * bits a code may continue in the next word (a reading: the pages do not
+ * show how such widths straddle words).
+ */
 int orc_pack(const uint8_t* q, int64_t N, int64_t K, int bits, uint32_t* out)
 {
     if (!orc_bits_ok(bits) || N < 0 || K < 0 || (K * bits) % 32 != 0)
@@ -119,6 +160,8 @@ int orc_pack(const uint8_t* q, int64_t N, int64_t K, int bits, uint32_t* out)
                 return ORC_EINVAL;
             int64_t bitpos = k * bits;
             out[n * words + bitpos / 32] |= code << (bitpos % 32);
+            if (bitpos % 32 + bits > 32)  /* the high bits continue in the next word */
+                out[n * words + bitpos / 32 + 1] |= code >> (32 - bitpos % 32);
         }
     }
     return 0;
@@ -134,7 +177,10 @@ int orc_unpack(const uint32_t* packed, int64_t N, int64_t K, int bits, uint8_t* 
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) {
             int64_t bitpos = k * bits;
-            q[n * K + k] = (uint8_t)((packed[n * words + bitpos / 32] >> (bitpos % 32)) & mask);
+            uint32_t v = packed[n * words + bitpos / 32] >> (bitpos % 32);
+            if (bitpos % 32 + bits > 32)
+                v |= packed[n * words + bitpos / 32 + 1] << (32 - bitpos % 32);
+            q[n * K + k] = (uint8_t)(v & mask);
         }
     return 0;
 }
@@ -149,8 +195,9 @@ static int orc_group_ok(int g)
 }
 
 /*
- * w: [N, K] values (fp32, or the fp32 value of a bf16 input).
- * bf16_params: 0 -> scales/biases stored as fp32; 1 -> stored as bf16.
+ * w: [N, K] values (fp32, or the fp32 value of a bf16 / fp16 input).
+ * bf16_params: 0 -> scales/biases stored as fp32; 1 -> stored as bf16;
+ * 2 -> stored as fp16.
  * codes: [N, K*bits/32]; scales, biases: [N, K/g], the STORED values written
  * as fp32 (a bf16-stored parameter is written as its exact fp32 value).
  *
@@ -183,9 +230,12 @@ int orc_affine_quantize(const float* w, int64_t N, int64_t K, int bits, int g,
             }
             float scale = (mx - mn) / qmax;
             float bias = mn;
-            if (bf16_params) {
+            if (bf16_params == 1) {
                 scale = orc_round_bf16(scale);
                 bias = orc_round_bf16(bias);
+            } else if (bf16_params == 2) {
+                scale = orc_round_f16(scale);
+                bias = orc_round_f16(bias);
             }
             if (scale == 0.0f)
                 scale = 1.0f;

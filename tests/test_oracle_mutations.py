@@ -36,6 +36,12 @@ MUTATIONS = [
      "int c = (k % 2 == 0) ? (byte & 15) : (byte >> 4);"),
     ("int8_absmax_scale", "float s = amax / 127.0f;\n        if (s == 0.0f)\n            s = 1.0f;\n        scale[r] = s;",
      "float s = amax / 128.0f;\n        if (s == 0.0f)\n            s = 1.0f;\n        scale[r] = s;"),
+    ("pack_drops_straddle", "                out[n * words + bitpos / 32 + 1] |= code >> (32 - bitpos % 32);",
+     "                out[n * words + bitpos / 32 + 1] |= 0u;"),
+    ("unpack_drops_straddle", "                v |= packed[n * words + bitpos / 32 + 1] << (32 - bitpos % 32);",
+     "                v |= 0u;"),
+    ("f16_ties_away", "    if (frac > 0.5 || (frac == 0.5 && fmod(fl, 2.0) != 0.0))", "    if (frac >= 0.5)"),
+    ("f16_subnormal_spacing", "    if (q < -24)\n        q = -24;", "    if (q < -25)\n        q = -25;"),
     ("percentile_index_n", "const float h = (float)(n - 1) * q;", "const float h = (float)n * q;"),
     ("percentile_lerp_side", "r = t < 0.5f ? a + d * t : b - d * (1.0f - t);", "r = t < 0.5f ? a + d * t : b - d * t;"),
     ("percentile_no_zero_fallback", "        if (row_clip == 0.0f)\n            row_clip = amax;", "        if (row_clip < 0.0f)\n            row_clip = amax;"),

@@ -44,7 +44,7 @@ def test_pack_golden_words(orc):
         assert np.array_equal(orc.unpack(got, q.shape[1], bits), q)
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 8])
 def test_pack_is_a_little_endian_bitstream(orc, bits):
     """Row of words == sum_k q[k] << (bits*k) as one integer; unpack inverts pack."""
     rng = np.random.default_rng(bits)
@@ -104,8 +104,8 @@ def _dyadic_case(N, K, g, bits, seed):
     return q, scale, bias, w
 
 
-@pytest.mark.parametrize("bits,g", [(2, 32), (4, 64), (8, 128), (4, 128)])
-@pytest.mark.parametrize("bf16", [False, True])
+@pytest.mark.parametrize("bits,g", [(2, 32), (4, 64), (8, 128), (4, 128), (1, 32), (3, 64), (5, 32), (6, 128)])
+@pytest.mark.parametrize("bf16", [False, True, "f16"])
 def test_quantize_recovers_dyadic_grid(orc, bits, g, bf16):
     """Weights on an exact grid come back as the same codes, scale and bias."""
     q, scale, bias, w = _dyadic_case(6, 2 * g, g, bits, seed=bits * 1000 + g)
@@ -117,7 +117,8 @@ def test_quantize_recovers_dyadic_grid(orc, bits, g, bf16):
     assert np.array_equal(orc.affine_dequantize(codes, s, b, w.shape[1], bits, g), w)
 
 
-@pytest.mark.parametrize("bits,g", [(2, 64), (4, 64), (4, 128), (8, 64), (4, 32)])
+@pytest.mark.parametrize("bits,g", [(2, 64), (4, 64), (4, 128), (8, 64), (4, 32), (1, 32), (3, 64), (5, 128),
+                                    (6, 32)])
 def test_quantize_roundtrip_within_half_scale(orc, bits, g):
     """|w - dequant(quant(w))| <= scale/2 (plus fp32 rounding of the step) for fp32 params."""
     w = synth.normal(11, (64, 4 * g), 0.02)
@@ -182,7 +183,8 @@ def _bitstream_codes(words_row, K, bits):
     return [(v >> (bits * k)) & ((1 << bits) - 1) for k in range(K)]
 
 
-@pytest.mark.parametrize("bits,g,M,N,K", [(4, 32, 3, 5, 64), (2, 64, 2, 7, 128), (8, 32, 4, 3, 96)])
+@pytest.mark.parametrize("bits,g,M,N,K", [(4, 32, 3, 5, 64), (2, 64, 2, 7, 128), (8, 32, 4, 3, 96), (3, 32, 2, 4, 64),
+                                          (5, 64, 2, 3, 128), (6, 32, 3, 2, 96), (1, 32, 2, 5, 64)])
 def test_affine_matmul_brute_force_exact(orc, bits, g, M, N, K):
     """Tiny layers with dyadic x and grid weights: the double sums are exact,
     so the oracle must equal an exact rational brute force."""
@@ -533,3 +535,19 @@ def test_quantize_clip_properties(orc):
     q100, s100 = orc.quantize_weight_int8_clip(w, 100.0)
     qa, sa = orc.quantize_int8_rows(w)
     assert np.array_equal(q100, qa) and np.array_equal(s100, sa)
+
+
+
+def test_round_f16_equals_numpy(orc):
+    """fp16 rounding of the oracle (written from the binary16 format) equals numpy's float32 ->
+    float16 conversion on normals, subnormals, ties, the overflow edge and signed zeros."""
+    rng = np.random.default_rng(13)
+    v = np.concatenate([
+        (rng.standard_normal(100000) * np.exp(rng.uniform(-25, 12, 100000))).astype(np.float32),
+        np.array([65504, 65519.99, 65520, 65536, -65520, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26, 2.0 ** -14,
+                  1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 0.0, -0.0, 2.0 ** -26], np.float32)])
+    with np.errstate(over="ignore"):
+        want = v.astype(np.float16).astype(np.float32)
+    got = orc.round_f16(v)
+    assert np.array_equal(np.signbit(got[np.isfinite(got)]), np.signbit(want[np.isfinite(want)]))
+    assert np.array_equal(got, want)
