@@ -566,8 +566,9 @@ struct W8Params {
     CUtensorMap tm_x;  // qx [M][K] int8, box {128 B, M rows}
     const float* s_x;
     const float* s_w;
-    const __nv_bfloat16* bias;
-    __nv_bfloat16* y;
+    const unsigned short* bias;  // [N] bf16, or fp16 when out_f16
+    unsigned short* y;           // [M][N] bf16, or fp16 when out_f16
+    int out_f16;
     int M, K, N;
     unsigned* status;
 };
@@ -684,8 +685,8 @@ __global__ void __launch_bounds__(kThreads, 2) w8_gemv_kernel(const __grid_const
             if (tok < M && n < p.N) {
                 float out = (float)sum * (p.s_x[tok] * p.s_w[n]);
                 if (p.bias)
-                    out += __bfloat162float(p.bias[n]);
-                p.y[(size_t)tok * p.N + n] = __float2bfloat16_rn(out);
+                    out += h16_to_float(p.bias[n], p.out_f16);
+                p.y[(size_t)tok * p.N + n] = to_h16(out, p.out_f16);
             }
         }
     }
@@ -726,8 +727,9 @@ struct W4Params {
     CUtensorMap tm_x;  // qx [M][K] int8, box {128 B, M rows}
     const float* s_x;
     const float* s_w;
-    const __nv_bfloat16* bias;
-    __nv_bfloat16* y;
+    const unsigned short* bias;  // [N] bf16, or fp16 when out_f16
+    unsigned short* y;           // [M][N] bf16, or fp16 when out_f16
+    int out_f16;
     int M, K, N;
     unsigned* status;
 };
@@ -843,8 +845,8 @@ __global__ void __launch_bounds__(kThreads, 2) w4_gemv_kernel(const __grid_const
             if (tok < M && col < p.N) {
                 float out = (float)(sum >> 4) * (p.s_x[tok] * p.s_w[col]);
                 if (p.bias)
-                    out += __bfloat162float(p.bias[col]);
-                p.y[(size_t)tok * p.N + col] = __float2bfloat16_rn(out);
+                    out += h16_to_float(p.bias[col], p.out_f16);
+                p.y[(size_t)tok * p.N + col] = to_h16(out, p.out_f16);
             }
         }
     }
@@ -874,10 +876,17 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, int smem, cudaStream_t st, const Pa
 }
 
 template <int BITS, int G, typename XT, typename PT, int NT, int RT>
-cudaError_t affine_launch_t(const AffineGemvArgs& a, int m0, int mcount, cudaStream_t st, const DeviceInfo& dev)
+cudaError_t affine_launch_t(const AffineGemvArgs& a, int m0, int mcount, cudaStream_t st, const DeviceInfo& dev,
+                            bool dry)
 {
     using Cfg = AffineCfg<BITS, G, XT, PT, NT, RT>;
     (void)dev;
+    // the CTA's group parameters live in shared memory beside the ring: long rows of small
+    // groups do not fit (the caller then takes the general kernel)
+    if (Cfg::smem_bytes((int)(a.K / G)) > 227 * 1024)
+        return cudaErrorNotSupported;
+    if (dry)
+        return cudaSuccess;
     AffineParams prm;
     const void* x = static_cast<const uint8_t*>(a.x) + (size_t)m0 * a.K * sizeof(XT);
     prm.scales = a.scales;
@@ -900,7 +909,7 @@ cudaError_t affine_launch_t(const AffineGemvArgs& a, int m0, int mcount, cudaStr
 }
 
 template <int BITS, int G, typename XT, typename PT>
-cudaError_t affine_launch_nt(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
+cudaError_t affine_launch_nt(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev, bool dry)
 {
     // 64-row CTAs when that still gives about one CTA per SM, 32-row CTAs, or 16-row CTAs (two
     // working CTAs per SM) when even 32-row CTAs would leave SMs idle
@@ -910,15 +919,15 @@ cudaError_t affine_launch_nt(const AffineGemvArgs& a, cudaStream_t st, const Dev
         const int mc = (int)(a.M - m0 < 16 ? a.M - m0 : 16);
         cudaError_t e;
         if (mc <= 8 && sizeof(XT) == 2)
-            e = wide     ? affine_launch_t<BITS, G, XT, PT, 1, 4>(a, (int)m0, mc, st, dev)
-                : narrow ? affine_launch_t<BITS, G, XT, PT, 1, 1>(a, (int)m0, mc, st, dev)
-                         : affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev);
+            e = wide     ? affine_launch_t<BITS, G, XT, PT, 1, 4>(a, (int)m0, mc, st, dev, dry)
+                : narrow ? affine_launch_t<BITS, G, XT, PT, 1, 1>(a, (int)m0, mc, st, dev, dry)
+                         : affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev, dry);
         else if (mc <= 8)
-            e = affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev);
+            e = affine_launch_t<BITS, G, XT, PT, 1, 2>(a, (int)m0, mc, st, dev, dry);
         else if (narrow && sizeof(XT) == 2)
-            e = affine_launch_t<BITS, G, XT, PT, 2, 1>(a, (int)m0, mc, st, dev);
+            e = affine_launch_t<BITS, G, XT, PT, 2, 1>(a, (int)m0, mc, st, dev, dry);
         else
-            e = affine_launch_t<BITS, G, XT, PT, 2, 2>(a, (int)m0, mc, st, dev);
+            e = affine_launch_t<BITS, G, XT, PT, 2, 2>(a, (int)m0, mc, st, dev, dry);
         if (e != cudaSuccess)
             return e;
     }
@@ -926,26 +935,26 @@ cudaError_t affine_launch_nt(const AffineGemvArgs& a, cudaStream_t st, const Dev
 }
 
 template <int BITS, typename XT, typename PT>
-cudaError_t affine_launch_g(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
+cudaError_t affine_launch_g(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev, bool dry)
 {
     switch (a.g) {
     case 32:
         if constexpr (BITS == 2)
             return cudaErrorNotSupported;
         else
-            return affine_launch_nt<BITS, 32, XT, PT>(a, st, dev);
-    case 64: return affine_launch_nt<BITS, 64, XT, PT>(a, st, dev);
-    default: return affine_launch_nt<BITS, 128, XT, PT>(a, st, dev);
+            return affine_launch_nt<BITS, 32, XT, PT>(a, st, dev, dry);
+    case 64: return affine_launch_nt<BITS, 64, XT, PT>(a, st, dev, dry);
+    default: return affine_launch_nt<BITS, 128, XT, PT>(a, st, dev, dry);
     }
 }
 
 template <typename XT, typename PT>
-cudaError_t affine_launch_b(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
+cudaError_t affine_launch_b(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev, bool dry)
 {
     switch (a.bits) {
-    case 2: return affine_launch_g<2, XT, PT>(a, st, dev);
-    case 4: return affine_launch_g<4, XT, PT>(a, st, dev);
-    default: return affine_launch_g<8, XT, PT>(a, st, dev);
+    case 2: return affine_launch_g<2, XT, PT>(a, st, dev, dry);
+    case 4: return affine_launch_g<4, XT, PT>(a, st, dev, dry);
+    default: return affine_launch_g<8, XT, PT>(a, st, dev, dry);
     }
 }
 
@@ -953,11 +962,18 @@ cudaError_t affine_launch_b(const AffineGemvArgs& a, cudaStream_t st, const Devi
 
 cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
-    if (a.x_dt == QLIN_BF16)
-        return a.p_dt == QLIN_BF16 ? affine_launch_b<__nv_bfloat16, __nv_bfloat16>(a, st, dev)
-                                   : affine_launch_b<__nv_bfloat16, float>(a, st, dev);
-    return a.p_dt == QLIN_BF16 ? affine_launch_b<float, __nv_bfloat16>(a, st, dev)
-                               : affine_launch_b<float, float>(a, st, dev);
+    auto run = [&](bool dry) {
+        if (a.x_dt == QLIN_BF16)
+            return a.p_dt == QLIN_BF16 ? affine_launch_b<__nv_bfloat16, __nv_bfloat16>(a, st, dev, dry)
+                                       : affine_launch_b<__nv_bfloat16, float>(a, st, dev, dry);
+        return a.p_dt == QLIN_BF16 ? affine_launch_b<float, __nv_bfloat16>(a, st, dev, dry)
+                                   : affine_launch_b<float, float>(a, st, dev, dry);
+    };
+    // every launch of the call checked first, so that a call runs wholly on one kernel
+    const cudaError_t e = run(true);
+    if (e == cudaErrorNotSupported)
+        return launch_affine_gemv_any(a, st, dev);
+    return e != cudaSuccess ? e : run(false);
 }
 
 cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev)
@@ -968,8 +984,9 @@ cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInf
         W8Params prm;
         prm.s_x = a.s_x + m0;
         prm.s_w = a.s_w;
-        prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
-        prm.y = static_cast<__nv_bfloat16*>(a.y) + m0 * a.N;
+        prm.bias = static_cast<const unsigned short*>(a.bias);
+        prm.y = static_cast<unsigned short*>(a.y) + m0 * a.N;
+        prm.out_f16 = a.out_f16;
         prm.M = mc;
         prm.K = (int)a.K;
         prm.N = (int)a.N;
@@ -1002,8 +1019,9 @@ cudaError_t launch_w4_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInf
         W4Params prm;
         prm.s_x = a.s_x + m0;
         prm.s_w = a.s_w;
-        prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
-        prm.y = static_cast<__nv_bfloat16*>(a.y) + m0 * a.N;
+        prm.bias = static_cast<const unsigned short*>(a.bias);
+        prm.y = static_cast<unsigned short*>(a.y) + m0 * a.N;
+        prm.out_f16 = a.out_f16;
         prm.M = mc;
         prm.K = (int)a.K;
         prm.N = (int)a.N;

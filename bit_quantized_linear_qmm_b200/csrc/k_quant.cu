@@ -13,6 +13,8 @@
 // half to even), so codes match the CPU reference bit for bit.
 #include "qlin_common.cuh"
 
+#include <type_traits>
+
 namespace qlin {
 namespace {
 
@@ -20,6 +22,7 @@ template <typename T> struct Vec;  // loads of N consecutive elements as floats
 
 QLIN_DEV float load_elem(const float* p, int64_t i) { return p[i]; }
 QLIN_DEV float load_elem(const __nv_bfloat16* p, int64_t i) { return __bfloat162float(p[i]); }
+QLIN_DEV float load_elem(const __half* p, int64_t i) { return __half2float(p[i]); }
 
 // ---------------------------------------------------------------- affine quantize
 // One warp per (row, group).  Lane l holds CPL = g/32 consecutive values.
@@ -117,6 +120,115 @@ __global__ void __launch_bounds__(256) affine_dequantize_kernel(const uint32_t* 
         } else {
             *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(vals);
         }
+    }
+}
+
+// ---------------------------------------------------------------- affine quantize, 3 / 5 / 6 bits
+// A row's codes form one LSB-first bitstream (code k at bits k*BITS ..), so a code may continue in
+// the next word; a group of G codes fills exactly WPG = G*BITS/32 whole words.  One warp per
+// (row, group) as above: lane l packs its CPL codes into v (bits l*CPL*BITS ..), and word j of the
+// group is the warp-wide OR of every lane's part that falls inside it.
+template <typename TW, typename TP, int BITS, int G>
+__global__ void __launch_bounds__(256) affine_quantize_odd_kernel(const TW* __restrict__ w, int64_t N, int64_t K,
+                                                                  uint32_t* __restrict__ codes,
+                                                                  TP* __restrict__ scales, TP* __restrict__ biases)
+{
+    constexpr int CPL = G / 32;
+    constexpr int NB = CPL * BITS;  // bits per lane, at most 24
+    constexpr int WPG = G * BITS / 32;
+    constexpr float QMAX = float((1 << BITS) - 1);
+    const int64_t groups_per_row = K / G;
+    const int64_t gid = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    if (gid >= N * groups_per_row)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int64_t n = gid / groups_per_row;
+    const int64_t gi = gid % groups_per_row;
+    const TW* wg = w + n * K + gi * G + lane * CPL;
+    float v[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i)
+        v[i] = load_elem(wg, i);
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 1; i < CPL; ++i) {
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    float scale = to_float(from_float<TP>(__fdiv_rn(__fsub_rn(mx, mn), QMAX)));
+    const float bias = to_float(from_float<TP>(mn));
+    if (scale == 0.0f)
+        scale = 1.0f;
+    if (lane == 0) {
+        scales[n * groups_per_row + gi] = from_float<TP>(scale);
+        biases[n * groups_per_row + gi] = from_float<TP>(bias);
+    }
+    uint32_t part = 0;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        float t = rintf(__fdiv_rn(__fsub_rn(v[i], bias), scale));
+        t = fminf(fmaxf(t, 0.0f), QMAX);
+        part |= static_cast<uint32_t>(t) << (BITS * i);
+    }
+    const int o = lane * NB;  // first bit of this lane's part within the group
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < WPG; ++j) {
+        const int lo = 32 * j;
+        uint32_t c = 0;
+        if (o >= lo && o < lo + 32)
+            c = part << (o - lo);  // the part starts in word j (its high bits may spill over)
+        else if (o < lo && o + NB > lo)
+            c = part >> (lo - o);  // the part started in word j-1 and ends in word j
+        const uint32_t word = __reduce_or_sync(0xffffffffu, c);
+        if (lane == j)
+            mine = word;
+    }
+    if (lane < WPG)
+        codes[n * (K * BITS / 32) + gi * WPG + lane] = mine;
+}
+
+// Dequantize for widths whose codes straddle words: one thread per 32 codes, which are BITS
+// whole words of one group (groups are multiples of 32 codes).
+template <typename TP, typename TO, int BITS>
+__global__ void __launch_bounds__(256) affine_dequantize_odd_kernel(const uint32_t* __restrict__ codes,
+                                                                    const TP* __restrict__ scales,
+                                                                    const TP* __restrict__ biases, int64_t N,
+                                                                    int64_t K, int g, TO* __restrict__ out)
+{
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    const int64_t chunks_per_row = K / 32;
+    const int64_t total = N * chunks_per_row;
+    const int64_t groups_per_row = K / g;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = idx / chunks_per_row;
+        const int64_t k0 = (idx % chunks_per_row) * 32;
+        const float s = to_float(scales[n * groups_per_row + k0 / g]);
+        const float b = to_float(biases[n * groups_per_row + k0 / g]);
+        uint32_t wd[BITS];
+#pragma unroll
+        for (int i = 0; i < BITS; ++i)
+            wd[i] = __ldg(codes + idx * BITS + i);  // the row's words k0*BITS/32 ..; rows are whole chunks
+        __align__(16) TO vals[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int bp = i * BITS, wi = bp / 32, sh = bp % 32;
+            uint32_t q = wd[wi] >> sh;
+            if (sh + BITS > 32)
+                q |= wd[wi + 1] << (32 - sh);
+            vals[i] = from_float<TO>(__fmaf_rn(static_cast<float>(q & MASK), s, b));
+        }
+        // 64 or 128 bytes at out + n*K + k0, a multiple of 64 bytes from the 16-byte aligned base
+        uint4* dst = reinterpret_cast<uint4*>(out + n * K + k0);
+#pragma unroll
+        for (int c = 0; c < 32 * (int)sizeof(TO) / 16; ++c)
+            dst[c] = reinterpret_cast<const uint4*>(vals)[c];
     }
 }
 
@@ -468,10 +580,27 @@ cudaError_t quantize_dispatch_g(const TW* w, int64_t N, int64_t K, int g, uint32
 {
     const int64_t groups = N * (K / g);
     const unsigned blocks = (unsigned)((groups + 7) / 8);
+    // power-of-two widths never straddle a word: lanes share whole words
+    constexpr bool pow2 = (BITS & (BITS - 1)) == 0;
     switch (g) {
-    case 32: affine_quantize_kernel<TW, TP, BITS, 32><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b); break;
-    case 64: affine_quantize_kernel<TW, TP, BITS, 64><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b); break;
-    default: affine_quantize_kernel<TW, TP, BITS, 128><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b); break;
+    case 32:
+        if constexpr (pow2)
+            affine_quantize_kernel<TW, TP, BITS, 32><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b);
+        else
+            affine_quantize_odd_kernel<TW, TP, BITS, 32><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b);
+        break;
+    case 64:
+        if constexpr (pow2)
+            affine_quantize_kernel<TW, TP, BITS, 64><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b);
+        else
+            affine_quantize_odd_kernel<TW, TP, BITS, 64><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b);
+        break;
+    default:
+        if constexpr (pow2)
+            affine_quantize_kernel<TW, TP, BITS, 128><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b);
+        else
+            affine_quantize_odd_kernel<TW, TP, BITS, 128><<<blocks, 256, 0, st>>>(w, N, K, codes, s, b);
+        break;
     }
     return cudaGetLastError();
 }
@@ -484,9 +613,24 @@ cudaError_t quantize_dispatch_b(const void* w, int64_t N, int64_t K, int bits, i
     TP* sp = static_cast<TP*>(s);
     TP* bp = static_cast<TP*>(b);
     switch (bits) {
+    case 1: return quantize_dispatch_g<TW, TP, 1>(wp, N, K, g, codes, sp, bp, st);
     case 2: return quantize_dispatch_g<TW, TP, 2>(wp, N, K, g, codes, sp, bp, st);
+    case 3: return quantize_dispatch_g<TW, TP, 3>(wp, N, K, g, codes, sp, bp, st);
     case 4: return quantize_dispatch_g<TW, TP, 4>(wp, N, K, g, codes, sp, bp, st);
+    case 5: return quantize_dispatch_g<TW, TP, 5>(wp, N, K, g, codes, sp, bp, st);
+    case 6: return quantize_dispatch_g<TW, TP, 6>(wp, N, K, g, codes, sp, bp, st);
     default: return quantize_dispatch_g<TW, TP, 8>(wp, N, K, g, codes, sp, bp, st);
+    }
+}
+
+template <typename TW>
+cudaError_t quantize_dispatch_p(const void* w, int64_t N, int64_t K, int bits, int g, uint32_t* codes, void* s,
+                                void* b, qlin_dtype p_dt, cudaStream_t st)
+{
+    switch (p_dt) {
+    case QLIN_F32: return quantize_dispatch_b<TW, float>(w, N, K, bits, g, codes, s, b, st);
+    case QLIN_BF16: return quantize_dispatch_b<TW, __nv_bfloat16>(w, N, K, bits, g, codes, s, b, st);
+    default: return quantize_dispatch_b<TW, __half>(w, N, K, bits, g, codes, s, b, st);
     }
 }
 
@@ -494,18 +638,34 @@ template <typename TP, typename TO>
 cudaError_t dequantize_dispatch(const uint32_t* codes, const void* s, const void* b, int64_t N, int64_t K, int bits,
                                 int g, void* out, cudaStream_t st, const DeviceInfo& dev)
 {
+    const int64_t cap = (int64_t)dev.sm_count * 16;
     const int64_t words = N * K * bits / 32;
-    const int64_t want = (words + 255) / 256;
-    const unsigned blocks = (unsigned)(want < (int64_t)dev.sm_count * 16 ? want : (int64_t)dev.sm_count * 16);
+    const int64_t want = (bits & (bits - 1)) == 0 ? (words + 255) / 256 : (N * (K / 32) + 255) / 256;
+    const unsigned blocks = (unsigned)(want < cap ? want : cap);
     const TP* sp = static_cast<const TP*>(s);
     const TP* bp = static_cast<const TP*>(b);
     TO* op = static_cast<TO*>(out);
     switch (bits) {
+    case 1: affine_dequantize_odd_kernel<TP, TO, 1><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
     case 2: affine_dequantize_kernel<TP, TO, 2><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    case 3: affine_dequantize_odd_kernel<TP, TO, 3><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
     case 4: affine_dequantize_kernel<TP, TO, 4><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    case 5: affine_dequantize_odd_kernel<TP, TO, 5><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    case 6: affine_dequantize_odd_kernel<TP, TO, 6><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
     default: affine_dequantize_kernel<TP, TO, 8><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
     }
     return cudaGetLastError();
+}
+
+template <typename TP>
+cudaError_t dequantize_dispatch_o(const uint32_t* codes, const void* s, const void* b, int64_t N, int64_t K,
+                                  int bits, int g, void* out, qlin_dtype o_dt, cudaStream_t st, const DeviceInfo& dev)
+{
+    switch (o_dt) {
+    case QLIN_F32: return dequantize_dispatch<TP, float>(codes, s, b, N, K, bits, g, out, st, dev);
+    case QLIN_BF16: return dequantize_dispatch<TP, __nv_bfloat16>(codes, s, b, N, K, bits, g, out, st, dev);
+    default: return dequantize_dispatch<TP, __half>(codes, s, b, N, K, bits, g, out, st, dev);
+    }
 }
 
 }  // namespace
@@ -514,26 +674,23 @@ cudaError_t launch_affine_quantize(const void* w, qlin_dtype w_dt, int64_t N, in
                                    uint32_t* codes, void* scales, void* biases, qlin_dtype p_dt, cudaStream_t st,
                                    const DeviceInfo&)
 {
-    if (w_dt == QLIN_F32)
-        return p_dt == QLIN_F32 ? quantize_dispatch_b<float, float>(w, N, K, bits, g, codes, scales, biases, st)
-                                : quantize_dispatch_b<float, __nv_bfloat16>(w, N, K, bits, g, codes, scales, biases, st);
-    return p_dt == QLIN_F32
-               ? quantize_dispatch_b<__nv_bfloat16, float>(w, N, K, bits, g, codes, scales, biases, st)
-               : quantize_dispatch_b<__nv_bfloat16, __nv_bfloat16>(w, N, K, bits, g, codes, scales, biases, st);
+    switch (w_dt) {
+    case QLIN_F32: return quantize_dispatch_p<float>(w, N, K, bits, g, codes, scales, biases, p_dt, st);
+    case QLIN_BF16: return quantize_dispatch_p<__nv_bfloat16>(w, N, K, bits, g, codes, scales, biases, p_dt, st);
+    default: return quantize_dispatch_p<__half>(w, N, K, bits, g, codes, scales, biases, p_dt, st);
+    }
 }
 
 cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, const void* biases, qlin_dtype p_dt,
                                      int64_t N, int64_t K, int bits, int g, void* out, qlin_dtype o_dt,
                                      cudaStream_t st, const DeviceInfo& dev)
 {
-    if (p_dt == QLIN_F32)
-        return o_dt == QLIN_F32
-                   ? dequantize_dispatch<float, float>(codes, scales, biases, N, K, bits, g, out, st, dev)
-                   : dequantize_dispatch<float, __nv_bfloat16>(codes, scales, biases, N, K, bits, g, out, st, dev);
-    return o_dt == QLIN_F32
-               ? dequantize_dispatch<__nv_bfloat16, float>(codes, scales, biases, N, K, bits, g, out, st, dev)
-               : dequantize_dispatch<__nv_bfloat16, __nv_bfloat16>(codes, scales, biases, N, K, bits, g, out, st,
-                                                                   dev);
+    switch (p_dt) {
+    case QLIN_F32: return dequantize_dispatch_o<float>(codes, scales, biases, N, K, bits, g, out, o_dt, st, dev);
+    case QLIN_BF16:
+        return dequantize_dispatch_o<__nv_bfloat16>(codes, scales, biases, N, K, bits, g, out, o_dt, st, dev);
+    default: return dequantize_dispatch_o<__half>(codes, scales, biases, N, K, bits, g, out, o_dt, st, dev);
+    }
 }
 
 cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
@@ -557,6 +714,9 @@ cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R,
     else if (w_dt == QLIN_BF16)
         quantize_int8_rows_kernel<__nv_bfloat16>
             <<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q, scale, rowsum, rel);
+    else if (w_dt == QLIN_F16)
+        quantize_int8_rows_kernel<__half>
+            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __half*>(w), C, q, scale, rowsum, rel);
     else
         quantize_int8_rows_kernel<float><<<(unsigned)R, 256, 0, st>>>(static_cast<const float*>(w), C, q, scale,
                                                                       rowsum, rel);
@@ -570,22 +730,20 @@ cudaError_t launch_quantize_weight_int8_clip(const void* w, qlin_dtype w_dt, int
     while (p2 < C)
         p2 <<= 1;
     const size_t smem = (size_t)p2 * 4;
-    if (w_dt == QLIN_BF16) {
-        cudaError_t e = cudaFuncSetAttribute(quantize_weight_int8_clip_kernel<__nv_bfloat16>,
+    auto run = [&](auto* typed) {
+        using TW = std::remove_const_t<std::remove_pointer_t<decltype(typed)>>;
+        cudaError_t e = cudaFuncSetAttribute(quantize_weight_int8_clip_kernel<TW>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
-        quantize_weight_int8_clip_kernel<__nv_bfloat16><<<(unsigned)R, 256, smem, st>>>(
-            static_cast<const __nv_bfloat16*>(w), C, p2, pct, q, scale);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(quantize_weight_int8_clip_kernel<float>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-        quantize_weight_int8_clip_kernel<float><<<(unsigned)R, 256, smem, st>>>(static_cast<const float*>(w), C, p2,
-                                                                              pct, q, scale);
+        quantize_weight_int8_clip_kernel<TW><<<(unsigned)R, 256, smem, st>>>(typed, C, p2, pct, q, scale);
+        return cudaGetLastError();
+    };
+    switch (w_dt) {
+    case QLIN_F32: return run(static_cast<const float*>(w));
+    case QLIN_BF16: return run(static_cast<const __nv_bfloat16*>(w));
+    default: return run(static_cast<const __half*>(w));
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int g, int8_t* q,
@@ -596,6 +754,8 @@ cudaError_t launch_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t 
     quantize_int8_groups_kernel<TW, G><<<blocks, 256, 0, st>>>(static_cast<const TW*>(w), N, K, q, scale_w)
     if (w_dt == QLIN_BF16) {
         if (g == 64) QLIN_QG(__nv_bfloat16, 64); else if (g == 128) QLIN_QG(__nv_bfloat16, 128); else QLIN_QG(__nv_bfloat16, 256);
+    } else if (w_dt == QLIN_F16) {
+        if (g == 64) QLIN_QG(__half, 64); else if (g == 128) QLIN_QG(__half, 128); else QLIN_QG(__half, 256);
     } else {
         if (g == 64) QLIN_QG(float, 64); else if (g == 128) QLIN_QG(float, 128); else QLIN_QG(float, 256);
     }
@@ -610,6 +770,8 @@ cudaError_t launch_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int
     if (w_dt == QLIN_BF16)
         pack_int4_cols_kernel<__nv_bfloat16>
             <<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), K, N, packed, scale);
+    else if (w_dt == QLIN_F16)
+        pack_int4_cols_kernel<__half><<<blocks, 256, 0, st>>>(static_cast<const __half*>(w), K, N, packed, scale);
     else
         pack_int4_cols_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(w), K, N, packed, scale);
     return cudaGetLastError();

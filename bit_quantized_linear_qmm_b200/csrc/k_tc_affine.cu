@@ -105,8 +105,8 @@ struct TsParams {
     const float* tok_scale;           // [M] 2^E_m
     const float* row_scale;           // [N] 2^F_n
     const void* bias;                 // [N] or null, the output dtype
-    void* out;                        // [M][N] bf16, or fp32 when out_f32
-    int out_f32;
+    void* out;                        // [M][N] of out_dt (fp32, bf16 or fp16)
+    int out_dt;                       // a qlin_dtype; also the dtype of bias
     int M, N, K;
     int g_shift, ng;                  // log2 g, K / g
     int tiles_t, tiles_w;
@@ -518,9 +518,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             // output row of TMEM lane 32 q + lane: ternary -> packed row 32 wt + lane, field q
             const int n = F::kTernary ? wt * 32 + lane + q * p.R : wt * kTW + 32 * q + lane;
             const bool n_ok = F::kTernary ? wt * 32 + lane < p.R : n < p.N;
-            const float bn = (p.bias && n_ok) ? (p.out_f32 ? static_cast<const float*>(p.bias)[n]
-                                                           : __bfloat162float(static_cast<const __nv_bfloat16*>(p.bias)[n]))
-                                              : 0.f;
+            float bn = 0.f;
+            if (p.bias && n_ok)
+                bn = p.out_dt == QLIN_F32    ? static_cast<const float*>(p.bias)[n]
+                     : p.out_dt == QLIN_BF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.bias)[n])
+                                             : __half2float(static_cast<const __half*>(p.bias)[n]);
             float rs = 0.f;
             if (n_ok) {
                 if constexpr (F::kTernary) {
@@ -561,10 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                     if (m < p.M) {  // 2^E_m 2^F_n is an exact power of two: one rounding in the fma
                         const float out = fmaf(__uint_as_float(v[j]), ts[j], bn);
                         const size_t oi = o0 + (size_t)(c * 16 + j) * p.N;
-                        if (p.out_f32)
+                        if (p.out_dt == QLIN_F32)
                             static_cast<float*>(p.out)[oi] = out;
-                        else
+                        else if (p.out_dt == QLIN_BF16)
                             static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(out);
+                        else
+                            static_cast<__half*>(p.out)[oi] = __float2half_rn(out);
                     }
                 }
             }
@@ -618,6 +622,17 @@ QLIN_DEV void load8(const __nv_bfloat16* p, float (&v)[8])
     for (int i = 0; i < 4; ++i) {
         v[2 * i] = __uint_as_float(w[i] << 16);
         v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+QLIN_DEV void load8(const __half* p, float (&v)[8])
+{
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
     }
 }
 QLIN_DEV void load8(const float* p, float (&v)[8])
@@ -779,7 +794,7 @@ cudaError_t launch_tc_bitlinear(const BitlinearArgs& a, cudaStream_t st, const D
     prm.row_scale = nullptr;
     prm.bias = a.bias;
     prm.out = a.y;
-    prm.out_f32 = 0;
+    prm.out_dt = QLIN_BF16;
     prm.M = (int)a.M;
     prm.N = (int)a.N;
     prm.K = (int)a.K;
@@ -815,21 +830,25 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
         const unsigned blocks = (unsigned)(a.M + (a.N + 7) / 8);
         const float qmax = (float)((1 << a.bits) - 1);
         const __nv_bfloat16* bb = static_cast<const __nv_bfloat16*>(a.biases);
-        // (x dtype, activation handling, parameter format)
-        const int form = (a.x_f32 ? 1 : 0) | (a.pergroup && a.M > 1 ? 2 : 0) | (a.pergroup ? 4 : 0);
-        switch (form) {
+        // (activation handling, parameter format) x (x dtype)
+        const int form = (a.pergroup && a.M > 1 ? 2 : 0) | (a.pergroup ? 1 : 0);
 #define QLIN_PREP(XT, QX, PG)                                                                                   \
     affine_prefill_prep_kernel<XT, 2, QX, PG><<<blocks, 256, 0, st>>>(static_cast<const XT*>(a.a), (int)a.M,    \
                                                                       (int)a.K, a.scales, bb, (int)a.N, ng, qmax, \
                                                                       x16, s16, b16, tok_scale, row_scale)
-        case 0: QLIN_PREP(__nv_bfloat16, 0, 0); break;
-        case 1: QLIN_PREP(float, 0, 0); break;
-        case 4: QLIN_PREP(__nv_bfloat16, 0, 1); break;
-        case 5: QLIN_PREP(float, 0, 1); break;
-        case 6: QLIN_PREP(__nv_bfloat16, 1, 1); break;
-        default: QLIN_PREP(float, 1, 1); break;
-#undef QLIN_PREP
+#define QLIN_PREP_X(QX, PG)                                                                                     \
+    switch (a.x_dt) {                                                                                           \
+    case QLIN_F32: QLIN_PREP(float, QX, PG); break;                                                             \
+    case QLIN_BF16: QLIN_PREP(__nv_bfloat16, QX, PG); break;                                                    \
+    default: QLIN_PREP(__half, QX, PG); break;                                                                  \
+    }
+        switch (form) {
+        case 0: QLIN_PREP_X(0, 0); break;
+        case 1: QLIN_PREP_X(0, 1); break;
+        default: QLIN_PREP_X(1, 1); break;
         }
+#undef QLIN_PREP_X
+#undef QLIN_PREP
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
@@ -842,7 +861,7 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     prm.row_scale = row_scale;
     prm.bias = a.bias;
     prm.out = a.out;
-    prm.out_f32 = a.x_f32;
+    prm.out_dt = a.x_dt;
     prm.M = (int)a.M;
     prm.N = (int)a.N;
     prm.K = (int)a.K;

@@ -92,7 +92,8 @@ struct TcParams {
     void* out;
     const float* s_x;
     const float* s_w;
-    const __nv_bfloat16* bias;
+    const unsigned short* bias;     // [N] bf16, or fp16 when out_f16
+    int out_f16;                    // y and bias are fp16 (else bf16)
     int vec_sw, vec_bias, vec_out;  // 16-byte alignment of s_w, bias and out
     unsigned* status;
 };
@@ -101,12 +102,6 @@ QLIN_DEV void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t
 {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
-}
-
-QLIN_DEV uint32_t pack_bf16x2(float lo, float hi)
-{
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // Grouped tile order: kGroupM consecutive M-tiles walk the N-tiles together.
@@ -285,14 +280,14 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                                 for (int j = 0; j < 4; ++j) {
-                                    bb[8 * h + 2 * j] = __uint_as_float(w4[j] << 16);
-                                    bb[8 * h + 2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
+                                    bb[8 * h + 2 * j] = h16_to_float(w4[j], p.out_f16);
+                                    bb[8 * h + 2 * j + 1] = h16_to_float(w4[j] >> 16, p.out_f16);
                                 }
                             }
                         } else {
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
-                                bb[j] = p.bias ? __bfloat162float(p.bias[min(n + j, p.N - 1)]) : 0.f;
+                                bb[j] = p.bias ? h16_to_float(p.bias[min(n + j, p.N - 1)], p.out_f16) : 0.f;
                         }
                     }
                 }
@@ -323,18 +318,20 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                             a = __uint_as_float(r[j]);
                         v[j] = a + bb[j];
                     }
-                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + n;
+                    unsigned short* o = static_cast<unsigned short*>(p.out) + (size_t)row * p.N + n;
+                    const int f16 = p.out_f16;
                     if (full16) {
-                        *reinterpret_cast<uint4*>(o) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                                                  pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                        *reinterpret_cast<uint4*>(o) =
+                            make_uint4(pack_h16x2(v[0], v[1], f16), pack_h16x2(v[2], v[3], f16),
+                                       pack_h16x2(v[4], v[5], f16), pack_h16x2(v[6], v[7], f16));
                         *reinterpret_cast<uint4*>(o + 8) =
-                            make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                                       pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+                            make_uint4(pack_h16x2(v[8], v[9], f16), pack_h16x2(v[10], v[11], f16),
+                                       pack_h16x2(v[12], v[13], f16), pack_h16x2(v[14], v[15], f16));
                     } else {
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             if (n + j < p.N)
-                                o[j] = __float2bfloat16_rn(v[j]);
+                                o[j] = to_h16(v[j], f16);
                     }
                 }
             }
@@ -488,7 +485,8 @@ cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const 
     prm.out = a.out;
     prm.s_x = a.s_x;
     prm.s_w = a.s_w;
-    prm.bias = static_cast<const __nv_bfloat16*>(a.bias);
+    prm.bias = static_cast<const unsigned short*>(a.bias);
+    prm.out_f16 = a.x_dt == QLIN_F16;
     prm.vec_sw = aligned16p(a.s_w);
     prm.vec_bias = aligned16p(a.bias);
     prm.vec_out = aligned16p(a.out);

@@ -64,9 +64,9 @@ qlin_status current_device(DeviceInfo& out)
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool dtype_ok(qlin_dtype d) { return d == QLIN_F32 || d == QLIN_BF16; }
+bool dtype_ok(qlin_dtype d) { return d == QLIN_F32 || d == QLIN_BF16 || d == QLIN_F16; }
 size_t dtype_size(qlin_dtype d) { return d == QLIN_F32 ? 4 : 2; }
-bool bits_ok(int b) { return b == 2 || b == 4 || b == 8; }
+bool bits_ok(int b) { return (b >= 1 && b <= 6) || b == 8; }
 bool group_ok(int g) { return g == 32 || g == 64 || g == 128; }
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -188,14 +188,19 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
     qlin_status s = check_affine(N, K, bits, group_size, param_dt);
     if (s != QLIN_OK)
         return s;
-    if (bits == 2 && group_size == 32)
-        return QLIN_ERR_UNSUPPORTED;
-    if (!aligned16(codes) || !aligned16(x) || (K * bits / 8) % 16 != 0 || (K * (int64_t)dtype_size(x_dt)) % 16 != 0)
+    // the specialized paths: power-of-two widths (not 2 bits in groups of 32), fp32 / bf16 operands,
+    // TMA-loaded rows (16-byte pitch); the tensor-core prefill also takes fp16 x.  Everything else
+    // runs the general decode kernel, which needs 4-byte aligned codes and 16-byte x rows.
+    const bool tma_rows = aligned16(codes) && (K * bits / 8) % 16 == 0;
+    const bool prefill = M > 16 && bits == 4 && param_dt == QLIN_BF16 && tma_rows;
+    const bool special = (bits == 2 || bits == 4 || bits == 8) && !(bits == 2 && group_size == 32) &&
+                         x_dt != QLIN_F16 && param_dt != QLIN_F16 && tma_rows;
+    if (!aligned16(x) || (K * (int64_t)dtype_size(x_dt)) % 16 != 0 || (reinterpret_cast<uintptr_t>(codes) & 3u) != 0)
         return QLIN_ERR_MISALIGNED;
     DeviceInfo dev;
     if ((s = current_device(dev)) != QLIN_OK)
         return s;
-    if (M > 16 && bits == 4 && param_dt == QLIN_BF16) {
+    if (prefill) {
         const size_t need = qlin_workspace_size(QLIN_OP_MATMUL, M, N, K, bits, group_size);
         if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
             return QLIN_ERR_WORKSPACE;
@@ -211,7 +216,7 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
         t.biases = biases;
         t.g = group_size;
         t.bits = bits;
-        t.x_f32 = x_dt == QLIN_F32 ? 1 : 0;
+        t.x_dt = x_dt;
         t.workspace = workspace;
         return from_cuda(launch_tc_affine(t, static_cast<cudaStream_t>(stream), dev));
     }
@@ -229,7 +234,8 @@ qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, co
     a.g = group_size;
     a.bias = bias;
     a.y = y;
-    return from_cuda(launch_affine_gemv(a, static_cast<cudaStream_t>(stream), dev));
+    return from_cuda(special ? launch_affine_gemv(a, static_cast<cudaStream_t>(stream), dev)
+                             : launch_affine_gemv_any(a, static_cast<cudaStream_t>(stream), dev));
 }
 
 qlin_status bitlinear_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K, const uint8_t* packed, int64_t N,
@@ -366,7 +372,7 @@ qlin_status pergroup_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K
     t.biases = nullptr;
     t.g = group_size;
     t.bits = 8;
-    t.x_f32 = x_dt == QLIN_F32 ? 1 : 0;
+    t.x_dt = x_dt;
     t.pergroup = 1;
     t.workspace = workspace;
     return from_cuda(launch_tc_affine(t, static_cast<cudaStream_t>(stream), dev));
@@ -408,7 +414,7 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
         return QLIN_ERR_INVALID_ARG;
     if (op == TC_W4A8 ? (K % 32 != 0 || N % 16 != 0) : (K % 16 != 0))
         return QLIN_ERR_INVALID_ARG;
-    if (x_dt != QLIN_BF16)
+    if (x_dt != QLIN_BF16 && x_dt != QLIN_F16)  // y and bias take x's 16-bit dtype
         return QLIN_ERR_UNSUPPORTED;
     if (!aligned16(x) || !aligned16(w) || !aligned16(y))
         return QLIN_ERR_MISALIGNED;
@@ -437,6 +443,7 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
         g.M = M;
         g.K = K;
         g.N = N;
+        g.out_f16 = x_dt == QLIN_F16;
         return from_cuda(op == TC_W8A8 ? launch_w8_gemv(g, st, dev) : launch_w4_gemv(g, st, dev));
     }
     TcGemmArgs t = {};
@@ -449,6 +456,7 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
     t.s_x = sx;
     t.s_w = scale_w;
     t.bias = bias;
+    t.x_dt = x_dt;
     return from_cuda(launch_tc_gemm(op, t, st, dev));
 }
 

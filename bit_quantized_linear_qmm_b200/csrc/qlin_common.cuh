@@ -37,10 +37,31 @@ QLIN_DEV uint32_t smem_u32(const void* p)
 template <typename T> QLIN_DEV float to_float(T v);
 template <> QLIN_DEV float to_float<float>(float v) { return v; }
 template <> QLIN_DEV float to_float<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <> QLIN_DEV float to_float<__half>(__half v) { return __half2float(v); }
 
 template <typename T> QLIN_DEV T from_float(float v);
 template <> QLIN_DEV float from_float<float>(float v) { return v; }
 template <> QLIN_DEV __nv_bfloat16 from_float<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <> QLIN_DEV __half from_float<__half>(float v) { return __float2half_rn(v); }
+
+// 16-bit output / bias values of the int8 layers: bf16, or fp16 when f16 is set (the dtype of x)
+QLIN_DEV float h16_to_float(uint32_t u, int f16)
+{
+    return f16 ? __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu))) : __uint_as_float(u << 16);
+}
+QLIN_DEV uint32_t pack_h16x2(float lo, float hi, int f16)
+{
+    if (f16) {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+QLIN_DEV unsigned short to_h16(float v, int f16)
+{
+    return f16 ? __half_as_ushort(__float2half_rn(v)) : __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
 
 // ---------------------------------------------------------------- mbarrier
 
@@ -318,6 +339,8 @@ struct AffineGemvArgs {
     void* y;
 };
 cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
+// any width 1..6, 8 and any dtypes (k_affine_any.cu); 4-byte aligned codes, 16-byte aligned x rows
+cudaError_t launch_affine_gemv_any(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
 
 // int8 decode GEMV (M <= 16): y = (float)(qx . w) * s_x[m] * s_w[n] + bias[n], bf16 out
 struct W8GemvArgs {
@@ -325,9 +348,10 @@ struct W8GemvArgs {
     const float* s_x;  // [M]
     const int8_t* w;   // [N][K] int8 (W8), or packed [K/2][N] bytes (W4)
     const float* s_w;  // [N]
-    const void* bias;  // bf16 [N] or NULL
-    void* y;           // bf16 [M][N]
+    const void* bias;  // [N] or NULL, bf16 (fp16 when out_f16)
+    void* y;           // [M][N], bf16 (fp16 when out_f16)
     int64_t M, K, N;
+    int out_f16;
 };
 cudaError_t launch_w8_gemv(const W8GemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
 // int4 decode GEMV (M <= 16): the same arguments, w = packed [K/2][N] bytes
@@ -366,7 +390,7 @@ struct TcGemmArgs {
     const void* biases;
     int g;
     int bits;                 // affine code width (8 with pergroup)
-    int x_f32;                // affine: x is fp32 (else bf16)
+    int x_dt;                 // affine / per-group: dtype of x, bias and y (a qlin_dtype)
     int pergroup;             // per-group int8 weights [N][K], fp32 scales [K/g][N] (group-major), no biases
     void* workspace;          // affine prefill: tc_affine_workspace() bytes, 256-byte aligned
 };

@@ -29,6 +29,7 @@ QLIN_ERR_WORKSPACE = 7
 
 QLIN_F32 = 0
 QLIN_BF16 = 1
+QLIN_F16 = 2
 
 QLIN_OP_MATMUL = 0
 QLIN_OP_BITLINEAR = 1
@@ -111,11 +112,13 @@ def _dt(t: torch.Tensor) -> int:
         return QLIN_F32
     if t.dtype == torch.bfloat16:
         return QLIN_BF16
+    if t.dtype == torch.float16:
+        return QLIN_F16
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
 def _torch_dt(code: int):
-    return torch.float32 if code == QLIN_F32 else torch.bfloat16
+    return {QLIN_F32: torch.float32, QLIN_BF16: torch.bfloat16, QLIN_F16: torch.float16}[code]
 
 
 def _cuda(*ts):

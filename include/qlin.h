@@ -81,7 +81,8 @@ typedef enum {
 
 typedef enum {
     QLIN_F32 = 0,
-    QLIN_BF16 = 1
+    QLIN_BF16 = 1,
+    QLIN_F16 = 2               /* IEEE binary16 */
 } qlin_dtype;
 
 typedef enum {
@@ -112,9 +113,14 @@ size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits
  *   both rounded to param_dt; a stored scale of 0 becomes 1;
  *   q = clip(round_half_even((w - bias) / scale), 0, 2^bits - 1) from the
  *   STORED scale and bias, fp32 subtract and IEEE divide.
- * w: [N, K] of w_dt.  codes: uint32 [N, K*bits/32].  scales, biases:
- * [N, K/group_size] of param_dt.  bits in {2, 4, 8}; group_size in
- * {32, 64, 128}; K % group_size == 0.  Bit-exact with the CPU reference.
+ * w: [N, K] of w_dt.  codes: uint32 [N, K*bits/32]; a row is one
+ * LSB-first bitstream, code k at bits k*bits .. k*bits+bits-1 of the row
+ * read as a little-endian sequence of 32-bit words, so for 3, 5 and 6 bits a
+ * code may continue in the next word (a group of group_size codes is always
+ * whole words).  scales, biases: [N, K/group_size] of param_dt.  bits in
+ * {1, 2, 3, 4, 5, 6, 8}; group_size in {32, 64, 128}; K % group_size == 0;
+ * every dtype (fp32, bf16, fp16) for w and the parameters.  Bit-exact with
+ * the CPU reference.
  */
 qlin_status qlin_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int bits,
                           int group_size, uint32_t* codes, void* scales, void* biases,
@@ -123,8 +129,9 @@ qlin_status qlin_quantize(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, 
 /*
  * Dequantised weight [nuvec-nn QuantizedLinear, dequantized_weight; cider
  * pergroup_linear docstring, dequantize formula]: w_out[n, k] =
- * fma(q, scale, bias) in fp32, rounded once to out_dt.  w_out: [N, K].
- * Bit-exact with the CPU reference.
+ * fma(q, scale, bias) in fp32, rounded once to out_dt.  w_out: [N, K],
+ * 16-byte aligned; codes 4-byte aligned.  Widths and dtypes as
+ * qlin_quantize.  Bit-exact with the CPU reference.
  */
 qlin_status qlin_dequantize(const uint32_t* codes, const void* scales, const void* biases,
                             qlin_dtype param_dt, int64_t N, int64_t K, int bits, int group_size,
@@ -144,10 +151,18 @@ qlin_status qlin_dequantize(const uint32_t* codes, const void* scales, const voi
  * registers, writes them to tensor memory as the A operand of tcgen05 MMA
  * and accumulates in fp32 in tensor memory -- every product within 2^-11 of
  * the exact one.  Other M > 16 calls run the decode kernel on 16-token
- * slices.  Requires (K*bits/8) % 16 == 0 and, for x, (K*sizeof(x_dt)) % 16
- * == 0.  workspace: at least qlin_workspace_size(QLIN_OP_MATMUL, M, N, K,
- * bits, group_size) bytes, 256-byte aligned (QLIN_ERR_WORKSPACE otherwise);
- * NULL is accepted when that size is 0 (M <= 16, or bits != 4).
+ * slices.  The decode kernel and the prefill GEMM take 2-, 4- and 8-bit
+ * codes whose rows are 16-byte aligned ((K*bits/8) % 16 == 0, codes 16-byte
+ * aligned), fp32 or bf16 x and parameters (the prefill also fp16 x), and not
+ * 2 bits in groups of 32.  Every other call -- widths 1, 3, 5, 6, fp16
+ * activations or parameters at M <= 16, rows whose group parameters do not
+ * fit the decode kernel's shared memory (long K in small groups) -- runs a
+ * general decode kernel (eight codes per lane, fp32 dequantisation exactly
+ * as qlin_dequantize, fp32 accumulation; slower).  x: 16-byte aligned;
+ * codes: 4-byte aligned (QLIN_ERR_MISALIGNED otherwise).  workspace: at
+ * least qlin_workspace_size(QLIN_OP_MATMUL, M, N, K, bits, group_size)
+ * bytes, 256-byte aligned (QLIN_ERR_WORKSPACE otherwise) when the call runs
+ * the prefill; NULL is accepted when that size is 0 (M <= 16, or bits != 4).
  */
 qlin_status qlin_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
                         const uint32_t* codes, const void* scales, const void* biases,
@@ -174,7 +189,8 @@ qlin_status bitlinear_matmul(const void* x, qlin_dtype x_dt, int64_t M, int64_t 
  * scale[r] = max_c |w[r, c]| / 127 (zero -> 1), q = clip(round_half_even(w /
  * scale), -128, 127).  Used for weights (rows = output features) and, with
  * the same rule, for activations (rows = tokens; the pages' quant_a).
- * w: [R, C] of w_dt; q: int8 [R, C]; scale: fp32 [R].  Bit-exact.
+ * w: [R, C] of w_dt (fp32, bf16 or fp16); q: int8 [R, C]; scale: fp32 [R].
+ * Bit-exact.
  */
 qlin_status qlin_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C,
                                     int8_t* q, float* scale, void* stream);
@@ -201,7 +217,8 @@ qlin_status qlin_int8_matmul_int32(const int8_t* a, const int8_t* b, int64_t M, 
  * W8A8 linear [cider/ops.py perchannel_linear]: y = dequant(quant_a(x) @
  * w^T) + bias, quant_a = per-token qlin_quantize_int8_rows of x (kept in the
  * workspace), int32 accumulation, then y = acc * s_x[m] * scale_w[n] + bias
- * in fp32 and one rounding to x_dt.  x: [M, K] of x_dt; w: int8 [N, K];
+ * in fp32 and one rounding to x_dt.  x: [M, K] of x_dt, bf16 or fp16
+ * (QLIN_ERR_UNSUPPORTED for fp32); w: int8 [N, K];
  * scale_w: fp32 [N]; bias: [N] of x_dt or NULL; y: [M, N] of x_dt.
  * K % 16 == 0.  workspace >= qlin_workspace_size(QLIN_OP_W8A8, M, N, K, 0, 0).
  * M <= 16 runs a weight-streaming GEMV (int8 mma.sync), larger M the tcgen05

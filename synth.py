@@ -34,6 +34,14 @@ def to_bf16(a: np.ndarray):
     return vals, bits
 
 
+def to_f16(a: np.ndarray):
+    """Round fp32 -> IEEE binary16 (round to nearest even, numpy's conversion).
+
+    Returns (values as fp32, raw fp16 bits as uint16)."""
+    h = np.ascontiguousarray(a, dtype=np.float32).astype(np.float16)
+    return h.astype(np.float32), h.view(np.uint16).copy()
+
+
 def outlier_weights(seed: int, N: int, K: int, sigma: float = 0.02,
                     frac: float = 0.001, factor: float = 20.0) -> np.ndarray:
     """N(0, sigma) weights with round(frac*N*K) positions, drawn uniformly
@@ -77,12 +85,14 @@ def ternary_codes(seed: int, N: int, K: int) -> np.ndarray:
 @dataclass
 class Activations:
     vals: np.ndarray            # fp32 values (exactly representable in `dtype`)
-    bits: np.ndarray | None     # uint16 bf16 bits when dtype == "bf16"
+    bits: np.ndarray | None     # uint16 bf16 / fp16 bits when dtype is "bf16" / "f16"
     dtype: str
 
     def torch(self, device="cpu"):
         if self.dtype == "bf16":
             t = torch.from_numpy(self.bits.view(np.int16)).view(torch.bfloat16)
+        elif self.dtype == "f16":
+            t = torch.from_numpy(self.bits.view(np.int16)).view(torch.float16)
         else:
             t = torch.from_numpy(self.vals)
         return t.to(device)
@@ -93,6 +103,9 @@ def activations(seed: int, shape, dtype: str, sigma: float = 1.0) -> Activations
     if dtype == "bf16":
         vals, bits = to_bf16(v)
         return Activations(vals, bits, "bf16")
+    if dtype == "f16":
+        vals, bits = to_f16(v)
+        return Activations(vals, bits, "f16")
     if dtype == "f32":
         return Activations(v, None, "f32")
     raise ValueError(dtype)
@@ -109,8 +122,8 @@ class AffineCase:
     N: int
     bits: int
     group_size: int
-    x_dtype: str        # "f32" | "bf16" (output and bias use the same dtype)
-    param_dtype: str    # "f32" | "bf16" (scales, biases)
+    x_dtype: str        # "f32" | "bf16" | "f16" (output and bias use the same dtype)
+    param_dtype: str    # "f32" | "bf16" | "f16" (scales, biases)
     bias: bool = True
     outliers: bool = False
     seed: int = 0

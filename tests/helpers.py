@@ -15,10 +15,13 @@ ABS = 1e-5
 
 
 def half_ulp(v: np.ndarray, dtype: torch.dtype) -> np.ndarray:
-    """Half a unit in the last place of |v| in `dtype` (bf16: 8 significant bits, fp32: 24)."""
-    bits = 8 if dtype == torch.bfloat16 else 24
+    """Half a unit in the last place of |v| in `dtype` (bf16: 8 significant bits, fp16: 11 with
+    subnormal spacing 2^-24, fp32: 24)."""
+    bits = {torch.bfloat16: 8, torch.float16: 11}.get(dtype, 24)
     a = np.abs(np.asarray(v, np.float64))
     _, e = np.frexp(a)  # a = f 2^e, f in [0.5, 1)
+    if dtype == torch.float16:
+        e = np.maximum(e, -13)  # below 2^-14 the spacing stays 2^-24
     return np.where(a > 0, np.ldexp(1.0, e - 1 - bits), 0.0)
 
 
@@ -49,6 +52,8 @@ def bf16_dev_from_f32_values(v: np.ndarray) -> torch.Tensor:
 def params_dev(vals: np.ndarray, dtype: str) -> torch.Tensor:
     if dtype == "bf16":
         return bf16_dev_from_f32_values(vals)
+    if dtype == "f16":  # fp32 values that are exactly fp16
+        return torch.from_numpy(np.ascontiguousarray(vals, np.float32).astype(np.float16)).cuda()
     return to_dev(vals.astype(np.float32))
 
 

@@ -49,12 +49,17 @@ def test_validation_before_device(ql):
     # null pointers
     assert L.qlin_quantize(None, 0, 4, 64, 4, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_INVALID_ARG
     # unsupported bits / group
-    assert L.qlin_quantize(P16, 0, 4, 64, 3, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize(P16, 0, 4, 64, 7, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize(P16, 0, 4, 64, 0, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize(P16, 3, 4, 64, 4, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_UNSUPPORTED  # no dtype 3
     assert L.qlin_quantize(P16, 0, 4, 64, 4, 48, P16, P16, P16, 0, None) == ql.QLIN_ERR_UNSUPPORTED
     # K not a multiple of the group
     assert L.qlin_dequantize(P16, P16, P16, 0, 4, 96, 4, 64, P16, 0, None) == ql.QLIN_ERR_INVALID_ARG
-    # misaligned codes pointer
-    assert L.qlin_matmul(P16, 1, 1, 128, C.c_void_p(260), P16, P16, 1, 64, 4, 64, None, P16, None, 0,
+    # codes not 4-byte aligned (a 4-byte aligned pointer that breaks the 16-byte rule takes the
+    # general kernel instead), x not 16-byte aligned
+    assert L.qlin_matmul(P16, 1, 1, 128, C.c_void_p(258), P16, P16, 1, 64, 4, 64, None, P16, None, 0,
+                         None) == ql.QLIN_ERR_MISALIGNED
+    assert L.qlin_matmul(C.c_void_p(264), 2, 1, 96, P16, P16, P16, 1, 64, 3, 32, None, P16, None, 0,
                          None) == ql.QLIN_ERR_MISALIGNED
     # BitLinear needs N % 4 == 0 and K % 16 == 0
     assert L.bitlinear_matmul(P16, 1, 1, 64, P16, 6, P16, 0, None, P16, None) == ql.QLIN_ERR_INVALID_ARG

@@ -86,7 +86,7 @@ def test_affine_rejects_bad_args(ql):
         ql.matmul(x, codes, s, s, 4, 64)  # K % g != 0
     assert e.value.status == ql.QLIN_ERR_INVALID_ARG
     with pytest.raises(ql.QlinError) as e:
-        ql.matmul(x, codes, s, s, 3, 32)
+        ql.matmul(x, codes, s, s, 7, 32)  # 7-bit codes
     assert e.value.status == ql.QLIN_ERR_UNSUPPORTED
     assert ql.device_status() == ql.QLIN_OK
 
