@@ -150,53 +150,54 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- timing
 
-def _graphs(step_fn, steps: int, per_graph: int):
-    """CUDA graphs holding `steps` steps: (graph of per_graph steps, count, remainder graph)."""
-    per_graph = max(1, min(per_graph, steps))
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for i in range(per_graph):
-            step_fn(i)
-    rem = steps % per_graph
-    g_rem = None
-    if rem:
-        g_rem = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_rem):
-            for i in range(rem):
-                step_fn(i)
-    return g, steps // per_graph, g_rem
-
-
-def time_steps(step_fn, steps: int, warmup: int, per_graph: int = 200, soak_s: float = 0.0, barrier=None):
-    """Milliseconds per step over exactly `steps` steps (graph replays between CUDA events)."""
+def time_windows(step_fn, steps: int, warmup: int, windows: int = 5, soak_s: float = 0.0, barrier=None) -> dict:
+    """Times exactly `steps` steps as `windows` back-to-back CUDA-graph replays (each a window of
+    steps // windows steps; the last also takes the remainder), with a CUDA event between windows on
+    the launching stream.  Returns ms per step over all the steps ("ms") and the median, min and
+    max of the windows' ms per step."""
+    windows = max(1, min(windows, steps))
+    per = steps // windows
+    sizes = [per] * windows
+    sizes[-1] += steps - per * windows
     for i in range(warmup):
         step_fn(i)
     torch.cuda.synchronize()
-    g, reps, g_rem = _graphs(step_fn, steps, per_graph)
-    g.replay()  # untimed: first replay uploads the graph
+    graphs = {}
+    for n in set(sizes):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                step_fn(i)
+        graphs[n] = g
+    for g in graphs.values():
+        g.replay()  # untimed: the first replay uploads the graph
     torch.cuda.synchronize()
     if soak_s > 0:
         t0 = time.time()
         while time.time() - t0 < soak_s:
-            g.replay()
+            graphs[sizes[0]].replay()
             torch.cuda.synchronize()
     if barrier:
         barrier()
     torch.cuda.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record()
-    for _ in range(reps):
-        g.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    ev1.record()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(windows + 1)]
+    ev[0].record()
+    for w, n in enumerate(sizes):
+        graphs[n].replay()
+        ev[w + 1].record()
     torch.cuda.synchronize()
     if barrier:
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    del g, g_rem
-    return ms / steps
+    per_step = [ev[w].elapsed_time(ev[w + 1]) / n for w, n in enumerate(sizes)]
+    total = ev[0].elapsed_time(ev[-1])
+    del graphs
+    return {"ms": total / steps, "median": float(np.median(per_step)), "min": float(np.min(per_step)),
+            "max": float(np.max(per_step)), "windows": windows}
+
+
+def time_steps(step_fn, steps: int, warmup: int, **kw) -> float:
+    """Median over 5 windows of ms per step (see time_windows)."""
+    return time_windows(step_fn, steps, warmup, **kw)["median"]
 
 
 def _copies(bytes_per_copy: int, l2_bytes: int, minimum: int = 2) -> int:
@@ -286,11 +287,128 @@ def cpu_baseline(budget_s: float = 12.0):
             "sample": f"{steps} full step(s) of the workload (4 BitLinear layers) on the host cores, {dt:.1f} s"}
 
 
+# ---------------------------------------------------------------- CPU oracle, every config
+
+def _cpu_rate(fn, units: float, min_s: float = 1.0):
+    """Calls fn until min_s has passed (at least twice); returns (units per second, calls, seconds)."""
+    fn()  # untimed: warms caches and the OpenMP pool
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s and n >= 2:
+            return units * n / dt, n, dt
+
+
+def _cpu_affine(case, rows: int, toks: int):
+    import oracle
+    w = case.weight()[:rows]
+    codes, s, b = oracle.affine_quantize(w, case.bits, case.group_size, case.param_dtype)
+    x = case.x().vals[:toks]
+    lb = case.layer_bias()
+    bias = None if lb is None else lb.vals[:rows]
+    return (lambda: oracle.affine_matmul(x, codes, s, b, case.bits, case.group_size, bias)), codes, s
+
+
+def cpu_config_rate(name: str) -> dict:
+    """The oracle on a bounded sample of one config, in the config's metric unit."""
+    import oracle
+    oracle.build()
+    kind, arg = CPU_CONFIGS[name]
+    if kind == "affine":  # GB/s of weight bytes (codes + scales + biases) in the sample
+        case, rows, toks = arg
+        fn, codes, s = _cpu_affine(case, rows, toks)
+        pbytes = 2 if case.param_dtype == "bf16" else 4
+        units, unit = codes.nbytes + 2 * s.size * pbytes, "GB/s"
+        sample = f"{rows} of {case.N} output rows, {toks} of {case.M} tokens, K = {case.K}"
+    elif kind == "prefill":  # TFLOP/s
+        case, rows, toks = arg
+        fn, _, _ = _cpu_affine(case, rows, toks)
+        units, unit = 2.0 * rows * toks * case.K, "TFLOP/s"
+        sample = f"{toks} of {case.M} tokens x {rows} of {case.N} output rows, K = {case.K}"
+    elif kind == "bitlinear":
+        rows = arg
+        cases = synth.BITLINEAR_DECODE
+        P = cases[0].packed()[:rows]
+        xs = [c.x().vals for c in cases]
+
+        def fn():
+            for c, x in zip(cases, xs):
+                oracle.bitlinear(x, P, 4 * rows, c.weight_scale, c.invert)
+        units, unit = 4.0 * P.nbytes, "GB/s"
+        sample = f"packed rows 0..{rows - 1} of 1024 ({4 * rows} of 4096 outputs) of each of the 4 layers"
+    else:  # "w8a8" / "w4a8": (case, rows, toks)
+        case, rows, toks = arg
+        w = case.weight()
+        x = case.x().vals[:toks]
+        if kind == "w8a8":
+            qw, sw = oracle.quantize_int8_rows(w[:rows])
+            fn = lambda: oracle.w8a8_linear(x, qw, sw)  # noqa: E731
+            wbytes = qw.nbytes + sw.nbytes
+        else:
+            P, sw = oracle.pack_int4_cols(np.ascontiguousarray(w[:rows].T))
+            fn = lambda: oracle.w4a8_linear(x, P, sw)  # noqa: E731
+            wbytes = P.nbytes + sw.nbytes
+        if case.M <= 16:
+            units, unit = float(wbytes), "GB/s"
+        else:
+            units, unit = 2.0 * rows * toks * case.K, "TFLOP/s"
+        sample = f"{toks} of {case.M} tokens x {rows} of {case.N} outputs, K = {case.K}"
+    rate, n, dt = _cpu_rate(fn, units)
+    scale = 1e9 if unit == "GB/s" else 1e12
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"config": name, "value": rate / scale, "unit": unit, "cores": threads,
+            "sample": f"{sample}; {n} calls in {dt:.2f} s"}
+
+
+def _cpu_configs():
+    d = synth.AFFINE_DECODE
+    il = synth.INT_LINEAR
+    return {
+        "cfg1_affine_b4_g64_M4_K512_N512_f32": ("affine", (synth.AFFINE_SMALL, 512, 4)),
+        "cfg2_bitlinear_decode_K4096_N4096": ("bitlinear", 64),
+        **{f"cfg3_{c.name}": ("affine", (c, 128, c.M)) for c in d},
+        "cfg4_affine_prefill_M2048_K4096_N14336": ("prefill", (synth.AFFINE_PREFILL, 64, 64)),
+        **{f"cfg5_w8a8_{c.name}": ("w8a8", (c, 256 if c.M == 1 else 64, min(c.M, 32))) for c in il},
+        **{f"cfg5_w4a8_{c.name}": ("w4a8", (c, 256 if c.M == 1 else 64, min(c.M, 32))) for c in il},
+    }
+
+
+CPU_CONFIGS = _cpu_configs()
+
+
+def cpu_table() -> dict:
+    """Every config's oracle sample on 1 thread and on all host cores (child processes, so each
+    OpenMP runtime starts with its own thread count)."""
+    allc = os.cpu_count() or 1
+    rows = []
+    for name in CPU_CONFIGS:
+        row = {"config": name}
+        for tag, threads in (("one", 1), ("all", allc)):
+            env = dict(os.environ, OMP_NUM_THREADS=str(threads))
+            r = subprocess.run([sys.executable, os.path.abspath(__file__), "--cpu-config", name], env=env,
+                               capture_output=True, text=True, timeout=600)
+            d = json.loads(r.stdout.strip().splitlines()[-1])
+            row[tag] = round(d["value"], 4)
+            row["unit"] = d["unit"]
+            row["sample"] = d["sample"]
+        row["cores_all"] = allc
+        rows.append(row)
+    return {"cpu_table": rows, "cores": allc}
+
+
 # ---------------------------------------------------------------- suite
 
-def _entry(name, us, units, unit, bound, peak, note=None):
-    val = units / (us * 1e-6) / (1e9 if unit == "GB/s" else 1e12)
-    e = {"case": name, "us": round(us, 3), "value": round(val, 1), "unit": unit, "bound": bound,
+def _entry(name, t, units, unit, bound, peak, note=None):
+    """Suite line from time_windows() stats `t` (ms per call): value and frac from the median window,
+    the spread as the windows' fastest and slowest."""
+    scale = 1e9 if unit == "GB/s" else 1e12
+    us = t["median"] * 1e3
+    val = units / (us * 1e-6) / scale
+    e = {"case": name, "us": round(us, 3), "us_min": round(t["min"] * 1e3, 3), "us_max": round(t["max"] * 1e3, 3),
+         "windows": t["windows"], "value": round(val, 1), "unit": unit, "bound": bound,
          "frac": round(val / peak, 4), "peak": peak}
     if note:
         e["note"] = note
@@ -303,6 +421,7 @@ def suite(l2: int, peaks: dict, int8_peak: float):
     bf16 = float(peaks["bf16_tflops"])
     out = []
     dev = "cuda"
+    tw = time_windows
 
     # --- MLX-affine layer, small (fp32)
     c = synth.AFFINE_SMALL
@@ -312,19 +431,27 @@ def suite(l2: int, peaks: dict, int8_peak: float):
     bias = c.layer_bias().torch(dev)
     y = torch.empty((c.M, c.N), dtype=torch.float32, device=dev)
     wb = codes.numel() * 4 + s.numel() * 8
-    us = time_steps(lambda i: ql.matmul(x, codes, s, b, 4, 64, bias, out=y), 200, 5) * 1e3
-    out.append(_entry(c.name, us, wb, "GB/s", "hbm", hbm, "launch-bound (0.16 MB)"))
+    t = tw(lambda i: ql.matmul(x, codes, s, b, 4, 64, bias, out=y), 200, 5)
+    out.append(_entry(c.name, t, wb, "GB/s", "hbm", hbm, "launch-bound (0.16 MB)"))
 
-    # --- BitLinear, each case alone
+    # --- BitLinear decode, each case alone
     P = torch.from_numpy(synth.BITLINEAR_DECODE[0].packed()).to(dev)
     pool = [P.clone() for _ in range(_copies(P.numel(), l2, 8))]
     ws = torch.tensor([0.5], device=dev)
     for c in synth.BITLINEAR_DECODE:
         x = c.x().torch(dev)
         y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
-        us = time_steps(lambda i: ql.bitlinear_matmul(x, pool[i % len(pool)], c.N, ws, c.invert, out=y), 400, 5) * 1e3
-        out.append(_entry(c.name, us, P.numel(), "GB/s", "hbm", hbm))
+        t = tw(lambda i: ql.bitlinear_matmul(x, pool[i % len(pool)], c.N, ws, c.invert, out=y), 400, 5)
+        out.append(_entry(c.name, t, P.numel(), "GB/s", "hbm", hbm))
     del pool
+
+    # --- BitLinear prefill (tcgen05 bf16, exact ternary operands), M = 2048, K = N = 4096
+    x = synth.activations(11, (2048, 4096), "bf16").torch(dev)
+    y = torch.empty((2048, 4096), dtype=torch.bfloat16, device=dev)
+    t = tw(lambda i: ql.bitlinear_matmul(x, P, 4096, ws, False, out=y), 20, 3)
+    out.append(_entry("bitlinear_prefill_M2048_K4096_N4096", t, 2.0 * 2048 * 4096 * 4096, "TFLOP/s", "tensor",
+                      bf16, "bf16 tcgen05 with exact {-1, 0, 1} operands; inputs L2-resident (x 16.8 MB, W 4.2 MB)"))
+    del x, y, P
 
     # --- MLX-affine decode
     for c in synth.AFFINE_DECODE:
@@ -340,23 +467,44 @@ def suite(l2: int, peaks: dict, int8_peak: float):
         def st(i, pool=pool, x=x, bias=bias, y=y, c=c):
             cc, ss, bb = pool[i % len(pool)]
             ql.matmul(x, cc, ss, bb, c.bits, c.group_size, bias, out=y)
-        us = time_steps(st, 200, 5) * 1e3
-        out.append(_entry(c.name, us, wb, "GB/s", "hbm", hbm))
+        t = tw(st, 200, 5)
+        out.append(_entry(c.name, t, wb, "GB/s", "hbm", hbm))
         del pool
         torch.cuda.empty_cache()
 
-    # --- MLX-affine prefill (tcgen05 bf16)
+    # --- MLX-affine decode, general kernel (3-bit codes straddling words; fp16 x)
+    for bits, xd in ((3, "bf16"), (5, "f16")):
+        c = synth.AffineCase(f"affine_b{bits}_g64_M1_K4096_N4096_{xd}_general", 1, 4096, 4096, bits, 64, xd, "bf16",
+                             True, seed=5)
+        wd = torch.from_numpy(c.weight()).to(dev)
+        codes, s, b = ql.quantize(wd, bits, 64, torch.bfloat16)
+        del wd
+        wb = codes.numel() * 4 + s.numel() * 2 + b.numel() * 2
+        pool = [(codes.clone(), s.clone(), b.clone()) for _ in range(_copies(wb, l2, 8))]
+        x = c.x().torch(dev)
+        bias = c.layer_bias().torch(dev)
+        y = torch.empty((1, 4096), dtype=x.dtype, device=dev)
+
+        def sg(i, pool=pool, x=x, bias=bias, y=y, bits=bits):
+            cc, ss, bb = pool[i % len(pool)]
+            ql.matmul(x, cc, ss, bb, bits, 64, bias, out=y)
+        t = tw(sg, 200, 5)
+        out.append(_entry(c.name, t, wb, "GB/s", "hbm", hbm, "general decode kernel (any width / dtype)"))
+        del pool
+        torch.cuda.empty_cache()
+
+    # --- MLX-affine prefill (tcgen05, fp16 operands)
     c = synth.AFFINE_PREFILL
     wd = torch.from_numpy(c.weight()).to(dev)
     codes, s, b = ql.quantize(wd, 4, 64, torch.bfloat16)
-    us_q = time_steps(lambda i: ql.quantize(wd, 4, 64, torch.bfloat16), 10, 2) * 1e3
+    t = tw(lambda i: ql.quantize(wd, 4, 64, torch.bfloat16), 10, 2)
     qbytes = wd.numel() * 4 + codes.numel() * 4 + s.numel() * 4
-    out.append(_entry("quantize_f32_b4_g64_N14336_K4096", us_q, qbytes, "GB/s", "hbm", hbm,
+    out.append(_entry("quantize_f32_b4_g64_N14336_K4096", t, qbytes, "GB/s", "hbm", hbm,
                       "reads fp32 W, writes codes + bf16 params"))
     wdq = torch.empty((c.N, c.K), dtype=torch.bfloat16, device=dev)
-    us_d = time_steps(lambda i: ql.dequantize(codes, s, b, c.K, 4, 64, torch.bfloat16), 10, 2) * 1e3
+    t = tw(lambda i: ql.dequantize(codes, s, b, c.K, 4, 64, torch.bfloat16), 10, 2)
     dbytes = codes.numel() * 4 + s.numel() * 4 + wdq.numel() * 2
-    out.append(_entry("dequantize_b4_g64_N14336_K4096_bf16", us_d, dbytes, "GB/s", "hbm", hbm))
+    out.append(_entry("dequantize_b4_g64_N14336_K4096_bf16", t, dbytes, "GB/s", "hbm", hbm))
     del wd, wdq
     x = c.x().torch(dev)
     bias = c.layer_bias().torch(dev)
@@ -367,53 +515,85 @@ def suite(l2: int, peaks: dict, int8_peak: float):
     def stp(i):
         cc, ss, bb = pool[i % 3]
         ql.matmul(x, cc, ss, bb, 4, 64, bias, out=y, workspace=wsp)
-    us = time_steps(stp, 20, 3) * 1e3
+    t = tw(stp, 20, 3)
     flops = 2.0 * c.M * c.N * c.K
-    out.append(_entry(c.name, us, flops, "TFLOP/s", "tensor", bf16, "bf16 tcgen05, fp32 accumulate; dequant fused"))
-    del pool, x, y
+    out.append(_entry(c.name, t, flops, "TFLOP/s", "tensor", bf16,
+                      "fp16 operands (x 2^-E, fp16(s q + b)), fp32 accumulate in TMEM; includes the prep kernel"))
+    del pool, x, y, wsp
     torch.cuda.empty_cache()
 
-    # --- W8A8 / W4A8, K = N = 8192, M in {1, 256, 4096}
+    # --- per-group INT8 (K = N = 4096, group 128): M = 1 FP-activation branch, M = 2048 act-quant branch
+    wf = torch.from_numpy(synth.normal(61, (4096, 4096), 0.02)).to(dev)
+    qg, sg_ = ql.quantize_int8_groups(wf, 128)
+    t = tw(lambda i: ql.quantize_int8_groups(wf, 128), 10, 2)
+    out.append(_entry("quantize_int8_groups_N4096_K4096_g128", t, wf.numel() * 5 + sg_.numel() * 4, "GB/s", "hbm",
+                      hbm, "reads fp32 W, writes int8 + scales"))
+    t = tw(lambda i: ql.quantize_weight_int8(wf, 99.9), 5, 2)
+    out.append(_entry("quantize_weight_int8_clip99.9_4096x4096", t, wf.numel() * 5 + 4096 * 4, "GB/s", "hbm", hbm,
+                      "per-row percentile: bitonic sort of each row in shared memory"))
+    del wf
+    pgb = qg.numel() + sg_.numel() * 4
+    pool = [(qg.clone(), sg_.clone()) for _ in range(_copies(pgb, l2, 4))]
+    for M in (1, 2048):
+        x = synth.activations(62, (M, 4096), "bf16").torch(dev)
+        y = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
+        wsz = torch.empty(ql.workspace_size(ql.QLIN_OP_PERGROUP, M, 4096, 4096, 8, 128), dtype=torch.uint8, device=dev)
+
+        def spg(i, x=x, y=y, wsz=wsz):
+            qq, ss = pool[i % len(pool)]
+            ql.pergroup_linear(x, qq, ss, 128, out=y, workspace=wsz)
+        t = tw(spg, 100 if M == 1 else 20, 3)
+        if M == 1:
+            out.append(_entry("pergroup_M1_K4096_N4096_g128", t, pgb, "GB/s", "hbm", hbm,
+                              "fp activation; runs the tcgen05 GEMM on a 1-token tile (no GEMV)"))
+        else:
+            out.append(_entry("pergroup_M2048_K4096_N4096_g128", t, 2.0 * M * 4096 * 4096, "TFLOP/s", "tensor", bf16,
+                              "fp16 operands (int8 x, fp16(s w)); includes act quant + prep"))
+        del x, y, wsz
+    del pool
+    torch.cuda.empty_cache()
+
+    # --- W8A8 / W4A8, K = N = 8192, M in {1, 256, 4096}; weights rotate over copies > 2 x L2
     base = synth.INT_LINEAR[0]
     wf = torch.from_numpy(base.weight()).to(dev)
     qw, sw = ql.quantize_int8_rows(wf)
     P4, s4 = ql.pack_int4_cols(wf.t().contiguous())
     del wf
+    n8, n4 = _copies(qw.numel(), l2), _copies(P4.numel(), l2)
+    p8 = [qw.clone() for _ in range(n8)]
+    p4 = [P4.clone() for _ in range(n4)]
     for c in synth.INT_LINEAR:
         x = c.x().torch(dev)
         y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
         wsz = ql.workspace_size(ql.QLIN_OP_W8A8, c.M, c.N, c.K)
         ws_ = torch.empty(wsz, dtype=torch.uint8, device=dev)
-        n8 = 4 if c.M == 1 else 2
-        p8 = [qw.clone() for _ in range(n8)]
-        p4 = [P4.clone() for _ in range(n8)]
-        for name, fn, wbytes in (
-                ("w8a8", lambda i: ql.w8a8_linear(x, p8[i % n8], sw, out=y, workspace=ws_), qw.numel() + 4 * c.N),
-                ("w4a8", lambda i: ql.w4a8_linear(x, p4[i % n8], s4, out=y, workspace=ws_), P4.numel() + 4 * c.N)):
-            us = time_steps(fn, 50 if c.M < 4096 else 10, 3) * 1e3
+        for name, fn, wbytes, ncp in (
+                ("w8a8", lambda i: ql.w8a8_linear(x, p8[i % n8], sw, out=y, workspace=ws_), qw.numel() + 4 * c.N, n8),
+                ("w4a8", lambda i: ql.w4a8_linear(x, p4[i % n4], s4, out=y, workspace=ws_), P4.numel() + 4 * c.N, n4)):
+            t = tw(fn, 50 if c.M < 4096 else 10, 3)
+            rot = f"weights rotate over {ncp} copies ({ncp * wbytes / 1e6:.0f} MB)"
             if c.M <= 16:
-                out.append(_entry(f"{name}_{c.name}", us, wbytes, "GB/s", "hbm", hbm,
-                                  "includes the activation-quant kernel"))
+                out.append(_entry(f"{name}_{c.name}", t, wbytes, "GB/s", "hbm", hbm,
+                                  f"includes the activation-quant kernel; {rot}"))
             else:
                 ops = 2.0 * c.M * c.N * c.K
                 roof = min(int8_peak, hbm * 1e9 * ops / (wbytes + c.M * c.K * 3 + c.M * c.N * 2) / 1e12)
-                out.append(_entry(f"{name}_{c.name}", us, ops, "TFLOP/s", "tensor", round(roof, 1),
-                                  "TOPS; includes the activation-quant kernel; peak = min(int8 peak, BW x AI)"))
+                out.append(_entry(f"{name}_{c.name}", t, ops, "TFLOP/s", "tensor", round(roof, 1),
+                                  f"TOPS; includes the activation-quant kernel; peak = min(int8 peak, BW x AI); {rot}"))
         # activation quantiser alone at this M
         if c.M == 4096:
-            qx = torch.empty((c.M, c.K), dtype=torch.int8, device=dev)
-            us = time_steps(lambda i: ql.quantize_int8_rows(x), 10, 3) * 1e3
-            out.append(_entry("act_quant_M4096_K8192", us, c.M * c.K * 3 + c.M * 4, "GB/s", "hbm", hbm))
-            del qx
-        del p8, p4, ws_, x, y
+            t = tw(lambda i: ql.quantize_int8_rows(x), 10, 3)
+            out.append(_entry("act_quant_M4096_K8192", t, c.M * c.K * 3 + c.M * 4, "GB/s", "hbm", hbm))
+        del ws_, x, y
         torch.cuda.empty_cache()
+    del p8, p4
 
     # --- raw int8 GEMM 4096 x 8192 x 8192
     a8 = torch.randint(-128, 128, (4096, 8192), dtype=torch.int8, device=dev)
     b8 = torch.randint(-128, 128, (8192, 8192), dtype=torch.int8, device=dev)
     c32 = torch.empty((4096, 8192), dtype=torch.int32, device=dev)
-    us = time_steps(lambda i: ql.int8_matmul_int32(a8, b8, out=c32), 10, 3) * 1e3
-    out.append(_entry("int8_matmul_int32_M4096_N8192_K8192", us, 2.0 * 4096 * 8192 * 8192, "TFLOP/s", "tensor",
+    t = tw(lambda i: ql.int8_matmul_int32(a8, b8, out=c32), 10, 3)
+    out.append(_entry("int8_matmul_int32_M4096_N8192_K8192", t, 2.0 * 4096 * 8192 * 8192, "TFLOP/s", "tensor",
                       int8_peak, "TOPS"))
     return out
 
@@ -522,10 +702,17 @@ def main():
     ap.add_argument("--no-suite", action="store_true")
     ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
                     help="run a few launches of one case (for ncu), print nothing else")
+    ap.add_argument("--cpu-table", action="store_true",
+                    help="time the CPU oracle on a sample of every config, 1 thread and all cores (no GPU)")
+    ap.add_argument("--cpu-config", default=None, choices=sorted(CPU_CONFIGS), help=argparse.SUPPRESS)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.profile:
         return profile_case(args.profile)
+    if args.cpu_config:
+        return print(json.dumps(cpu_config_rate(args.cpu_config)), flush=True)
+    if args.cpu_table:
+        return print(json.dumps(cpu_table()), flush=True)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -555,7 +742,8 @@ def main():
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    ms = time_steps(wl.step, args.steps, args.warmup, soak_s=1.0, barrier=barrier)
+    tm = time_windows(wl.step, args.steps, args.warmup, soak_s=1.0, barrier=barrier)
+    ms = tm["ms"]
     clocks = sampler.stop()
 
     ms_max = max_over_ranks(ms, dist)
@@ -570,7 +758,7 @@ def main():
                 "kernel": wl.key, "peak_source": f"{peaks['source']} hbm_gbs (of measured)"}
 
     wl.e2e_prepare()
-    ms_e2e = time_steps(wl.e2e_step, max(1, min(args.steps, 1000)), args.warmup, barrier=barrier)
+    ms_e2e = time_windows(wl.e2e_step, max(1, min(args.steps, 1000)), args.warmup, barrier=barrier)["ms"]
     e2e_value = whole_job_rate(world, wl.units_per_step, max_over_ranks(ms_e2e, dist))
 
     suite_out = None
@@ -597,6 +785,9 @@ def main():
         "e2e": {"value": round(e2e_value, 1), "unit": wl.unit, "h2d_bytes_per_step": wl.h2d,
                 "d2h_bytes_per_step": wl.d2h},
         "clocks": clocks, "gpu_launches": wl.launches_per_step * args.steps,
+        "ms_per_step_windows": {"median": round(tm["median"], 6), "min": round(tm["min"], 6),
+                                "max": round(tm["max"], 6), "windows": tm["windows"],
+                                "note": "rank 0's K steps split into back-to-back graph replays"},
     }
     if suite_out is not None:
         line["suite"] = suite_out

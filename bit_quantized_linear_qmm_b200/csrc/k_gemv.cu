@@ -969,6 +969,10 @@ cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const D
         return a.p_dt == QLIN_BF16 ? affine_launch_b<float, __nv_bfloat16>(a, st, dev, dry)
                                    : affine_launch_b<float, float>(a, st, dev, dry);
     };
+    // layers whose codes fit in shared memory over the SMs: the resident-weight kernel
+    const cudaError_t ed = launch_affine_dec(a, st, dev);
+    if (ed != cudaErrorNotSupported)
+        return ed;
     // every launch of the call checked first, so that a call runs wholly on one kernel
     const cudaError_t e = run(true);
     if (e == cudaErrorNotSupported)

@@ -339,6 +339,9 @@ struct AffineGemvArgs {
     void* y;
 };
 cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
+// all codes in shared memory, one CTA per SM (k_affine_dec.cu); cudaErrorNotSupported for
+// layers outside it (x not bf16, codes too large for shared memory, ...), launching nothing
+cudaError_t launch_affine_dec(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
 // any width 1..6, 8 and any dtypes (k_affine_any.cu); 4-byte aligned codes, 16-byte aligned x rows
 cudaError_t launch_affine_gemv_any(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
 

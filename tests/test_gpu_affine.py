@@ -78,6 +78,26 @@ def test_affine_m_above_16_sliced(ql, orc, case):
     _run_case(ql, orc, case)
 
 
+# the resident-weight decode kernel (bf16 x, M <= 8, every code block in shared memory, one CTA
+# per SM, at most two 16-row tiles per CTA): N = 1000 -> 63 CTAs of 15-16 rows, 2400 -> 148 of
+# 16-17, 4096 -> 27-28, 4736 -> exactly 32 (no spare row); K / g even; M = 1 (token-0 epilogue)
+# and M = 5, 8 (the general one)
+RESIDENT = [synth.AffineCase(f"resident_b{b}_g{g}_M{M}_K{K}_N{N}_{pd}", M, K, N, b, g, "bf16", pd, bias, seed=b + M + N)
+            for (b, g, K, N) in [(4, 128, 1024, 4096), (4, 64, 512, 4736), (4, 32, 256, 2400), (2, 64, 768, 4096),
+                                 (2, 128, 512, 1000), (8, 64, 512, 4096), (8, 128, 256, 4736), (8, 32, 384, 2400)]
+            for M in (1, 5, 8)
+            for (pd, bias) in [("bf16", True), ("f32", False)]]
+
+
+@pytest.mark.parametrize("case", RESIDENT, ids=[c.name for c in RESIDENT])
+def test_affine_resident_decode(ql, orc, case):
+    rng = np.random.default_rng(case.N)
+    rows = None if case.N * case.K <= 4096 * 1024 else np.sort(rng.choice(case.N, size=600, replace=False))
+    if rows is not None:
+        rows[-1] = case.N - 1
+    _run_case(ql, orc, case, rows)
+
+
 def test_affine_rejects_bad_args(ql):
     x = torch.zeros((1, 96), dtype=torch.bfloat16, device="cuda")
     codes = torch.zeros((4, 12), dtype=torch.int32, device="cuda")

@@ -121,6 +121,24 @@ def test_w8a8_full_m4096_sampled_rows_and_tokens(ql, orc):
     assert_fp_close(ys, yr, mag, None, "w8a8 M4096 sampled")
 
 
+def test_w4a8_full_m4096_sampled_cols_and_tokens(ql, orc):
+    """The W4A8 M=4096 layer (K = N = 8192) through one call -- the tcgen05 GEMM with the nibble
+    transform -- checked on sampled tokens x sampled output columns (the last included)."""
+    case = synth.INT_LINEAR[2]
+    w = case.weight()
+    P, sw = orc.pack_int4_cols(np.ascontiguousarray(w.T))
+    x = case.x()
+    y = ql.w4a8_linear(x.torch("cuda"), to_dev(P), to_dev(sw))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    toks = np.sort(rng.choice(case.M, size=64, replace=False))
+    cols = np.sort(rng.choice(case.N, size=64, replace=False))
+    cols[-1] = case.N - 1
+    yr, mag, _, _ = orc.w4a8_linear(x.vals[toks], np.ascontiguousarray(P[:, cols]), sw[cols])
+    ys = y[torch.as_tensor(toks, device="cuda")][:, torch.as_tensor(cols, device="cuda")]
+    assert_fp_close(ys, yr, mag, None, "w4a8 M4096 sampled")
+
+
 def test_int_linear_rejects(ql):
     x = torch.zeros((2, 100), dtype=torch.bfloat16, device="cuda")
     w = torch.zeros((16, 100), dtype=torch.int8, device="cuda")
