@@ -653,7 +653,49 @@ def _prof_int(kind, M):
     return lambda: ql.w4a8_linear(x, P, s4)
 
 
+def _prof_affine_b8():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    c = synth.AffineCase("p", 1, 4096, 4096, 8, 64, "bf16", "bf16", True)
+    codes, s, b = ql.quantize(torch.from_numpy(c.weight()).cuda(), 8, 64, torch.bfloat16)
+    x = c.x().torch("cuda")
+    bias = c.layer_bias().torch("cuda")
+    return lambda: ql.matmul(x, codes, s, b, 8, 64, bias)
+
+
+def _prof_quantize():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    w = torch.from_numpy(synth.AFFINE_PREFILL.weight()).cuda()
+    return lambda: ql.quantize(w, 4, 64, torch.bfloat16)
+
+
+def _prof_act_quant():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    x = synth.INT_LINEAR[2].x().torch("cuda")
+    return lambda: ql.quantize_int8_rows(x)
+
+
+def _prof_bitlinear_prefill():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    P = torch.from_numpy(synth.BITLINEAR_DECODE[0].packed()).cuda()
+    x = synth.activations(11, (2048, 4096), "bf16").torch("cuda")
+    ws = torch.tensor([0.5], device="cuda")
+    return lambda: ql.bitlinear_matmul(x, P, 4096, ws, False)
+
+
+def _prof_pergroup(M):
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    q, s = ql.quantize_int8_groups(torch.from_numpy(synth.normal(61, (4096, 4096), 0.02)).cuda(), 128)
+    x = synth.activations(62, (M, 4096), "bf16").torch("cuda")
+    return lambda: ql.pergroup_linear(x, q, s, 128)
+
+
 PROFILE_CASES = {
+    "affine_decode_m1_b8": _prof_affine_b8,
+    "affine_quantize_n14336": _prof_quantize,
+    "act_quant_m4096": _prof_act_quant,
+    "bitlinear_prefill_m2048": _prof_bitlinear_prefill,
+    "pergroup_m2048": lambda: _prof_pergroup(2048),
+    "pergroup_m1": lambda: _prof_pergroup(1),
     "bitlinear_m1": lambda: _prof_bitlinear(1),
     "bitlinear_m8": lambda: _prof_bitlinear(8),
     "affine_decode_m1": lambda: _prof_affine(1, 4096, 4096),
