@@ -6,6 +6,11 @@
 //   y[m,n] = sum_g [ s[n,g] * sum_{k in g} x[m,k] q[n,k] + b[n,g] * sum_{k in g} x[m,k] ] + bias[n]
 //   [nuvec-nn QuantizedLinear: forward, dequantized_weight (w = scale q + bias per group)]
 //
+// The same kernel runs the one-token branch of the per-group INT8 layer [cider/ops.py
+// pergroup_linear: M == 1 -> per-group MV, FP activation, weight dequant on the fly]: an int8
+// weight c is the 8-bit code c ^ 0x80 = c + 128 with the group's scale s and bias -128 s, the
+// scales read from their group-major [K/g, N] layout.
+//
 // Design (B200; a decode layer is a few MB and sits in a chain of dependent layers, so the
 // weight fetch has to overlap the previous layer and what follows the dependency wait has to be
 // short):
@@ -61,6 +66,7 @@ struct DecParams {
     int rowbytes, pitch;         // code bytes per row; shared-memory row pitch (16 mod 128)
     int rows_max, T, RG, KG;     // rows per CTA at most, 16-row tiles, warp row groups x group split
     int p_f32;                   // group parameters are fp32 (else bf16)
+    int pg;                      // per-group INT8: int8 codes, fp32 scales [NG][N], bias -128 s
     int code_bytes, x_bytes, param_bytes, aux_bytes;  // shared-memory areas
     int xpitch;                  // shared-memory pitch of an x row
     unsigned* status;
@@ -161,7 +167,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) affine_dec_kernel(const __grid
             bulk_g2s(codes_s + (size_t)r * p.pitch, p.codes + (size_t)(r0 + r) * p.rowbytes, (unsigned)p.rowbytes,
                      bar);
     }
-    {
+    if (p.pg) {  // group-major fp32 scales -> [row][NG], one element per copy (consecutive rows)
+        const float* sg = static_cast<const float*>(p.scales);
+        float* ss = reinterpret_cast<float*>(params_s);
+        for (int e = tid; e < rows * p.NG; e += kDecThreads) {
+            const int g = e / rows, r = e % rows;
+            cp_async4(ss + r * p.NG + g, sg + (size_t)g * p.N + r0 + r);
+        }
+    } else {
         const int words = rows * p.NG * psz / 4;  // scales block, then biases block
         const size_t off = (size_t)r0 * p.NG * psz;
         const uint8_t* sg = static_cast<const uint8_t*>(p.scales) + off;
@@ -239,6 +252,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) affine_dec_kernel(const __grid
                     }
                 }
             }
+        if constexpr (BITS == 8) {
+            if (p.pg) {  // int8 weights c read as the unsigned codes c ^ 0x80 = c + 128
+#pragma unroll
+                for (int t = 0; t < kTPW; ++t)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int j = 0; j < WPL; ++j)
+                            cw[t][h][j] ^= 0x80808080u;
+            }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             // token rows past M read row 0 and are zeroed with a mask (no branch)
@@ -348,8 +372,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) affine_dec_kernel(const __grid
                 sb = __bfloat162float(S_[rb * p.NG + gi]);
                 bb = __bfloat162float(B_[rb * p.NG + gi]);
             }
-            ba = fmaf(-OFF, sa, ba);
-            bb = fmaf(-OFF, sb, bb);
+            if (p.pg) {  // w = s (c ^ 0x80) - 128 s for the int8 weight c
+                ba = -128.0f * sa;
+                bb = -128.0f * sb;
+            } else {
+                ba = fmaf(-OFF, sa, ba);
+                bb = fmaf(-OFF, sb, bb);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -447,6 +476,8 @@ bool affine_dec_plan(const AffineGemvArgs& a, const DeviceInfo& dev, int& grid, 
         return false;
     if (a.p_dt != QLIN_BF16 && a.p_dt != QLIN_F32)
         return false;
+    if (a.pergroup && (a.bits != 8 || a.p_dt != QLIN_F32))
+        return false;
     const int64_t NG = a.K / a.g;
     if (a.p_dt == QLIN_BF16 && NG % 2 != 0)  // 4-byte copies of whole rows of bf16 parameters
         return false;
@@ -500,6 +531,7 @@ bool affine_dec_plan(const AffineGemvArgs& a, const DeviceInfo& dev, int& grid, 
         p.RG = RG;
         p.KG = kDecWarps / RG;
         p.p_f32 = a.p_dt == QLIN_F32;
+        p.pg = a.pergroup;
         p.code_bytes = code_bytes;
         p.x_bytes = x_bytes;
         p.param_bytes = param_bytes;

@@ -360,6 +360,26 @@ qlin_status pergroup_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K
     qlin_status s;
     if ((s = current_device(dev)) != QLIN_OK)
         return s;
+    if (M == 1 && x_dt == QLIN_BF16) {  // the FP-activation branch as a weight-resident decode GEMV
+        AffineGemvArgs a;
+        a.x = x;
+        a.x_dt = x_dt;
+        a.M = M;
+        a.K = K;
+        a.N = N;
+        a.codes = reinterpret_cast<const uint32_t*>(w);
+        a.scales = scale_w;
+        a.biases = scale_w;  // not read
+        a.p_dt = QLIN_F32;
+        a.bits = 8;
+        a.g = group_size;
+        a.bias = bias;
+        a.y = y;
+        a.pergroup = 1;
+        const cudaError_t e = launch_affine_dec(a, static_cast<cudaStream_t>(stream), dev);
+        if (e != cudaErrorNotSupported)
+            return from_cuda(e);
+    }
     TcGemmArgs t = {};
     t.M = M;
     t.N = N;

@@ -337,6 +337,10 @@ struct AffineGemvArgs {
     int bits, g;
     const void* bias;
     void* y;
+    // per-group INT8 at one token (pergroup_linear's FP-activation branch): codes are the int8
+    // weights [N][K], scales the fp32 [K/g][N] group-major scale_w, no biases; only
+    // launch_affine_dec takes it
+    int pergroup = 0;
 };
 cudaError_t launch_affine_gemv(const AffineGemvArgs& a, cudaStream_t st, const DeviceInfo& dev);
 // all codes in shared memory, one CTA per SM (k_affine_dec.cu); cudaErrorNotSupported for
