@@ -76,6 +76,12 @@ def any_bytes(seed: int, rows: int, K: int) -> np.ndarray:
     return rng.integers(0, 256, size=(rows, K)).astype(np.uint8)
 
 
+def random_words(seed: int, shape) -> np.ndarray:
+    """uint32 words with every bit uniform (packed codes of any width, drawn directly)."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 2**32, size=shape, dtype=np.uint32)
+
+
 def ternary_codes(seed: int, N: int, K: int) -> np.ndarray:
     """uint8 [N, K] codes uniform in {0, 1, 2} (unpacked form)."""
     rng = np.random.default_rng(seed)

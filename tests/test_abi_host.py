@@ -76,3 +76,23 @@ def test_valid_call_without_gpu_reports_device(ql):
     assert L.qlin_matmul(P16, 1, 1, 128, P16, P16, P16, 1, 64, 4, 64, None, P16, None, 0,
                          None) == ql.QLIN_ERR_DEVICE
     assert L.qlin_get_device_status(None) == ql.QLIN_ERR_DEVICE
+
+
+def test_empty_inputs_rejected_before_device(ql):
+    """M, N or K = 0 is an invalid argument for every entry (checked before any device access)."""
+    L = ql.lib()
+    assert L.qlin_matmul(P16, 1, 0, 128, P16, P16, P16, 1, 64, 4, 64, None, P16, None, 0, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_matmul(P16, 1, 1, 128, P16, P16, P16, 1, 0, 4, 64, None, P16, None, 0, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_matmul(P16, 1, 1, 0, P16, P16, P16, 1, 64, 4, 64, None, P16, None, 0, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.bitlinear_matmul(P16, 1, 0, 64, P16, 8, P16, 0, None, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.bitlinear_matmul(P16, 1, 1, 64, P16, 0, P16, 0, None, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize(P16, 0, 0, 64, 4, 64, P16, P16, P16, 0, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_dequantize(P16, P16, P16, 0, 4, 0, 4, 64, P16, 0, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_int8_rows(P16, 1, 0, 64, P16, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_pack_int4_cols(P16, 1, 64, 0, P16, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_int8_matmul_int32(P16, P16, 0, 16, 16, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.w8a8_linear(P16, 1, 0, 64, P16, P16, 16, None, P16, P16, 4096, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.w4a8_linear(P16, 1, 1, 64, P16, P16, 0, None, P16, P16, 4096, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.pergroup_linear(P16, 1, 0, 128, P16, P16, 16, 64, None, P16, P16, 4096, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_int8_groups(P16, 1, 16, 0, 64, P16, P16, None) == ql.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_weight_int8(P16, 1, 0, 64, -1.0, P16, P16, None) == ql.QLIN_ERR_INVALID_ARG
