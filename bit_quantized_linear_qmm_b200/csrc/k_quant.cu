@@ -440,53 +440,128 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __
 // ---------------------------------------------------------------- per-column int4
 // Block = 32 columns x 8 row slices.
 // ---------------------------------------------------------------- per-row int8 with a percentile clip
-// One CTA per row [cider/ops.py quantize_weight_int8, clip_percentile]: |w| of the row is sorted in
-// shared memory (bitonic, as uint32 bit patterns: non-negative floats order like their bits; the
-// pad is +inf), the clip is the linear-interpolated percentile at (C - 1) p / 100 in float32 with
-// every operation rounded separately (as numpy does it for a float32 row), 0 -> max |w|; then
-// scale = clip / 127 (zero -> 1), w clipped to [-clip, clip], q = clip(round(w / scale), -128,
-// 127) with IEEE divisions.  P2 = the power of two >= C that the sort runs over.
+// One CTA per row [cider/ops.py quantize_weight_int8, clip_percentile]: the clip is the
+// linear-interpolated percentile of |w| at h = (C - 1) p / 100, which needs only the order
+// statistics v_(j) and v_(j+1), j = floor(h).  |w| of the row is held in shared memory as uint32
+// bit patterns (non-negative floats order like their bits); v_(j) is found by a radix select (four
+// passes of a 256-bin histogram of one byte, most significant first, over the values that match
+// the bytes found so far) and v_(j+1) is v_(j) again when more than j + 1 values are <= it, else
+// the smallest value above it.  The interpolation runs in float32 with every operation rounded
+// separately (as numpy does it for a float32 row), 0 -> max |w|; then scale = clip / 127 (zero ->
+// 1), w clipped to [-clip, clip], q = clip(round(w / scale), -128, 127) with IEEE divisions.
 template <typename TW>
-__global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW* __restrict__ w, int64_t C, int P2,
+__global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW* __restrict__ w, int64_t C,
                                                                        float pct, int8_t* __restrict__ q,
                                                                        float* __restrict__ scale)
 {
-    extern __shared__ uint32_t sv[];
+    extern __shared__ uint32_t sv[];  // [C] bit patterns of |w|
+    __shared__ unsigned hist[256];
+    __shared__ uint32_t sel_s, rank_s;
+    __shared__ unsigned cnt_le_s;
+    __shared__ uint32_t next_s, max_s;
     __shared__ float row_clip_s, scale_s;
+    const int n = (int)C;
     const TW* row = w + (int64_t)blockIdx.x * C;
-    for (int i = threadIdx.x; i < P2; i += blockDim.x)
-        sv[i] = i < C ? __float_as_uint(fabsf(to_float(row[i]))) : 0x7F800000u;
-    __syncthreads();
-    for (int k = 2; k <= P2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < P2; i += blockDim.x) {
-                const int l = i ^ j;
-                if (l > i) {
-                    const uint32_t a = sv[i], b = sv[l];
-                    if (((i & k) == 0) == (a > b)) {
-                        sv[i] = b;
-                        sv[l] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
+    uint32_t mx = 0u;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint32_t b = __float_as_uint(fabsf(to_float(row[i])));
+        sv[i] = b;
+        mx = max(mx, b);
     }
+    // the rank of v_(j): j = floor((n - 1) q) when that is below n - 1 (else the maximum is used)
+    const float qq = __fdiv_rn(pct, 100.0f);
+    const float h = __fmul_rn((float)(n - 1), qq);
+    const bool interior = h < (float)(n - 1);
+    const int j = interior ? (int)floorf(h) : n - 1;
     if (threadIdx.x == 0) {
-        const float qq = __fdiv_rn(pct, 100.0f);
-        const float h = __fmul_rn((float)(C - 1), qq);
+        sel_s = 0u;
+        rank_s = (uint32_t)j;
+        max_s = 0u;
+        next_s = 0xFFFFFFFFu;
+        cnt_le_s = 0u;
+    }
+    __syncthreads();
+    atomicMax(&max_s, mx);
+    // radix select of v_(j), one byte per pass from the top
+    for (int pass = 3; pass >= 0; --pass) {
+        const int sh = 8 * pass;
+        const uint32_t hi_mask = pass == 3 ? 0u : 0xFFFFFFFFu << (sh + 8);
+        for (int b = threadIdx.x; b < 256; b += blockDim.x)
+            hist[b] = 0u;
+        __syncthreads();
+        const uint32_t prefix = sel_s;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint32_t v = sv[i];
+            if ((v & hi_mask) == prefix) {
+                // one shared atomic per distinct byte in the warp (the top bytes of a row's |w|
+                // are nearly all equal: per-lane atomics would serialise)
+                const uint32_t key = (v >> sh) & 0xFFu;
+                const unsigned peers = __match_any_sync(__activemask(), key);
+                if ((threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1))
+                    atomicAdd(&hist[key], (unsigned)__popc(peers));
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {  // the bucket holding rank_s among the matching values: a warp scan
+            const int ln = threadIdx.x;
+            unsigned c[8], tot = 0u;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                c[b] = hist[8 * ln + b];
+                tot += c[b];
+            }
+            unsigned inc = tot;  // inclusive prefix of the lanes' bin totals
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
+                if (ln >= o)
+                    inc += t;
+            }
+            const uint32_t r = rank_s;
+            const unsigned excl = inc - tot;
+            __syncwarp();
+            if (r >= excl && r < inc) {  // exactly one lane: rank_s < the matching count
+                uint32_t rr = r - excl;
+                int b = 0;
+                for (; b < 7; ++b) {
+                    if (rr < c[b])
+                        break;
+                    rr -= c[b];
+                }
+                sel_s = prefix | ((uint32_t)(8 * ln + b) << sh);
+                rank_s = rr;
+            }
+        }
+        __syncthreads();
+    }
+    const uint32_t vj = sel_s;
+    // v_(j+1): vj again when more than j + 1 values are <= vj, else the smallest value above it
+    {
+        unsigned c = 0u;
+        uint32_t nx = 0xFFFFFFFFu;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint32_t v = sv[i];
+            c += v <= vj ? 1u : 0u;
+            if (v > vj)
+                nx = min(nx, v);
+        }
+        atomicAdd(&cnt_le_s, c);
+        atomicMin(&next_s, nx);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
         float r;
-        if (h >= (float)(C - 1)) {
-            r = __uint_as_float(sv[C - 1]);
+        if (!interior) {
+            r = __uint_as_float(vj);  // the largest value
         } else {
-            const float j = floorf(h);
-            const float t = __fsub_rn(h, j);
-            const float a = __uint_as_float(sv[(int64_t)j]), b = __uint_as_float(sv[(int64_t)j + 1]);
+            const uint32_t vj1 = cnt_le_s > (unsigned)(j + 1) ? vj : next_s;
+            const float t = __fsub_rn(h, floorf(h));
+            const float a = __uint_as_float(vj), b = __uint_as_float(vj1);
             const float d = __fsub_rn(b, a);
             r = t < 0.5f ? __fadd_rn(a, __fmul_rn(d, t)) : __fsub_rn(b, __fmul_rn(d, __fsub_rn(1.0f, t)));
         }
         if (r == 0.0f)
-            r = __uint_as_float(sv[C - 1]);  // max |w|
+            r = __uint_as_float(max_s);  // max |w|
         float sc = __fdiv_rn(r, 127.0f);
         if (sc == 0.0f)
             sc = 1.0f;
@@ -726,17 +801,14 @@ cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R,
 cudaError_t launch_quantize_weight_int8_clip(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, float pct,
                                              int8_t* q, float* scale, cudaStream_t st, const DeviceInfo&)
 {
-    int p2 = 1;
-    while (p2 < C)
-        p2 <<= 1;
-    const size_t smem = (size_t)p2 * 4;
+    const size_t smem = (size_t)C * 4;  // the row's |w| bit patterns
     auto run = [&](auto* typed) {
         using TW = std::remove_const_t<std::remove_pointer_t<decltype(typed)>>;
         cudaError_t e = cudaFuncSetAttribute(quantize_weight_int8_clip_kernel<TW>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
-        quantize_weight_int8_clip_kernel<TW><<<(unsigned)R, 256, smem, st>>>(typed, C, p2, pct, q, scale);
+        quantize_weight_int8_clip_kernel<TW><<<(unsigned)R, 256, smem, st>>>(typed, C, pct, q, scale);
         return cudaGetLastError();
     };
     switch (w_dt) {

@@ -316,7 +316,7 @@ qlin_status qlin_quantize_weight_int8(const void* w, qlin_dtype w_dt, int64_t R,
     if (clip_percentile < 0.0)  // no clip: the absmax rule
         return from_cuda(
             launch_quantize_int8_rows(w, w_dt, R, C, q, scale, nullptr, static_cast<cudaStream_t>(stream), dev));
-    if (C > 32768)  // the row is sorted in shared memory
+    if (C > 32768)  // the row is held in shared memory
         return QLIN_ERR_UNSUPPORTED;
     // numpy converts the percentile to the row's float32 before dividing by 100
     return from_cuda(launch_quantize_weight_int8_clip(w, w_dt, R, C, (float)clip_percentile, q, scale,

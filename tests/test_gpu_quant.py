@@ -129,3 +129,21 @@ def test_quantize_weight_int8_no_clip_is_absmax(ql, orc):
     q, s = ql.quantize_weight_int8(torch.from_numpy(w).cuda(), None)
     torch.cuda.synchronize()
     assert np.array_equal(q.cpu().numpy(), q_ref) and np.array_equal(s.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("p", [0.0, 12.5, 50.0, 66.7, 99.0, 100.0])
+def test_quantize_weight_int8_clip_ties(ql, orc, p):
+    """Rows of few distinct magnitudes (every order statistic tied with its neighbours), one row of a
+    single value and one with a lone nonzero: the percentile's two order statistics at every rank."""
+    import synth
+    rng = np.random.default_rng(int(p * 10) + 3)
+    w = rng.choice(np.array([-0.5, -0.25, 0.0, 0.25, 0.5, 1.0], np.float32), size=(6, 777)).astype(np.float32)
+    w[1, :] = 0.125
+    w[2, :] = 0.0
+    w[2, 400] = -3.0
+    w[3] = synth.normal(5, (777,), 1.0)
+    q_ref, s_ref = orc.quantize_weight_int8_clip(w, p)
+    q, s = ql.quantize_weight_int8(torch.from_numpy(w).cuda(), p)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
