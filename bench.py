@@ -247,17 +247,25 @@ class BitlinearDecode:
             self.ql.bitlinear_matmul(self.xs[c], w, case.N, self.ws, case.invert, out=self.ys[c])
 
     def e2e_prepare(self):
-        self.hx = [x.cpu().pin_memory() for x in self.xs]
-        self.hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in self.ys]
-        self.h2d = sum(t.numel() * t.element_size() for t in self.hx)
-        self.d2h = sum(t.numel() * t.element_size() for t in self.hy)
+        """The step's inputs (x of the 4 layers) in one pinned host buffer and its results (y) in
+        another, so each step moves them with one copy each way; the layers read and write views
+        of the matching device buffers."""
+        nx = [x.numel() for x in self.xs]
+        ny = [y.numel() for y in self.ys]
+        self.hx = torch.cat([x.reshape(-1).cpu() for x in self.xs]).pin_memory()
+        self.dx = torch.empty_like(self.hx, device="cuda")
+        self.hy = torch.empty(sum(ny), dtype=self.ys[0].dtype).pin_memory()
+        self.dy = torch.empty_like(self.hy, device="cuda")
+        self.xs = [v.view(c.M, c.K) for v, c in zip(torch.split(self.dx, nx), self.cases)]
+        self.ys = [v.view(c.M, c.N) for v, c in zip(torch.split(self.dy, ny), self.cases)]
+        self.dx.copy_(self.hx)
+        self.h2d = self.hx.numel() * self.hx.element_size()
+        self.d2h = self.hy.numel() * self.hy.element_size()
 
     def e2e_step(self, i: int):
-        for c in range(len(self.cases)):
-            self.xs[c].copy_(self.hx[c], non_blocking=True)
+        self.dx.copy_(self.hx, non_blocking=True)
         self.step(i)
-        for c in range(len(self.cases)):
-            self.hy[c].copy_(self.ys[c], non_blocking=True)
+        self.hy.copy_(self.dy, non_blocking=True)
 
 
 def cpu_bitlinear_step():
