@@ -168,7 +168,19 @@ __global__ void __launch_bounds__(kThreads, 2) bitlinear_kernel(const __grid_con
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             const int m = 8 * t + gid;
-            if (ci < my && m < p.M && (FAST || k < p.K)) {
+            if constexpr (FAST) {
+                // token rows past M read row 0 and are zeroed with a mask: no divergent branch in
+                // the straight-line loop (ci < MY is compile-time here)
+                const uint32_t keep = m < p.M ? 0xFFFFFFFFu : 0u;
+                const __nv_bfloat16* src = p.x + (size_t)(m < p.M ? m : 0) * p.K + k;
+                if (ci < my) {
+                    const uint4 a = ldg_cg_v4(src), b = ldg_cg_v4(src + 8);
+                    dst[t][0] = make_uint4(a.x & keep, a.y & keep, a.z & keep, a.w & keep);
+                    dst[t][1] = make_uint4(b.x & keep, b.y & keep, b.z & keep, b.w & keep);
+                } else {
+                    dst[t][0] = dst[t][1] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            } else if (ci < my && m < p.M && k < p.K) {
                 const __nv_bfloat16* src = p.x + (size_t)m * p.K + k;
                 dst[t][0] = ldg_cg_v4(src);
                 dst[t][1] = ldg_cg_v4(src + 8);
