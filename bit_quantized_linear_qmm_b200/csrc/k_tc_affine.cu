@@ -92,8 +92,10 @@ struct Bars {
     uint64_t mma_done;
     uint32_t tmem;
     int abort_flag;
+    int epi_abort;  // written by epilogue warps only: their common break decision
 };
-constexpr int kSmem = kXStages * kXBytes + kCodeRing + (int)sizeof(Bars) + 1024;
+constexpr int kTokScaleBytes = kTT * 4;  // the epilogue's token scales of the current tile
+constexpr int kSmem = kXStages * kXBytes + kCodeRing + kTokScaleBytes + (int)sizeof(Bars) + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(kAccCols + kAStages * kACols <= kTmemCols, "tensor memory");
 
@@ -194,7 +196,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint4* code_ring = reinterpret_cast<uint4*>(smem + kXStages * kXBytes);
-    Bars& bars = *reinterpret_cast<Bars*>(smem + kXStages * kXBytes + kCodeRing);
+    float* tok_s = reinterpret_cast<float*>(smem + kXStages * kXBytes + kCodeRing);
+    Bars& bars = *reinterpret_cast<Bars*>(smem + kXStages * kXBytes + kCodeRing + kTokScaleBytes);
     auto X = [&](int s) { return smem + s * kXBytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -216,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
         mbar_init(&bars.acc_empty, kEpiWarps);
         mbar_init(&bars.mma_done, 1);
         bars.abort_flag = 0;
+        bars.epi_abort = 0;
         fence_mbar_init();
     }
     if (warp == 1)
@@ -503,15 +507,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             bars.abort_flag = 1;
     } else {
         // ------------------------------------------------------------ epilogue
+        // Everything a tile's epilogue reads from global memory -- the token scales (into shared
+        // memory, one per thread), the bias and the row scale -- is fetched before it waits for the
+        // tile's accumulator, so those loads overlap the MMAs instead of following them.
         const int q = warp & 3;                        // TMEM lane quarter this warp may access
         const int th = (warp - 2 - kXformWarps) >> 2;  // token half
+        const int et = threadIdx.x - (2 + kXformWarps) * 32;  // 0 .. 255 among the epilogue threads
+        auto epi_bar = [] { asm volatile("bar.sync 2, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
         pdl_wait_prior_grids();  // bias / out may be touched by the previous kernel
         for (int ti = 0; ti < my_tiles; ++ti) {
-            if (!mbar_wait_bounded(&bars.acc_full, (unsigned)(ti & 1), p.status) || aborted(&bars.abort_flag)) {
-                bars.abort_flag = 1;
-                break;
-            }
-            tc_fence_after();
             int tt, wt;
             tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_t, p.tiles_w, tt, wt);
             const int m0 = tt * kTT + th * (kTT / 2);
@@ -532,6 +536,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                     rs = p.row_scale[n];
                 }
             }
+            if constexpr (!F::kTernary)  // the workspace holds token scales for whole 256-token tiles
+                tok_s[et] = __ldg(p.tok_scale + tt * kTT + et);
+            epi_bar();  // the tile's token scales are in shared memory
+            // the epilogue warps meet at named barriers, so they break together: a warp whose wait
+            // failed (or that saw another role stop) records it in epi_abort, which only they write,
+            // and all of them read it after the next barrier
+            if (!mbar_wait_bounded(&bars.acc_full, (unsigned)(ti & 1), p.status) || aborted(&bars.abort_flag))
+                bars.epi_abort = 1;
+            epi_bar();
+            if (*reinterpret_cast<volatile int*>(&bars.epi_abort)) {
+                bars.abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
             const uint32_t acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(th * (kTT / 2));
             const size_t o0 = (size_t)m0 * p.N + n;
 #pragma unroll 1
@@ -540,17 +558,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                 tmem_ld16(acc + (uint32_t)(c * 16), v);
                 if (!n_ok)
                     continue;
-                // token scales of the chunk (the workspace holds them for whole 256-token tiles)
+                // token scales of the chunk, times the row scale
                 float ts[16];
                 if constexpr (F::kTernary) {
 #pragma unroll
                     for (int u = 0; u < 16; ++u)
                         ts[u] = rs;
                 } else {
-                    const float4* tsp = reinterpret_cast<const float4*>(p.tok_scale + m0 + c * 16);
+                    const float4* tsp = reinterpret_cast<const float4*>(tok_s + th * (kTT / 2) + c * 16);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const float4 t4 = __ldg(tsp + u);
+                        const float4 t4 = tsp[u];
                         ts[4 * u] = t4.x * rs;
                         ts[4 * u + 1] = t4.y * rs;
                         ts[4 * u + 2] = t4.z * rs;
@@ -576,6 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&bars.acc_empty);
+            epi_bar();  // every epilogue warp is done with this tile's token scales
         }
     }
     tc_fence_before();
