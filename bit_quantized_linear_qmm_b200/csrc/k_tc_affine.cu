@@ -42,6 +42,25 @@
 #include "qlin_common.cuh"
 
 namespace qlin {
+
+#ifdef QLIN_TRACE
+// Trace build: %globaltimer per CTA and tile of the last launch -- [cta][tile][4]: the MMA thread
+// starts the tile (its accumulator free), has issued the tile's last MMA, the epilogue (warp 10)
+// sees the accumulator complete, hands it back.  Host side: qlin_trace_read_ts().
+constexpr int kTsTraceCtas = 160;
+constexpr int kTsTraceTiles = 16;
+__device__ unsigned long long g_ts_trace[kTsTraceCtas * kTsTraceTiles * 4];
+#define TS_TRACE(ti, i)                                                                             \
+    do {                                                                                            \
+        if ((int)blockIdx.x < kTsTraceCtas && (ti) < kTsTraceTiles)                                 \
+            g_ts_trace[((int)blockIdx.x * kTsTraceTiles + (ti)) * 4 + (i)] = globaltimer_ns();      \
+    } while (0)
+#else
+#define TS_TRACE(ti, i) \
+    do {                \
+    } while (0)
+#endif
+
 namespace {
 
 constexpr int kTW = 128;            // weight rows (outputs n) per tile: MMA M
@@ -270,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                 // the epilogue has read the previous tile's accumulators
                 ok = mbar_wait_bounded(&bars.acc_empty, (unsigned)(ti & 1) ^ 1u, p.status);
                 tc_fence_after();
+                TS_TRACE(ti, 0);
                 for (int kb = 0; kb < nk && ok; ++kb) {
                     ok = mbar_wait_bounded(&bars.xfull[xs], xph, p.status) &&
                          mbar_wait_bounded(&bars.afull[as], aph, p.status);
@@ -292,6 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                         aph ^= 1u;
                     }
                 }
+                TS_TRACE(ti, 1);
                 if (ok)
                     tc_commit(&bars.acc_full);  // fires when this tile's MMAs are done
             }
@@ -550,16 +571,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                 break;
             }
             tc_fence_after();
+            if (warp == 2 + kXformWarps && lane == 0)
+                TS_TRACE(ti, 2);
             const uint32_t acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(th * (kTT / 2));
             const size_t o0 = (size_t)m0 * p.N + n;
-#pragma unroll 1
-            for (int c = 0; c < kTT / 32; ++c) {
-                uint32_t v[16];
-                tmem_ld16(acc + (uint32_t)(c * 16), v);
+            // chunk c = 16 tokens of this warp's token half: its accumulators are scaled by
+            // 2^E_m 2^F_n (an exact power of two: one rounding in the fma), biased and stored
+            auto chunk_out = [&](int c, const uint32_t (&v)[16]) {
                 if (!n_ok)
-                    continue;
-                // token scales of the chunk, times the row scale
-                float ts[16];
+                    return;
+                float ts[16];  // token scales of the chunk, times the row scale
                 if constexpr (F::kTernary) {
 #pragma unroll
                     for (int u = 0; u < 16; ++u)
@@ -575,25 +596,56 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                         ts[4 * u + 3] = t4.w * rs;
                     }
                 }
+                // tokens of the chunk that exist (all 16 except in the last token tile); the output
+                // dtype and the token bound are settled once per chunk, the address advances by N
+                const int mleft = p.M - (m0 + c * 16);
+                const int cnt = mleft < 16 ? mleft : 16;
+                const size_t step = (size_t)p.N;
+                if (p.out_dt == QLIN_BF16) {
+                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + o0 + (size_t)(c * 16) * step;
+                    if (cnt == 16) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int m = m0 + c * 16 + j;
-                    if (m < p.M) {  // 2^E_m 2^F_n is an exact power of two: one rounding in the fma
-                        const float out = fmaf(__uint_as_float(v[j]), ts[j], bn);
-                        const size_t oi = o0 + (size_t)(c * 16 + j) * p.N;
-                        if (p.out_dt == QLIN_F32)
-                            static_cast<float*>(p.out)[oi] = out;
-                        else if (p.out_dt == QLIN_BF16)
-                            static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(out);
-                        else
-                            static_cast<__half*>(p.out)[oi] = __float2half_rn(out);
+                        for (int j = 0; j < 16; ++j, o += step)
+                            *o = __float2bfloat16_rn(fmaf(__uint_as_float(v[j]), ts[j], bn));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j, o += step)
+                            if (j < cnt)
+                                *o = __float2bfloat16_rn(fmaf(__uint_as_float(v[j]), ts[j], bn));
                     }
+                } else if (p.out_dt == QLIN_F16) {
+                    __half* o = static_cast<__half*>(p.out) + o0 + (size_t)(c * 16) * step;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j, o += step)
+                        if (j < cnt)
+                            *o = __float2half_rn(fmaf(__uint_as_float(v[j]), ts[j], bn));
+                } else {
+                    float* o = static_cast<float*>(p.out) + o0 + (size_t)(c * 16) * step;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j, o += step)
+                        if (j < cnt)
+                            *o = fmaf(__uint_as_float(v[j]), ts[j], bn);
                 }
+            };
+            // two chunks per tensor-memory round trip; the accumulator is handed back to the MMA
+            // thread as soon as the last loads have landed, before their chunks are written out
+#pragma unroll 1
+            for (int c = 0; c < kTT / 32; c += 2) {
+                uint32_t v0[16], v1[16];
+                tmem_ld16_nowait(acc + (uint32_t)(c * 16), v0);
+                tmem_ld16_nowait(acc + (uint32_t)((c + 1) * 16), v1);
+                tmem_wait_ld();
+                if (c + 2 >= kTT / 32) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars.acc_empty);
+                    if (warp == 2 + kXformWarps && lane == 0)
+                        TS_TRACE(ti, 3);
+                }
+                chunk_out(c, v0);
+                chunk_out(c + 1, v1);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bars.acc_empty);
             epi_bar();  // every epilogue warp is done with this tile's token scales
         }
     }
@@ -902,3 +954,15 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
 }
 
 }  // namespace qlin
+
+#ifdef QLIN_TRACE
+// Trace build only: the prefill GEMM's per-tile timestamps of the last launch ([cta][tile][4]
+// uint64, see g_ts_trace); returns the number of CTAs and tiles recorded per CTA as 1000 c + t.
+extern "C" int qlin_trace_read_ts(void* host, size_t bytes)
+{
+    const size_t need = sizeof(qlin::g_ts_trace);
+    if (!host || bytes < need || cudaMemcpyFromSymbol(host, qlin::g_ts_trace, need) != cudaSuccess)
+        return -1;
+    return qlin::kTsTraceCtas * 1000 + qlin::kTsTraceTiles;
+}
+#endif
