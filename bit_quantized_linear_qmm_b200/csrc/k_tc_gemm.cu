@@ -9,13 +9,13 @@
 //              [cider/ops.py w4a8_linear, pack_weight_int4]
 //
 // Persistent, warp-specialised kernel: one CTA per SM walks 128 x BN output
-// tiles (BN = 256, or 128 when there are too few tiles to fill the GPU) in a
+// tiles (BN = 256, or 128 / 112 when there are too few tiles to fill the GPU) in a
 // grouped order: kGroupM M-tiles walk the N-tiles together, so each weight
 // tile is fetched from HBM about once and reused from L2.
 //   warp 0       TMA producer: A tiles and the B source (int8 B or packed
 //                int4) into a shared-memory ring, mbarrier completion
 //                (expect-tx).
-//   warp 1       allocates 2 x BN TMEM columns (two accumulators); one thread
+//   warp 1       allocates two accumulators of BN TMEM columns; one thread
 //                issues tcgen05.mma (kind::i8, M = 128, N = BN, K = 32 per
 //                instruction); tcgen05.commit frees ring slots and transformed
 //                B buffers when their MMAs are done, and publishes each
@@ -23,11 +23,14 @@
 //   warps 2..5   epilogue: tcgen05.ld of one accumulator (warp q owns TMEM
 //                lanes 32q .. 32q+31 = 32 output rows) while the MMAs of the
 //                next tile fill the other one; scales, bias, 16-byte stores.
-//   warps 6..    (W4A8) 2 x BN transform threads turn the packed source into
-//                the K-major 128-byte-swizzled operand in a 2-deep buffer:
-//                nibbles -> int8 16 (c - 8) (the epilogue shifts the exact
-//                int32 sum back by 4 bits).  fence.proxy.async publishes the
-//                operand to the tensor core.
+//   warps 6..    (W4A8) BN transform threads turn the packed source into an
+//                MN-major 128-byte-swizzled operand in a 2-deep buffer: a
+//                packed row of k-pairs [K/2][N] is already N-contiguous, so
+//                each 16-byte chunk becomes one 16-byte chunk of K row 2i
+//                (high nibbles) and one of K row 2i + 1 (low nibbles), no
+//                transposition; nibble c -> int8 16 (c - 8) (the epilogue
+//                shifts the exact int32 sum back by 4 bits).
+//                fence.proxy.async publishes the operand to the tensor core.
 // Every mbarrier wait is bounded; on expiry the kernel records the timeout,
 // every role stops, the MMA thread waits for its MMAs in flight, and TMEM is
 // always freed.
@@ -54,7 +57,8 @@ __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 template <int BSRC, int BN>
 struct TcCfg {
     static constexpr int KE = 128;                          // K elements per stage (128 bytes of A)
-    static constexpr int XW = BSRC == B_TMA_I8 ? 0 : BN / 16;  // transform warps: two threads per B row
+    static constexpr int XW = BSRC == B_TMA_I8 ? 0 : BN / 32;  // transform warps: one thread per B column
+    static constexpr int B_ATOM = 128 * 128;                // MN-major B: one 128-column atom over K = 128
     static constexpr int A_BYTES = kBM * 128;
     static constexpr int B_BYTES = BN * 128;                // one K-major swizzled B operand
     static constexpr int RAW_BYTES = BSRC == B_W4 ? (KE / 2) * BN : B_BYTES;
@@ -62,11 +66,13 @@ struct TcCfg {
     static constexpr int BRING = XW > 0 ? kBDepth * B_BYTES : 0;  // transformed B ring
     static constexpr int NS = cmin(8, (kSmemBudget - BRING) / SLOT);
     static constexpr int THREADS = (2 + kEpiWarps + XW) * 32;
-    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int ACC_COLS = rup(BN, 128);             // TMEM columns between the two accumulators
+    static constexpr int TMEM_COLS = 2 * ACC_COLS;
     static constexpr uint32_t IDESC =
         (2u << 4) |                                         // D: s32
         (1u << 7) | (1u << 10) |                            // A, B: s8 (signed)
-        ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);  // K-major A and B
+        (BSRC == B_W4 ? (1u << 16) : 0u) |                  // B MN-major (W4A8), else K-major
+        ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);  // K-major A
     struct Bars {
         uint64_t full[NS];
         uint64_t empty[NS];
@@ -201,7 +207,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                 const int buf = ti & 1;
                 ok = mbar_wait_bounded(&bars.acc_empty[buf], ((ti >> 1) & 1) ^ 1, p.status);
                 tc_fence_after();
-                const uint32_t acc = tmem + (uint32_t)(buf * BN);
+                const uint32_t acc = tmem + (uint32_t)(buf * Cfg::ACC_COLS);
                 for (int kb = 0; kb < nk && ok; ++kb, ++it) {
                     const int slot = it % Cfg::NS;
                     ok = mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status);
@@ -213,9 +219,13 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                     const uint32_t a0 = smem_u32(A(slot));
                     const uint32_t b0 = smem_u32(Cfg::XW > 0 ? BT(it % kBDepth) : RAW(slot));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc_mma<true>(acc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
-                                        Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        // K = 32 per instruction: 32 bytes along a K-major row, or 32 rows (4 swizzle
+                        // groups of 1024 bytes) of the MN-major W4A8 operand
+                        const uint64_t bd = Cfg::XW > 0 ? umma_desc_sw128_mn(b0 + kk * 4096, Cfg::B_ATOM)
+                                                        : umma_desc_sw128(b0 + kk * 32);
+                        tc_mma<true>(acc, umma_desc_sw128(a0 + kk * 32), bd, Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    }
                     tc_commit(&bars.empty[slot]);
                     if (Cfg::XW > 0)
                         tc_commit(&bars.bempty[it % kBDepth]);
@@ -247,7 +257,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             float sx = 0.f;
             if constexpr (EPI == E_SCALED)
                 sx = row_ok ? p.s_x[row] : 0.f;
-            const uint32_t acc = tmem + (uint32_t)(buf * BN) + ((uint32_t)(32 * q) << 16);
+            const uint32_t acc = tmem + (uint32_t)(buf * Cfg::ACC_COLS) + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
             for (int c = 0; c < BN / 16; ++c) {
                 const int n = nt * BN + c * 16;
@@ -342,15 +352,11 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         }
     } else if constexpr (Cfg::XW > 0) {
         // ------------------------------------------------------------ B transform
-        const int tt = threadIdx.x - (2 + kEpiWarps) * 32;  // 0 .. 2 BN - 1
-        const int wt = tt >> 5;                             // transform warp
-        // W4: warp wt takes 128-column half wt % (BN/128) and 16-k unit wt / (BN/128)
-        const int w4_q = 32 * (wt % (BN / 128)) + lane;  // column quad
-        const int w4_u = wt / (BN / 128);
-        const int w4_rot = (lane >> 1) & 3;
-        const uint32_t c0 = w4_rot, c1 = (w4_rot + 1) & 3, c2 = (w4_rot + 2) & 3, c3 = (w4_rot + 3) & 3;
-        const uint32_t w4_selA = c0 | ((4 + c0) << 4) | (c1 << 8) | ((4 + c1) << 12);
-        const uint32_t w4_selB = c2 | ((4 + c2) << 4) | (c3 << 8) | ((4 + c3) << 12);
+        const int tt = threadIdx.x - (2 + kEpiWarps) * 32;  // 0 .. BN - 1
+        constexpr int CPR = BN / 16;                        // 16-byte chunks per packed row
+        constexpr int UNITS = 64 * CPR / (32 * Cfg::XW);    // chunks per thread per stage
+        static_assert(UNITS * 32 * Cfg::XW == 64 * CPR, "transform split");
+        const uint32_t kHi = 0xF0F0F0F0u, kSign = 0x80808080u;
         pdl_wait_prior_grids();  // the packed weights may come from the previous kernel
         // one stage: RAW(slot) -> BT(it % kBDepth)
         // ring positions of stage it: slot / phase of the code ring, buffer / phase of the operand ring
@@ -361,43 +367,30 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                 !mbar_wait_bounded(&bars.bempty[bslot], bph ^ 1u, p.status) || aborted(&bars.abort_flag))
                 return false;
             uint8_t* dst = BT(bslot);
-            {
-                // raw[i][n]: k-pair row i (k = 2i high nibble, 2i+1 low) of column n; 64 rows x BN bytes.
-                // Eight 32-bit loads (the k-pair rows of unit u for columns 4q .. 4q+3; a warp's lanes
-                // hit 32 distinct banks) are byte-transposed by PRMT into per-column words; slot sl
-                // holds column (rot + sl) & 3 so that the 16-byte stores of each 8-lane phase land in 8
-                // distinct swizzle chunks.  Nibble c -> int8 16 (c - 8): bit 3 flipped, kept in the
-                // high half of the byte.
-                const uint32_t* raw32 = reinterpret_cast<const uint32_t*>(RAW(slot));
-                const int u = w4_u;
-                uint32_t W[8];
+            const uint8_t* raw = RAW(slot);
+            // raw[i][n]: packed row i (k = 2i high nibble, 2i + 1 low) of column n, 64 rows x BN bytes.
+            // Consecutive lanes take consecutive 16-byte chunks of a row, so every 8-lane phase of a
+            // store writes 8 distinct swizzle chunks of one K row.
+            uint4 v[UNITS];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    W[i] = raw32[(8 * u + i) * (BN / 4) + w4_q];
-                uint32_t Ar[4], Br[4];  // row pairs (0,1), (2,3), (4,5), (6,7)
+            for (int u = 0; u < UNITS; ++u)
+                v[u] = *reinterpret_cast<const uint4*>(raw + 16 * (tt + u * 32 * Cfg::XW));
 #pragma unroll
-                for (int pr2 = 0; pr2 < 4; ++pr2) {
-                    Ar[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selA);
-                    Br[pr2] = prmt(W[2 * pr2], W[2 * pr2 + 1], w4_selB);
+            for (int u = 0; u < UNITS; ++u) {
+                const int idx = tt + u * 32 * Cfg::XW;
+                const int i = idx / CPR, c = idx % CPR;
+                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    hi[j] = (w[j] & kHi) ^ kSign;         // k = 2i:     16 (c - 8)
+                    lo[j] = ((w[j] << 4) & kHi) ^ kSign;  // k = 2i + 1
                 }
-#pragma unroll
-                for (int sl = 0; sl < 4; ++sl) {
-                    const uint32_t* src = sl < 2 ? Ar : Br;
-                    const uint32_t sel2 = (sl & 1) ? 0x7632u : 0x5410u;
-                    const uint32_t t0 = prmt(src[0], src[1], sel2);  // k-pair rows 0..3 of the column
-                    const uint32_t t1 = prmt(src[2], src[3], sel2);  // rows 4..7
-                    uint32_t o[4];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const uint32_t x = (hh ? t1 : t0) ^ 0x88888888u;
-                        const uint32_t hi = x & 0xF0F0F0F0u;         // k = 2i
-                        const uint32_t lo = (x << 4) & 0xF0F0F0F0u;  // k = 2i + 1
-                        o[2 * hh] = prmt(hi, lo, 0x5140u);
-                        o[2 * hh + 1] = prmt(hi, lo, 0x7362u);
-                    }
-                    const int n = 4 * w4_q + ((w4_rot + sl) & 3);
-                    st_shared_v4(dst + swz128(n, u), o[0], o[1], o[2], o[3]);
-                }
+                // MN-major swizzled operand: K row r of atom a at a * 16 KB + (r / 8) * 1024 + (r % 8) * 128
+                uint8_t* at = dst + (c >> 3) * Cfg::B_ATOM + (i >> 2) * 1024;
+                const int r0 = (2 * i) & 7;
+                st_shared_v4(at + r0 * 128 + (((c & 7) ^ r0) << 4), hi[0], hi[1], hi[2], hi[3]);
+                st_shared_v4(at + (r0 + 1) * 128 + (((c & 7) ^ (r0 + 1)) << 4), lo[0], lo[1], lo[2], lo[3]);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -494,12 +487,30 @@ cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const 
     if (!encode_tmap_2d(&prm.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K,
                         128, kBM))
         return cudaErrorInvalidValue;
-    // 256-column tiles when they still give every SM a tile, else 128
+    // 256-column tiles when they still give every SM a tile; else the width that
+    // minimises the per-SM work, (tile rounds) x (tile width): 128, or for an
+    // int8 B operand also 112 (e.g. 2 x 74 tiles = 148 SMs for N = 8192)
     const int64_t tiles_m = (a.M + kBM - 1) / kBM;
-    const bool wide = tiles_m * ((a.N + 255) / 256) >= dev.sm_count;
-    if (!encode_b(op, &prm.tm_b, a, wide ? 256 : 128))
+    int bn = 256;
+    if (tiles_m * ((a.N + 255) / 256) < dev.sm_count) {
+        auto cost = [&](int w) {
+            const int64_t tiles = tiles_m * ((a.N + w - 1) / w);
+            return (tiles + dev.sm_count - 1) / dev.sm_count * w;
+        };
+        bn = 128;
+        if (op != TC_W4A8 && cost(112) < cost(128))
+            bn = 112;
+    }
+    if (!encode_b(op, &prm.tm_b, a, bn))
         return cudaErrorInvalidValue;
-    return wide ? launch_bn<256>(op, prm, st, dev) : launch_bn<128>(op, prm, st, dev);
+    if (bn == 256)
+        return launch_bn<256>(op, prm, st, dev);
+    if (bn == 112) {
+        if (op == TC_I8_RAW)
+            return launch_t<B_TMA_I8, E_I32, 112>(prm, st, dev);
+        return launch_t<B_TMA_I8, E_SCALED, 112>(prm, st, dev);
+    }
+    return launch_bn<128>(op, prm, st, dev);
 }
 
 }  // namespace qlin

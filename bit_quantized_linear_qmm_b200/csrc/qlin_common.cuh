@@ -250,6 +250,16 @@ QLIN_DEV uint64_t umma_desc_sw128(uint32_t smem_addr)
            ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
+// Shared-memory matrix descriptor of an MN-major operand tile written with the
+// 128-byte swizzle: each K row holds 128 consecutive M / N bytes, 8-row groups
+// are 1024 bytes apart (SBO) and successive 128-byte M / N atoms lbo bytes
+// apart (LBO).
+QLIN_DEV uint64_t umma_desc_sw128_mn(uint32_t smem_addr, uint32_t lbo)
+{
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the
 // async proxy (TMA, tensor cores).
 QLIN_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
