@@ -180,10 +180,28 @@ def test_bitlinear_fields_every_byte():
 # ---------------------------------------------------------------- W4 nibbles -> int8 16 (c - 8)
 
 def test_w4_decode_constants_in_source():
-    for name in ("k_tc_gemm.cu", "k_gemv.cu"):
-        s = _src(name)
-        assert "^ 0x88888888u" in s and "& 0xF0F0F0F0u" in s and "(x << 4) & 0xF0F0F0F0u" in s, name
-        assert "prmt(hi, lo, 0x5140u)" in s and "prmt(hi, lo, 0x7362u)" in s, name
+    s = _src("k_gemv.cu")
+    assert "^ 0x88888888u" in s and "& 0xF0F0F0F0u" in s and "(x << 4) & 0xF0F0F0F0u" in s
+    assert "prmt(hi, lo, 0x5140u)" in s and "prmt(hi, lo, 0x7362u)" in s
+    s = _src("k_tc_gemm.cu")
+    assert "kHi = 0xF0F0F0F0u, kSign = 0x80808080u" in s
+    assert "hi[j] = (w[j] & kHi) ^ kSign;" in s and "lo[j] = ((w[j] << 4) & kHi) ^ kSign;" in s
+
+
+def test_w4_mn_major_split_every_byte():
+    """The GEMM's MN-major operand: a packed word holds four columns of one k-pair row; the
+    high nibbles give K row 2i and the low nibbles K row 2i + 1, each byte int8 16 (c - 8)."""
+    rng = np.random.default_rng(7)
+    for byte in range(256):
+        for pos in range(4):
+            w = int(rng.integers(0, 2**32))
+            w = (w & ~(0xFF << (8 * pos)) | (byte << (8 * pos))) & 0xFFFFFFFF
+            hi = (w & 0xF0F0F0F0) ^ 0x80808080
+            lo = ((w << 4) & 0xF0F0F0F0) ^ 0x80808080
+            for col in range(4):
+                b = (w >> (8 * col)) & 0xFF
+                assert int(np.int8(np.uint8((hi >> (8 * col)) & 0xFF))) == 16 * ((b >> 4) - 8)
+                assert int(np.int8(np.uint8((lo >> (8 * col)) & 0xFF))) == 16 * ((b & 15) - 8)
 
 
 def test_w4_nibbles_every_byte():
