@@ -1,7 +1,9 @@
 // k_affine_dec.cu -- MLX-affine decode GEMV for up to 8 tokens per launch (one for 2-bit codes),
-// bf16 activations, 2-, 4- or 8-bit codes, on layers of at most 32 output rows per SM (N <= 4736 on B200) whose
-// codes fit in shared memory when spread over the SMs (the Llama-7B layers into 4096 features,
-// K = 4096 or 11008).  Wider layers and more tokens take the ring-streaming kernel (k_gemv.cu).
+// bf16 activations, 2-, 4- or 8-bit codes, on layers whose codes fit in shared memory when spread
+// over the SMs: up to 32 output rows per SM (N <= 4736 on B200) with 8 warps, up to 128 with 16
+// warps when the codes fill more than half of an SM's shared memory (the Llama-7B layers: 4096 ->
+// 4096, 11008 -> 4096, 4096 -> 11008).  Other layers and more tokens take the ring-streaming
+// kernel (k_gemv.cu).
 //
 //   y[m,n] = sum_g [ s[n,g] * sum_{k in g} x[m,k] q[n,k] + b[n,g] * sum_{k in g} x[m,k] ] + bias[n]
 //   [nuvec-nn QuantizedLinear: forward, dequantized_weight (w = scale q + bias per group)]
@@ -18,8 +20,10 @@
 //    griddepcontrol.wait one warp issues a bulk copy (cp.async.bulk, no tensor map) per row of the
 //    CTA's codes into shared memory and every thread copies a slice of the rows' group scales and
 //    biases (cp.async, 4 bytes): the layer's whole weight is on its way before the previous kernel
-//    has finished.  Under about 100 registers a thread, the next layer's CTA fits beside this one
-//    and does the same while this one computes.
+//    has finished.  Under about 100 registers a thread and half the shared memory, the next
+//    layer's CTA fits beside this one (8 warps) and does the same while this one computes; a CTA
+//    whose codes fill more than half the shared memory cannot share the SM, and runs 16 warps
+//    (measured 4-8 % faster there than 8: more warps to hide the loop's latency).
 //  * After the wait the CTA copies the launch's token rows of x into shared memory (one round
 //    trip) and the layer bias too, so neither the main loop nor the epilogue waits on memory.
 //  * Rows sit in shared memory at a pitch of 16 * WPL (mod 128) bytes (16 for WPL = 8), WPL the
@@ -39,8 +43,9 @@
 //  * Measured on B200: mma.sync m16n8k16 issues once per ~8.7 cycles per SM sub-partition; with
 //    two warps per sub-partition the loop is bound by the MMA and decode dependency chains, not
 //    by the pipe.  (Alternatives measured slower: a second register set loading a group ahead --
-//    the register count then keeps the next layer's CTA off the SM; group sums of x computed by
-//    the threads; four accumulator chains; one tile per warp; 16 warps.)
+//    the register count then keeps the next layer's CTA off the SM; group sums of x computed once
+//    per CTA by the threads instead of the all-ones MMA, with 8 and with 16 warps; four accumulator
+//    chains; one tile per warp; 16 warps on layers that can share the SM.)
 //  * Partial sums of the warps that share rows meet in shared memory (the code area, once every
 //    warp has left the main loop); the bias is added in fp32 and y rounded once to bf16.
 //  * The bulk copies complete on an mbarrier whose wait is bounded (qlin::kWaitLimitNs): on expiry
@@ -50,8 +55,7 @@
 namespace qlin {
 namespace {
 
-constexpr int kDecWarps = 8;
-constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecWarpsMax = 16;
 constexpr int kTPW = 2;  // 16-row tiles per warp
 constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 (1, 1)
 
@@ -65,6 +69,7 @@ struct DecParams {
     int M, K, N, NG;
     int rowbytes, pitch;         // code bytes per row; shared-memory row pitch (16 mod 128)
     int rows_max, T, RG, KG;     // rows per CTA at most, 16-row tiles, warp row groups x group split
+    int W;                       // warps per CTA (8 or 16)
     int p_f32;                   // group parameters are fp32 (else bf16)
     int pg;                      // per-group INT8: int8 codes, fp32 scales [NG][N], bias -128 s
     int code_bytes, x_bytes, param_bytes, aux_bytes;  // shared-memory areas
@@ -119,10 +124,13 @@ QLIN_DEV uint32_t code_pair(uint32_t w, int i)
     }
 }
 
-// ONE: a one-token launch
-template <int BITS, int G, int NT, bool ONE>
-__global__ void __launch_bounds__(kDecThreads, 1) affine_dec_kernel(const __grid_constant__ DecParams p)
+// ONE: a one-token launch.  W warps: 8 while the CTA leaves room on the SM for the next layer's
+// CTA (its weight fetch then overlaps this layer), 16 when its codes alone fill more than half of
+// the SM's shared memory (no overlap is possible; more warps hide the loop's latency instead).
+template <int BITS, int G, int NT, bool ONE, int W>
+__global__ void __launch_bounds__(W * 32, 1) affine_dec_kernel(const __grid_constant__ DecParams p)
 {
+    constexpr int kDecThreads = W * 32;
     static_assert(!ONE || NT == 1, "one token fits one token tile");
     constexpr int CPW = 32 / BITS;          // codes per word
     constexpr int WPL = G * BITS / 128;     // words per lane per row per group
@@ -208,9 +216,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) affine_dec_kernel(const __grid
 #pragma unroll
     for (int t = 0; t < kTPW; ++t)
         trow[t] = min(16 * (kTPW * rg + t), 16 * p.T - 16);
-    // warps past RG x KG (when RG does not divide 8) have no work
+    // warps past RG x KG (when RG does not divide W) have no work
     const int ngw = (warp < p.RG * p.KG && p.NG > kg) ? (p.NG - 1 - kg) / p.KG + 1 : 0;  // groups of this warp
-    const int S = ngw * WPL;                                      // word steps of this warp
 
     if (!mbar_wait_bounded(bar, 0, p.status))
         abort_s = 1;
@@ -443,14 +450,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) affine_dec_kernel(const __grid
 }
 
 template <typename Kern>
-cudaError_t launch_dec(Kern kern, unsigned grid, int smem, cudaStream_t st, const DecParams& prm)
+cudaError_t launch_dec(Kern kern, unsigned grid, int warps, int smem, cudaStream_t st, const DecParams& prm)
 {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.blockDim = dim3((unsigned)(32 * warps), 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -464,8 +471,11 @@ cudaError_t launch_dec(Kern kern, unsigned grid, int smem, cudaStream_t st, cons
 template <int BITS, int G>
 cudaError_t dec_launch_nt(const DecParams& prm, unsigned grid, int smem, cudaStream_t st)
 {
-    return prm.M == 1 ? launch_dec(affine_dec_kernel<BITS, G, 1, true>, grid, smem, st, prm)
-                      : launch_dec(affine_dec_kernel<BITS, G, 1, false>, grid, smem, st, prm);
+    if (prm.W == 16)
+        return prm.M == 1 ? launch_dec(affine_dec_kernel<BITS, G, 1, true, 16>, grid, 16, smem, st, prm)
+                          : launch_dec(affine_dec_kernel<BITS, G, 1, false, 16>, grid, 16, smem, st, prm);
+    return prm.M == 1 ? launch_dec(affine_dec_kernel<BITS, G, 1, true, 8>, grid, 8, smem, st, prm)
+                      : launch_dec(affine_dec_kernel<BITS, G, 1, false, 8>, grid, 8, smem, st, prm);
 }
 
 // Plans the launch; false when the layer is outside this kernel (the caller then takes another).
@@ -491,17 +501,15 @@ bool affine_dec_plan(const AffineGemvArgs& a, const DeviceInfo& dev, int& grid, 
     grid = (int)(a.N >= 16LL * dev.sm_count ? dev.sm_count : (a.N + 15) / 16);
     const int rows_max = (int)((a.N + grid - 1) / grid);
     const int T = (rows_max + 15) / 16;
-    if (T > 2)  // more than one row group of two tiles per CTA: measured slower than the ring kernel
+    if (T > 8)
         return false;
     const int RG = (T + kTPW - 1) / kTPW;  // row groups of kTPW tiles; KG = warps / RG share each
-    if (RG > kDecWarps)
-        return false;
     // code rows at 16 * WPL (mod 128): a warp's vector loads of 8 rows fall in distinct banks
     const int wpl = a.g * a.bits / 128;
     const int ct = wpl >= 8 ? 16 : 16 * wpl;
     const int pitch = (int)(rowbytes + ((ct - rowbytes % 128) + 128) % 128);
     const int mmax = (int)a.M;
-    const int red = kDecWarps * kTPW * 4 * 32 * 4;
+    const int red = kDecWarpsMax * kTPW * 4 * 32 * 4;
     int code_bytes = 16 * T * pitch;  // tiles past T are never read
     code_bytes = code_bytes > red ? code_bytes : red;
     // x rows at a pitch that spreads the 16-byte loads of a warp's token rows over the banks
@@ -513,6 +521,11 @@ bool affine_dec_plan(const AffineGemvArgs& a, const DeviceInfo& dev, int& grid, 
     const int param_bytes = (int)((2LL * rows_max * NG * psz + 15) / 16 * 16);
     const int aux_bytes = (rows_max * 4 + 15) / 16 * 16;
     smem = code_bytes + x_bytes + param_bytes + aux_bytes + 16;
+    // 8 warps while two CTAs fit on an SM (the next layer's fetch overlaps this one); else 16.
+    // More than one row group of two tiles on 8 warps measured slower than the ring kernel.
+    const int W = 2 * smem <= 227 * 1024 ? 8 : 16;
+    if (W == 8 && T > 2)
+        return false;
     if (smem > 227 * 1024)
         return false;
     if (out) {
@@ -529,7 +542,8 @@ bool affine_dec_plan(const AffineGemvArgs& a, const DeviceInfo& dev, int& grid, 
         p.rows_max = rows_max;
         p.T = T;
         p.RG = RG;
-        p.KG = kDecWarps / RG;
+        p.KG = W / RG;
+        p.W = W;
         p.p_f32 = a.p_dt == QLIN_F32;
         p.pg = a.pergroup;
         p.code_bytes = code_bytes;

@@ -20,6 +20,8 @@ averaged over the layers:
   x+chunk0      wait return -> first 64-k chunk done (x arrival + one chunk)
   loop          rest of the main loop
   reduce        CTA reduction, scaling, bias and y stores
+  start->wait   CTA start -> its griddepcontrol.wait return (mean over CTAs)
+  start->chunk0 CTA start -> first chunk done (affine: codes and x landed)
   critical      last CTA end minus first wait return
   end spread    last CTA end minus first CTA end
   doubled       SMs that ran two CTAs of the same layer (summed over layers)
@@ -109,9 +111,12 @@ def main():
     grid = int(np.count_nonzero(buf[0, :, 0]))
     t = buf[:, :grid, :].astype(np.int64)
     rel, x0, loop, red, crit, spread, dbl = [], [], [], [], [], [], 0
+    s2w, s2c = [], []
     for i in range(1, args.layers):
         rel.append(t[i, :, 2].min() - t[i - 1, :, 5].max())
         x0.append((t[i, :, 3] - t[i, :, 2]).mean())
+        s2w.append((t[i, :, 2] - t[i, :, 0]).mean())
+        s2c.append((t[i, :, 3] - t[i, :, 0]).mean())
         loop.append((t[i, :, 4] - t[i, :, 3]).mean())
         red.append((t[i, :, 5] - t[i, :, 4]).mean())
         crit.append(t[i, :, 5].max() - t[i, :, 2].min())
@@ -120,6 +125,7 @@ def main():
         dbl += int(np.sum(np.bincount(sm) > 1))
     out = {"kind": args.kind, "layers": args.layers, "ctas": grid, "period_us": round(period_us, 3),
            "release_ns": round(float(np.mean(rel))), "x_chunk0_ns": round(float(np.mean(x0))),
+           "start_to_wait_ns": round(float(np.mean(s2w))), "start_to_chunk0_ns": round(float(np.mean(s2c))),
            "loop_ns": round(float(np.mean(loop))), "reduce_ns": round(float(np.mean(red))),
            "critical_ns": round(float(np.mean(crit))), "end_spread_ns": round(float(np.mean(spread))),
            "doubled_sms": dbl}

@@ -98,6 +98,27 @@ def test_affine_resident_decode(ql, orc, case):
     _run_case(ql, orc, case, rows)
 
 
+# the same kernel with 16 warps, for code blocks that fill more than half of an SM's shared memory
+# (one CTA per SM), and with up to 8 row tiles per CTA: N = 11008 -> 74-75 rows (5 tiles, 3 row
+# groups of 5 warps, the 16th warp idle), 9472 -> 64, 13000 -> 87-88 (6 tiles), 8000 -> 54, 7400 -> 50
+BIG_RESIDENT = [synth.AffineCase(f"resident16_b{b}_g{g}_M{M}_K{K}_N{N}_{pd}", M, K, N, b, g, "bf16", pd, bias,
+                                 seed=b + M + N)
+                for (b, g, K, N, M, pd, bias) in [(4, 128, 4096, 11008, 1, "bf16", True),
+                                                  (4, 64, 4096, 9472, 5, "f32", False),
+                                                  (8, 64, 2048, 9472, 8, "bf16", True),
+                                                  (2, 128, 8192, 8000, 1, "bf16", True),
+                                                  (4, 32, 3072, 13000, 1, "bf16", False),
+                                                  (8, 128, 2048, 7400, 1, "f32", True)]]
+
+
+@pytest.mark.parametrize("case", BIG_RESIDENT, ids=[c.name for c in BIG_RESIDENT])
+def test_affine_resident_decode_16_warps(ql, orc, case):
+    rng = np.random.default_rng(case.N)
+    rows = np.sort(rng.choice(case.N, size=400, replace=False))
+    rows[0], rows[-1] = 0, case.N - 1
+    _run_case(ql, orc, case, rows)
+
+
 def test_affine_rejects_bad_args(ql):
     x = torch.zeros((1, 96), dtype=torch.bfloat16, device="cuda")
     codes = torch.zeros((4, 12), dtype=torch.int32, device="cuda")
