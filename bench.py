@@ -538,7 +538,7 @@ def suite(l2: int, peaks: dict, int8_peak: float):
                       hbm, "reads fp32 W, writes int8 + scales"))
     t = tw(lambda i: ql.quantize_weight_int8(wf, 99.9), 5, 2)
     out.append(_entry("quantize_weight_int8_clip99.9_4096x4096", t, wf.numel() * 5 + 4096 * 4, "GB/s", "hbm", hbm,
-                      "per-row percentile: bitonic sort of each row in shared memory"))
+                      "per-row percentile: a radix select of each row's order statistics in shared memory"))
     del wf
     pgb = qg.numel() + sg_.numel() * 4
     pool = [(qg.clone(), sg_.clone()) for _ in range(_copies(pgb, l2, 4))]
@@ -553,7 +553,7 @@ def suite(l2: int, peaks: dict, int8_peak: float):
         t = tw(spg, 100 if M == 1 else 20, 3)
         if M == 1:
             out.append(_entry("pergroup_M1_K4096_N4096_g128", t, pgb, "GB/s", "hbm", hbm,
-                              "fp activation; runs the tcgen05 GEMM on a 1-token tile (no GEMV)"))
+                              "fp activation; the resident-weight decode kernel (int8 c as the code c ^ 0x80)"))
         else:
             out.append(_entry("pergroup_M2048_K4096_N4096_g128", t, 2.0 * M * 4096 * 4096, "TFLOP/s", "tensor", bf16,
                               "fp16 operands (int8 x, fp16(s w)); includes act quant + prep"))
@@ -676,6 +676,25 @@ def _prof_quantize():
     return lambda: ql.quantize(w, 4, 64, torch.bfloat16)
 
 
+def _prof_quantize_bf16():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    w = torch.from_numpy(synth.AFFINE_PREFILL.weight()).cuda().to(torch.bfloat16)
+    return lambda: ql.quantize(w, 4, 64, torch.bfloat16)
+
+
+def _prof_dequantize():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    c = synth.AFFINE_PREFILL
+    codes, s, b = ql.quantize(torch.from_numpy(c.weight()).cuda(), 4, 64, torch.bfloat16)
+    return lambda: ql.dequantize(codes, s, b, c.K, 4, 64, torch.bfloat16)
+
+
+def _prof_clip():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    w = torch.from_numpy(synth.normal(61, (4096, 4096), 0.02)).cuda()
+    return lambda: ql.quantize_weight_int8(w, 99.9)
+
+
 def _prof_act_quant():
     from bit_quantized_linear_qmm_b200 import qlin as ql
     x = synth.INT_LINEAR[2].x().torch("cuda")
@@ -701,6 +720,9 @@ PROFILE_CASES = {
     "affine_decode_m1_b8": _prof_affine_b8,
     "affine_quantize_n14336": _prof_quantize,
     "act_quant_m4096": _prof_act_quant,
+    "affine_quantize_bf16_n14336": _prof_quantize_bf16,
+    "dequantize_n14336": _prof_dequantize,
+    "clip_4096": _prof_clip,
     "bitlinear_prefill_m2048": _prof_bitlinear_prefill,
     "pergroup_m2048": lambda: _prof_pergroup(2048),
     "pergroup_m1": lambda: _prof_pergroup(1),

@@ -24,7 +24,125 @@ QLIN_DEV float load_elem(const float* p, int64_t i) { return p[i]; }
 QLIN_DEV float load_elem(const __nv_bfloat16* p, int64_t i) { return __bfloat162float(p[i]); }
 QLIN_DEV float load_elem(const __half* p, int64_t i) { return __half2float(p[i]); }
 
+// 16 consecutive elements from a 16-byte aligned address, as floats
+QLIN_DEV void load16(const float* p, float (&v)[16])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(p) + q);
+        v[4 * q] = f.x;
+        v[4 * q + 1] = f.y;
+        v[4 * q + 2] = f.z;
+        v[4 * q + 3] = f.w;
+    }
+}
+QLIN_DEV float lo_half_to_float(uint32_t u, const __nv_bfloat16*) { return __uint_as_float(u << 16); }
+QLIN_DEV float hi_half_to_float(uint32_t u, const __nv_bfloat16*) { return __uint_as_float(u & 0xffff0000u); }
+QLIN_DEV float lo_half_to_float(uint32_t u, const __half*)
+{
+    return __half2float(__ushort_as_half((unsigned short)(u & 0xffffu)));
+}
+QLIN_DEV float hi_half_to_float(uint32_t u, const __half*) { return __half2float(__ushort_as_half((unsigned short)(u >> 16))); }
+template <typename T>
+QLIN_DEV void load16(const T* p, float (&v)[16])  // bf16 / fp16: element 2j in the low half of word j
+{
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + q);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[8 * q + 2 * j] = lo_half_to_float(w4[j], p);
+            v[8 * q + 2 * j + 1] = hi_half_to_float(w4[j], p);
+        }
+    }
+}
+
+// rint(d / s) of the quotient rounded once, as an IEEE single division rounds it, for s > 0.
+// With r = 1/s and m = d * r each rounded once, m = q (1 + e1)(1 + e2) for the exact quotient q
+// and |e1|, |e2| <= 2^-24, while the rounded quotient is q (1 + e3), |e3| <= 2^-24: the two differ
+// by less than 1.8e-7 |q|, under 1e-4 while |m| < 512.  rint changes value only at half-integers,
+// so rint(m) is rint of the rounded quotient whenever m lies more than 1e-4 from a half-integer,
+// i.e. whenever its distance to the nearest integer, |m - rint(m)| (exact for |m| < 2^23), is
+// under 0.4999; within that band (and for |m| >= 512) the division itself is done.  r must come
+// from a normal s (fast = false otherwise, and every element divides): r is then finite and both
+// roundings are relative.
+QLIN_DEV bool rcp_ok(float s) { return s >= 1.17549435e-38f && s <= 8.0e37f; }  // s and 1/s normal
+QLIN_DEV float rint_div(float d, float s, float r, bool fast)
+{
+    if (fast) {
+        const float m = __fmul_rn(d, r);
+        const float t = rintf(m);
+        if (fabsf(__fsub_rn(m, t)) < 0.4999f && fabsf(m) < 512.0f)
+            return t;
+    }
+    return rintf(__fdiv_rn(d, s));
+}
+
 // ---------------------------------------------------------------- affine quantize
+// G/16 lanes per group, each holding 16 consecutive values (16-byte loads) and storing its own
+// 16 codes as whole words (2-, 4- and 8-bit codes; 16-byte aligned weights).  The matrix is a flat
+// run of N*K/G groups: the parameters [N][K/G] and the code words [N][K*BITS/32] follow the same
+// order.  The group's lanes find its min and max with G/16 - 1 butterfly steps.
+template <typename TW, typename TP, int BITS, int G>
+__global__ void __launch_bounds__(256) affine_quantize_vec_kernel(const TW* __restrict__ w, int64_t groups,
+                                                                  uint32_t* __restrict__ codes,
+                                                                  TP* __restrict__ scales, TP* __restrict__ biases)
+{
+    constexpr int LPG = G / 16;               // lanes per group
+    constexpr int WPT = 16 * BITS / 32;       // code words per lane
+    constexpr float QMAX = float((1 << BITS) - 1);
+    static_assert(BITS == 2 || BITS == 4 || BITS == 8, "whole words per lane");
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t gi = t / LPG;
+    const int sub = (int)(t % LPG);
+    // lanes past the last group (in the last warp only) work on the last group and store nothing,
+    // so that every lane takes part in the butterfly
+    const bool ok = gi < groups;
+    const int64_t gq = ok ? gi : groups - 1;
+    float v[16];
+    load16(w + gq * G + 16 * sub, v);
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+    }
+#pragma unroll
+    for (int off = 1; off < LPG; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    float scale = __fdiv_rn(__fsub_rn(mx, mn), QMAX);
+    float bias = mn;
+    scale = to_float(from_float<TP>(scale));
+    bias = to_float(from_float<TP>(bias));
+    if (scale == 0.0f)
+        scale = 1.0f;
+    if (ok && sub == 0) {
+        scales[gi] = from_float<TP>(scale);
+        biases[gi] = from_float<TP>(bias);
+    }
+    uint32_t word[WPT];
+#pragma unroll
+    for (int j = 0; j < WPT; ++j)
+        word[j] = 0u;
+    const float rs = __frcp_rn(scale);
+    const bool fast = rcp_ok(scale);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float q = rint_div(__fsub_rn(v[i], bias), scale, rs, fast);
+        q = fminf(fmaxf(q, 0.0f), QMAX);
+        word[i * BITS / 32] |= static_cast<uint32_t>(q) << ((i * BITS) % 32);
+    }
+    if (ok) {
+        uint32_t* dst = codes + gi * (G * BITS / 32) + sub * WPT;
+#pragma unroll
+        for (int j = 0; j < WPT; ++j)
+            dst[j] = word[j];
+    }
+}
+
 // One warp per (row, group).  Lane l holds CPL = g/32 consecutive values.
 template <typename TW, typename TP, int BITS, int G>
 __global__ void __launch_bounds__(256) affine_quantize_kernel(const TW* __restrict__ w, int64_t N, int64_t K,
@@ -86,33 +204,30 @@ __global__ void __launch_bounds__(256) affine_quantize_kernel(const TW* __restri
 }
 
 // ---------------------------------------------------------------- affine dequantize
-// One thread per packed word.
-template <typename TP, typename TO, int BITS>
+// One thread per packed word, in flat form: code c of the [N][K] matrix is field c % CPW of word
+// c / CPW and belongs to group c / G of the [N][K/G] parameters (K is a multiple of G), and out[c]
+// is its value -- no row / column arithmetic.  A word never straddles a group (CPW <= G).
+template <typename TP, typename TO, int BITS, int G>
 __global__ void __launch_bounds__(256) affine_dequantize_kernel(const uint32_t* __restrict__ codes,
                                                                 const TP* __restrict__ scales,
-                                                                const TP* __restrict__ biases, int64_t N, int64_t K,
-                                                                int g, TO* __restrict__ out)
+                                                                const TP* __restrict__ biases, int64_t total,
+                                                                TO* __restrict__ out)
 {
     constexpr int CPW = 32 / BITS;
     constexpr uint32_t MASK = (1u << BITS) - 1u;
-    const int64_t words_per_row = K / CPW;
-    const int64_t total = N * words_per_row;
-    const int64_t groups_per_row = K / g;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t n = idx / words_per_row;
-        const int64_t wi = idx % words_per_row;
-        const int64_t k0 = wi * CPW;
-        const float s = to_float(scales[n * groups_per_row + k0 / g]);
-        const float b = to_float(biases[n * groups_per_row + k0 / g]);
+        const int64_t c0 = idx * CPW;
+        const float s = to_float(scales[c0 / G]);
+        const float b = to_float(biases[c0 / G]);
         const uint32_t word = __ldg(codes + idx);
         TO vals[CPW];
 #pragma unroll
         for (int i = 0; i < CPW; ++i)
             vals[i] = from_float<TO>(__fmaf_rn(static_cast<float>((word >> (BITS * i)) & MASK), s, b));
-        // CPW * sizeof(TO) is 8..64 bytes and out + n*K + k0 is aligned to it.
+        // CPW * sizeof(TO) is 8..64 bytes and out + c0 is aligned to it.
         constexpr int BYTES = CPW * (int)sizeof(TO);
-        TO* dst = out + n * K + k0;
+        TO* dst = out + c0;
         if constexpr (BYTES >= 16) {
 #pragma unroll
             for (int c = 0; c < BYTES / 16; ++c)
@@ -233,89 +348,31 @@ __global__ void __launch_bounds__(256) affine_dequantize_odd_kernel(const uint32
 }
 
 // ---------------------------------------------------------------- per-row int8
-// One block per row: absmax, then quantise (second read comes from L1/L2).
-template <typename TW>
-__global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __restrict__ w, int64_t C,
-                                                                 int8_t* __restrict__ q, float* __restrict__ scale,
-                                                                 int32_t* __restrict__ rowsum, int release)
+// The symmetric int8 code clamp(rint(x / s), -128, 127) of an element with |x| <= amax, s = amax /
+// 127 rounded once (or 1 for amax = 0), r = 1/s rounded once.  On the multiply path (rint_div's
+// argument, with s and 1/s normal) |x r| <= 127 (1 + 3 2^-24), so the code already lies in
+// [-127, 127] and needs no clamp; the division path clamps (a NaN element gives
+// fminf(fmaxf(NaN, -128), 127) = -128, as the division form always did).
+QLIN_DEV int sym_code(float x, float s, float r, bool fast)
 {
-    if (release)
-        pdl_launch_dependents();
-    __shared__ float red[8];
-    __shared__ int ired[8];
-    const int64_t r = blockIdx.x;
-    const TW* row = w + r * C;
-    float amax = 0.0f;
-    for (int64_t c = threadIdx.x; c < C; c += blockDim.x)
-        amax = fmaxf(amax, fabsf(load_elem(row, c)));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if ((threadIdx.x & 31) == 0)
-        red[threadIdx.x / 32] = amax;
-    __syncthreads();
-    amax = red[0];
-    for (int i = 1; i < (int)(blockDim.x / 32); ++i)
-        amax = fmaxf(amax, red[i]);
-    float s = __fdiv_rn(amax, 127.0f);
-    if (s == 0.0f)
-        s = 1.0f;
-    if (threadIdx.x == 0)
-        scale[r] = s;
-    int sum = 0;
-    int8_t* qrow = q + r * C;
-    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
-        float t = rintf(__fdiv_rn(load_elem(row, c), s));
-        t = fminf(fmaxf(t, -128.0f), 127.0f);
-        const int qi = static_cast<int>(t);
-        qrow[c] = static_cast<int8_t>(qi);
-        sum += qi;
+    if (fast) {
+        const float m = __fmul_rn(x, r);
+        const float t = rintf(m);
+        if (fabsf(__fsub_rn(m, t)) < 0.4999f)
+            return (int)t;
     }
-    if (rowsum) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if ((threadIdx.x & 31) == 0)
-            ired[threadIdx.x / 32] = sum;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int t = 0;
-            for (int i = 0; i < (int)(blockDim.x / 32); ++i)
-                t += ired[i];
-            rowsum[r] = t;
-        }
-    }
+    return (int)fminf(fmaxf(rintf(__fdiv_rn(x, s)), -128.0f), 127.0f);
 }
 
-// Single-pass variant for bf16 rows with C % 8 == 0 and C <= 256 * 8 * VPT: each
-// thread keeps its VPT 16-byte pieces of the row in registers between the
-// absmax reduction and the quantisation, so the row is read from memory once.
-template <int VPT>
-__global__ void __launch_bounds__(256) quantize_int8_rows_bf16_reg_kernel(const __nv_bfloat16* __restrict__ w,
-                                                                         int64_t C, int8_t* __restrict__ q,
-                                                                         float* __restrict__ scale,
-                                                                         int32_t* __restrict__ rowsum, int release)
+// four int8 codes -> one word, code i in byte i
+QLIN_DEV uint32_t pack4(int a, int b, int c, int d)
 {
-    if (release)
-        pdl_launch_dependents();
-    __shared__ float red[8];
-    __shared__ int ired[8];
-    const int64_t r = blockIdx.x;
-    const uint4* row = reinterpret_cast<const uint4*>(w + r * C);
-    const int C8 = (int)(C / 8);
-    uint4 v[VPT];
-    float amax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-        const int c = (int)threadIdx.x + j * 256;
-        v[j] = c < C8 ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] << 16)));
-            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] & 0xffff0000u)));
-        }
-    }
+    return prmt(prmt((uint32_t)a, (uint32_t)b, 0x0040u), prmt((uint32_t)c, (uint32_t)d, 0x0040u), 0x5410u);
+}
+
+// the row's absmax over the block (256 threads) from each thread's partial
+QLIN_DEV float block_amax(float amax, float* red)
+{
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -326,115 +383,122 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16_reg_kernel(const 
 #pragma unroll
     for (int i = 1; i < 8; ++i)
         amax = fmaxf(amax, red[i]);
+    return amax;
+}
+
+// eight bf16 of a 16-byte piece -> four code words pair: codes of elements 0..3 and 4..7
+QLIN_DEV uint2 sym_codes8(const uint4& v, float s, float r, bool fast)
+{
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    int c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        c[i] = sym_code(__uint_as_float((i & 1) ? (u[i / 2] & 0xffff0000u) : (u[i / 2] << 16)), s, r, fast);
+    return make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+}
+
+QLIN_DEV float amax8(const uint4& v, float amax)
+{
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        amax = fmaxf(amax, fabsf(__uint_as_float(u[i] << 16)));
+        amax = fmaxf(amax, fabsf(__uint_as_float(u[i] & 0xffff0000u)));
+    }
+    return amax;
+}
+
+// One block (256 threads) per row: absmax, then quantise (second read comes from L1/L2).
+template <typename TW>
+__global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __restrict__ w, int64_t C,
+                                                                 int8_t* __restrict__ q, float* __restrict__ scale,
+                                                                 int release)
+{
+    if (release)
+        pdl_launch_dependents();
+    __shared__ float red[8];
+    const int64_t r = blockIdx.x;
+    const TW* row = w + r * C;
+    float amax = 0.0f;
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x)
+        amax = fmaxf(amax, fabsf(load_elem(row, c)));
+    amax = block_amax(amax, red);
     float s = __fdiv_rn(amax, 127.0f);
     if (s == 0.0f)
         s = 1.0f;
     if (threadIdx.x == 0)
         scale[r] = s;
-    int sum = 0;
-    uint2* qrow = reinterpret_cast<uint2*>(q + r * C);
+    int8_t* qrow = q + r * C;
+    const float rs = __frcp_rn(s);
+    const bool fast = rcp_ok(s);
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x)
+        qrow[c] = static_cast<int8_t>(sym_code(load_elem(row, c), s, rs, fast));
+}
+
+// Single-pass variant for bf16 rows with C % 8 == 0 and C <= 256 * 8 * VPT: each
+// thread keeps its VPT 16-byte pieces of the row in registers between the
+// absmax reduction and the quantisation, so the row is read from memory once.
+template <int VPT>
+__global__ void __launch_bounds__(256) quantize_int8_rows_bf16_reg_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                         int64_t C, int8_t* __restrict__ q,
+                                                                         float* __restrict__ scale, int release)
+{
+    if (release)
+        pdl_launch_dependents();
+    __shared__ float red[8];
+    const int64_t r = blockIdx.x;
+    const uint4* row = reinterpret_cast<const uint4*>(w + r * C);
+    const int C8 = (int)(C / 8);
+    uint4 v[VPT];
+    float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
         const int c = (int)threadIdx.x + j * 256;
-        if (c < C8) {
-            const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-            uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t bits = (i & 1) ? (u[i / 2] & 0xffff0000u) : (u[i / 2] << 16);
-                float t = rintf(__fdiv_rn(__uint_as_float(bits), s));
-                t = fminf(fmaxf(t, -128.0f), 127.0f);
-                const int qi = static_cast<int>(t);
-                sum += qi;
-                packed[i / 4] |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * (i % 4));
-            }
-            qrow[c] = make_uint2(packed[0], packed[1]);
-        }
+        v[j] = c < C8 ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+        amax = amax8(v[j], amax);
     }
-    if (rowsum) {
+    amax = block_amax(amax, red);
+    float s = __fdiv_rn(amax, 127.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    if (threadIdx.x == 0)
+        scale[r] = s;
+    uint2* qrow = reinterpret_cast<uint2*>(q + r * C);
+    const float rs = __frcp_rn(s);
+    const bool fast = rcp_ok(s);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if ((threadIdx.x & 31) == 0)
-            ired[threadIdx.x / 32] = sum;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int t = 0;
-            for (int i = 0; i < 8; ++i)
-                t += ired[i];
-            rowsum[r] = t;
-        }
+    for (int j = 0; j < VPT; ++j) {
+        const int c = (int)threadIdx.x + j * 256;
+        if (c < C8)
+            qrow[c] = sym_codes8(v[j], s, rs, fast);
     }
 }
 
 // Vectorised variant for bf16 rows with C % 8 == 0 (16-byte loads, 8-byte stores).
 __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __nv_bfloat16* __restrict__ w,
                                                                         int64_t C, int8_t* __restrict__ q,
-                                                                        float* __restrict__ scale,
-                                                                        int32_t* __restrict__ rowsum, int release)
+                                                                        float* __restrict__ scale, int release)
 {
     if (release)
         pdl_launch_dependents();
     __shared__ float red[8];
-    __shared__ int ired[8];
     const int64_t r = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(w + r * C);
     const int64_t C8 = C / 8;
     float amax = 0.0f;
-    for (int64_t c = threadIdx.x; c < C8; c += blockDim.x) {
-        const uint4 v = __ldg(row + c);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] << 16)));
-            amax = fmaxf(amax, fabsf(__uint_as_float(u[i] & 0xffff0000u)));
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if ((threadIdx.x & 31) == 0)
-        red[threadIdx.x / 32] = amax;
-    __syncthreads();
-    amax = red[0];
-    for (int i = 1; i < (int)(blockDim.x / 32); ++i)
-        amax = fmaxf(amax, red[i]);
+    for (int64_t c = threadIdx.x; c < C8; c += blockDim.x)
+        amax = amax8(__ldg(row + c), amax);
+    amax = block_amax(amax, red);
     float s = __fdiv_rn(amax, 127.0f);
     if (s == 0.0f)
         s = 1.0f;
     if (threadIdx.x == 0)
         scale[r] = s;
-    int sum = 0;
     uint2* qrow = reinterpret_cast<uint2*>(q + r * C);
-    for (int64_t c = threadIdx.x; c < C8; c += blockDim.x) {
-        const uint4 v = __ldg(row + c);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-        uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t bits = (i & 1) ? (u[i / 2] & 0xffff0000u) : (u[i / 2] << 16);
-            float t = rintf(__fdiv_rn(__uint_as_float(bits), s));
-            t = fminf(fmaxf(t, -128.0f), 127.0f);
-            const int qi = static_cast<int>(t);
-            sum += qi;
-            packed[i / 4] |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * (i % 4));
-        }
-        qrow[c] = make_uint2(packed[0], packed[1]);
-    }
-    if (rowsum) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if ((threadIdx.x & 31) == 0)
-            ired[threadIdx.x / 32] = sum;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int t = 0;
-            for (int i = 0; i < (int)(blockDim.x / 32); ++i)
-                t += ired[i];
-            rowsum[r] = t;
-        }
-    }
+    const float rs = __frcp_rn(s);
+    const bool fast = rcp_ok(s);
+    for (int64_t c = threadIdx.x; c < C8; c += blockDim.x)
+        qrow[c] = sym_codes8(__ldg(row + c), s, rs, fast);
 }
 
 // ---------------------------------------------------------------- per-column int4
@@ -571,9 +635,11 @@ __global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW
     }
     __syncthreads();
     const float rc = row_clip_s, sc = scale_s;
+    const float rsc = __frcp_rn(sc);
+    const bool fast = rcp_ok(sc);
     for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
         const float v = fminf(fmaxf(to_float(row[c]), -rc), rc);
-        q[(int64_t)blockIdx.x * C + c] = (int8_t)fminf(fmaxf(rintf(__fdiv_rn(v, sc)), -128.f), 127.f);
+        q[(int64_t)blockIdx.x * C + c] = (int8_t)sym_code(v, sc, rsc, fast);
     }
 }
 
@@ -606,11 +672,55 @@ __global__ void __launch_bounds__(256) quantize_int8_groups_kernel(const TW* __r
     float sc = __fdiv_rn(amax, 127.0f);
     if (sc == 0.f)
         sc = 1.f;
+    const float rsc = __frcp_rn(sc);
+    const bool fast = rcp_ok(sc);
 #pragma unroll
     for (int i = 0; i < PER; ++i)
-        q[n * K + grp * G + i * 32 + lane] = (int8_t)fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -128.f), 127.f);
+        q[n * K + grp * G + i * 32 + lane] = (int8_t)sym_code(v[i], sc, rsc, fast);
     if (lane == 0)
         scale_w[grp * N + n] = sc;
+}
+
+// The same with G/16 lanes per group, 16 consecutive values each (16-byte loads, one 16-byte store
+// of the lane's int8 codes); 16-byte aligned w and q.
+template <typename TW, int G>
+__global__ void __launch_bounds__(256) quantize_int8_groups_vec_kernel(const TW* __restrict__ w, int64_t N, int64_t K,
+                                                                      int8_t* __restrict__ q,
+                                                                      float* __restrict__ scale_w)
+{
+    constexpr int LPG = G / 16;
+    const int64_t ng = K / G, groups = N * ng;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t gi = t / LPG;
+    const int sub = (int)(t % LPG);
+    // lanes past the last group take part in the butterfly on the last group and store nothing
+    const bool ok = gi < groups;
+    const int64_t gq = ok ? gi : groups - 1;
+    float v[16];
+    load16(w + gq * G + 16 * sub, v);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float sc = __fdiv_rn(amax, 127.0f);
+    if (sc == 0.f)
+        sc = 1.f;
+    const float rsc = __frcp_rn(sc);
+    const bool fast = rcp_ok(sc);
+    int c[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        c[i] = sym_code(v[i], sc, rsc, fast);
+    const uint32_t word[4] = {pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]),
+                              pack4(c[8], c[9], c[10], c[11]), pack4(c[12], c[13], c[14], c[15])};
+    if (ok) {
+        *reinterpret_cast<uint4*>(q + gi * G + 16 * sub) = make_uint4(word[0], word[1], word[2], word[3]);
+        if (sub == 0)
+            scale_w[(gi % ng) * N + gi / ng] = sc;
+    }
 }
 
 template <typename TW>
@@ -637,11 +747,13 @@ __global__ void __launch_bounds__(256) pack_int4_cols_kernel(const TW* __restric
         return;
     if (ty == 0)
         scale[n] = s;
+    const float rs = __frcp_rn(s);
+    const bool fast = rcp_ok(s);
     for (int64_t i = ty; i < K / 2; i += 8) {
         uint32_t c[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            float t = __fadd_rn(rintf(__fdiv_rn(load_elem(w, (2 * i + h) * N + n), s)), 8.0f);
+            float t = __fadd_rn(rint_div(load_elem(w, (2 * i + h) * N + n), s, rs, fast), 8.0f);
             t = fminf(fmaxf(t, 0.0f), 15.0f);
             c[h] = static_cast<uint32_t>(t);
         }
@@ -657,6 +769,18 @@ cudaError_t quantize_dispatch_g(const TW* w, int64_t N, int64_t K, int g, uint32
     const unsigned blocks = (unsigned)((groups + 7) / 8);
     // power-of-two widths never straddle a word: lanes share whole words
     constexpr bool pow2 = (BITS & (BITS - 1)) == 0;
+    if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
+        if ((reinterpret_cast<uintptr_t>(w) & 15u) == 0) {  // groups start 16-byte aligned (g >= 32)
+            const int64_t threads = groups * (g / 16);
+            const unsigned vb = (unsigned)((threads + 255) / 256);
+            switch (g) {
+            case 32: affine_quantize_vec_kernel<TW, TP, BITS, 32><<<vb, 256, 0, st>>>(w, groups, codes, s, b); break;
+            case 64: affine_quantize_vec_kernel<TW, TP, BITS, 64><<<vb, 256, 0, st>>>(w, groups, codes, s, b); break;
+            default: affine_quantize_vec_kernel<TW, TP, BITS, 128><<<vb, 256, 0, st>>>(w, groups, codes, s, b); break;
+            }
+            return cudaGetLastError();
+        }
+    }
     switch (g) {
     case 32:
         if constexpr (pow2)
@@ -720,14 +844,22 @@ cudaError_t dequantize_dispatch(const uint32_t* codes, const void* s, const void
     const TP* sp = static_cast<const TP*>(s);
     const TP* bp = static_cast<const TP*>(b);
     TO* op = static_cast<TO*>(out);
+    auto pow2 = [&](auto bits_c) {
+        constexpr int B = decltype(bits_c)::value;
+        switch (g) {
+        case 32: affine_dequantize_kernel<TP, TO, B, 32><<<blocks, 256, 0, st>>>(codes, sp, bp, words, op); break;
+        case 64: affine_dequantize_kernel<TP, TO, B, 64><<<blocks, 256, 0, st>>>(codes, sp, bp, words, op); break;
+        default: affine_dequantize_kernel<TP, TO, B, 128><<<blocks, 256, 0, st>>>(codes, sp, bp, words, op); break;
+        }
+    };
     switch (bits) {
     case 1: affine_dequantize_odd_kernel<TP, TO, 1><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
-    case 2: affine_dequantize_kernel<TP, TO, 2><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    case 2: pow2(std::integral_constant<int, 2>{}); break;
     case 3: affine_dequantize_odd_kernel<TP, TO, 3><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
-    case 4: affine_dequantize_kernel<TP, TO, 4><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    case 4: pow2(std::integral_constant<int, 4>{}); break;
     case 5: affine_dequantize_odd_kernel<TP, TO, 5><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
     case 6: affine_dequantize_odd_kernel<TP, TO, 6><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
-    default: affine_dequantize_kernel<TP, TO, 8><<<blocks, 256, 0, st>>>(codes, sp, bp, N, K, g, op); break;
+    default: pow2(std::integral_constant<int, 8>{}); break;
     }
     return cudaGetLastError();
 }
@@ -769,7 +901,7 @@ cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, 
 }
 
 cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
-                                      int32_t* rowsum, cudaStream_t st, const DeviceInfo&, bool release_dependents)
+                                      cudaStream_t st, const DeviceInfo&, bool release_dependents)
 {
     // The kernel itself starts only after its predecessor completes; with
     // release_dependents it lets the next (programmatic-dependent) kernel start
@@ -779,22 +911,22 @@ cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R,
                      (reinterpret_cast<uintptr_t>(q) & 7) == 0;
     if (vec && C <= 256 * 8 * 4)
         quantize_int8_rows_bf16_reg_kernel<4><<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
-                                                                          scale, rowsum, rel);
+                                                                          scale, rel);
     else if (vec && C <= 256 * 8 * 8)
         quantize_int8_rows_bf16_reg_kernel<8><<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
-                                                                          scale, rowsum, rel);
+                                                                          scale, rel);
     else if (vec)
         quantize_int8_rows_bf16x8_kernel<<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
-                                                                       scale, rowsum, rel);
+                                                                       scale, rel);
     else if (w_dt == QLIN_BF16)
         quantize_int8_rows_kernel<__nv_bfloat16>
-            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q, scale, rowsum, rel);
+            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q, scale, rel);
     else if (w_dt == QLIN_F16)
         quantize_int8_rows_kernel<__half>
-            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __half*>(w), C, q, scale, rowsum, rel);
+            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __half*>(w), C, q, scale, rel);
     else
         quantize_int8_rows_kernel<float><<<(unsigned)R, 256, 0, st>>>(static_cast<const float*>(w), C, q, scale,
-                                                                      rowsum, rel);
+                                                                      rel);
     return cudaGetLastError();
 }
 
@@ -821,9 +953,17 @@ cudaError_t launch_quantize_weight_int8_clip(const void* w, qlin_dtype w_dt, int
 cudaError_t launch_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int g, int8_t* q,
                                         float* scale_w, cudaStream_t st, const DeviceInfo&)
 {
+    const bool vec = ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(q)) & 15u) == 0;
     const unsigned blocks = (unsigned)((N * (K / g) + 7) / 8);
-#define QLIN_QG(TW, G) \
-    quantize_int8_groups_kernel<TW, G><<<blocks, 256, 0, st>>>(static_cast<const TW*>(w), N, K, q, scale_w)
+    const unsigned vblocks = (unsigned)((N * (K / g) * (g / 16) + 255) / 256);
+#define QLIN_QG(TW, G)                                                                                               \
+    do {                                                                                                             \
+        if (vec)                                                                                                     \
+            quantize_int8_groups_vec_kernel<TW, G>                                                                   \
+                <<<vblocks, 256, 0, st>>>(static_cast<const TW*>(w), N, K, q, scale_w);                              \
+        else                                                                                                         \
+            quantize_int8_groups_kernel<TW, G><<<blocks, 256, 0, st>>>(static_cast<const TW*>(w), N, K, q, scale_w); \
+    } while (0)
     if (w_dt == QLIN_BF16) {
         if (g == 64) QLIN_QG(__nv_bfloat16, 64); else if (g == 128) QLIN_QG(__nv_bfloat16, 128); else QLIN_QG(__nv_bfloat16, 256);
     } else if (w_dt == QLIN_F16) {

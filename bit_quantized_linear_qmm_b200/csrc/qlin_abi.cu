@@ -283,7 +283,7 @@ qlin_status qlin_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, i
     if ((s = current_device(dev)) != QLIN_OK)
         return s;
     return from_cuda(
-        launch_quantize_int8_rows(w, w_dt, R, C, q, scale, nullptr, static_cast<cudaStream_t>(stream), dev));
+        launch_quantize_int8_rows(w, w_dt, R, C, q, scale, static_cast<cudaStream_t>(stream), dev));
 }
 
 qlin_status qlin_pack_int4_cols(const void* w, qlin_dtype w_dt, int64_t K, int64_t N, uint8_t* packed, float* scale,
@@ -315,7 +315,7 @@ qlin_status qlin_quantize_weight_int8(const void* w, qlin_dtype w_dt, int64_t R,
         return s;
     if (clip_percentile < 0.0)  // no clip: the absmax rule
         return from_cuda(
-            launch_quantize_int8_rows(w, w_dt, R, C, q, scale, nullptr, static_cast<cudaStream_t>(stream), dev));
+            launch_quantize_int8_rows(w, w_dt, R, C, q, scale, static_cast<cudaStream_t>(stream), dev));
     if (C > 32768)  // the row is held in shared memory
         return QLIN_ERR_UNSUPPORTED;
     // numpy converts the percentile to the row's float32 before dividing by 100
@@ -449,7 +449,7 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
     float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)M * (size_t)K));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the quantiser lets the next kernel start its prologue (fetching the layer's weights) early
-    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, nullptr, st, dev, true);
+    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, st, dev, true);
     if (e != cudaSuccess)
         return from_cuda(e);
     if (M <= 16) {  // decode: weight-streaming GEMV on int8 mma.sync

@@ -17,7 +17,8 @@ def ql():
 
 @pytest.mark.parametrize("g", [64, 128, 256])
 @pytest.mark.parametrize("wdt", ["f32", "bf16"])
-def test_quantize_int8_groups_bit_exact(ql, orc, g, wdt):
+@pytest.mark.parametrize("aligned", [True, False])
+def test_quantize_int8_groups_bit_exact(ql, orc, g, wdt, aligned):
     w = synth.normal(41, (96, 1024), 0.02)
     w[3, 128:256] = 0.0           # zero groups -> scale 1
     w[5, 700] = 0.9               # one group dominated by an outlier
@@ -25,6 +26,9 @@ def test_quantize_int8_groups_bit_exact(ql, orc, g, wdt):
         w = torch.from_numpy(w).to(torch.bfloat16).float().numpy()
     q_ref, s_ref = orc.quantize_int8_groups(w, g)
     wt = torch.from_numpy(w).to(torch.bfloat16 if wdt == "bf16" else torch.float32).cuda()
+    if not aligned:  # data one element past a 16-byte boundary: the warp-per-group kernel
+        flat = torch.empty(wt.numel() + 1, dtype=wt.dtype, device="cuda")
+        wt = flat[1:].view(wt.shape).copy_(wt)
     q, s = ql.quantize_int8_groups(wt, g)
     torch.cuda.synchronize()
     assert np.array_equal(q.cpu().numpy(), q_ref)

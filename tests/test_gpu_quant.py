@@ -56,6 +56,48 @@ def test_dequantize_bit_exact(ql, orc, bits, g, p_dt, o_dt):
         assert np.array_equal(out.cpu().numpy(), ref)
 
 
+def _offset_copy(t, elems=1):
+    """A contiguous copy of t whose data starts `elems` elements past an allocation (not 16-byte
+    aligned): the quantiser and dequantiser then take their per-group / per-word kernels."""
+    flat = torch.empty(t.numel() + elems, dtype=t.dtype, device=t.device)
+    v = flat[elems:].view(t.shape)
+    v.copy_(t)
+    assert v.data_ptr() % 16 != 0
+    return v
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("w_dt", ["f32", "bf16"])
+def test_quantize_unaligned_weights_bit_exact(ql, orc, bits, w_dt):
+    g = 64
+    N, K = 9, 3 * g
+    w = synth.outlier_weights(150 + bits, N, K, frac=0.02)
+    wv, wd = _w_dev(w, w_dt)
+    codes, s, b = ql.quantize(_offset_copy(wd), bits, g, torch.float32)
+    torch.cuda.synchronize()
+    rc, rs, rb = orc.affine_quantize(wv, bits, g, False)
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), rc)
+    assert np.array_equal(host_f32(s), rs)
+    assert np.array_equal(host_f32(b), rb)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("aligned", [True, False])
+def test_dequantize_word_tail_and_unaligned_bit_exact(ql, orc, bits, aligned):
+    # K = g = 32: 32 * bits / 32 words per row; 53 rows give a word count that is not a multiple of 4
+    # for 2-bit codes (the vector kernel's tail); unaligned codes take the per-word kernel
+    g, N, K = 32, 53, 32
+    w = synth.normal(250 + bits, (N, K), 0.02)
+    rc, rs, rb = orc.affine_quantize(w, bits, g, True)
+    cd = u32_dev(rc)
+    if not aligned:
+        cd = _offset_copy(cd)
+    out = ql.dequantize(cd, params_dev(rs, "bf16"), params_dev(rb, "bf16"), K, bits, g, torch.bfloat16)
+    torch.cuda.synchronize()
+    ref = orc.affine_dequantize(rc, rs, rb, K, bits, g)
+    assert np.array_equal(host_bits16(out), orc.f32_to_bf16_bits(ref))
+
+
 @pytest.mark.parametrize("w_dt", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", [(1, 8192), (7, 1000), (33, 4096), (3, 24)])
 def test_quantize_int8_rows_bit_exact(ql, orc, w_dt, shape):
