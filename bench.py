@@ -695,6 +695,12 @@ def _prof_clip():
     return lambda: ql.quantize_weight_int8(w, 99.9)
 
 
+def _prof_int8_groups():
+    from bit_quantized_linear_qmm_b200 import qlin as ql
+    w = torch.from_numpy(synth.normal(61, (4096, 4096), 0.02)).cuda()
+    return lambda: ql.quantize_int8_groups(w, 128)
+
+
 def _prof_act_quant():
     from bit_quantized_linear_qmm_b200 import qlin as ql
     x = synth.INT_LINEAR[2].x().torch("cuda")
@@ -723,6 +729,7 @@ PROFILE_CASES = {
     "affine_quantize_bf16_n14336": _prof_quantize_bf16,
     "dequantize_n14336": _prof_dequantize,
     "clip_4096": _prof_clip,
+    "int8_groups_4096": _prof_int8_groups,
     "bitlinear_prefill_m2048": _prof_bitlinear_prefill,
     "pergroup_m2048": lambda: _prof_pergroup(2048),
     "pergroup_m1": lambda: _prof_pergroup(1),

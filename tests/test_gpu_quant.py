@@ -99,7 +99,7 @@ def test_dequantize_word_tail_and_unaligned_bit_exact(ql, orc, bits, aligned):
 
 
 @pytest.mark.parametrize("w_dt", ["f32", "bf16"])
-@pytest.mark.parametrize("shape", [(1, 8192), (7, 1000), (33, 4096), (3, 24)])
+@pytest.mark.parametrize("shape", [(1, 8192), (7, 1000), (33, 4096), (3, 24), (700, 1000), (1024, 8192), (600, 24)])
 def test_quantize_int8_rows_bit_exact(ql, orc, w_dt, shape):
     R, Cc = shape
     w = synth.normal(300 + R, (R, Cc), 1.0)
