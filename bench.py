@@ -834,7 +834,7 @@ def main():
     peak = float(peaks["hbm_gbs"])
     roofline = {"bound": wl.bound, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(wl.key),
-                "kernel": wl.key, "peak_source": f"{peaks['source']} hbm_gbs (of measured)"}
+                "kernel": wl.key, "peak_source": f"{peaks['source']} hbm_gbs (of {peaks['source']})"}
 
     wl.e2e_prepare()
     ms_e2e = time_windows(wl.e2e_step, max(1, min(args.steps, 1000)), args.warmup, barrier=barrier)["ms"]
