@@ -64,17 +64,13 @@ __device__ unsigned long long g_ts_trace[kTsTraceCtas * kTsTraceTiles * 4];
 namespace {
 
 constexpr int kTW = 128;            // weight rows (outputs n) per tile: MMA M
-constexpr int kTT = 256;            // tokens per tile: MMA N
 constexpr int kKE = 64;             // k per stage (128 bytes of bf16 x)
-constexpr int kXStages = 6;         // x ring depth
-constexpr int kAStages = 8;         // TMEM A ring depth
 constexpr int kACols = kKE / 2;     // TMEM columns of one A stage (two bf16 per column)
-constexpr int kXBytes = kTT * 128;  // one x stage
 constexpr int kXformWarps = 8;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kXformWarps + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;
-constexpr int kAccCols = kTT;       // A ring starts here
+constexpr int kXStagesMax = 6, kAStagesMax = 8;
 // Code formats of the A operand: CB = 4, the MLX affine 4-bit codes with a group scale and bias;
 // CB = 8, signed int8 weights with a group scale (the per-group INT8 format).  A transform thread
 // covers 32 k of one weight row per stage: 4 * CB bytes of codes, kept kCodePF(CB) stages ahead in
@@ -92,20 +88,16 @@ template <int CB> struct CodeFmt {
     static constexpr int kKPerCopy = CB == 4 ? 32 : 16;      // k covered by one 16-byte copy
 };
 constexpr int kGroupT = 4;          // token tiles that walk the weight tiles together
-// kind::f16: D f32, A and B f16 (format 0; bf16 = format 1 for the ternary format), both K-major,
-// N = 256, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-constexpr uint32_t kIdescBf16 = kIdesc | (1u << 7) | (1u << 10);
 
 // per transform thread, kPF stages of its code bytes: [stage][copy][transform thread] x 16 bytes
 constexpr int kCodeRing = 6 * kXformWarps * 32 * 16;
 static_assert(CodeFmt<4>::kPF * CodeFmt<4>::kCopies <= 6 && CodeFmt<8>::kPF * CodeFmt<8>::kCopies <= 6, "ring");
 
 struct Bars {
-    uint64_t xfull[kXStages];
-    uint64_t xempty[kXStages];
-    uint64_t afull[kAStages];
-    uint64_t aempty[kAStages];
+    uint64_t xfull[kXStagesMax];
+    uint64_t xempty[kXStagesMax];
+    uint64_t afull[kAStagesMax];
+    uint64_t aempty[kAStagesMax];
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t mma_done;
@@ -113,10 +105,31 @@ struct Bars {
     int abort_flag;
     int epi_abort;  // written by epilogue warps only: their common break decision
 };
-constexpr int kTokScaleBytes = kTT * 4;  // the epilogue's token scales of the current tile
-constexpr int kSmem = kXStages * kXBytes + kCodeRing + kTokScaleBytes + (int)sizeof(Bars) + 1024;
-static_assert(kSmem <= 227 * 1024, "shared memory");
-static_assert(kAccCols + kAStages * kACols <= kTmemCols, "tensor memory");
+// Tile shapes.  TT = 256 tokens: one 256-column accumulator, an 8-stage A ring and a 6-stage x
+// ring.  TT = 384 tokens: two 192-column accumulators (two MMAs of N = 192 per 16-wide k step on
+// the same A stage, so each decoded weight serves 384 tokens), a 4-stage A ring and a 4-stage x
+// ring of two 192-row boxes per stage -- for shapes where it takes fewer rounds of tiles over the
+// SMs (the weight decode, not the MMA, bounds a stage).
+template <int TT> struct TsCfg {
+    static constexpr int kTT = TT;                        // tokens per tile
+    static constexpr int kNMma = TT == 384 ? 2 : 1;       // MMAs (accumulators) per 16-wide k step
+    static constexpr int kNT = TT / kNMma;                // MMA N; also the x TMA box rows
+    static constexpr int kXStages = TT == 384 ? 4 : 6;    // x ring depth
+    static constexpr int kAStages = TT == 384 ? 4 : 8;    // TMEM A ring depth
+    static constexpr int kXBytes = TT * 128;              // one x stage
+    static constexpr int kAccCols = TT;                   // A ring starts here
+    static constexpr int kTokScaleBytes = TT * 4;         // the epilogue's token scales of a tile
+    static constexpr int kSmem = kXStages * kXBytes + kCodeRing + kTokScaleBytes + (int)sizeof(Bars) + 1024;
+    // kind::f16: D f32, A and B f16 (format 0; bf16 = format 1 for the ternary format), both
+    // K-major, N = kNT, M = 128
+    static constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kNT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    static constexpr uint32_t kIdescBf16 = kIdesc | (1u << 7) | (1u << 10);
+    static_assert(TT == 256 || TT == 384, "tile widths");
+    static_assert(kXStages <= kXStagesMax && kAStages <= kAStagesMax, "barrier slots");
+    static_assert(kSmem <= 227 * 1024, "shared memory");
+    static_assert(kAccCols + kAStages * kACols <= kTmemCols, "tensor memory");
+    static_assert(kNT % 16 == 0 && kNT <= 256 && (kNT * 128) % 1024 == 0, "MMA N and box alignment");
+};
 
 struct TsParams {
     CUtensorMap tm_x;                 // x16 [M][K] fp16 (workspace), box {64, 256}, 128-byte swizzle
@@ -207,16 +220,19 @@ QLIN_DEV void tile_coords(int t, int tiles_t, int tiles_w, int& tt, int& wt)
     wt = r / gt;
 }
 
-template <int CB>
+template <int CB, int TT>
 __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_constant__ TsParams p)
 {
     using F = CodeFmt<CB>;
+    using C = TsCfg<TT>;
+    constexpr int kTT = C::kTT, kXStages = C::kXStages, kAStages = C::kAStages, kXBytes = C::kXBytes;
+    constexpr int kAccCols = C::kAccCols;
     constexpr int kCodePF = F::kPF;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint4* code_ring = reinterpret_cast<uint4*>(smem + kXStages * kXBytes);
     float* tok_s = reinterpret_cast<float*>(smem + kXStages * kXBytes + kCodeRing);
-    Bars& bars = *reinterpret_cast<Bars*>(smem + kXStages * kXBytes + kCodeRing + kTokScaleBytes);
+    Bars& bars = *reinterpret_cast<Bars*>(smem + kXStages * kXBytes + kCodeRing + C::kTokScaleBytes);
     auto X = [&](int s) { return smem + s * kXBytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -267,7 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                         break;
                     }
                     mbar_arrive_expect_tx(&bars.xfull[slot], kXBytes);
-                    tma_load_2d(X(slot), &p.tm_x, kb * kKE, tt * kTT, &bars.xfull[slot]);
+#pragma unroll
+                    for (int b = 0; b < C::kNMma; ++b)  // boxes of kNT token rows
+                        tma_load_2d(X(slot) + b * C::kNT * 128, &p.tm_x, kb * kKE, tt * kTT + b * C::kNT,
+                                    &bars.xfull[slot]);
                     if (++slot == kXStages) {
                         slot = 0;
                         ph ^= 1u;
@@ -299,8 +318,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                     const uint32_t b0 = smem_u32(X(xs));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_ts(tmem, tmem + (uint32_t)(kAccCols + as * kACols + kk * 8), umma_desc_sw128(b0 + kk * 32),
-                                  CodeFmt<CB>::kTernary ? kIdescBf16 : kIdesc, (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+                        for (int b = 0; b < C::kNMma; ++b)  // accumulator b: tokens b kNT .. +kNT-1
+                            tc_mma_ts(tmem + (uint32_t)(b * C::kNT), tmem + (uint32_t)(kAccCols + as * kACols + kk * 8),
+                                      umma_desc_sw128(b0 + b * C::kNT * 128 + kk * 32),
+                                      CodeFmt<CB>::kTernary ? C::kIdescBf16 : C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
                     tc_commit(&bars.xempty[xs]);
                     tc_commit(&bars.aempty[as]);
                     if (++xs == kXStages) {
@@ -557,8 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_affine_ts_kernel(const __grid_
                     rs = p.row_scale[n];
                 }
             }
-            if constexpr (!F::kTernary)  // the workspace holds token scales for whole 256-token tiles
-                tok_s[et] = __ldg(p.tok_scale + tt * kTT + et);
+            if constexpr (!F::kTernary) {  // the tile's token scales (zero past the last token)
+                for (int i = et; i < kTT; i += kEpiWarps * 32)
+                    tok_s[i] = tt * kTT + i < p.M ? __ldg(p.tok_scale + tt * kTT + i) : 0.f;
+            }
             epi_bar();  // the tile's token scales are in shared memory
             // the epilogue warps meet at named barriers, so they break together: a warp whose wait
             // failed (or that saw another role stop) records it in epi_abort, which only they write,
@@ -828,14 +852,24 @@ size_t tc_affine_workspace(int64_t M, int64_t N, int64_t K, int g)
 {
     auto a256 = [](size_t v) { return (v + 255) & ~size_t(255); };
     const size_t ng = (size_t)(K / g);
-    const size_t mt = (size_t)(M + kTT - 1) / kTT * kTT;  // token scales of whole tiles (read in 16s)
+    const size_t mt = (size_t)(M + 255) / 256 * 256;  // token scales (the epilogue reads none past M)
     return a256((size_t)M * K * 2) + 2 * a256((size_t)N * ng * 2) + a256(mt * 4) + a256((size_t)N * 4);
 }
 
 namespace {
 
+// 384-token tiles when they take fewer rounds of tiles over the SMs than 256-token ones (e.g.
+// 2048 tokens x 112 weight tiles: 5 rounds instead of 7), else 256
+int tile_tokens(int64_t M, int tiles_w, const DeviceInfo& dev)
+{
+    auto rounds = [&](int tt) { return ((M + tt - 1) / tt * tiles_w + dev.sm_count - 1) / dev.sm_count; };
+    return rounds(384) < rounds(256) ? 384 : 256;
+}
+
+template <int TT>
 cudaError_t launch_ts(void (*kern)(TsParams), const TsParams& prm, cudaStream_t st, const DeviceInfo& dev)
 {
+    constexpr int kSmem = TsCfg<TT>::kSmem;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess)
         return e;
@@ -872,22 +906,24 @@ cudaError_t launch_tc_bitlinear(const BitlinearArgs& a, cudaStream_t st, const D
     prm.R = (int)(a.N / 4);
     prm.g_shift = 0;
     prm.ng = 1;
-    prm.tiles_t = (int)((a.M + kTT - 1) / kTT);
     prm.tiles_w = (prm.R + 31) / 32;
+    const int tt = tile_tokens(a.M, prm.tiles_w, dev);
+    prm.tiles_t = (int)((a.M + tt - 1) / tt);
     prm.vec_params = 0;
     prm.weight_scale = a.weight_scale;
     prm.invert = a.invert;
     prm.status = dev.status;
     if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
-                        (uint64_t)a.K * 2, kKE, kTT))
+                        (uint64_t)a.K * 2, kKE, tt == 384 ? TsCfg<384>::kNT : TsCfg<256>::kNT))
         return cudaErrorInvalidValue;
-    return launch_ts(tc_affine_ts_kernel<2>, prm, st, dev);
+    return tt == 384 ? launch_ts<384>(tc_affine_ts_kernel<2, 384>, prm, st, dev)
+                     : launch_ts<256>(tc_affine_ts_kernel<2, 256>, prm, st, dev);
 }
 
 cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
     // workspace: x16 [M][K], s16 / b16 [N][ng] (fp16), tok_scale [M rounded up to 256 tokens],
-    // row_scale [N] (fp32)
+    // row_scale [N] (fp32) -- the layout tc_affine_workspace sizes
     auto a256 = [](size_t v) { return (v + 255) & ~size_t(255); };
     const int ng = (int)(a.K / a.g);
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
@@ -895,7 +931,7 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     __half* s16 = reinterpret_cast<__half*>(ws + a256((size_t)a.M * a.K * 2));
     __half* b16 = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(s16) + a256((size_t)a.N * ng * 2));
     float* tok_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(b16) + a256((size_t)a.N * ng * 2));
-    const size_t mt = (size_t)(a.M + kTT - 1) / kTT * kTT;
+    const size_t mt = (size_t)(a.M + 255) / 256 * 256;
     float* row_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(tok_scale) + a256(mt * 4));
     {
         const unsigned blocks = (unsigned)(a.M + (a.N + 7) / 8);
@@ -940,17 +976,20 @@ cudaError_t launch_tc_affine(const TcGemmArgs& a, cudaStream_t st, const DeviceI
     while ((1 << prm.g_shift) < a.g)
         ++prm.g_shift;
     prm.ng = (int)(a.K / a.g);
-    prm.tiles_t = (int)((a.M + kTT - 1) / kTT);
     prm.tiles_w = (int)((a.N + kTW - 1) / kTW);
+    const int tt = tile_tokens(a.M, prm.tiles_w, dev);
+    prm.tiles_t = (int)((a.M + tt - 1) / tt);
     prm.vec_params = prm.ng % 8 == 0;  // workspace rows are then 16-byte aligned
     prm.status = dev.status;
     if (!encode_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)a.K, (uint64_t)a.M,
-                        (uint64_t)a.K * 2, kKE, kTT))
+                        (uint64_t)a.K * 2, kKE, tt == 384 ? TsCfg<384>::kNT : TsCfg<256>::kNT))
         return cudaErrorInvalidValue;
     prm.weight_scale = nullptr;
     prm.invert = 0;
     prm.R = 0;
-    return launch_ts(a.bits == 8 ? tc_affine_ts_kernel<8> : tc_affine_ts_kernel<4>, prm, st, dev);
+    if (tt == 384)
+        return launch_ts<384>(a.bits == 8 ? tc_affine_ts_kernel<8, 384> : tc_affine_ts_kernel<4, 384>, prm, st, dev);
+    return launch_ts<256>(a.bits == 8 ? tc_affine_ts_kernel<8, 256> : tc_affine_ts_kernel<4, 256>, prm, st, dev);
 }
 
 }  // namespace qlin

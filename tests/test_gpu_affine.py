@@ -143,7 +143,10 @@ PREFILL_SMALL = [
                              # short K: few terms, little cancellation -- the products' own error must meet the bar
                              (1280, 128, 4096, 32, "bf16"), (300, 64, 520, 32, "bf16"), (64, 128, 128, 64, "bf16"),
                              # fp32 x (and output, bias) through the same fp16 tensor-core path
-                             (100, 512, 384, 64, "f32"), (33, 128, 64, 128, "f32")]
+                             (100, 512, 384, 64, "f32"), (33, 128, 64, 128, "f32"),
+                             # 384-token tiles (two 192-column accumulators): 1280 tokens -> 4 x 32 tiles
+                             # instead of 5 x 32 on 148 SMs; 1100 leaves a last tile of 332 tokens
+                             (1100, 256, 4096, 64, "bf16"), (1100, 128, 4096, 32, "f32")]
 ]
 @pytest.mark.parametrize("case", PREFILL_SMALL, ids=[c.name for c in PREFILL_SMALL])
 def test_affine_prefill_small(ql, orc, case):

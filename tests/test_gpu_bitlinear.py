@@ -104,7 +104,10 @@ PREFILL = [synth.BitLinearCase(f"prefill_M{M}_K{K}_N{N}_{'div' if inv else 'mul'
            for (M, K, N, inv, b, ab) in [(300, 1040, 600, False, True, True),   # K % 32 == 16, ragged tiles
                                          (256, 512, 4096, True, False, False),
                                          (33, 2048, 136, False, False, True),
-                                         (512, 4096, 512, False, True, False)]]
+                                         (512, 4096, 512, False, True, False),
+                                         # 384-token tiles (4 x 32 tiles instead of 5 x 32 on 148 SMs):
+                                         # the last tile holds 332 tokens, its second 192-row box 140
+                                         (1100, 512, 4096, False, True, False)]]
 
 
 @pytest.mark.parametrize("case", PREFILL, ids=[c.name for c in PREFILL])
