@@ -248,24 +248,34 @@ class BitlinearDecode:
 
     def e2e_prepare(self):
         """The step's inputs (x of the 4 layers) in one pinned host buffer and its results (y) in
-        another, so each step moves them with one copy each way; the layers read and write views
-        of the matching device buffers."""
+        another, so each step moves them with one copy each way.  Two device copies of the input
+        buffer: while a step runs its 4 layers on one, the next step's input is copied into the
+        other on a side stream; the step then reads its own result back.  Every step still moves
+        exactly its input in and its result out."""
         nx = [x.numel() for x in self.xs]
         ny = [y.numel() for y in self.ys]
         self.hx = torch.cat([x.reshape(-1).cpu() for x in self.xs]).pin_memory()
-        self.dx = torch.empty_like(self.hx, device="cuda")
+        self.dx2 = [torch.empty_like(self.hx, device="cuda") for _ in range(2)]
         self.hy = torch.empty(sum(ny), dtype=self.ys[0].dtype).pin_memory()
         self.dy = torch.empty_like(self.hy, device="cuda")
-        self.xs = [v.view(c.M, c.K) for v, c in zip(torch.split(self.dx, nx), self.cases)]
+        self.xs2 = [[v.view(c.M, c.K) for v, c in zip(torch.split(d, nx), self.cases)] for d in self.dx2]
         self.ys = [v.view(c.M, c.N) for v, c in zip(torch.split(self.dy, ny), self.cases)]
-        self.dx.copy_(self.hx)
+        for d in self.dx2:
+            d.copy_(self.hx)
+        self.side = torch.cuda.Stream()
         self.h2d = self.hx.numel() * self.hx.element_size()
         self.d2h = self.hy.numel() * self.hy.element_size()
 
     def e2e_step(self, i: int):
-        self.dx.copy_(self.hx, non_blocking=True)
+        cur = torch.cuda.current_stream()
+        b = i % 2
+        self.side.wait_stream(cur)  # the other input buffer was last read by the previous step
+        with torch.cuda.stream(self.side):
+            self.dx2[1 - b].copy_(self.hx, non_blocking=True)  # the next step's input
+        self.xs = self.xs2[b]
         self.step(i)
-        self.hy.copy_(self.dy, non_blocking=True)
+        self.hy.copy_(self.dy, non_blocking=True)  # this step's result
+        cur.wait_stream(self.side)
 
 
 def cpu_bitlinear_step():
