@@ -548,7 +548,7 @@ def suite(l2: int, peaks: dict, int8_peak: float):
                       hbm, "reads fp32 W, writes int8 + scales"))
     t = tw(lambda i: ql.quantize_weight_int8(wf, 99.9), 5, 2)
     out.append(_entry("quantize_weight_int8_clip99.9_4096x4096", t, wf.numel() * 5 + 4096 * 4, "GB/s", "hbm", hbm,
-                      "per-row percentile: a radix select of each row's order statistics in shared memory"))
+                      "per-row percentile: an 11-bit histogram and a counted bin (radix select for dense bins) per row in shared memory"))
     del wf
     pgb = qg.numel() + sg_.numel() * 4
     pool = [(qg.clone(), sg_.clone()) for _ in range(_copies(pgb, l2, 4))]

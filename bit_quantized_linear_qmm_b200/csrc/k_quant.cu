@@ -507,10 +507,14 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __
 // One CTA per row [cider/ops.py quantize_weight_int8, clip_percentile]: the clip is the
 // linear-interpolated percentile of |w| at h = (C - 1) p / 100, which needs only the order
 // statistics v_(j) and v_(j+1), j = floor(h).  |w| of the row is held in shared memory as uint32
-// bit patterns (non-negative floats order like their bits); v_(j) is found by a radix select (four
+// bit patterns (non-negative floats order like their bits).  First one pass builds a 2048-bin
+// histogram of the top 11 bits (the exponent and three mantissa bits) and a block scan finds the
+// bin B holding rank j; when B holds at most 256 values they are gathered and ranked by counting
+// (v_(j) and, inside B, v_(j+1); past B, v_(j+1) is the smallest value of a higher bin, a minimum
+// taken in the same gather pass).  A denser bin takes the general route: a radix select (four
 // passes of a 256-bin histogram of one byte, most significant first, over the values that match
-// the bytes found so far) and v_(j+1) is v_(j) again when more than j + 1 values are <= it, else
-// the smallest value above it.  The interpolation runs in float32 with every operation rounded
+// the bytes found so far), with v_(j+1) = v_(j) again when more than j + 1 values are <= it, else
+// the smallest value above it.  Both routes select on the same bit patterns.  The interpolation runs in float32 with every operation rounded
 // separately (as numpy does it for a float32 row), 0 -> max |w|; then scale = clip / 127 (zero ->
 // 1), w clipped to [-clip, clip], q = clip(round(w / scale), -128, 127) with IEEE divisions.
 template <typename TW>
@@ -518,19 +522,23 @@ __global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW
                                                                        float pct, int8_t* __restrict__ q,
                                                                        float* __restrict__ scale)
 {
-    extern __shared__ uint32_t sv[];  // [C] bit patterns of |w|
+    extern __shared__ uint32_t sv[];  // [C] fp32 bit patterns of w (|w| is the pattern & 0x7FFFFFFF)
     __shared__ unsigned hist[256];
+    __shared__ unsigned hist11[2048];  // by the top 11 bits of the pattern (bit 31 is 0)
+    __shared__ uint32_t cand[256];     // the values of bin B (fast route)
+    __shared__ unsigned wsum[8];
     __shared__ uint32_t sel_s, rank_s;
     __shared__ unsigned cnt_le_s;
-    __shared__ uint32_t next_s, max_s;
+    __shared__ uint32_t next_s, max_s, vj_s, vj1_s;
+    __shared__ unsigned fbin_s, frank_s, fcnt_s, gcount_s;
     __shared__ float row_clip_s, scale_s;
     const int n = (int)C;
     const TW* row = w + (int64_t)blockIdx.x * C;
     uint32_t mx = 0u;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const uint32_t b = __float_as_uint(fabsf(to_float(row[i])));
+        const uint32_t b = __float_as_uint(to_float(row[i]));
         sv[i] = b;
-        mx = max(mx, b);
+        mx = max(mx, b & 0x7FFFFFFFu);
     }
     // the rank of v_(j): j = floor((n - 1) q) when that is below n - 1 (else the maximum is used)
     const float qq = __fdiv_rn(pct, 100.0f);
@@ -543,11 +551,84 @@ __global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW
         max_s = 0u;
         next_s = 0xFFFFFFFFu;
         cnt_le_s = 0u;
+        gcount_s = 0u;
+        fcnt_s = 0xFFFFFFFFu;
     }
+    for (int b = threadIdx.x; b < 2048; b += blockDim.x)
+        hist11[b] = 0u;
     __syncthreads();
     atomicMax(&max_s, mx);
-    // radix select of v_(j), one byte per pass from the top
-    for (int pass = 3; pass >= 0; --pass) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        atomicAdd(&hist11[(sv[i] & 0x7FFFFFFFu) >> 20], 1u);
+    __syncthreads();
+    {  // block scan of the bins (thread t: bins 8t .. 8t+7) to the bin holding rank j
+        unsigned c8[8], tot = 0u;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            c8[b] = hist11[8 * threadIdx.x + b];
+            tot += c8[b];
+        }
+        const int ln = threadIdx.x & 31, wp = threadIdx.x >> 5;
+        unsigned inc = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
+            if (ln >= o)
+                inc += t;
+        }
+        if (ln == 31)
+            wsum[wp] = inc;
+        __syncthreads();
+        for (int k = 0; k < wp; ++k)
+            inc += wsum[k];
+        const unsigned excl = inc - tot, r = (unsigned)j;
+        if (r >= excl && r < inc) {  // exactly one thread
+            unsigned rr = r - excl;
+            int b = 0;
+            for (; b < 7; ++b) {
+                if (rr < c8[b])
+                    break;
+                rr -= c8[b];
+            }
+            fbin_s = 8u * threadIdx.x + (unsigned)b;
+            frank_s = rr;
+            fcnt_s = c8[b];
+        }
+    }
+    __syncthreads();
+    const bool fast = fcnt_s <= 256u;  // the same for every thread
+    if (fast) {
+        const uint32_t B = fbin_s;
+        uint32_t nx = 0xFFFFFFFFu;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint32_t v = sv[i] & 0x7FFFFFFFu;
+            if ((v >> 20) == B)
+                cand[atomicAdd(&gcount_s, 1u)] = v;
+            else if ((v >> 20) > B)
+                nx = min(nx, v);
+        }
+        atomicMin(&next_s, nx);
+        __syncthreads();
+        const unsigned cn = fcnt_s, rr = frank_s;
+        if (threadIdx.x < cn) {  // rank by counting: v sits at ranks [less, less + eq) of bin B
+            const uint32_t e = cand[threadIdx.x];
+            unsigned less = 0u, eq = 0u;
+            for (unsigned u = 0; u < cn; ++u) {
+                const uint32_t o = cand[u];
+                less += o < e ? 1u : 0u;
+                eq += o == e ? 1u : 0u;
+            }
+            if (less <= rr && rr < less + eq)
+                vj_s = e;
+            if (rr + 1 < cn && less <= rr + 1 && rr + 1 < less + eq)
+                vj1_s = e;
+        }
+        if (threadIdx.x == 0 && rr + 1 >= cn)
+            vj1_s = next_s;  // v_(j+1) is the smallest value of a higher bin
+        __syncthreads();
+    }
+    // radix select of v_(j), one byte per pass from the top (bins denser than 256 values)
+    for (int pass = 3; pass >= 0 && !fast; --pass) {
         const int sh = 8 * pass;
         const uint32_t hi_mask = pass == 3 ? 0u : 0xFFFFFFFFu << (sh + 8);
         for (int b = threadIdx.x; b < 256; b += blockDim.x)
@@ -555,7 +636,7 @@ __global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW
         __syncthreads();
         const uint32_t prefix = sel_s;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const uint32_t v = sv[i];
+            const uint32_t v = sv[i] & 0x7FFFFFFFu;
             if ((v & hi_mask) == prefix) {
                 // one shared atomic per distinct byte in the warp (the top bytes of a row's |w|
                 // are nearly all equal: per-lane atomics would serialise)
@@ -598,27 +679,33 @@ __global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW
         }
         __syncthreads();
     }
-    const uint32_t vj = sel_s;
-    // v_(j+1): vj again when more than j + 1 values are <= vj, else the smallest value above it
-    {
+    if (!fast) {
+        // v_(j+1): vj again when more than j + 1 values are <= vj, else the smallest value above it
+        const uint32_t vj = sel_s;
         unsigned c = 0u;
         uint32_t nx = 0xFFFFFFFFu;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const uint32_t v = sv[i];
+            const uint32_t v = sv[i] & 0x7FFFFFFFu;
             c += v <= vj ? 1u : 0u;
             if (v > vj)
                 nx = min(nx, v);
         }
         atomicAdd(&cnt_le_s, c);
         atomicMin(&next_s, nx);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            vj_s = vj;
+            vj1_s = cnt_le_s > (unsigned)(j + 1) ? vj : next_s;
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
+        const uint32_t vj = vj_s;
         float r;
         if (!interior) {
             r = __uint_as_float(vj);  // the largest value
         } else {
-            const uint32_t vj1 = cnt_le_s > (unsigned)(j + 1) ? vj : next_s;
+            const uint32_t vj1 = vj1_s;
             const float t = __fsub_rn(h, floorf(h));
             const float a = __uint_as_float(vj), b = __uint_as_float(vj1);
             const float d = __fsub_rn(b, a);
@@ -636,10 +723,10 @@ __global__ void __launch_bounds__(256) quantize_weight_int8_clip_kernel(const TW
     __syncthreads();
     const float rc = row_clip_s, sc = scale_s;
     const float rsc = __frcp_rn(sc);
-    const bool fast = rcp_ok(sc);
-    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
-        const float v = fminf(fmaxf(to_float(row[c]), -rc), rc);
-        q[(int64_t)blockIdx.x * C + c] = (int8_t)sym_code(v, sc, rsc, fast);
+    const bool mul_ok = rcp_ok(sc);
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {  // the row from shared memory
+        const float v = fminf(fmaxf(__uint_as_float(sv[c]), -rc), rc);
+        q[(int64_t)blockIdx.x * C + c] = (int8_t)sym_code(v, sc, rsc, mul_ok);
     }
 }
 

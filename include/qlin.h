@@ -251,8 +251,9 @@ qlin_status w4a8_linear(const void* x, qlin_dtype x_dt, int64_t M, int64_t K,
  * float32 row), replaced by max |w| when 0; scale = clip / 127 (zero -> 1);
  * w clipped to [-clip, clip]; q = clip(round_half_even(w / scale), -128, 127).
  * w: [R, C] of w_dt; q: int8 [R, C]; scale: fp32 [R].  The clip path holds a
- * row in shared memory (a radix select finds the two order statistics the
- * interpolation needs): C <= 32768 (QLIN_ERR_UNSUPPORTED otherwise);
+ * row in shared memory (a histogram of its top bits, then a count or a radix
+ * select inside the bin, finds the two order statistics the interpolation
+ * needs): C <= 32768 (QLIN_ERR_UNSUPPORTED otherwise);
  * p > 100 or NaN -> QLIN_ERR_INVALID_ARG.  Bit-exact.
  */
 qlin_status qlin_quantize_weight_int8(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, double clip_percentile,
