@@ -171,13 +171,36 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             pdl_launch_dependents();
+            auto load_b = [&](int slot, int kb, int nt) {
+                if constexpr (BSRC == B_TMA_I8)
+                    tma_load_2d(RAW(slot), &p.tm_b, kb * 128, nt * BN, &bars.full[slot]);
+                else
+                    tma_load_2d(RAW(slot), &p.tm_b, nt * BN, kb * (Cfg::KE / 2), &bars.full[slot]);
+            };
+            // W8A8 / W4A8: a layer's weights are not written by the previous kernels of the stream
+            // (the ordering rule), so the first stages' weight boxes go out before the dependency
+            // wait and stream while the activation quantiser runs; the raw int8 GEMM's B may be
+            // an activation and waits first
+            int pre = 0, mt0 = 0, nt0 = 0;
+            if (EPI == E_SCALED && my_tiles > 0) {
+                tile_coords((int)blockIdx.x, p.tiles_m, p.tiles_n, mt0, nt0);
+                pre = nk < Cfg::NS ? nk : Cfg::NS;
+                for (int kb = 0; kb < pre; ++kb) {
+                    mbar_arrive_expect_tx(&bars.full[kb], Cfg::A_BYTES + Cfg::RAW_BYTES);
+                    load_b(kb, kb, nt0);
+                }
+            }
             pdl_wait_prior_grids();  // A (activations) may come from the previous kernel
+            for (int kb = 0; kb < pre; ++kb)
+                tma_load_2d(A(kb), &p.tm_a, kb * Cfg::KE, mt0 * kBM, &bars.full[kb]);
             int it = 0;
             for (int ti = 0; ti < my_tiles && !aborted(&bars.abort_flag); ++ti) {
                 int mt, nt;
                 tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
                 int kb = 0;
                 for (; kb < nk; ++kb, ++it) {
+                    if (it < pre)
+                        continue;  // issued above (the first stages of tile 0)
                     const int slot = it % Cfg::NS;
                     if (it >= Cfg::NS && !mbar_wait_bounded(&bars.empty[slot], ((it / Cfg::NS) & 1) ^ 1, p.status)) {
                         bars.abort_flag = 1;
@@ -185,10 +208,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                     }
                     mbar_arrive_expect_tx(&bars.full[slot], Cfg::A_BYTES + Cfg::RAW_BYTES);
                     tma_load_2d(A(slot), &p.tm_a, kb * Cfg::KE, mt * kBM, &bars.full[slot]);
-                    if constexpr (BSRC == B_TMA_I8)
-                        tma_load_2d(RAW(slot), &p.tm_b, kb * 128, nt * BN, &bars.full[slot]);
-                    else
-                        tma_load_2d(RAW(slot), &p.tm_b, nt * BN, kb * (Cfg::KE / 2), &bars.full[slot]);
+                    load_b(slot, kb, nt);
                 }
                 if (kb < nk)
                     break;
@@ -357,7 +377,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         constexpr int UNITS = 64 * CPR / (32 * Cfg::XW);    // chunks per thread per stage
         static_assert(UNITS * 32 * Cfg::XW == 64 * CPR, "transform split");
         const uint32_t kHi = 0xF0F0F0F0u, kSign = 0x80808080u;
-        pdl_wait_prior_grids();  // the packed weights may come from the previous kernel
+        pdl_wait_prior_grids();  // (a stage is complete only once its activations have landed too)
         // one stage: RAW(slot) -> BT(it % kBDepth)
         // ring positions of stage it: slot / phase of the code ring, buffer / phase of the operand ring
         int slot = 0, bslot = 0;

@@ -45,8 +45,11 @@
  *     call, the activation quantiser that opens each w8a8 / w4a8 call or
  *     the preparation kernel that opens a qlin_matmul prefill, a
  *     copy, an event wait, another library's kernel -- because such an
- *     operation starts only after everything before it has completed and
- *     releases nothing early.
+ *     operation starts only after everything before it has completed.  (The
+ *     activation quantiser and the preparation kernel do let the second
+ *     kernel of their own call start early: it fetches the call's weights
+ *     meanwhile and reads the quantiser's or preparation's output only after
+ *     its wait.)
  *   - Every call validates its arguments before launching anything and
  *     returns a qlin_status; nothing is launched when it is not QLIN_OK.
  *     No C++ exception crosses this interface.
