@@ -144,9 +144,11 @@ PREFILL_SMALL = [
                              (1280, 128, 4096, 32, "bf16"), (300, 64, 520, 32, "bf16"), (64, 128, 128, 64, "bf16"),
                              # fp32 x (and output, bias) through the same fp16 tensor-core path
                              (100, 512, 384, 64, "f32"), (33, 128, 64, 128, "f32"),
-                             # 384-token tiles (two 192-column accumulators): 1280 tokens -> 4 x 32 tiles
-                             # instead of 5 x 32 on 148 SMs; 1100 leaves a last tile of 332 tokens
-                             (1100, 256, 4096, 64, "bf16"), (1100, 128, 4096, 32, "f32")]
+                             # 384-token tiles (two 192-column accumulators), taken when they need fewer
+                             # tile rounds: 1100 tokens x 32 weight tiles -> 3 x 32 (1 round instead of 2),
+                             # the last tile holding 332 tokens; 740 x 112 -> 2 x 112 (2 rounds, not 3)
+                             (1100, 256, 4096, 64, "bf16"), (1100, 128, 4096, 32, "f32"),
+                             (740, 64, 14336, 64, "bf16")]
 ]
 @pytest.mark.parametrize("case", PREFILL_SMALL, ids=[c.name for c in PREFILL_SMALL])
 def test_affine_prefill_small(ql, orc, case):

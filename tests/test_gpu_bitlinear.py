@@ -105,8 +105,8 @@ PREFILL = [synth.BitLinearCase(f"prefill_M{M}_K{K}_N{N}_{'div' if inv else 'mul'
                                          (256, 512, 4096, True, False, False),
                                          (33, 2048, 136, False, False, True),
                                          (512, 4096, 512, False, True, False),
-                                         # 384-token tiles (4 x 32 tiles instead of 5 x 32 on 148 SMs):
-                                         # the last tile holds 332 tokens, its second 192-row box 140
+                                         # 384-token tiles (3 x 32 tiles instead of 5 x 32 of 256 on 148
+                                         # SMs): the last holds 332 tokens, its second 192-row box 140
                                          (1100, 512, 4096, False, True, False)]]
 
 

@@ -69,8 +69,8 @@ def test_pergroup_llm_shape_sampled_rows(ql, orc, M):
     _case(ql, orc, M, 4096, 4096, 128, "bf16", True, seed=47, rows=rows)
 
 
-def test_pergroup_384_token_tiles(ql, orc):
-    """1100 tokens, N = 4096: 4 x 32 tiles of 384 tokens (two 192-column accumulators) instead of
+def test_pergroup_two_accumulator_tiles(ql, orc):
+    """1100 tokens, N = 4096: 3 x 32 tiles of 384 tokens (two 192-column accumulators) instead of
     5 x 32 of 256 on 148 SMs; the last tile holds 332 tokens.  256 sampled output rows."""
     rng = np.random.default_rng(5)
     rows = np.sort(rng.choice(4096, size=256, replace=False))
