@@ -8,22 +8,24 @@
 //   W4A8:      y[m,n] = acc * s_x[m] * s_w[n] (+ bias[n]),   acc = qx . (c - 8)
 //              [cider/ops.py w4a8_linear, pack_weight_int4]
 //
-// Persistent, warp-specialised kernel: one CTA per SM walks 128 x BN output
-// tiles (BN = 256, or 128 / 112 when there are too few tiles to fill the GPU) in a
+// Persistent, warp-specialised kernel: one CTA per SM walks MT*128 x BN output
+// tiles (128 x 256; or, when there are too few tiles to fill the GPU, 128 x 128,
+// 128 x 112 or 256 x 112, two 128-token sub-tiles sharing each weight stage) in a
 // grouped order: kGroupM M-tiles walk the N-tiles together, so each weight
 // tile is fetched from HBM about once and reused from L2.
 //   warp 0       TMA producer: A tiles and the B source (int8 B or packed
 //                int4) into a shared-memory ring, mbarrier completion
 //                (expect-tx).
-//   warp 1       allocates two accumulators of BN TMEM columns; one thread
+//   warp 1       allocates two accumulators of MT x BN TMEM columns; one thread
 //                issues tcgen05.mma (kind::i8, M = 128, N = BN, K = 32 per
-//                instruction); tcgen05.commit frees ring slots and transformed
-//                B buffers when their MMAs are done, and publishes each
-//                finished accumulator to the epilogue.
-//   warps 2..5   epilogue: tcgen05.ld of one accumulator (warp q owns TMEM
-//                lanes 32q .. 32q+31 = 32 output rows) while the MMAs of the
-//                next tile fill the other one; scales, bias, 16-byte stores.
-//   warps 6..    (W4A8) BN transform threads turn the packed source into an
+//                instruction, once per sub-tile); tcgen05.commit frees ring
+//                slots and transformed B buffers when their MMAs are done, and
+//                publishes each finished accumulator to the epilogue.
+//   warps 2..    4 MT epilogue warps: tcgen05.ld of one accumulator (warp w owns
+//                TMEM lanes 32 (w % 4) .. +31 = 32 output rows of one sub-tile)
+//                while the MMAs of the next tile fill the other one; scales,
+//                bias, 16-byte stores.
+//   then         (W4A8) BN transform threads turn the packed source into an
 //                MN-major 128-byte-swizzled operand in a 2-deep buffer: a
 //                packed row of k-pairs [K/2][N] is already N-contiguous, so
 //                each 16-byte chunk becomes one 16-byte chunk of K row 2i
@@ -54,20 +56,22 @@ enum Epi { E_I32 = 0, E_SCALED = 1 };
 __host__ __device__ constexpr int rup(int a, int b) { return (a + b - 1) / b * b; }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
-template <int BSRC, int BN>
+template <int BSRC, int BN, int MT>
 struct TcCfg {
     static constexpr int KE = 128;                          // K elements per stage (128 bytes of A)
     static constexpr int XW = BSRC == B_TMA_I8 ? 0 : BN / 32;  // transform warps: one thread per B column
     static constexpr int B_ATOM = 128 * 128;                // MN-major B: one 128-column atom over K = 128
-    static constexpr int A_BYTES = kBM * 128;
+    static constexpr int TM = MT * kBM;                     // tokens per CTA tile: MT sub-tiles of 128
+    static constexpr int EW = MT * kEpiWarps;               // epilogue warps: one per (sub-tile, lane quarter)
+    static constexpr int A_BYTES = TM * 128;
     static constexpr int B_BYTES = BN * 128;                // one K-major swizzled B operand
     static constexpr int RAW_BYTES = BSRC == B_W4 ? (KE / 2) * BN : B_BYTES;
     static constexpr int SLOT = rup(A_BYTES + RAW_BYTES, 1024);
     static constexpr int BRING = XW > 0 ? kBDepth * B_BYTES : 0;  // transformed B ring
     static constexpr int NS = cmin(8, (kSmemBudget - BRING) / SLOT);
-    static constexpr int THREADS = (2 + kEpiWarps + XW) * 32;
-    static constexpr int ACC_COLS = rup(BN, 128);             // TMEM columns between the two accumulators
-    static constexpr int TMEM_COLS = 2 * ACC_COLS;
+    static constexpr int THREADS = (2 + EW + XW) * 32;
+    static constexpr int ACC_COLS = rup(BN, 128);             // TMEM columns between two accumulators
+    static constexpr int TMEM_COLS = 2 * MT * ACC_COLS;       // 2 buffers x MT sub-tiles
     static constexpr uint32_t IDESC =
         (2u << 4) |                                         // D: s32
         (1u << 7) | (1u << 10) |                            // A, B: s8 (signed)
@@ -86,6 +90,7 @@ struct TcCfg {
     };
     static constexpr int SMEM = NS * SLOT + BRING + (int)sizeof(Bars) + 1024;
     static_assert(NS >= 2, "ring too shallow");
+    static_assert(TMEM_COLS <= 512, "tensor memory");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -124,10 +129,10 @@ QLIN_DEV void tile_coords(int t, int tiles_m, int tiles_n, int& mt, int& nt)
 
 QLIN_DEV bool aborted(int* flag) { return *reinterpret_cast<volatile int*>(flag) != 0; }
 
-template <int BSRC, int EPI, int BN>
-__global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(const __grid_constant__ TcParams p)
+template <int BSRC, int EPI, int BN, int MT>
+__global__ void __launch_bounds__(TcCfg<BSRC, BN, MT>::THREADS, 1) tc_gemm_kernel(const __grid_constant__ TcParams p)
 {
-    using Cfg = TcCfg<BSRC, BN>;
+    using Cfg = TcCfg<BSRC, BN, MT>;
     using Bars = typename Cfg::Bars;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -142,6 +147,9 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
     // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
     const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int total = my_tiles * nk;  // ring stages this CTA runs
+    // 128-token sub-tiles of M-tile mt that hold rows (those wholly past M are neither loaded nor
+    // multiplied)
+    auto subtiles = [&](int mt) { return min(MT, (p.M - mt * Cfg::TM + kBM - 1) / kBM); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::NS; ++s) {
@@ -154,7 +162,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.acc_full[b], 1);
-            mbar_init(&bars.acc_empty[b], kEpiWarps);
+            mbar_init(&bars.acc_empty[b], Cfg::EW);
         }
         mbar_init(&bars.mma_done, 1);
         bars.abort_flag = 0;
@@ -181,22 +189,28 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             // (the ordering rule), so the first stages' weight boxes go out before the dependency
             // wait and stream while the activation quantiser runs; the raw int8 GEMM's B may be
             // an activation and waits first
+            auto load_a = [&](int slot, int kb, int mt, int ms) {
+                for (int m = 0; m < ms; ++m)
+                    tma_load_2d(A(slot) + m * (kBM * 128), &p.tm_a, kb * Cfg::KE, mt * Cfg::TM + m * kBM,
+                                &bars.full[slot]);
+            };
             int pre = 0, mt0 = 0, nt0 = 0;
             if (EPI == E_SCALED && my_tiles > 0) {
                 tile_coords((int)blockIdx.x, p.tiles_m, p.tiles_n, mt0, nt0);
                 pre = nk < Cfg::NS ? nk : Cfg::NS;
                 for (int kb = 0; kb < pre; ++kb) {
-                    mbar_arrive_expect_tx(&bars.full[kb], Cfg::A_BYTES + Cfg::RAW_BYTES);
+                    mbar_arrive_expect_tx(&bars.full[kb], subtiles(mt0) * (kBM * 128) + Cfg::RAW_BYTES);
                     load_b(kb, kb, nt0);
                 }
             }
             pdl_wait_prior_grids();  // A (activations) may come from the previous kernel
             for (int kb = 0; kb < pre; ++kb)
-                tma_load_2d(A(kb), &p.tm_a, kb * Cfg::KE, mt0 * kBM, &bars.full[kb]);
+                load_a(kb, kb, mt0, subtiles(mt0));
             int it = 0;
             for (int ti = 0; ti < my_tiles && !aborted(&bars.abort_flag); ++ti) {
                 int mt, nt;
                 tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
+                const int ms = subtiles(mt);
                 int kb = 0;
                 for (; kb < nk; ++kb, ++it) {
                     if (it < pre)
@@ -206,8 +220,8 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
                         bars.abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars.full[slot], Cfg::A_BYTES + Cfg::RAW_BYTES);
-                    tma_load_2d(A(slot), &p.tm_a, kb * Cfg::KE, mt * kBM, &bars.full[slot]);
+                    mbar_arrive_expect_tx(&bars.full[slot], ms * (kBM * 128) + Cfg::RAW_BYTES);
+                    load_a(slot, kb, mt, ms);
                     load_b(slot, kb, nt);
                 }
                 if (kb < nk)
@@ -225,9 +239,12 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             bool ok = true;
             for (int ti = 0; ti < my_tiles && ok; ++ti) {
                 const int buf = ti & 1;
+                int mt, nt;
+                tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
+                const int ms = subtiles(mt);
                 ok = mbar_wait_bounded(&bars.acc_empty[buf], ((ti >> 1) & 1) ^ 1, p.status);
                 tc_fence_after();
-                const uint32_t acc = tmem + (uint32_t)(buf * Cfg::ACC_COLS);
+                const uint32_t acc = tmem + (uint32_t)(buf * MT * Cfg::ACC_COLS);
                 for (int kb = 0; kb < nk && ok; ++kb, ++it) {
                     const int slot = it % Cfg::NS;
                     ok = mbar_wait_bounded(&bars.full[slot], (it / Cfg::NS) & 1, p.status);
@@ -241,10 +258,16 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         // K = 32 per instruction: 32 bytes along a K-major row, or 32 rows (4 swizzle
-                        // groups of 1024 bytes) of the MN-major W4A8 operand
+                        // groups of 1024 bytes) of the MN-major W4A8 operand; every sub-tile of
+                        // tokens multiplies the same B operand
                         const uint64_t bd = Cfg::XW > 0 ? umma_desc_sw128_mn(b0 + kk * 4096, Cfg::B_ATOM)
                                                         : umma_desc_sw128(b0 + kk * 32);
-                        tc_mma<true>(acc, umma_desc_sw128(a0 + kk * 32), bd, Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+                        for (int m = 0; m < MT; ++m)
+                            if (m < ms)
+                                tc_mma<true>(acc + (uint32_t)(m * Cfg::ACC_COLS),
+                                             umma_desc_sw128(a0 + m * (kBM * 128) + kk * 32), bd, Cfg::IDESC,
+                                             (kb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(&bars.empty[slot]);
                     if (Cfg::XW > 0)
@@ -259,9 +282,10 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             mbar_wait_bounded(&bars.mma_done, 0, p.status);
         }
         __syncwarp();
-    } else if (warp < 2 + kEpiWarps) {
+    } else if (warp < 2 + Cfg::EW) {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int msub = (warp - 2) / kEpiWarps;  // token sub-tile this warp reads back
         pdl_wait_prior_grids();  // scales / bias / out may be touched by the previous kernel
         for (int ti = 0; ti < my_tiles; ++ti) {
             const int buf = ti & 1;
@@ -272,14 +296,17 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
             tc_fence_after();
             int mt, nt;
             tile_coords((int)blockIdx.x + ti * (int)gridDim.x, p.tiles_m, p.tiles_n, mt, nt);
-            const int row = mt * kBM + 32 * q + lane;
+            const int row = mt * Cfg::TM + msub * kBM + 32 * q + lane;
             const bool row_ok = row < p.M;
             float sx = 0.f;
             if constexpr (EPI == E_SCALED)
                 sx = row_ok ? p.s_x[row] : 0.f;
-            const uint32_t acc = tmem + (uint32_t)(buf * Cfg::ACC_COLS) + ((uint32_t)(32 * q) << 16);
+            const uint32_t acc =
+                tmem + (uint32_t)((buf * MT + msub) * Cfg::ACC_COLS) + ((uint32_t)(32 * q) << 16);
+            // a sub-tile wholly past M was not multiplied: nothing to read back
+            const int ncols = msub < subtiles(mt) ? BN / 16 : 0;
 #pragma unroll 1
-            for (int c = 0; c < BN / 16; ++c) {
+            for (int c = 0; c < ncols; ++c) {
                 const int n = nt * BN + c * 16;
                 // 16 whole columns with 16-byte aligned rows: vector loads and stores
                 const bool full16 = n + 16 <= p.N && p.vec_out && (p.N % (EPI == E_I32 ? 4 : 8)) == 0;
@@ -372,7 +399,7 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         }
     } else if constexpr (Cfg::XW > 0) {
         // ------------------------------------------------------------ B transform
-        const int tt = threadIdx.x - (2 + kEpiWarps) * 32;  // 0 .. BN - 1
+        const int tt = threadIdx.x - (2 + Cfg::EW) * 32;  // 0 .. BN - 1
         constexpr int CPR = BN / 16;                        // 16-byte chunks per packed row
         constexpr int UNITS = 64 * CPR / (32 * Cfg::XW);    // chunks per thread per stage
         static_assert(UNITS * 32 * Cfg::XW == 64 * CPR, "transform split");
@@ -438,15 +465,15 @@ __global__ void __launch_bounds__(TcCfg<BSRC, BN>::THREADS, 1) tc_gemm_kernel(co
         tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
 
-template <int BSRC, int EPI, int BN>
+template <int BSRC, int EPI, int BN, int MT>
 cudaError_t launch_t(TcParams& prm, cudaStream_t st, const DeviceInfo& dev)
 {
-    using Cfg = TcCfg<BSRC, BN>;
-    auto kern = tc_gemm_kernel<BSRC, EPI, BN>;
+    using Cfg = TcCfg<BSRC, BN, MT>;
+    auto kern = tc_gemm_kernel<BSRC, EPI, BN, MT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess)
         return e;
-    prm.tiles_m = (prm.M + kBM - 1) / kBM;
+    prm.tiles_m = (prm.M + Cfg::TM - 1) / Cfg::TM;
     prm.tiles_n = (prm.N + BN - 1) / BN;
     const int tiles = prm.tiles_m * prm.tiles_n;
     cudaLaunchConfig_t cfg = {};
@@ -475,14 +502,22 @@ bool encode_b(TcOp op, CUtensorMap* tm, const TcGemmArgs& a, int bn)
     }
 }
 
-template <int BN>
+template <int BN, int MT>
 cudaError_t launch_bn(TcOp op, TcParams& prm, cudaStream_t st, const DeviceInfo& dev)
 {
     switch (op) {
-    case TC_I8_RAW: return launch_t<B_TMA_I8, E_I32, BN>(prm, st, dev);
-    case TC_W8A8: return launch_t<B_TMA_I8, E_SCALED, BN>(prm, st, dev);
-    default: return launch_t<B_W4, E_SCALED, BN>(prm, st, dev);  // TC_W4A8
+    case TC_I8_RAW: return launch_t<B_TMA_I8, E_I32, BN, MT>(prm, st, dev);
+    case TC_W8A8: return launch_t<B_TMA_I8, E_SCALED, BN, MT>(prm, st, dev);
+    default: return launch_t<B_W4, E_SCALED, BN, MT>(prm, st, dev);  // TC_W4A8
     }
+}
+
+template <int MT>
+cudaError_t launch_i8_112(TcOp op, TcParams& prm, cudaStream_t st, const DeviceInfo& dev)
+{
+    if (op == TC_I8_RAW)
+        return launch_t<B_TMA_I8, E_I32, 112, MT>(prm, st, dev);
+    return launch_t<B_TMA_I8, E_SCALED, 112, MT>(prm, st, dev);
 }
 
 bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -507,30 +542,45 @@ cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const 
     if (!encode_tmap_2d(&prm.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K,
                         128, kBM))
         return cudaErrorInvalidValue;
-    // 256-column tiles when they still give every SM a tile; else the width that
-    // minimises the per-SM work, (tile rounds) x (tile width): 128, or for an
-    // int8 B operand also 112 (e.g. 2 x 74 tiles = 148 SMs for N = 8192)
-    const int64_t tiles_m = (a.M + kBM - 1) / kBM;
-    int bn = 256;
-    if (tiles_m * ((a.N + 255) / 256) < dev.sm_count) {
-        auto cost = [&](int w) {
-            const int64_t tiles = tiles_m * ((a.N + w - 1) / w);
-            return (tiles + dev.sm_count - 1) / dev.sm_count * w;
-        };
-        bn = 128;
-        if (op != TC_W4A8 && cost(112) < cost(128))
-            bn = 112;
+    // 128 x 256 tiles when they still give every SM a tile. Otherwise the tile shape, MT sub-tiles
+    // of 128 tokens by BN columns, with the least estimated time per SM: (tile rounds) x (the
+    // longer of a K stage's tensor-core work and the time one SM takes to draw the stage's operand
+    // bytes from L2). At these shapes the intake of one SM, about 65 GB/s, is the bound whether
+    // 148 or 74 SMs are busy, so the bytes a tile draws per K step (MT x 128 token rows plus the
+    // weight rows) decide: e.g. for 8192 x 8192 weights, 128 x 112 tiles at 256 tokens (148 tiles,
+    // 240 rows each) and 256 x 112 tiles at 384 or 512 tokens (148 tiles, 368 rows each, instead
+    // of two rounds of 240). Two sub-tiles share each weight stage between two accumulators.
+    const int64_t sms = dev.sm_count;
+    int mt = 1, bn = 256;
+    if (((a.M + kBM - 1) / kBM) * ((a.N + 255) / 256) < sms) {
+        constexpr double kMmaNs = 128.0 * 128 * 2 / 21.5e3;  // ns per token x column of one stage (int8)
+        constexpr double kIntakeNs = 128.0 / 65.0;           // ns per operand row of one stage, one SM
+        double best = 0;
+        for (int m = 1; m <= 2; ++m)
+            for (int w : {256, 128, 112}) {
+                // two sub-tiles with 112-column int8 B tiles only (the other two-sub-tile shapes
+                // were slower wherever they were measured)
+                if ((w == 112 && op == TC_W4A8) || (m == 2 && w != 112))
+                    continue;
+                const int64_t tiles = ((a.M + m * kBM - 1) / (m * kBM)) * ((a.N + w - 1) / w);
+                const int64_t rounds = (tiles + sms - 1) / sms;
+                const double rows = m * kBM + (op == TC_W4A8 ? w / 2 : w);
+                const double mma = kMmaNs * m * w, intake = kIntakeNs * rows;
+                const double t = (double)rounds * (mma > intake ? mma : intake);
+                if (best == 0 || t < best) {
+                    best = t;
+                    mt = m;
+                    bn = w;
+                }
+            }
     }
     if (!encode_b(op, &prm.tm_b, a, bn))
         return cudaErrorInvalidValue;
     if (bn == 256)
-        return launch_bn<256>(op, prm, st, dev);
-    if (bn == 112) {
-        if (op == TC_I8_RAW)
-            return launch_t<B_TMA_I8, E_I32, 112>(prm, st, dev);
-        return launch_t<B_TMA_I8, E_SCALED, 112>(prm, st, dev);
-    }
-    return launch_bn<128>(op, prm, st, dev);
+        return launch_bn<256, 1>(op, prm, st, dev);
+    if (bn == 112)
+        return mt == 2 ? launch_i8_112<2>(op, prm, st, dev) : launch_i8_112<1>(op, prm, st, dev);
+    return launch_bn<128, 1>(op, prm, st, dev);
 }
 
 }  // namespace qlin

@@ -16,7 +16,10 @@ def ql():
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (130, 200, 272), (256, 384, 512), (5, 1000, 4096),
                                    (1280, 4096, 256),  # 160 tiles of 128 x 256: the wide tile path
-                                   (128, 128, 16), (333, 129, 1040)])
+                                   (128, 128, 16), (333, 129, 1040),
+                                   # tiles of two 128-token sub-tiles: the second sub-tile partly past M;
+                                   # a last M-tile of one sub-tile, ragged N and a part stage of K
+                                   (400, 8192, 256), (300, 8000, 160)])
 def test_int8_matmul_int32_bit_exact(ql, orc, M, N, K):
     rng = np.random.default_rng(M * 7 + N)
     a = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
@@ -69,7 +72,9 @@ SMALL = [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
 # a k32 step half past K, rows past N
 SMALL_W8 = SMALL + [synth.IntCase(f"M{M}_K{K}_N{N}", M, K, N, seed=M + K) for (M, K, N) in
                     [(16, 272, 100), (9, 1040, 64), (8, 4096, 520),
-                     (1280, 256, 4096)]]  # the wide (128 x 256) tile path
+                     (1280, 256, 4096),  # the wide (128 x 256) tile path
+                     # two 128-token sub-tiles per tile (one weight stage, two accumulators)
+                     (400, 256, 8192), (300, 160, 8000)]]
 
 
 @pytest.mark.parametrize("case", SMALL_W8, ids=[c.name for c in SMALL_W8])
