@@ -370,7 +370,8 @@ QLIN_DEV uint32_t pack4(int a, int b, int c, int d)
     return prmt(prmt((uint32_t)a, (uint32_t)b, 0x0040u), prmt((uint32_t)c, (uint32_t)d, 0x0040u), 0x5410u);
 }
 
-// the row's absmax over the block (256 threads) from each thread's partial
+// the row's absmax over the block (NW warps) from each thread's partial
+template <int NW = 8>
 QLIN_DEV float block_amax(float amax, float* red)
 {
 #pragma unroll
@@ -381,19 +382,38 @@ QLIN_DEV float block_amax(float amax, float* red)
     __syncthreads();
     amax = red[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i)
+    for (int i = 1; i < NW; ++i)
         amax = fmaxf(amax, red[i]);
     return amax;
 }
 
-// eight bf16 of a 16-byte piece -> four code words pair: codes of elements 0..3 and 4..7
+// eight bf16 of a 16-byte piece -> four code words pair: codes of elements 0..3 and 4..7.
+// The multiply path is tested once for the whole piece (one branch, not eight): when every
+// product lies clear of a half-integer its codes are those sym_code gives; otherwise every
+// element goes through sym_code.
 QLIN_DEV uint2 sym_codes8(const uint4& v, float s, float r, bool fast)
 {
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-    int c[8];
+    float x[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-        c[i] = sym_code(__uint_as_float((i & 1) ? (u[i / 2] & 0xffff0000u) : (u[i / 2] << 16)), s, r, fast);
+        x[i] = __uint_as_float((i & 1) ? (u[i / 2] & 0xffff0000u) : (u[i / 2] << 16));
+    int c[8];
+    if (fast) {
+        bool clear = true;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float m = __fmul_rn(x[i], r);
+            const float t = rintf(m);
+            clear &= fabsf(__fsub_rn(m, t)) < 0.4999f;
+            c[i] = (int)t;
+        }
+        if (clear)
+            return make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        c[i] = sym_code(x[i], s, r, fast);
     return make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
 }
 
@@ -416,6 +436,7 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __res
 {
     if (release)
         pdl_launch_dependents();
+    pdl_wait_prior_grids();  // w and the outputs belong to the stream's earlier kernels until they complete
     __shared__ float red[8];
     const int64_t r = blockIdx.x;
     const TW* row = w + r * C;
@@ -435,17 +456,21 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_kernel(const TW* __res
         qrow[c] = static_cast<int8_t>(sym_code(load_elem(row, c), s, rs, fast));
 }
 
-// Single-pass variant for bf16 rows with C % 8 == 0 and C <= 256 * 8 * VPT: each
+// Single-pass variant for bf16 rows with C % 8 == 0 and C <= NT * 8 * VPT: each
 // thread keeps its VPT 16-byte pieces of the row in registers between the
 // absmax reduction and the quantisation, so the row is read from memory once.
-template <int VPT>
-__global__ void __launch_bounds__(256) quantize_int8_rows_bf16_reg_kernel(const __nv_bfloat16* __restrict__ w,
-                                                                         int64_t C, int8_t* __restrict__ q,
-                                                                         float* __restrict__ scale, int release)
+// A launch of few rows takes NT = 512 or 1024 threads per row: a thread's
+// dependent chain (load, absmax, codes) is then a few pieces long, and the
+// GPU holds enough warps to hide its latency.
+template <int NT, int VPT>
+__global__ void __launch_bounds__(NT) quantize_int8_rows_bf16_reg_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                        int64_t C, int8_t* __restrict__ q,
+                                                                        float* __restrict__ scale, int release)
 {
     if (release)
         pdl_launch_dependents();
-    __shared__ float red[8];
+    pdl_wait_prior_grids();  // w and the outputs belong to the stream's earlier kernels until they complete
+    __shared__ float red[NT / 32];
     const int64_t r = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(w + r * C);
     const int C8 = (int)(C / 8);
@@ -453,11 +478,11 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16_reg_kernel(const 
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-        const int c = (int)threadIdx.x + j * 256;
+        const int c = (int)threadIdx.x + j * NT;
         v[j] = c < C8 ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
         amax = amax8(v[j], amax);
     }
-    amax = block_amax(amax, red);
+    amax = block_amax<NT / 32>(amax, red);
     float s = __fdiv_rn(amax, 127.0f);
     if (s == 0.0f)
         s = 1.0f;
@@ -468,7 +493,7 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16_reg_kernel(const 
     const bool fast = rcp_ok(s);
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-        const int c = (int)threadIdx.x + j * 256;
+        const int c = (int)threadIdx.x + j * NT;
         if (c < C8)
             qrow[c] = sym_codes8(v[j], s, rs, fast);
     }
@@ -481,6 +506,7 @@ __global__ void __launch_bounds__(256) quantize_int8_rows_bf16x8_kernel(const __
 {
     if (release)
         pdl_launch_dependents();
+    pdl_wait_prior_grids();  // w and the outputs belong to the stream's earlier kernels until they complete
     __shared__ float red[8];
     const int64_t r = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(w + r * C);
@@ -987,34 +1013,64 @@ cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, 
     }
 }
 
-cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
-                                      cudaStream_t st, const DeviceInfo&, bool release_dependents)
+// One row per CTA.  With release_dependents (the activation quantiser of an int8 linear) the CTAs
+// let the next kernel of the call start its prologue early -- that kernel waits before reading q
+// and scale.  With as_dependent the launch is itself a programmatic dependent of the stream's
+// previous kernel: its CTAs may be placed while that kernel runs and wait (griddepcontrol.wait)
+// before touching memory.  (Behind the decode GEMVs that made the pair of calls slower: 20.3
+// against 18.0 us at 16 tokens, K = N = 8192; behind the tcgen05 GEMMs it hides the launch.)
+template <typename... KArgs, typename... Args>
+cudaError_t launch_rows(void (*kern)(KArgs...), int64_t R, int nt, cudaStream_t st, bool pdl, Args... args)
 {
-    // The kernel itself starts only after its predecessor completes; with
-    // release_dependents it lets the next (programmatic-dependent) kernel start
-    // its prologue early -- that kernel waits before reading q and scale.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)R, 1, 1);
+    cfg.blockDim = dim3((unsigned)nt, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
+                                      cudaStream_t st, const DeviceInfo& dev, bool release_dependents,
+                                      bool as_dependent)
+{
     const int rel = release_dependents ? 1 : 0;
+    const bool pdl = as_dependent;
     const bool vec = w_dt == QLIN_BF16 && C % 8 == 0 && (reinterpret_cast<uintptr_t>(w) & 15) == 0 &&
                      (reinterpret_cast<uintptr_t>(q) & 7) == 0;
-    if (vec && C <= 256 * 8 * 4)
-        quantize_int8_rows_bf16_reg_kernel<4><<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
-                                                                          scale, rel);
-    else if (vec && C <= 256 * 8 * 8)
-        quantize_int8_rows_bf16_reg_kernel<8><<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
-                                                                          scale, rel);
-    else if (vec)
-        quantize_int8_rows_bf16x8_kernel<<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q,
-                                                                       scale, rel);
-    else if (w_dt == QLIN_BF16)
-        quantize_int8_rows_kernel<__nv_bfloat16>
-            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w), C, q, scale, rel);
-    else if (w_dt == QLIN_F16)
-        quantize_int8_rows_kernel<__half>
-            <<<(unsigned)R, 256, 0, st>>>(static_cast<const __half*>(w), C, q, scale, rel);
-    else
-        quantize_int8_rows_kernel<float><<<(unsigned)R, 256, 0, st>>>(static_cast<const float*>(w), C, q, scale,
-                                                                      rel);
-    return cudaGetLastError();
+    const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(w);
+    const int64_t C8 = C / 8, sms = dev.sm_count;
+    if (vec && R <= 2 * sms && C8 <= 1024 * 4) {  // few rows: 1024 threads per row
+        if (C8 <= 1024)
+            return launch_rows(quantize_int8_rows_bf16_reg_kernel<1024, 1>, R, 1024, st, pdl, wb, C, q, scale, rel);
+        if (C8 <= 2048)
+            return launch_rows(quantize_int8_rows_bf16_reg_kernel<1024, 2>, R, 1024, st, pdl, wb, C, q, scale, rel);
+        return launch_rows(quantize_int8_rows_bf16_reg_kernel<1024, 4>, R, 1024, st, pdl, wb, C, q, scale, rel);
+    }
+    if (vec && R <= 4 * sms && C8 <= 512 * 8) {
+        if (C8 <= 1024)
+            return launch_rows(quantize_int8_rows_bf16_reg_kernel<512, 2>, R, 512, st, pdl, wb, C, q, scale, rel);
+        if (C8 <= 2048)
+            return launch_rows(quantize_int8_rows_bf16_reg_kernel<512, 4>, R, 512, st, pdl, wb, C, q, scale, rel);
+        return launch_rows(quantize_int8_rows_bf16_reg_kernel<512, 8>, R, 512, st, pdl, wb, C, q, scale, rel);
+    }
+    if (vec && C8 <= 256 * 4)
+        return launch_rows(quantize_int8_rows_bf16_reg_kernel<256, 4>, R, 256, st, pdl, wb, C, q, scale, rel);
+    if (vec && C8 <= 256 * 8)
+        return launch_rows(quantize_int8_rows_bf16_reg_kernel<256, 8>, R, 256, st, pdl, wb, C, q, scale, rel);
+    if (vec)
+        return launch_rows(quantize_int8_rows_bf16x8_kernel, R, 256, st, pdl, wb, C, q, scale, rel);
+    if (w_dt == QLIN_BF16)
+        return launch_rows(quantize_int8_rows_kernel<__nv_bfloat16>, R, 256, st, pdl, wb, C, q, scale, rel);
+    if (w_dt == QLIN_F16)
+        return launch_rows(quantize_int8_rows_kernel<__half>, R, 256, st, pdl, static_cast<const __half*>(w), C, q,
+                           scale, rel);
+    return launch_rows(quantize_int8_rows_kernel<float>, R, 256, st, pdl, static_cast<const float*>(w), C, q, scale,
+                       rel);
 }
 
 cudaError_t launch_quantize_weight_int8_clip(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, float pct,

@@ -448,8 +448,9 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
     int8_t* qx = static_cast<int8_t*>(workspace);
     float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)M * (size_t)K));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the quantiser lets the next kernel start its prologue (fetching the layer's weights) early
-    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, st, dev, true);
+    // the quantiser lets the next kernel start its prologue (fetching the layer's weights) early;
+    // ahead of a tcgen05 GEMM it is also placed early itself, behind the stream's previous kernel
+    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, st, dev, true, M > 16);
     if (e != cudaSuccess)
         return from_cuda(e);
     if (M <= 16) {  // decode: weight-streaming GEMV on int8 mma.sync

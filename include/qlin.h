@@ -42,14 +42,17 @@
  *     completed).  Rule: the packed weights and group parameters of a call
  *     must not be written by ANY earlier call of the same run.  A run ends at
  *     every other operation on the stream -- a quantize, dequantize or pack
- *     call, the activation quantiser that opens each w8a8 / w4a8 call or
- *     the preparation kernel that opens a qlin_matmul prefill, a
- *     copy, an event wait, another library's kernel -- because such an
- *     operation starts only after everything before it has completed.  (The
- *     activation quantiser and the preparation kernel do let the second
- *     kernel of their own call start early: it fetches the call's weights
- *     meanwhile and reads the quantiser's or preparation's output only after
- *     its wait.)
+ *     call, the activation quantiser that opens a w8a8 / w4a8 call of at
+ *     most 16 tokens, the preparation kernel that opens a qlin_matmul
+ *     prefill, a copy, an event wait, another library's kernel -- because
+ *     such an operation starts only after everything before it has
+ *     completed.  The activation quantiser of a w8a8 / w4a8 call of more
+ *     than 16 tokens is itself a programmatic dependent: it waits for its
+ *     predecessors before it reads x or writes anything, but it does not
+ *     end the run.  (The activation quantiser and the preparation kernel let
+ *     the second kernel of their own call start early: it fetches the call's
+ *     weights meanwhile and reads the quantiser's or preparation's output
+ *     only after its wait.)
  *   - Every call validates its arguments before launching anything and
  *     returns a qlin_status; nothing is launched when it is not QLIN_OK.
  *     No C++ exception crosses this interface.

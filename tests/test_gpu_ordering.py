@@ -53,3 +53,38 @@ def test_three_chained_calls_with_ordering_point(orc, between):
         yr, mag = orc.bitlinear(c3.x().vals, P3_host, 256, 0.25, False)
         assert_fp_close(y3, yr, mag, None, f"call3 rep {rep}")
     assert ql.device_status() == ql.QLIN_OK
+
+
+@pytest.mark.parametrize("M", [16, 256])
+@pytest.mark.parametrize("op", ["w8a8", "w4a8"])
+def test_int8_linear_chain_shares_workspace(op, M):
+    """Three chained int8 linears on one stream, each layer's output the next one's input and one
+    workspace for all three: the activation quantiser of a call rewrites the workspace that the
+    previous call's GEMM reads, so it must wait for that GEMM (above 16 tokens it is placed early,
+    as a programmatic dependent).  The chain run back to back gives the bits of the same calls
+    separated by synchronisations."""
+    ql = build_lib()
+    K = N = 2048
+    layers = []
+    for l in range(3):
+        w = torch.from_numpy(synth.normal(40 + l, (N, K), 1.0 / np.sqrt(K))).cuda()
+        layers.append(ql.quantize_int8_rows(w) if op == "w8a8" else ql.pack_int4_cols(w.t().contiguous()))
+    f = ql.w8a8_linear if op == "w8a8" else ql.w4a8_linear
+    x0 = synth.activations(44, (M, K), "bf16").torch("cuda")
+    ws = torch.empty(ql.workspace_size(ql.QLIN_OP_W8A8, M, N, K), dtype=torch.uint8, device="cuda")
+
+    def chain(sync):
+        x = x0
+        for wq, sw in layers:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            f(x, wq, sw, out=y, workspace=ws)
+            if sync:
+                torch.cuda.synchronize()
+            x = y
+        torch.cuda.synchronize()
+        return x
+
+    ref = chain(True)
+    assert torch.isfinite(ref.float()).all() and ref.float().abs().max() > 0
+    for _ in range(5):
+        assert torch.equal(chain(False), ref)

@@ -99,7 +99,12 @@ def test_dequantize_word_tail_and_unaligned_bit_exact(ql, orc, bits, aligned):
 
 
 @pytest.mark.parametrize("w_dt", ["f32", "bf16"])
-@pytest.mark.parametrize("shape", [(1, 8192), (7, 1000), (33, 4096), (3, 24), (700, 1000), (1024, 8192), (600, 24)])
+@pytest.mark.parametrize("shape", [(1, 8192), (7, 1000), (33, 4096), (3, 24), (700, 1000), (1024, 8192), (600, 24),
+                                   # launches of few rows: 1024 threads per row with 1, 2 and 4 pieces each
+                                   # (the last ragged), then 512 threads with 2, 4 and 8; the 296 / 297 rows
+                                   # step between the two on a 148-SM part
+                                   (150, 12000), (50, 30000), (296, 8192), (297, 8192), (400, 4096),
+                                   (500, 9000), (300, 20000)])
 def test_quantize_int8_rows_bit_exact(ql, orc, w_dt, shape):
     R, Cc = shape
     w = synth.normal(300 + R, (R, Cc), 1.0)
@@ -110,6 +115,25 @@ def test_quantize_int8_rows_bit_exact(ql, orc, w_dt, shape):
     q, s = ql.quantize_int8_rows(wd)
     torch.cuda.synchronize()
     rq, rs = orc.quantize_int8_rows(wv)
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy(), rs)
+
+
+@pytest.mark.parametrize("w_dt", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(3, 64), (200, 4096), (700, 1000)])
+def test_quantize_int8_rows_half_integer_ties(ql, orc, w_dt, shape):
+    """Rows whose absmax is 127 have scale 1, so half-integers x.5 quantise exactly at a tie (rint
+    rounds to even): every piece of eight leaves the multiply path for the division path."""
+    R, Cc = shape
+    rng = np.random.default_rng(R + Cc)
+    w = (rng.integers(-127, 127, size=(R, Cc)) + 0.5).astype(np.float32)
+    w[:, 0] = 127.0
+    w[::3, 1:9] = np.float32(2.5)  # one piece of ties only
+    wv, wd = _w_dev(w, w_dt)
+    q, s = ql.quantize_int8_rows(wd)
+    torch.cuda.synchronize()
+    rq, rs = orc.quantize_int8_rows(wv)
+    assert np.all(rs == 1.0)
     assert np.array_equal(q.cpu().numpy(), rq)
     assert np.array_equal(s.cpu().numpy(), rs)
 
