@@ -1020,7 +1020,7 @@ cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, 
 // before touching memory.  (Behind the decode GEMVs that made the pair of calls slower: 20.3
 // against 18.0 us at 16 tokens, K = N = 8192; behind the tcgen05 GEMMs it hides the launch.)
 template <typename... KArgs, typename... Args>
-cudaError_t launch_rows(void (*kern)(KArgs...), int64_t R, int nt, cudaStream_t st, bool pdl, Args... args)
+static cudaError_t launch_rows(void (*kern)(KArgs...), int64_t R, int nt, cudaStream_t st, bool pdl, Args... args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)R, 1, 1);
@@ -1034,9 +1034,9 @@ cudaError_t launch_rows(void (*kern)(KArgs...), int64_t R, int nt, cudaStream_t 
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
-                                      cudaStream_t st, const DeviceInfo& dev, bool release_dependents,
-                                      bool as_dependent)
+static cudaError_t launch_quantize_int8_rows_as(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
+                                         float* scale, cudaStream_t st, const DeviceInfo& dev, bool release_dependents,
+                                         bool as_dependent)
 {
     const int rel = release_dependents ? 1 : 0;
     const bool pdl = as_dependent;
@@ -1071,6 +1071,18 @@ cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R,
                            scale, rel);
     return launch_rows(quantize_int8_rows_kernel<float>, R, 256, st, pdl, static_cast<const float*>(w), C, q, scale,
                        rel);
+}
+
+cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q, float* scale,
+                                      cudaStream_t st, const DeviceInfo& dev, bool release_dependents)
+{
+    return launch_quantize_int8_rows_as(w, w_dt, R, C, q, scale, st, dev, release_dependents, false);
+}
+
+cudaError_t launch_quantize_int8_rows_dependent(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
+                                                float* scale, cudaStream_t st, const DeviceInfo& dev)
+{
+    return launch_quantize_int8_rows_as(w, w_dt, R, C, q, scale, st, dev, true, true);
 }
 
 cudaError_t launch_quantize_weight_int8_clip(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, float pct,

@@ -11,6 +11,12 @@ namespace qlin {
 // gives up; qlin_get_device_status() reads and clears it.
 __device__ unsigned g_device_status;
 
+// k_quant.cu: the per-row int8 quantiser launched as a programmatic dependent of the stream's
+// previous kernel (its CTAs may be placed early and wait before touching memory); it also lets
+// the next kernel start its prologue early.
+cudaError_t launch_quantize_int8_rows_dependent(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
+                                                float* scale, cudaStream_t st, const DeviceInfo& dev);
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -450,7 +456,8 @@ qlin_status int_linear(TcOp op, const void* x, qlin_dtype x_dt, int64_t M, int64
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the quantiser lets the next kernel start its prologue (fetching the layer's weights) early;
     // ahead of a tcgen05 GEMM it is also placed early itself, behind the stream's previous kernel
-    cudaError_t e = launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, st, dev, true, M > 16);
+    cudaError_t e = M > 16 ? launch_quantize_int8_rows_dependent(x, x_dt, M, K, qx, sx, st, dev)
+                           : launch_quantize_int8_rows(x, x_dt, M, K, qx, sx, st, dev, true);
     if (e != cudaSuccess)
         return from_cuda(e);
     if (M <= 16) {  // decode: weight-streaming GEMV on int8 mma.sync

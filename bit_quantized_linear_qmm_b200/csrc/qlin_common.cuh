@@ -340,12 +340,8 @@ cudaError_t launch_affine_quantize(const void* w, qlin_dtype w_dt, int64_t N, in
 cudaError_t launch_affine_dequantize(const uint32_t* codes, const void* scales, const void* biases,
                                      qlin_dtype p_dt, int64_t N, int64_t K, int bits, int g, void* out,
                                      qlin_dtype o_dt, cudaStream_t st, const DeviceInfo& dev);
-// release_dependents: the next kernel of the stream may start its prologue before this one
-// ends. as_dependent: this launch is itself a programmatic dependent of the previous kernel
-// (its CTAs may be placed early; they wait before touching memory).
 cudaError_t launch_quantize_int8_rows(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
-                                      float* scale, cudaStream_t st, const DeviceInfo& dev,
-                                      bool release_dependents = false, bool as_dependent = false);
+                                      float* scale, cudaStream_t st, const DeviceInfo& dev, bool release_dependents = false);
 cudaError_t launch_quantize_weight_int8_clip(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, float pct,
                                              int8_t* q, float* scale, cudaStream_t st, const DeviceInfo& dev);
 cudaError_t launch_quantize_int8_groups(const void* w, qlin_dtype w_dt, int64_t N, int64_t K, int g, int8_t* q,
