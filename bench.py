@@ -711,9 +711,9 @@ def _prof_int8_groups():
     return lambda: ql.quantize_int8_groups(w, 128)
 
 
-def _prof_act_quant():
+def _prof_act_quant(M=None):
     from bit_quantized_linear_qmm_b200 import qlin as ql
-    x = synth.INT_LINEAR[2].x().torch("cuda")
+    x = synth.INT_LINEAR[2].x().torch("cuda") if M is None else synth.activations(5, (M, 8192), "bf16").torch("cuda")
     return lambda: ql.quantize_int8_rows(x)
 
 
@@ -736,6 +736,7 @@ PROFILE_CASES = {
     "affine_decode_m1_b8": _prof_affine_b8,
     "affine_quantize_n14336": _prof_quantize,
     "act_quant_m4096": _prof_act_quant,
+    "act_quant_m256": lambda: _prof_act_quant(256),
     "affine_quantize_bf16_n14336": _prof_quantize_bf16,
     "dequantize_n14336": _prof_dequantize,
     "clip_4096": _prof_clip,
