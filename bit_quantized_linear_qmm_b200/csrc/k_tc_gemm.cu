@@ -524,6 +524,43 @@ bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) =
 
 }  // namespace
 
+// The CTA tile of an M x N output on sms SMs: mt sub-tiles of 128 tokens by bn columns.
+void tc_tile_shape(TcOp op, int64_t M, int64_t N, int64_t sms, int& mt, int& bn)
+{
+    // 128 x 256 tiles when they still give every SM a tile. Otherwise the tile shape, MT sub-tiles
+    // of 128 tokens by BN columns, with the least estimated time per SM: (tile rounds) x (the
+    // longer of a K stage's tensor-core work and the time one SM takes to draw the stage's operand
+    // bytes from L2). At these shapes the intake of one SM, about 65 GB/s, is the bound whether
+    // 148 or 74 SMs are busy, so the bytes a tile draws per K step (MT x 128 token rows plus the
+    // weight rows) decide: e.g. for 8192 x 8192 weights, 128 x 112 tiles at 256 tokens (148 tiles,
+    // 240 rows each) and 256 x 112 tiles at 384 or 512 tokens (148 tiles, 368 rows each, instead
+    // of two rounds of 240). Two sub-tiles share each weight stage between two accumulators.
+    mt = 1;
+    bn = 256;
+    if (((M + kBM - 1) / kBM) * ((N + 255) / 256) < sms) {
+        constexpr double kMmaNs = 128.0 * 128 * 2 / 21.5e3;  // ns per token x column of one stage (int8)
+        constexpr double kIntakeNs = 128.0 / 65.0;           // ns per operand row of one stage, one SM
+        double best = 0;
+        for (int m = 1; m <= 2; ++m)
+            for (int w : {256, 128, 112}) {
+                // two sub-tiles with 112-column int8 B tiles only (the other two-sub-tile shapes
+                // were slower wherever they were measured)
+                if ((w == 112 && op == TC_W4A8) || (m == 2 && w != 112))
+                    continue;
+                const int64_t tiles = ((M + m * kBM - 1) / (m * kBM)) * ((N + w - 1) / w);
+                const int64_t rounds = (tiles + sms - 1) / sms;
+                const double rows = m * kBM + (op == TC_W4A8 ? w / 2 : w);
+                const double mma = kMmaNs * m * w, intake = kIntakeNs * rows;
+                const double t = (double)rounds * (mma > intake ? mma : intake);
+                if (best == 0 || t < best) {
+                    best = t;
+                    mt = m;
+                    bn = w;
+                }
+            }
+    }
+}
+
 cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const DeviceInfo& dev)
 {
     TcParams prm;
@@ -542,38 +579,8 @@ cudaError_t launch_tc_gemm(TcOp op, const TcGemmArgs& a, cudaStream_t st, const 
     if (!encode_tmap_2d(&prm.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K,
                         128, kBM))
         return cudaErrorInvalidValue;
-    // 128 x 256 tiles when they still give every SM a tile. Otherwise the tile shape, MT sub-tiles
-    // of 128 tokens by BN columns, with the least estimated time per SM: (tile rounds) x (the
-    // longer of a K stage's tensor-core work and the time one SM takes to draw the stage's operand
-    // bytes from L2). At these shapes the intake of one SM, about 65 GB/s, is the bound whether
-    // 148 or 74 SMs are busy, so the bytes a tile draws per K step (MT x 128 token rows plus the
-    // weight rows) decide: e.g. for 8192 x 8192 weights, 128 x 112 tiles at 256 tokens (148 tiles,
-    // 240 rows each) and 256 x 112 tiles at 384 or 512 tokens (148 tiles, 368 rows each, instead
-    // of two rounds of 240). Two sub-tiles share each weight stage between two accumulators.
-    const int64_t sms = dev.sm_count;
-    int mt = 1, bn = 256;
-    if (((a.M + kBM - 1) / kBM) * ((a.N + 255) / 256) < sms) {
-        constexpr double kMmaNs = 128.0 * 128 * 2 / 21.5e3;  // ns per token x column of one stage (int8)
-        constexpr double kIntakeNs = 128.0 / 65.0;           // ns per operand row of one stage, one SM
-        double best = 0;
-        for (int m = 1; m <= 2; ++m)
-            for (int w : {256, 128, 112}) {
-                // two sub-tiles with 112-column int8 B tiles only (the other two-sub-tile shapes
-                // were slower wherever they were measured)
-                if ((w == 112 && op == TC_W4A8) || (m == 2 && w != 112))
-                    continue;
-                const int64_t tiles = ((a.M + m * kBM - 1) / (m * kBM)) * ((a.N + w - 1) / w);
-                const int64_t rounds = (tiles + sms - 1) / sms;
-                const double rows = m * kBM + (op == TC_W4A8 ? w / 2 : w);
-                const double mma = kMmaNs * m * w, intake = kIntakeNs * rows;
-                const double t = (double)rounds * (mma > intake ? mma : intake);
-                if (best == 0 || t < best) {
-                    best = t;
-                    mt = m;
-                    bn = w;
-                }
-            }
-    }
+    int mt, bn;
+    tc_tile_shape(op, a.M, a.N, dev.sm_count, mt, bn);
     if (!encode_b(op, &prm.tm_b, a, bn))
         return cudaErrorInvalidValue;
     if (bn == 256)

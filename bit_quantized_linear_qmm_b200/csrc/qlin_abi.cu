@@ -16,6 +16,8 @@ __device__ unsigned g_device_status;
 // the next kernel start its prologue early.
 cudaError_t launch_quantize_int8_rows_dependent(const void* w, qlin_dtype w_dt, int64_t R, int64_t C, int8_t* q,
                                                 float* scale, cudaStream_t st, const DeviceInfo& dev);
+// k_tc_gemm.cu: the CTA tile of the int8 tcgen05 GEMM, mt sub-tiles of 128 tokens by bn columns.
+void tc_tile_shape(TcOp op, int64_t M, int64_t N, int64_t sms, int& mt, int& bn);
 
 namespace {
 
@@ -124,6 +126,17 @@ const char* qlin_status_string(qlin_status s)
 }
 
 int qlin_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+qlin_status qlin_int8_gemm_tile(qlin_op op, int64_t M, int64_t N, int sm_count, int* tokens, int* columns)
+{
+    if ((op != QLIN_OP_W8A8 && op != QLIN_OP_W4A8) || M < 1 || N < 1 || sm_count < 1 || !tokens || !columns)
+        return QLIN_ERR_INVALID_ARG;
+    int mt = 1, bn = 256;
+    tc_tile_shape(op == QLIN_OP_W4A8 ? TC_W4A8 : TC_W8A8, M, N, sm_count, mt, bn);
+    *tokens = 128 * mt;
+    *columns = bn;
+    return QLIN_OK;
+}
 
 size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size)
 {

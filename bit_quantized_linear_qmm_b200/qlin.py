@@ -66,6 +66,7 @@ def lib():
         "qlin_status_string": ([I], C.c_char_p),
         "qlin_version": ([], I),
         "qlin_workspace_size": ([I, I64, I64, I64, I, I], SZ),
+        "qlin_int8_gemm_tile": ([I, I64, I64, I, P, P], I),
         "qlin_quantize": ([P, I, I64, I64, I, I, P, P, P, I, P], I),
         "qlin_dequantize": ([P, P, P, I, I64, I64, I, I, P, I, P], I),
         "qlin_matmul": ([P, I, I64, I64, P, P, P, I, I64, I, I, P, P, P, SZ, P], I),
@@ -132,6 +133,13 @@ def _cuda(*ts):
 
 def workspace_size(op: int, M: int, N: int, K: int, bits: int = 0, group_size: int = 0) -> int:
     return int(lib().qlin_workspace_size(op, M, N, K, bits, group_size))
+
+
+def int8_gemm_tile(op: int, M: int, N: int, sm_count: int) -> tuple[int, int]:
+    """(tokens, columns) of the int8 tensor-core GEMM's CTA tile for an M x N output."""
+    t, c = C.c_int(0), C.c_int(0)
+    _check(lib().qlin_int8_gemm_tile(op, M, N, sm_count, C.byref(t), C.byref(c)), "qlin_int8_gemm_tile")
+    return t.value, c.value
 
 
 def quantize(w: torch.Tensor, bits: int, group_size: int, param_dtype=torch.bfloat16):

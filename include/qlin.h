@@ -112,6 +112,20 @@ int qlin_version(void);
 size_t qlin_workspace_size(qlin_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size);
 
 /*
+ * The CTA tile the int8 tensor-core GEMM takes for an M x N output on a GPU
+ * of sm_count SMs: *tokens = 128 or 256 rows, *columns = 256, 128 or 112.
+ * This GEMM serves qlin_int8_matmul_int32 and w8a8_linear / w4a8_linear
+ * above 16 tokens.  op: QLIN_OP_W8A8 for int8 weights (also the raw int8
+ * GEMM), QLIN_OP_W4A8 for packed int4 weights.  With fewer 128 x 256 tiles
+ * than SMs, the shape minimises (tile rounds) x (operand rows one SM draws
+ * per K step): one SM's intake from L2 bounds these shapes.  A 256-row tile
+ * is two 128-token sub-tiles sharing each weight stage.  A pure host
+ * function: no device call, any thread.  QLIN_ERR_INVALID_ARG for another
+ * op, M < 1, N < 1, sm_count < 1 or a NULL output.
+ */
+qlin_status qlin_int8_gemm_tile(qlin_op op, int64_t M, int64_t N, int sm_count, int* tokens, int* columns);
+
+/*
  * Affine group quantisation of a dense weight [nuvec-nn QuantizedLinear,
  * from_linear; cider/ops.py pergroup_linear docstring, quantize formula].
  * Per group of `group_size` consecutive inputs of one output row:

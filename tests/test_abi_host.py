@@ -96,3 +96,27 @@ def test_empty_inputs_rejected_before_device(ql):
     assert L.pergroup_linear(P16, 1, 0, 128, P16, P16, 16, 64, None, P16, P16, 4096, None) == ql.QLIN_ERR_INVALID_ARG
     assert L.qlin_quantize_int8_groups(P16, 1, 16, 0, 64, P16, P16, None) == ql.QLIN_ERR_INVALID_ARG
     assert L.qlin_quantize_weight_int8(P16, 1, 0, 64, -1.0, P16, P16, None) == ql.QLIN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("op,M,N,want", [
+    # int8 weights, K = N = 8192 on 148 SMs: 148 tiles of 128 x 112 at 256 tokens (one round; 256 x 112
+    # tiles took 41.6 us there against 30.9), 148 tiles of 256 x 112 at 384 and 512 tokens (41.6 / 43.6 us
+    # against 50.2 / 51.8 for two rounds of 128 x 112), 128 x 256 once they fill every SM
+    ("W8A8", 256, 8192, (128, 112)), ("W8A8", 384, 8192, (256, 112)), ("W8A8", 512, 8192, (256, 112)),
+    ("W8A8", 4096, 8192, (128, 256)), ("W8A8", 512, 4096, (128, 112)), ("W8A8", 1, 8192, (128, 112)),
+    # packed int4 weights: 128 x 128 at 256 tokens (39.1 us; 128 x 256: 48.5), 128 x 256 at 384 (49.4 us
+    # against 66.8 for two rounds of 128 x 128)
+    ("W4A8", 256, 8192, (128, 128)), ("W4A8", 384, 8192, (128, 256)), ("W4A8", 4096, 8192, (128, 256)),
+])
+def test_int8_gemm_tile_choice(ql, op, M, N, want):
+    """The int8 tensor-core GEMM's CTA tile on a 148-SM part, pinned to the shapes that timed fastest."""
+    assert ql.int8_gemm_tile(getattr(ql, "QLIN_OP_" + op), M, N, 148) == want
+
+
+def test_int8_gemm_tile_rejects(ql):
+    t, c = C.c_int(0), C.c_int(0)
+    L = ql.lib()
+    for args in [(ql.QLIN_OP_MATMUL, 256, 8192, 148), (ql.QLIN_OP_W8A8, 0, 8192, 148),
+                 (ql.QLIN_OP_W8A8, 256, 0, 148), (ql.QLIN_OP_W4A8, 256, 8192, 0)]:
+        assert L.qlin_int8_gemm_tile(*args, C.byref(t), C.byref(c)) == ql.QLIN_ERR_INVALID_ARG, args
+    assert L.qlin_int8_gemm_tile(ql.QLIN_OP_W8A8, 256, 8192, 148, None, C.byref(c)) == ql.QLIN_ERR_INVALID_ARG

@@ -29,6 +29,14 @@ def test_int8_matmul_int32_bit_exact(ql, orc, M, N, K):
     assert np.array_equal(c.cpu().numpy(), orc.int8_matmul(a, b))
 
 
+@pytest.mark.parametrize("op,M,N", [("W8A8", 400, 8192), ("W8A8", 300, 8000)])
+def test_two_subtile_cases_take_that_tile(ql, op, M, N):
+    """The parity cases above and below that stand for tiles of two 128-token sub-tiles get that
+    tile on this device."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert ql.int8_gemm_tile(getattr(ql, "QLIN_OP_" + op), M, N, sms) == (256, 112)
+
+
 def test_int8_matmul_extremes(ql, orc):
     """All -128 times all -128 over K = 4096 -> 2^26 per element (exact int32)."""
     a = np.full((130, 4096), -128, np.int8)
