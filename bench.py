@@ -756,6 +756,8 @@ PROFILE_CASES = {
     "w4a8_m1": lambda: _prof_int("w4a8", 1),
     "w8a8_m256": lambda: _prof_int("w8a8", 256),
     "w4a8_m256": lambda: _prof_int("w4a8", 256),
+    "w8a8_m384": lambda: _prof_int("w8a8", 384),  # 256 x 112 tiles of two token sub-tiles
+    "w4a8_m384": lambda: _prof_int("w4a8", 384),
 }
 
 
